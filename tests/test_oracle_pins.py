@@ -268,16 +268,18 @@ def test_two_loop_equals_dense_bfgs_inverse_update():
     np.testing.assert_allclose(O.two_loop_direction(g, [], []), -g)
 
 
-def test_armijo_halving_count_on_quadratic():
+@pytest.mark.parametrize("c1", [1e-4, 0.5])
+def test_armijo_halving_count_on_quadratic(c1):
     """f(x) = a x^2 / 2, empty history: d = -g, t0 = min(1, 1/|g|), the accepted
-    step is t0 / 2^j with j the least integer meeting the Armijo condition."""
+    step is t0 / 2^j with j the least integer meeting the Armijo condition.
+    With u = t a the condition reads (1-u)^2 <= 1 - 2 c1 u, so c1 = 0.5 rejects
+    the steps 1 < u < 2 that plain decrease would take (first case: u = 5/3)."""
     for a, x0 in [(50.0, 0.3), (3.0, 2.0), (400.0, -0.01)]:
         f = lambda x: 0.5 * a * float(x[0]) ** 2
         gr = lambda x: np.array([a * float(x[0])])
         st = O.LBFGSState(x=np.array([x0]), f=f([x0]), g=gr([x0]))
         g0 = a * x0
         t = min(1.0, 1.0 / abs(g0))
-        c1 = 1e-4
         while not (0.5 * a * (x0 - t * g0) ** 2 <= 0.5 * a * x0 ** 2 - c1 * t * g0 * g0):
             t *= 0.5
         assert O.lbfgs_step(st, f, gr, c1=c1)
