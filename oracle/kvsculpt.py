@@ -351,7 +351,8 @@ def _clamped_shares(w, lo, hi, total):
     else:
         return shares(cuts[-1])
     base = shares(prev)
-    free = pos & (prev * w >= lo) & (prev * w < hi)
+    mid = 0.5 * (prev + c)  # no breakpoint lies strictly inside (prev, c)
+    free = pos & (mid * w > lo) & (mid * w < hi)
     slope = w[free].sum()
     if slope <= 0.0:
         return shares(c)
@@ -365,7 +366,9 @@ def pilot_allocate(mse, total: int, k_min: int, k_max, alpha: float = 0.5) -> np
     The page gives the law (budget proportional to the square root of the pilot
     MSE, at layer and KV-head granularity); the bounds and the integer rounding
     are this restatement's reading: the real-valued shares are
-    x_b = clip(c * MSE_b^alpha, k_min, k_max_b) with sum x_b = total, and the
+    x_b = clip(c * MSE_b^alpha, k_min, k_max_b) with sum x_b = total (if the
+    problems with a positive MSE cannot absorb the budget even at k_max, the
+    zero-MSE problems share the remainder evenly), and the
     integers are floor(x_b) plus one unit for the largest fractional parts
     (ties to the lower problem index) until the total is met.
     """
@@ -378,7 +381,15 @@ def pilot_allocate(mse, total: int, k_min: int, k_max, alpha: float = 0.5) -> np
     w = np.where(np.isfinite(mse) & (mse > 0), mse, 0.0) ** alpha
     if w.sum() <= 0.0:
         w = np.ones(B)
-    ideal = _clamped_shares(w, lo, hi, float(total))
+    pos = w > 0
+    if hi[pos].sum() + lo[~pos].sum() < total:
+        # the problems with a positive signal cannot absorb the budget: they all get
+        # k_max and the zero-signal problems share the rest evenly
+        ideal = hi.copy()
+        ideal[~pos] = _clamped_shares(np.ones(int((~pos).sum())), lo[~pos], hi[~pos],
+                                      float(total - hi[pos].sum()))
+    else:
+        ideal = _clamped_shares(w, lo, hi, float(total))
     base = np.floor(ideal)
     frac = ideal - base
     k = base.astype(np.int64)

@@ -368,3 +368,33 @@ def test_allocation_brute_force(seed):
             best, best_cost = cand, cost
     assert tuple(got) == best
     assert got.sum() == total and np.all(got >= k_min) and np.all(got <= k_max)
+
+
+@pytest.mark.parametrize("seed", range(25))
+def test_allocation_spends_the_whole_budget(seed):
+    """The budget is redistributed, not reduced: the real shares sum to the
+    total, sit inside their bounds and are proportional to MSE^0.5 wherever
+    unclamped (compared with a bisection on the proportionality constant)."""
+    r = np.random.default_rng(900 + seed)
+    B = int(r.integers(5, 120))
+    k_min = int(r.integers(1, 20))
+    k_max = r.integers(k_min, 2000, size=B)
+    total = int(r.integers(B * k_min, int(k_max.sum()) + 1))
+    mse = np.exp(r.uniform(-8, 4, size=B))
+    from oracle.kvsculpt import _clamped_shares
+    w = np.sqrt(mse)
+    lo, hi = np.full(B, float(k_min)), k_max.astype(float)
+    x = _clamped_shares(w, lo, hi, float(total))
+    assert abs(x.sum() - total) < 1e-6 * total
+    np.testing.assert_allclose(x, _shares_by_bisection(w, lo, hi, total), rtol=1e-9, atol=1e-9)
+    k = O.pilot_allocate(mse, total, k_min, k_max, 0.5)
+    assert k.sum() == total and np.all(np.abs(k - x) < 1.0)
+
+
+def test_allocation_zero_signal_absorbs_leftover():
+    """Zero-MSE problems weigh 0; when the others are all at k_max the rest of
+    the budget is shared evenly among the zero-MSE problems (hand-derived)."""
+    k = O.pilot_allocate([0.0, 4.0, 0.0], 50, 5, [30, 10, 30], 0.5)
+    assert k.tolist() == [20, 10, 20]
+    k = O.pilot_allocate([0.0, 4.0, 0.0], 20, 5, [30, 10, 30], 0.5)
+    assert k.tolist() == [5, 10, 5]
