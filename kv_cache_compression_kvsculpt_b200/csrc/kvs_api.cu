@@ -1,0 +1,414 @@
+// C ABI of the KVSculpt library: argument validation, workspace layout and
+// the orchestration of the kernels for each call (see include/kvsculpt.h).
+#include <math.h>
+#include <stdio.h>
+#include <string.h>
+
+#include <algorithm>
+#include <cstddef>
+#include <vector>
+
+#include "kvs_internal.cuh"
+
+namespace kvs {
+
+static thread_local char g_err[256] = "no error";
+
+void set_cuda_error(cudaError_t e, const char *where) {
+  snprintf(g_err, sizeof g_err, "%s: %s (%s)", where, cudaGetErrorName(e), cudaGetErrorString(e));
+}
+
+static bool aligned(const void *p, size_t a) { return ((uintptr_t)p % a) == 0; }
+
+static int check_offsets(const int64_t *off, int B, int64_t *sum, int *mx, bool allow_empty) {
+  if (!off || off[0] != 0) return KVS_EINVAL;
+  int64_t m = 0;
+  for (int b = 0; b < B; ++b) {
+    const int64_t n = off[b + 1] - off[b];
+    if (n < (allow_empty ? 0 : 1) || n > (1 << 30)) return KVS_EINVAL;
+    m = std::max(m, n);
+  }
+  *sum = off[B];
+  *mx = (int)m;
+  return KVS_OK;
+}
+
+int geom_from_batch(const kvs_batch *b, HostGeom *g, bool need_c) {
+  if (!b || b->B < 1 || (b->d != 64 && b->d != 128)) return b && b->B >= 1 ? KVS_ENOTSUP : KVS_EINVAL;
+  if (!b->q_off || !b->z_off || !b->q_off_h || !b->z_off_h) return KVS_EINVAL;
+  *g = HostGeom{};
+  g->B = b->B;
+  g->d = b->d;
+  if (check_offsets(b->q_off_h, b->B, &g->sum_q, &g->max_q, false)) return KVS_EINVAL;
+  if (check_offsets(b->z_off_h, b->B, &g->sum_z, &g->max_z, false)) return KVS_EINVAL;
+  if (need_c) {
+    if (!b->c_off || !b->c_off_h) return KVS_EINVAL;
+    if (check_offsets(b->c_off_h, b->B, &g->sum_c, &g->max_c, false)) return KVS_EINVAL;
+  } else if (b->c_off_h) {
+    if (check_offsets(b->c_off_h, b->B, &g->sum_c, &g->max_c, true)) return KVS_EINVAL;
+  }
+  g->ld_s = align_up(std::max<int64_t>(std::max(g->max_z, g->max_c), 4), 4);
+  return KVS_OK;
+}
+
+// Bump allocator over a caller buffer (256-byte aligned pieces).
+struct Carver {
+  char *base;
+  size_t off = 0;
+  template <class T>
+  T *take(int64_t count) {
+    off = (size_t)align_up((int64_t)off, 256);
+    T *p = base ? reinterpret_cast<T *>(base + off) : nullptr;
+    off += (size_t)std::max<int64_t>(count, 0) * sizeof(T);
+    return p;
+  }
+};
+
+size_t carve_work(const HostGeom &g, void *base, Work *w) {
+  Carver c{static_cast<char *>(base)};
+  w->S = c.take<float>(g.sum_q * g.ld_s);
+  w->Yh = c.take<float>(g.sum_q * g.d);
+  w->Go = c.take<float>(g.sum_q * g.d);
+  w->lse_h = c.take<float>(g.sum_q);
+  w->delta = c.take<float>(g.sum_q);
+  w->row_out = c.take<float>(g.sum_q);
+  w->row_ls = c.take<float>(g.sum_q);
+  w->gram = c.take<float>(g.sum_c * g.max_c);
+  w->chol = c.take<double>(g.sum_c * g.max_c);
+  w->xs = c.take<double>(g.sum_c * g.d);
+  w->R = c.take<float>(g.sum_c * g.d);
+  w->fbuf = c.take<float>(g.B);
+  w->Yt = c.take<float>(g.sum_q * g.d);
+  w->lset = c.take<float>(g.sum_q);
+  w->imp = c.take<float>(g.sum_z);
+  w->idx = c.take<int32_t>(g.sum_c);
+  w->bytes = align_up((int64_t)c.off, 256);
+  return w->bytes;
+}
+
+size_t carve_state(const HostGeom &g, int h, void *base, State *s) {
+  Carver c{static_cast<char *>(base)};
+  const int64_t n = g.sum_c * g.d;
+  s->sc = c.take<LbfgsScal>(g.B);
+  s->x = c.take<float>(n);
+  s->g = c.take<float>(n);
+  s->dir = c.take<float>(n);
+  s->gn = c.take<float>(n);
+  s->ring_s = c.take<float>((int64_t)(h + 1) * n);
+  s->ring_y = c.take<float>((int64_t)(h + 1) * n);
+  s->h = h;
+  s->bytes = align_up((int64_t)c.off, 256);
+  return s->bytes;
+}
+
+static int prep(const kvs_batch *b, bool need_c, void *ws, size_t ws_bytes, void *stream,
+                Batch *Bt, Work *w) {
+  int rc = geom_from_batch(b, &Bt->g, need_c);
+  if (rc) return rc;
+  Bt->b = b;
+  Bt->st = static_cast<cudaStream_t>(stream);
+  if (!ws || !aligned(ws, 256)) return KVS_EINVAL;
+  if (carve_work(Bt->g, nullptr, w) > ws_bytes) return KVS_EWORKSPACE;
+  carve_work(Bt->g, ws, w);
+  return KVS_OK;
+}
+
+static bool ok_ptr(const void *p) { return p && aligned(p, 16); }
+
+static bool ok_sched(const kvs_schedule *s) {
+  return s && s->outer >= 0 && s->steps >= 0 && s->history >= 1 && s->history <= 15 &&
+         s->max_bt >= 1 && s->max_bt <= 64 && s->backtrack > 0.f && s->backtrack < 1.f &&
+         s->c1 > 0.f && s->c1 < 1.f && isfinite(s->lambda) && s->w_out >= 0.f && s->w_lse >= 0.f;
+}
+
+static Filter phase_filter(const State &s, int want) {
+  return Filter{reinterpret_cast<const int *>(reinterpret_cast<const char *>(s.sc) +
+                                              offsetof(LbfgsScal, phase)),
+                (int)(sizeof(LbfgsScal) / sizeof(int)), want};
+}
+
+static const Filter ALL{nullptr, 0, 0};
+
+// Loss and gradient at Kc into (w.fbuf, s.gn), then the state reset.
+static int lbfgs_restart(const Batch &Bt, const kvs_schedule &sc, const float *Q, const float *Y,
+                         const float *lse, const float *Vc, const float *Kc, const State &s,
+                         int clear, const Work &w) {
+  int rc = launch_forward(Bt, Q, Kc, Vc, Y, lse, sc.w_out, sc.w_lse, w.fbuf, nullptr, ALL, w);
+  if (rc) return rc;
+  rc = launch_backward(Bt, Q, Vc, s.gn, ALL, w);
+  if (rc) return rc;
+  return launch_lbfgs_reset(Bt, s, Kc, w.fbuf, s.gn, clear);
+}
+
+static int lbfgs_one_step(const Batch &Bt, const kvs_schedule &sc, const float *Q,
+                          const float *Y, const float *lse, const float *Vc, float *Kc,
+                          const State &s, int32_t *status, float *f_out, const Work &w) {
+  int rc = launch_lbfgs_direction(Bt, s, sc);
+  if (rc) return rc;
+  const Filter searching = phase_filter(s, PH_SEARCH);
+  for (int t = 0; t < sc.max_bt; ++t) {
+    if ((rc = launch_lbfgs_trial(Bt, s, Kc))) return rc;
+    if ((rc = launch_forward(Bt, Q, Kc, Vc, Y, lse, sc.w_out, sc.w_lse, w.fbuf, nullptr,
+                             searching, w)))
+      return rc;
+    if ((rc = launch_lbfgs_armijo(Bt, s, sc, w.fbuf))) return rc;
+  }
+  if ((rc = launch_backward(Bt, Q, Vc, s.gn, phase_filter(s, PH_ACCEPT), w))) return rc;
+  return launch_lbfgs_update(Bt, s, Kc, status, f_out);
+}
+
+}  // namespace kvs
+
+using namespace kvs;
+
+extern "C" {
+
+const char *kvs_version(void) { return "kvsculpt-b200 0.1 (sm_100a)"; }
+
+const char *kvs_last_cuda_error(void) { return g_err; }
+
+size_t kvs_workspace_bytes(const kvs_batch *batch, const kvs_schedule *) {
+  HostGeom g;
+  if (geom_from_batch(batch, &g, false)) return 0;
+  Work w;
+  return carve_work(g, nullptr, &w);
+}
+
+size_t kvs_lbfgs_state_bytes(const kvs_batch *batch, int32_t history) {
+  HostGeom g;
+  if (history < 1 || history > 15 || geom_from_batch(batch, &g, true)) return 0;
+  State s;
+  return carve_state(g, history, nullptr, &s);
+}
+
+int kvs_build_queries(const kvs_query_spec *sp, const float *q_retain, const float *q_ctx,
+                      const int32_t *pos, float *Q, void *stream) {
+  if (!sp || sp->B < 1 || sp->g < 1 || sp->m_q < 0 || sp->n_syn < 0 || sp->N < 1 ||
+      !(sp->rope_base > 1.f))
+    return KVS_EINVAL;
+  if (sp->d != 64 && sp->d != 128) return KVS_ENOTSUP;
+  if (!ok_ptr(Q) || (sp->m_q > 0 && !ok_ptr(q_retain)) ||
+      (sp->n_syn > 0 && (!ok_ptr(q_ctx) || !ok_ptr(pos))))
+    return KVS_EINVAL;
+  return launch_build_queries(sp, q_retain, q_ctx, pos, Q, static_cast<cudaStream_t>(stream));
+}
+
+int kvs_targets(const kvs_batch *batch, const float *Q, const float *Kz, const float *Vz,
+                float *Y, float *lse, float *importance, void *ws, size_t ws_bytes,
+                void *stream) {
+  Batch Bt;
+  Work w;
+  int rc = prep(batch, false, ws, ws_bytes, stream, &Bt, &w);
+  if (rc) return rc;
+  if (!ok_ptr(Q) || !ok_ptr(Kz) || !ok_ptr(Vz) || !ok_ptr(Y) || !ok_ptr(lse) ||
+      (importance && !ok_ptr(importance)))
+    return KVS_EINVAL;
+  return launch_targets(Bt, Q, Kz, Vz, Y, lse, importance, w);
+}
+
+int kvs_init_topk(const kvs_batch *batch, const float *importance, const float *Kz,
+                  int32_t *idx, float *Kc, void *stream) {
+  HostGeom g;
+  int rc = geom_from_batch(batch, &g, true);
+  if (rc) return rc;
+  if (!ok_ptr(importance) || !ok_ptr(Kz) || !ok_ptr(idx) || !ok_ptr(Kc)) return KVS_EINVAL;
+  if (g.max_z > 16384) return KVS_ENOTSUP;
+  for (int b = 0; b < g.B; ++b)
+    if (batch->c_off_h[b + 1] - batch->c_off_h[b] > batch->z_off_h[b + 1] - batch->z_off_h[b])
+      return KVS_EINVAL;
+  Batch Bt{g, batch, static_cast<cudaStream_t>(stream)};
+  return launch_topk(Bt, importance, Kz, idx, Kc);
+}
+
+int kvs_loss_grad(const kvs_batch *batch, const float *Q, const float *Kc, const float *Vc,
+                  const float *Y, const float *lse, float w_out, float w_lse, float *loss,
+                  float *parts, float *dKc, void *ws, size_t ws_bytes, void *stream) {
+  Batch Bt;
+  Work w;
+  int rc = prep(batch, true, ws, ws_bytes, stream, &Bt, &w);
+  if (rc) return rc;
+  if (!ok_ptr(Q) || !ok_ptr(Kc) || !ok_ptr(Vc) || !ok_ptr(Y) || !ok_ptr(lse) || !ok_ptr(loss) ||
+      (parts && !ok_ptr(parts)) || (dKc && !ok_ptr(dKc)))
+    return KVS_EINVAL;
+  rc = launch_forward(Bt, Q, Kc, Vc, Y, lse, w_out, w_lse, loss, parts, ALL, w);
+  if (rc || !dKc) return rc;
+  return launch_backward(Bt, Q, Vc, dKc, ALL, w);
+}
+
+int kvs_fit_values(const kvs_batch *batch, const float *Q, const float *Kc, const float *Y,
+                   float lambda, float *Vc, int32_t *status, void *ws, size_t ws_bytes,
+                   void *stream) {
+  Batch Bt;
+  Work w;
+  int rc = prep(batch, true, ws, ws_bytes, stream, &Bt, &w);
+  if (rc) return rc;
+  if (!ok_ptr(Q) || !ok_ptr(Kc) || !ok_ptr(Y) || !ok_ptr(Vc) || !ok_ptr(status) ||
+      !isfinite(lambda))
+    return KVS_EINVAL;
+  return launch_fit(Bt, Q, Kc, Y, lambda, Vc, status, w);
+}
+
+static int prep_state(const Batch &Bt, const kvs_schedule *sched, void *state,
+                      size_t state_bytes, State *s) {
+  if (!ok_sched(sched) || !state || !aligned(state, 256)) return KVS_EINVAL;
+  if (carve_state(Bt.g, sched->history, nullptr, s) > state_bytes) return KVS_EWORKSPACE;
+  carve_state(Bt.g, sched->history, state, s);
+  return KVS_OK;
+}
+
+int kvs_lbfgs_reset(const kvs_batch *batch, const kvs_schedule *sched, const float *Q,
+                    const float *Y, const float *lse, const float *Vc, const float *Kc,
+                    void *state, size_t state_bytes, int32_t clear_history, void *ws,
+                    size_t ws_bytes, void *stream) {
+  Batch Bt;
+  Work w;
+  State s;
+  int rc = prep(batch, true, ws, ws_bytes, stream, &Bt, &w);
+  if (rc) return rc;
+  if ((rc = prep_state(Bt, sched, state, state_bytes, &s))) return rc;
+  if (!ok_ptr(Q) || !ok_ptr(Y) || !ok_ptr(lse) || !ok_ptr(Vc) || !ok_ptr(Kc)) return KVS_EINVAL;
+  return lbfgs_restart(Bt, *sched, Q, Y, lse, Vc, Kc, s, clear_history != 0, w);
+}
+
+int kvs_lbfgs_step(const kvs_batch *batch, const kvs_schedule *sched, const float *Q,
+                   const float *Y, const float *lse, const float *Vc, float *Kc, void *state,
+                   size_t state_bytes, int32_t *status, float *f_out, void *ws, size_t ws_bytes,
+                   void *stream) {
+  Batch Bt;
+  Work w;
+  State s;
+  int rc = prep(batch, true, ws, ws_bytes, stream, &Bt, &w);
+  if (rc) return rc;
+  if ((rc = prep_state(Bt, sched, state, state_bytes, &s))) return rc;
+  if (!ok_ptr(Q) || !ok_ptr(Y) || !ok_ptr(lse) || !ok_ptr(Vc) || !ok_ptr(Kc) ||
+      (status && !ok_ptr(status)) || (f_out && !ok_ptr(f_out)))
+    return KVS_EINVAL;
+  return lbfgs_one_step(Bt, *sched, Q, Y, lse, Vc, Kc, s, status, f_out, w);
+}
+
+int kvs_compress_batch(const kvs_batch *batch, const kvs_schedule *sched, const float *Q,
+                       const float *Kz, const float *Vz, float *Kc, float *Vc, int32_t *idx,
+                       float *loss_trace, float *parts, int32_t *status, void *state,
+                       size_t state_bytes, void *ws, size_t ws_bytes, void *stream) {
+  Batch Bt;
+  Work w;
+  State s;
+  int rc = prep(batch, true, ws, ws_bytes, stream, &Bt, &w);
+  if (rc) return rc;
+  if ((rc = prep_state(Bt, sched, state, state_bytes, &s))) return rc;
+  if (!ok_ptr(Q) || !ok_ptr(Kz) || !ok_ptr(Vz) || !ok_ptr(Kc) || !ok_ptr(Vc) ||
+      !ok_ptr(status) || (idx && !ok_ptr(idx)) || (loss_trace && !ok_ptr(loss_trace)) ||
+      (parts && !ok_ptr(parts)))
+    return KVS_EINVAL;
+  if (Bt.g.max_z > 16384) return KVS_ENOTSUP;
+  for (int b = 0; b < Bt.g.B; ++b)
+    if (batch->c_off_h[b + 1] - batch->c_off_h[b] > batch->z_off_h[b + 1] - batch->z_off_h[b])
+      return KVS_EINVAL;
+  const kvs_schedule &sc = *sched;
+  int32_t *ix = idx ? idx : w.idx;
+  KVS_CUDA_TRY(cudaMemsetAsync(status, 0, sizeof(int32_t) * Bt.g.B, Bt.st));
+  if ((rc = launch_targets(Bt, Q, Kz, Vz, w.Yt, w.lset, w.imp, w))) return rc;
+  if ((rc = launch_topk(Bt, w.imp, Kz, ix, Kc))) return rc;
+  if ((rc = launch_fit(Bt, Q, Kc, w.Yt, sc.lambda, Vc, status, w))) return rc;
+  if ((rc = lbfgs_restart(Bt, sc, Q, w.Yt, w.lset, Vc, Kc, s, 1, w))) return rc;
+  const int64_t tstride = sc.outer + 1;
+  if (loss_trace && (rc = launch_copy_f(Bt, s, loss_trace, tstride, 0))) return rc;
+  for (int o = 0; o < sc.outer; ++o) {
+    for (int t = 0; t < sc.steps; ++t)
+      if ((rc = lbfgs_one_step(Bt, sc, Q, w.Yt, w.lset, Vc, Kc, s, status, nullptr, w)))
+        return rc;
+    if ((rc = launch_fit(Bt, Q, Kc, w.Yt, sc.lambda, Vc, status, w))) return rc;
+    if ((rc = lbfgs_restart(Bt, sc, Q, w.Yt, w.lset, Vc, Kc, s, sc.persist_history ? 0 : 1, w)))
+      return rc;
+    if (loss_trace && (rc = launch_copy_f(Bt, s, loss_trace, tstride, o + 1))) return rc;
+  }
+  if (parts)
+    rc = launch_forward(Bt, Q, Kc, Vc, w.Yt, w.lset, sc.w_out, sc.w_lse, w.fbuf, parts, ALL, w);
+  return rc;
+}
+
+// Host-only budget allocation.  The real shares x_b(c) = clip(c w_b, k_min,
+// k_max_b) are non-decreasing in c; c is found by bisection to the resolution
+// of double precision, then the integers are floors plus largest remainders.
+int kvs_pilot_allocate(int32_t B, const float *pilot_mse, int64_t total, int32_t k_min,
+                       const int32_t *k_max, float alpha, int32_t *k_out) {
+  if (B < 1 || !pilot_mse || !k_max || !k_out || k_min < 1 || !(alpha >= 0.f)) return KVS_EINVAL;
+  int64_t lo_sum = 0, hi_sum = 0;
+  for (int b = 0; b < B; ++b) {
+    if (k_max[b] < k_min) return KVS_EINVAL;
+    lo_sum += k_min;
+    hi_sum += k_max[b];
+  }
+  if (total < lo_sum || total > hi_sum) return KVS_EINVAL;
+  std::vector<double> w(B), x(B);
+  double wsum = 0.0;
+  for (int b = 0; b < B; ++b) {
+    const double m = pilot_mse[b];
+    w[b] = (isfinite(m) && m > 0.0) ? pow(m, (double)alpha) : 0.0;
+    wsum += w[b];
+  }
+  if (!(wsum > 0.0)) std::fill(w.begin(), w.end(), 1.0);
+  // When the problems with a positive signal cannot absorb the budget even at
+  // k_max, they take k_max and the zero-signal problems share the rest evenly.
+  int64_t cap_pos = 0, floor_zero = 0;
+  for (int b = 0; b < B; ++b) {
+    if (w[b] > 0.0) cap_pos += k_max[b];
+    else floor_zero += k_min;
+  }
+  std::vector<double> lo(B, (double)k_min), hi(B);
+  for (int b = 0; b < B; ++b) hi[b] = k_max[b];
+  if (cap_pos + floor_zero < total) {
+    for (int b = 0; b < B; ++b) {
+      if (w[b] > 0.0) lo[b] = hi[b];   // pinned at k_max
+      else w[b] = 1.0;
+    }
+  }
+  auto shares = [&](double c) {
+    double s = 0.0;
+    for (int b = 0; b < B; ++b) {
+      x[b] = std::min(hi[b], std::max(lo[b], c * w[b]));
+      s += x[b];
+    }
+    return s;
+  };
+  double clo = 0.0, chi = 1.0;
+  while (shares(chi) < (double)total && chi < 1e300) chi *= 2.0;
+  for (int it = 0; it < 2000; ++it) {
+    const double mid = 0.5 * (clo + chi);
+    if (mid <= clo || mid >= chi) break;
+    if (shares(mid) < (double)total) clo = mid;
+    else chi = mid;
+  }
+  // Between clo and chi the total is crossed; interpolate on the linear piece.
+  const double slo = shares(clo);
+  std::vector<double> xlo(x);
+  const double shi = shares(chi);
+  std::vector<double> ideal(B);
+  const double f = (shi > slo) ? ((double)total - slo) / (shi - slo) : 1.0;
+  for (int b = 0; b < B; ++b) ideal[b] = xlo[b] + f * (x[b] - xlo[b]);
+  std::vector<int64_t> k(B);
+  std::vector<double> frac(B);
+  int64_t sum = 0;
+  for (int b = 0; b < B; ++b) {
+    k[b] = (int64_t)floor(ideal[b]);
+    k[b] = std::min<int64_t>(std::max<int64_t>(k[b], k_min), k_max[b]);
+    frac[b] = ideal[b] - (double)k[b];
+    sum += k[b];
+  }
+  std::vector<int> order(B);
+  for (int b = 0; b < B; ++b) order[b] = b;
+  std::stable_sort(order.begin(), order.end(), [&](int a, int c) { return frac[a] > frac[c]; });
+  int64_t left = total - sum;
+  for (int i = 0; left > 0 && i < B; ++i) {
+    const int b = order[i];
+    if (k[b] < k_max[b]) {
+      ++k[b];
+      --left;
+    }
+  }
+  if (left != 0) return KVS_EINVAL;
+  for (int b = 0; b < B; ++b) k_out[b] = (int32_t)k[b];
+  return KVS_OK;
+}
+
+}  // extern "C"

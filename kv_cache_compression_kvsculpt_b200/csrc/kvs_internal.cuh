@@ -1,0 +1,101 @@
+// Internal launchers shared by the C-ABI layer (not part of the public ABI).
+#pragma once
+
+#include "kvs_common.cuh"
+
+namespace kvs {
+
+// L-BFGS line-search phase of a problem.
+enum Phase : int { PH_IDLE = 0, PH_SEARCH = 1, PH_ACCEPT = 2, PH_FAIL = 3 };
+
+// Per-problem scalar state of L-BFGS (lives in the caller's state buffer).
+struct LbfgsScal {
+  float f;        // loss at x
+  float ft;       // loss at the current trial point
+  float t;        // current trial step
+  float gtd;      // g . d of the current direction
+  float gamma;    // s . y / y . y of the newest stored pair (H0 = gamma I)
+  float rho[16];  // 1 / (s_i . y_i) per ring slot
+  int count;      // valid pairs in the ring
+  int head;       // next ring slot to write
+  int phase;      // Phase
+  int trials;     // trials of the current search
+  int pad[3];
+};
+
+// Scratch buffers carved from the caller's workspace.
+struct Work {
+  float *S;        // [sum_q, ld_s]  scores / probabilities / dS
+  float *Yh;       // [sum_q, d]     compressed attention output
+  float *Go;       // [sum_q, d]     dloss/dYh
+  float *lse_h;    // [sum_q]
+  float *delta;    // [sum_q]
+  float *row_out;  // [sum_q]        per-row squared output error
+  float *row_ls;   // [sum_q]        per-row squared LSE error
+  float *gram;     // [sum_c, max_c] A^T A + lam I (float)
+  double *chol;    // [sum_c, max_c] Cholesky factor (double)
+  double *xs;      // [sum_c, d]     right-hand sides / solution (double)
+  float *R;        // [sum_c, d]     A^T Y
+  float *fbuf;     // [B]            loss scratch
+  float *Yt;       // [sum_q, d]     targets (kvs_compress_batch)
+  float *lset;     // [sum_q]        target log-sum-exp (kvs_compress_batch)
+  float *imp;      // [sum_z]        importance (kvs_compress_batch)
+  int32_t *idx;    // [sum_c]        top-k positions (kvs_compress_batch)
+  size_t bytes;
+};
+
+// Persistent L-BFGS state carved from the caller's state buffer.
+struct State {
+  LbfgsScal *sc;   // [B]
+  float *x;        // [sum_c*d] accepted keys
+  float *g;        // [sum_c*d] gradient at x
+  float *dir;      // [sum_c*d] search direction
+  float *gn;       // [sum_c*d] gradient at the accepted trial point
+  float *ring_s;   // [h+1][sum_c*d]  ring of step differences (slot `head` is scratch)
+  float *ring_y;   // [h+1][sum_c*d]  ring of gradient differences
+  int h;
+  size_t bytes;
+};
+
+size_t carve_work(const HostGeom &g, void *base, Work *w);
+size_t carve_state(const HostGeom &g, int h, void *base, State *s);
+
+struct Batch {
+  HostGeom g;
+  const kvs_batch *b;
+  cudaStream_t st;
+};
+
+// ---- attention contractions (kvs_attn.cu) ----
+// targets: Y, lse and (optionally) importance.
+int launch_targets(const Batch &B, const float *Q, const float *Kz, const float *Vz, float *Y,
+                   float *lse, float *imp, const Work &w);
+// Forward over the compressed pairs for the problems selected by `flt`. Leaves A in w.S, lse_h, Yh, Go, delta and
+// writes loss[b] (and parts[2b..2b+1] if non-null).
+int launch_forward(const Batch &B, const float *Q, const float *Kc, const float *Vc,
+                   const float *Y, const float *lse, float w_out, float w_lse, float *loss,
+                   float *parts, Filter flt, const Work &w);
+// Backward: dKc from the state left by launch_forward for the same problems.
+int launch_backward(const Batch &B, const float *Q, const float *Vc, float *dKc,
+                    Filter flt, const Work &w);
+// Ridge fit: Vc = (A^T A + lam I)^-1 A^T Y.
+int launch_fit(const Batch &B, const float *Q, const float *Kc, const float *Y, float lam,
+               float *Vc, int32_t *status, const Work &w);
+
+// ---- other kernels ----
+int launch_build_queries(const kvs_query_spec *sp, const float *q_retain, const float *q_ctx,
+                         const int32_t *pos, float *Q, cudaStream_t st);
+int launch_topk(const Batch &B, const float *imp, const float *Kz, int32_t *idx, float *Kc);
+int launch_chol_solve(const Batch &B, float *Vc, int32_t *status, const Work &w);
+
+// L-BFGS pieces (kvs_lbfgs.cu)
+int launch_lbfgs_reset(const Batch &B, const State &s, const float *Kc, const float *f,
+                       const float *g, int clear);
+int launch_lbfgs_direction(const Batch &B, const State &s, const kvs_schedule &sc);
+int launch_lbfgs_trial(const Batch &B, const State &s, float *Kc);
+int launch_lbfgs_armijo(const Batch &B, const State &s, const kvs_schedule &sc, const float *ft);
+int launch_lbfgs_update(const Batch &B, const State &s, float *Kc, int32_t *status,
+                        float *f_out);
+int launch_copy_f(const Batch &B, const State &s, float *dst, int64_t stride, int64_t col);
+
+}  // namespace kvs
