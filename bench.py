@@ -1,0 +1,399 @@
+#!/usr/bin/env python
+"""Throughput of the KVSculpt distillation solve on B200.
+
+One step = the whole hot path over one batch of head-problems: training-query
+construction, targets and importance, top-k keys, the initial ridge fit, then
+`outer` x (`steps` L-BFGS steps + ridge re-fit), for every problem of the
+workload (default: 28 layers x 2 KV heads of a Qwen2.5-1.5B-shaped cache,
+N = 2048, m = 128, r = 0.5, 40 x 5 schedule).  Inputs are resident in HBM when
+the device-timed region starts; the e2e figure repeats the step through the
+same C-ABI calls with the inputs copied from pinned host memory and the
+compressed pairs copied back inside the timed region.
+
+Prints one JSON line (rank 0).  `--impl reference` times the float64 CPU
+oracle on a bounded sample of the same workload instead.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import workload as W  # noqa: E402
+
+METRIC = "head-problems compressed/sec at N=2048,r=0.5"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+# CUDA-core fp32 FMA peak from unit counts and clock: 148 SMs x 128 lanes x 2 flop x 1.965 GHz
+DERIVED_PEAKS = {"fp32_simt_tflops": 148 * 128 * 2 * 1.965e9 / 1e12}
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as fh:
+            d = json.load(fh)
+        return d, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+def describe(wl: W.Workload):
+    return (f"{wl.name}: {wl.B} head-problems ({wl.n_seq} seq x {wl.n_layers} layers x "
+            f"{wl.n_kv_heads} KV heads), d={wl.d}, N={wl.N}, m={wl.m}, z={wl.z}, k={wl.k}, "
+            f"n_q={wl.g}x({wl.m_q}+{wl.n_syn})={wl.n_q}, schedule {wl.outer}x{wl.steps} L-BFGS, "
+            f"history {wl.history}, lambda {wl.lam}")
+
+
+# ---------------------------------------------------------------- clocks
+
+class ClockSampler:
+    """nvidia-smi samples of SM clock and throttle reasons while running."""
+
+    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+         "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+         "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index):
+        self.index = index
+        self.rows = []
+        self.proc = None
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.index}", f"--query-gpu={self.Q}",
+                 "--format=csv,noheader,nounits", "-lms", "200"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.t = threading.Thread(target=self._read, daemon=True)
+            self.t.start()
+        except (OSError, FileNotFoundError):
+            self.proc = None
+        return self
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.rows.append([x.strip() for x in line.split(",")])
+
+    def __exit__(self, *a):
+        if self.proc:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+
+    def summary(self):
+        if not self.rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unavailable"]}
+        sm = [float(r[1]) for r in self.rows if len(r) > 8 and r[1].replace(".", "").isdigit()]
+        mx = [float(r[2]) for r in self.rows if len(r) > 8 and r[2].replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = set()
+        for r in self.rows:
+            if len(r) > 8:
+                for n, v in zip(names, r[5:9]):
+                    if v.strip().lower() == "active":
+                        reasons.add(n)
+        return {"sm_mhz": statistics.median(sm) if sm else None,
+                "sm_max_mhz": max(mx) if mx else None, "reasons": sorted(reasons),
+                "samples": len(self.rows)}
+
+
+# ---------------------------------------------------------------- GPU arm
+
+class Job:
+    """Device buffers of one rank's batch and the calls of one step."""
+
+    def __init__(self, wl, seq, dev):
+        import torch
+        import kv_cache_compression_kvsculpt_b200 as K
+        self.K, self.torch, self.wl = K, torch, wl
+        ids = [(seq, l, h) for l in range(wl.n_layers) for h in range(wl.n_kv_heads)]
+        self.bt = W.make_batch(wl, 0, ids)
+        B = self.bt.B
+        self.host = {
+            "q_retain": torch.from_numpy(self.bt.q_retain).pin_memory(),
+            "q_ctx": torch.from_numpy(self.bt.q_ctx).pin_memory(),
+            "pos": torch.from_numpy(self.bt.pos).pin_memory(),
+            "Kz": torch.from_numpy(self.bt.Kz).pin_memory(),
+            "Vz": torch.from_numpy(self.bt.Vz).pin_memory(),
+        }
+        self.dev = {k: v.to(dev) for k, v in self.host.items()}
+        self.batch = K.KvsBatch(wl.d, self.bt.q_off, self.bt.z_off,
+                                np.arange(B + 1, dtype=np.int64) * wl.k)
+        self.spec = K.QuerySpec(B, wl.d, wl.g, wl.m_q, wl.n_syn, wl.N, wl.rope_base)
+        self.sched = K.Schedule(outer=wl.outer, steps=wl.steps, history=wl.history, lam=wl.lam,
+                                w_out=wl.w_out, w_lse=wl.w_lse)
+        self.Q = torch.empty((self.batch.sum_q, wl.d), device=dev)
+        self.Kc = torch.empty((self.batch.sum_c, wl.d), device=dev)
+        self.Vc = torch.empty_like(self.Kc)
+        self.trace = torch.empty((B, wl.outer + 1), device=dev)
+        self.parts = torch.empty((B, 2), device=dev)
+        self.status = torch.empty(B, dtype=torch.int32, device=dev)
+        self.ws = K.alloc_workspace(self.batch, device=dev)
+        self.state = K.alloc_state(self.batch, wl.history, device=dev)
+        self.out_host = {"Kc": torch.empty(self.Kc.shape).pin_memory(),
+                         "Vc": torch.empty(self.Vc.shape).pin_memory()}
+
+    def step(self, d=None):
+        K = self.K
+        d = d or self.dev
+        K.kvs_build_queries(self.spec, d["q_retain"], d["q_ctx"], d["pos"], self.Q)
+        K.kvs_compress_batch(self.batch, self.sched, self.Q, d["Kz"], d["Vz"], self.Kc, self.Vc,
+                             None, self.trace, self.parts, self.status, self.state, self.ws)
+
+    def step_e2e(self):
+        """Same step from pinned host inputs, compressed pairs copied back."""
+        d = {k: self.dev[k].copy_(v, non_blocking=True) for k, v in self.host.items()}
+        self.step(d)
+        self.out_host["Kc"].copy_(self.Kc, non_blocking=True)
+        self.out_host["Vc"].copy_(self.Vc, non_blocking=True)
+
+    def h2d_bytes(self):
+        return sum(v.numel() * v.element_size() for v in self.host.values())
+
+    def d2h_bytes(self):
+        return sum(v.numel() * v.element_size() for v in self.out_host.values())
+
+
+def time_region(torch, fn, n, dist=None):
+    """Device time (ms) of n calls of fn on the current stream, max over ranks."""
+    st = torch.cuda.current_stream()
+    if dist:
+        dist.barrier()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(st)
+    for _ in range(n):
+        fn()
+    e1.record(st)
+    torch.cuda.synchronize()
+    ms = e0.elapsed_time(e1)
+    if dist:
+        t = torch.tensor([ms], device="cuda")
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms = float(t.item())
+        dist.barrier()
+    return ms
+
+
+def loss_grad_roofline(job, peaks, reps=20):
+    """Time kvs_loss_grad (the dominant evaluation) over the batch at the solved point."""
+    torch, K, wl = job.torch, job.K, job.wl
+    B = job.batch.B
+    Y = torch.empty_like(job.Q)
+    lse = torch.empty(job.batch.sum_q, device=job.Q.device)
+    K.kvs_targets(job.batch, job.Q, job.dev["Kz"], job.dev["Vz"], Y, lse, None, job.ws)
+    loss = torch.empty(B, device=job.Q.device)
+    dK = torch.empty_like(job.Kc)
+
+    def ev():
+        K.kvs_loss_grad(job.batch, job.Q, job.Kc, job.Vc, Y, lse, 1.0, 1.0, loss, None, dK, job.ws)
+
+    for _ in range(3):
+        ev()
+    ms = time_region(torch, ev, reps) / reps
+    flops = 8.0 * wl.n_q * wl.k * wl.d * B
+    achieved = flops / (ms * 1e-3) / 1e12
+    return ms, flops, achieved
+
+
+def run_gpu(args):
+    import torch
+    import kv_cache_compression_kvsculpt_b200 as K
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    dist = None
+    if world > 1:
+        import datetime
+        import torch.distributed as dist_mod
+        os.environ.setdefault("MASTER_ADDR", "127.0.0.1")
+        dist_mod.init_process_group("nccl", timeout=datetime.timedelta(seconds=300))
+        dist = dist_mod
+    torch.cuda.set_device(local)
+    wl = W.WORKLOADS[args.workload]
+    if args.outer is not None:
+        wl = wl.with_(outer=args.outer)
+    job = Job(wl, seq=rank, dev="cuda")
+    for _ in range(args.warmup):
+        job.step()
+    torch.cuda.synchronize()
+    st = int(torch.cuda.current_device())
+    n0 = K.kvs_launch_count()
+    with ClockSampler(st) as clk:
+        ms = time_region(torch, job.step, args.steps, dist)
+    launches = K.kvs_launch_count() - n0
+    status = job.status.cpu().numpy()
+    ms_step = ms / args.steps
+    problems = wl.B * world
+    value = problems / (ms_step * 1e-3)
+    # e2e through host buffers
+    job.step_e2e()
+    ms_e2e = time_region(torch, job.step_e2e, args.steps, dist) / args.steps
+    e2e_value = problems / (ms_e2e * 1e-3)
+    peaks, peak_src = load_peaks()
+    lg_ms, lg_flops, lg_tflops = loss_grad_roofline(job, peaks)
+    if args.peak_key in DERIVED_PEAKS:
+        peak, peak_src = DERIVED_PEAKS[args.peak_key], "derived"
+    else:
+        peak = peaks.get(args.peak_key, FALLBACK_PEAKS.get(args.peak_key))
+    final = job.trace[:, -1].cpu().numpy()
+    first = job.trace[:, 0].cpu().numpy()
+    out = {
+        "metric": METRIC,
+        "value": round(value, 4),
+        "unit": "head-problems/s",
+        "n_gpus": world,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": round(ms_step, 3),
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": args.dtype_label,
+        "data": "synthetic (seeded generator; stands in for Qwen2.5-1.5B-Instruct KV caches)",
+        "config": {"workload": describe(wl), "problems_per_gpu": wl.B,
+                   "l2": "inputs and per-step working set larger than L2 (126 MB)",
+                   "parallelism": f"problem-sharded x{world}, no collective"},
+        "e2e": {"value": round(e2e_value, 4), "unit": "head-problems/s",
+                "h2d_bytes_per_step": job.h2d_bytes(), "d2h_bytes_per_step": job.d2h_bytes()},
+        "loss_grad_evals_per_s": round(wl.B / (lg_ms * 1e-3), 1),
+        "roofline": {"kernel": "kvs_loss_grad (forward + dKc backward, whole batch)",
+                     "bound": args.bound, "achieved": round(lg_tflops, 3), "peak": peak,
+                     "unit": "TFLOP/s", "frac": round(lg_tflops / peak, 4),
+                     "traffic": None, "peak_source": f"{peak_src} {args.peak_key}",
+                     "ms_per_launch": round(lg_ms, 4),
+                     "algorithmic_flops_per_launch": lg_flops},
+        "gpu_launches": int(launches),
+        "clocks": clk.summary(),
+        "quality": {"select_fit_loss_mean": float(np.mean(first)),
+                    "final_loss_mean": float(np.mean(final)),
+                    "status_nonzero": int((status != 0).sum())},
+    }
+    if rank == 0 and not args.no_cpu_baseline:
+        out["cpu_baseline"] = cpu_baseline(wl, budget_s=args.cpu_budget)
+    if rank == 0:
+        print(json.dumps(out), flush=True)
+    if dist:
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+# ---------------------------------------------------------------- oracle
+
+def oracle_sample(wl, budget_s, pid=(0, 0, 0)):
+    """The oracle's schedule on one problem, run until budget_s of outer
+    iterations have elapsed; returns the per-problem time extrapolated to the
+    full schedule and a description of the sample."""
+    import oracle as O
+    t0 = time.perf_counter()
+    bt = W.make_batch(wl, 0, [pid])
+    p = bt.problem(0)
+    Q = O.build_queries(p["q_retain"], p["q_ctx"], p["pos"], wl.g, wl.m_q, wl.n_syn, wl.N,
+                        wl.rope_base)
+    Y, lse = O.targets(Q, p["Kz"], p["Vz"])
+    idx = O.topk_select(O.importance(Q, p["Kz"], lse), wl.k)
+    Kc = np.asarray(p["Kz"], np.float64)[idx]
+    Vc, _ = O.ridge_fit(Q, Kc, Y, wl.lam)
+    f, g, _ = O.loss_grad(Q, Kc, Vc, Y, lse)
+    st = O.LBFGSState(x=Kc.ravel().copy(), f=f, g=g.ravel())
+    d = wl.d
+    t_setup = time.perf_counter() - t0
+    done = 0
+    t1 = time.perf_counter()
+    while done < wl.outer and (done == 0 or time.perf_counter() - t1 < budget_s):
+        fl = lambda x: O.loss_only(Q, x.reshape(-1, d), Vc, Y, lse)
+        fg = lambda x: O.loss_grad(Q, x.reshape(-1, d), Vc, Y, lse)[1].ravel()
+        for _ in range(wl.steps):
+            O.lbfgs_step(st, fl, fg, wl.history)
+        Vc, _ = O.ridge_fit(Q, st.x.reshape(-1, d), Y, wl.lam)
+        f, g, _ = O.loss_grad(Q, st.x.reshape(-1, d), Vc, Y, lse)
+        st.f, st.g = f, g.ravel()
+        done += 1
+    t_outer = (time.perf_counter() - t1) / done
+    total = t_setup + t_outer * wl.outer
+    sample = (f"1 problem {pid} of {wl.name}: query build, targets, top-k, first fit, then "
+              f"{done} of {wl.outer} outer iterations ({wl.steps} L-BFGS steps + re-fit each) "
+              f"timed; per-problem time extrapolated to the full schedule")
+    return total, sample
+
+
+def _cores():
+    try:
+        from threadpoolctl import threadpool_info
+        n = [i.get("num_threads") for i in threadpool_info() if i.get("user_api") == "blas"]
+        if n:
+            return int(max(n))
+    except Exception:
+        pass
+    return os.cpu_count() or 1
+
+
+def cpu_baseline(wl, budget_s=20.0):
+    t, sample = oracle_sample(wl, budget_s)
+    return {"value": round(1.0 / t, 6), "unit": "head-problems/s", "cores": _cores(),
+            "kind": "oracle", "sample": sample, "seconds_per_problem": round(t, 2)}
+
+
+def run_reference(args):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    wl = W.WORKLOADS[args.workload]
+    if args.outer is not None:
+        wl = wl.with_(outer=args.outer)
+    budget = max(2.0, min(args.cpu_budget, 20.0))
+    for _ in range(args.warmup if args.warmup < 1 else 1):
+        oracle_sample(wl, 1.0)
+    times = []
+    sample = ""
+    for _ in range(args.steps):
+        t, sample = oracle_sample(wl, budget)
+        times.append(t)
+    per = float(np.mean(times))
+    value = 1.0 / per
+    out = {"impl": "reference", "metric": METRIC, "value": round(value, 6),
+           "unit": "head-problems/s", "n_gpus": int(os.environ.get("WORLD_SIZE", "1")),
+           "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(per * 1e3, 1),
+           "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+           "data": "synthetic (seeded generator)", "config": {"workload": describe(wl)},
+           "cpu_baseline": {"value": round(value, 6), "unit": "head-problems/s",
+                            "cores": _cores(), "kind": "oracle", "sample": sample},
+           "e2e": {"value": round(value, 6), "unit": "head-problems/s",
+                   "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(out), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=3)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--workload", default="qwen_cache_r05", choices=sorted(W.WORKLOADS))
+    ap.add_argument("--outer", type=int, default=None, help="override the outer iterations")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-budget", type=float, default=20.0)
+    ap.add_argument("--bound", default="alu")
+    ap.add_argument("--peak-key", default="fp32_simt_tflops")
+    ap.add_argument("--dtype-label", default="f32")
+    args = ap.parse_args()
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_gpu(args)
+
+
+if __name__ == "__main__":
+    main()

@@ -77,8 +77,8 @@ typedef struct kvs_batch {
 typedef struct kvs_schedule {
   int32_t outer;             /* outer iterations: value re-fits after the initial one */
   int32_t steps;             /* L-BFGS steps per outer iteration */
-  int32_t history;           /* L-BFGS pairs kept (1..16) */
-  int32_t max_bt;            /* Armijo trials per step (1..32) */
+  int32_t history;           /* L-BFGS pairs kept (1..15) */
+  int32_t max_bt;            /* Armijo trials per step (1..64) */
   int32_t persist_history;   /* 1: keep (s,y) pairs across value re-fits; 0: clear them */
   float lambda;              /* ridge penalty, absolute */
   float w_out;               /* weight of the output term, mean over n_q*d */
@@ -100,6 +100,7 @@ typedef struct kvs_query_spec {
 /* Library version / diagnostics. */
 const char *kvs_version(void);
 const char *kvs_last_cuda_error(void);     /* text of the last CUDA error seen by this thread */
+uint64_t kvs_launch_count(void);           /* kernels this library has launched in this process */
 
 /* Bytes of scratch workspace needed by every call below for this batch
  * (and schedule; may be NULL when no L-BFGS call will use the workspace).

@@ -18,7 +18,7 @@ import torch
 __all__ = [
     "KvsError", "KvsBatch", "Schedule", "QuerySpec", "LIB_PATH", "lib",
     "ST_NONFINITE", "ST_NOT_PD", "ST_LS_FAIL",
-    "kvs_version", "kvs_workspace_bytes", "kvs_lbfgs_state_bytes", "kvs_build_queries",
+    "kvs_version", "kvs_launch_count", "kvs_workspace_bytes", "kvs_lbfgs_state_bytes", "kvs_build_queries",
     "kvs_targets", "kvs_init_topk", "kvs_loss_grad", "kvs_fit_values", "kvs_lbfgs_reset",
     "kvs_lbfgs_step", "kvs_compress_batch", "kvs_pilot_allocate",
     "alloc_workspace", "alloc_state",
@@ -27,7 +27,7 @@ __all__ = [
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libkvsculpt.so")
 if not os.path.exists(LIB_PATH):
     raise ImportError(f"{LIB_PATH} is missing: build it with "
-                      "`python -m kv_cache_compression_kvsculpt_b200.build`")
+                      "`python kv_cache_compression_kvsculpt_b200/build.py`")
 lib = ctypes.CDLL(LIB_PATH)
 
 ST_NONFINITE, ST_NOT_PD, ST_LS_FAIL = 1, 2, 4
@@ -56,6 +56,7 @@ _BP, _SP, _QP = ctypes.POINTER(_Batch), ctypes.POINTER(_Sched), ctypes.POINTER(_
 _SIGS = {
     "kvs_version": (ctypes.c_char_p, []),
     "kvs_last_cuda_error": (ctypes.c_char_p, []),
+    "kvs_launch_count": (ctypes.c_uint64, []),
     "kvs_workspace_bytes": (_sz, [_BP, _SP]),
     "kvs_lbfgs_state_bytes": (_sz, [_BP, _i32]),
     "kvs_build_queries": (ctypes.c_int, [_QP, _vp, _vp, _vp, _vp, _vp]),
@@ -201,6 +202,10 @@ class QuerySpec:
 
 def kvs_version() -> str:
     return lib.kvs_version().decode()
+
+
+def kvs_launch_count() -> int:
+    return int(lib.kvs_launch_count())
 
 
 def kvs_workspace_bytes(batch: KvsBatch, sched: Optional[Schedule] = None) -> int:

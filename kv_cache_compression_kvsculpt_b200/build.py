@@ -1,6 +1,7 @@
 """Build libkvsculpt.so (all CUDA sources, sm_100a) in the package directory.
 
-Usage: python -m kv_cache_compression_kvsculpt_b200.build [--verbose]
+Usage: python kv_cache_compression_kvsculpt_b200/build.py [--verbose] [--ptxas]
+(run by path: importing the package needs the library this script builds)
 Each .cu is compiled to an object under <repo>/_build (skipped when the object
 is newer than its source and the shared headers), then linked with nvcc.
 """

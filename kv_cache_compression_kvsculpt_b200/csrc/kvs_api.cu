@@ -5,6 +5,7 @@
 #include <string.h>
 
 #include <algorithm>
+#include <atomic>
 #include <cstddef>
 #include <vector>
 
@@ -13,6 +14,9 @@
 namespace kvs {
 
 static thread_local char g_err[256] = "no error";
+static std::atomic<uint64_t> g_launches{0};
+
+void count_launch() { g_launches.fetch_add(1, std::memory_order_relaxed); }
 
 void set_cuda_error(cudaError_t e, const char *where) {
   snprintf(g_err, sizeof g_err, "%s: %s (%s)", where, cudaGetErrorName(e), cudaGetErrorString(e));
@@ -166,6 +170,8 @@ extern "C" {
 const char *kvs_version(void) { return "kvsculpt-b200 0.1 (sm_100a)"; }
 
 const char *kvs_last_cuda_error(void) { return g_err; }
+
+uint64_t kvs_launch_count(void) { return g_launches.load(std::memory_order_relaxed); }
 
 size_t kvs_workspace_bytes(const kvs_batch *batch, const kvs_schedule *) {
   HostGeom g;

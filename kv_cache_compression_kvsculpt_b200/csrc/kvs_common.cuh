@@ -10,6 +10,8 @@ namespace kvs {
 
 // Per-thread text of the last CUDA error (kvs_last_cuda_error).
 void set_cuda_error(cudaError_t e, const char *where);
+// Counts kernel launches (kvs_launch_count); called once per launch.
+void count_launch();
 
 #define KVS_CUDA_TRY(expr)                                     \
   do {                                                         \
@@ -22,6 +24,7 @@ void set_cuda_error(cudaError_t e, const char *where);
 
 #define KVS_LAUNCH_CHECK(where)                                \
   do {                                                         \
+    ::kvs::count_launch();                                     \
     cudaError_t _e = cudaGetLastError();                       \
     if (_e != cudaSuccess) {                                   \
       ::kvs::set_cuda_error(_e, where);                        \

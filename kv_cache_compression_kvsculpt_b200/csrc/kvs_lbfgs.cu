@@ -58,7 +58,8 @@ __global__ void __launch_bounds__(NT) k_direction(LbfgsScal *sc, const float *__
   const int b = blockIdx.x;
   LbfgsScal &s = sc[b];
   const int64_t o = seg0(c_off, b, d), n = c_off[b + 1] * (int64_t)d - o;
-  const int count = s.count, head = s.head, slots = h + 1;
+  const int slots = h + 1;
+  const int count = min(max(s.count, 0), h), head = min(max(s.head, 0), h);
   const float gamma = count > 0 ? s.gamma : 1.f;
   // loop 1, newest pair first: q <- q - alpha_j y_j ; alpha_j = rho_j s_j . q
   for (int p = 0; p <= count; ++p) {
@@ -174,7 +175,7 @@ __global__ void __launch_bounds__(NT) k_update(LbfgsScal *sc, float *__restrict_
   const int phase = s.phase;
   const int64_t o = seg0(c_off, b, d), n = c_off[b + 1] * (int64_t)d - o;
   if (phase == PH_ACCEPT) {
-    const int slot = s.head;
+    const int slot = min(max(s.head, 0), h);
     float *rs = ring_s + slot * rstride + o;
     float *ry = ring_y + slot * rstride + o;
     float sy = 0.f, yy = 0.f;
@@ -195,7 +196,7 @@ __global__ void __launch_bounds__(NT) k_update(LbfgsScal *sc, float *__restrict_
         s.rho[slot] = 1.f / sy;
         s.gamma = sy / yy;
         s.head = (slot + 1) % (h + 1);
-        s.count = min(s.count + 1, h);
+        s.count = min(max(s.count, 0) + 1, h);
       }
       s.f = s.ft;
       if (!isfinite(s.f) && status) status[b] |= KVS_ST_NONFINITE;

@@ -138,7 +138,8 @@ __global__ void __launch_bounds__(1024) k_topk(const float *__restrict__ imp,
       s_run_out = run;
     }
     __syncthreads();
-    if (sel) out[wsum[w] + __popc(bal & lt)] = j;
+    const uint32_t at = wsum[w] + __popc(bal & lt);
+    if (sel && at < (uint32_t)k) out[at] = j;
     __syncthreads();
   }
 }
@@ -151,7 +152,9 @@ __global__ void k_gather(const float *__restrict__ Kz, const int64_t *__restrict
   const int r = blockIdx.x * 8 + (threadIdx.x >> 5);
   const int64_t c0 = c_off[b];
   if (r >= c_off[b + 1] - c0) return;
-  const float *src = Kz + (z_off[b] + idx[c0 + r]) * d;
+  const int src_row = idx[c0 + r];
+  if (src_row < 0 || src_row >= z_off[b + 1] - z_off[b]) return;
+  const float *src = Kz + (z_off[b] + src_row) * d;
   float *dst = Kc + (c0 + r) * d;
   for (int c = threadIdx.x & 31; c < d; c += 32) dst[c] = src[c];
 }

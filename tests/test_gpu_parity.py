@@ -1,0 +1,325 @@
+"""Parity of the CUDA path (through the C ABI) with the float64 oracle.
+
+Tolerances (stated by the method's accuracy contract): loss within rel 1e-3,
+gradient cosine >= 0.999, V_c within rel 1e-3, final loss of the whole
+schedule within 5 %, top-k indices bit-exact on identical float32 scores.
+Inputs are the seeded synthetic workloads; every per-step comparison feeds
+both sides the same float32 tensors.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle as O
+import workload as W
+from gpu_common import Case, cosine, dev, host, rel
+
+pytestmark = pytest.mark.gpu
+
+RAGGED = W.Workload("ragged_small", 1, 3, 2, d=128, N=300, m=44, g=2, n_syn=61, k=64,
+                    layer_scale=True, outer=3, steps=4)
+RAGGED_NQ = [210, 173, 97, 210, 150, 201]
+RAGGED_K = [37, 100, 1, 256, 64, 129]
+SMALL64 = W.Workload("small_d64", 1, 2, 2, d=64, N=200, m=40, g=3, n_syn=30, k=50,
+                     layer_scale=True, outer=3, steps=4)
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _cuda():
+    assert torch.cuda.is_available(), "GPU tests need a CUDA device"
+    import kv_cache_compression_kvsculpt_b200 as K  # noqa: F401  (fails loudly without the .so)
+
+
+def cases():
+    return {
+        "single_d64": lambda: Case(W.WORKLOADS["single_d64"]),
+        "qwen_layer": lambda: Case(W.WORKLOADS["qwen_layer"]),
+        "ragged": lambda: Case(RAGGED, k=RAGGED_K, n_q=RAGGED_NQ),
+        "small_d64": lambda: Case(SMALL64, k=[50, 7, 160, 33]),
+    }
+
+
+@pytest.fixture(scope="module", params=["single_d64", "qwen_layer", "ragged", "small_d64"])
+def case(request):
+    return cases()[request.param]()
+
+
+# ------------------------------------------------------------------ queries
+
+@pytest.mark.parametrize("name", ["single_d64", "qwen_layer", "small_d64"])
+def test_build_queries(name):
+    import kv_cache_compression_kvsculpt_b200 as K
+    wl = W.WORKLOADS.get(name) or SMALL64
+    bt = W.make_batch(wl, 0)
+    spec = K.QuerySpec(bt.B, wl.d, wl.g, wl.m_q, wl.n_syn, wl.N, wl.rope_base)
+    Q = torch.empty((bt.B * wl.n_q, wl.d), device="cuda")
+    K.kvs_build_queries(spec, dev(bt.q_retain), dev(bt.q_ctx), dev(bt.pos, torch.int32), Q)
+    torch.cuda.synchronize()
+    got = host(Q)
+    from gpu_common import oracle_queries
+    want = np.concatenate(oracle_queries(wl, bt))
+    assert rel(got, want) < 2e-6
+    # retain rows are copied verbatim
+    nr = wl.g * wl.m_q
+    row0 = np.concatenate([np.arange(h * (wl.m_q + wl.n_syn), h * (wl.m_q + wl.n_syn) + wl.m_q)
+                           for h in range(wl.g)])
+    np.testing.assert_array_equal(got[:wl.n_q][row0], bt.q_retain[:nr])
+
+
+# ------------------------------------------------------------------ targets
+
+def run_targets(c):
+    K = c.K
+    Y = torch.empty_like(c.Q)
+    lse = torch.empty(c.Q.shape[0], device="cuda")
+    imp = torch.empty(c.Kz.shape[0], device="cuda")
+    K.kvs_targets(c.batch, c.Q, c.Kz, c.Vz, Y, lse, imp, c.ws)
+    torch.cuda.synchronize()
+    return host(Y), host(lse), host(imp)
+
+
+def test_targets(case):
+    c = case
+    Y, lse, imp = run_targets(c)
+    for b in range(c.bt.B):
+        Yo, lo = c.targets_oracle(b)
+        io = O.importance(c.Qs[b], c.Zk[b], lo)
+        q0, q1 = c.q_off[b], c.q_off[b + 1]
+        z0, z1 = c.bt.z_off[b], c.bt.z_off[b + 1]
+        assert rel(Y[q0:q1], Yo) < 1e-4
+        assert np.max(np.abs(lse[q0:q1] - lo) / (1 + np.abs(lo))) < 1e-5
+        assert rel(imp[z0:z1], io) < 1e-4
+        assert abs(imp[z0:z1].sum() - (q1 - q0)) < 1e-3 * (q1 - q0)
+
+
+# ------------------------------------------------------------------ top-k
+
+def test_topk_bit_exact(case):
+    c = case
+    K = c.K
+    r = np.random.default_rng(3)
+    imp = r.integers(0, 50, size=c.Kz.shape[0]).astype(np.float32) * np.float32(0.125)  # ties
+    _, _, imp_real = run_targets(c)
+    for variant in (imp, imp_real):
+        idx = torch.empty(c.batch.sum_c, dtype=torch.int32, device="cuda")
+        Kc = torch.empty((c.batch.sum_c, c.wl.d), device="cuda")
+        K.kvs_init_topk(c.batch, dev(variant), c.Kz, idx, Kc)
+        torch.cuda.synchronize()
+        gi, gk = host(idx), host(Kc)
+        co = c.batch.c_off_h
+        for b in range(c.bt.B):
+            z0, z1 = c.bt.z_off[b], c.bt.z_off[b + 1]
+            want = O.topk_select(variant[z0:z1].astype(np.float64), int(c.k[b]))
+            np.testing.assert_array_equal(gi[co[b]:co[b + 1]], want)
+            np.testing.assert_array_equal(gk[co[b]:co[b + 1]], c.Zk[b][want])
+
+
+# ----------------------------------------------------------- loss and grad
+
+def select_fit_point(c, perturb=0.0, seed=0):
+    """K_c = top-k keys of the oracle's importance, V_c = oracle ridge fit (float32)."""
+    r = np.random.default_rng(seed)
+    Kcs, Vcs, tgt = [], [], []
+    for b in range(c.bt.B):
+        Yo, lo = c.targets_oracle(b)
+        idx = O.topk_select(O.importance(c.Qs[b], c.Zk[b], lo), int(c.k[b]))
+        Kc = c.Zk[b][idx].astype(np.float64)
+        if perturb:
+            Kc = Kc + perturb * r.standard_normal(Kc.shape) * np.abs(Kc).mean()
+        Kc = Kc.astype(np.float32)
+        Vc, _ = O.ridge_fit(c.Qs[b], Kc, Yo, 1e-3)
+        Kcs.append(Kc)
+        Vcs.append(Vc.astype(np.float32))
+        tgt.append((Yo.astype(np.float32), lo.astype(np.float32)))
+    return Kcs, Vcs, tgt
+
+
+@pytest.mark.parametrize("perturb", [0.0, 0.3])
+def test_loss_grad(case, perturb):
+    c = case
+    K = c.K
+    Kcs, Vcs, tgt = select_fit_point(c, perturb)
+    Y = dev(np.concatenate([t[0] for t in tgt]))
+    lse = dev(np.concatenate([t[1] for t in tgt]))
+    B = c.bt.B
+    loss = torch.empty(B, device="cuda")
+    parts = torch.empty((B, 2), device="cuda")
+    dK = torch.empty((c.batch.sum_c, c.wl.d), device="cuda")
+    K.kvs_loss_grad(c.batch, c.Q, dev(np.concatenate(Kcs)), dev(np.concatenate(Vcs)), Y, lse,
+                    1.0, 1.0, loss, parts, dK, c.ws)
+    torch.cuda.synchronize()
+    gl, gp, gd = host(loss), host(parts), host(dK)
+    co = c.batch.c_off_h
+    for b in range(B):
+        f, g, info = O.loss_grad(c.Qs[b], Kcs[b], Vcs[b], tgt[b][0], tgt[b][1])
+        assert abs(gl[b] - f) <= 1e-3 * f, (b, gl[b], f)
+        assert abs(gp[b, 0] - info["out"]) <= 1e-3 * info["out"] + 1e-9
+        assert abs(gp[b, 1] - info["lse"]) <= 1e-3 * info["lse"] + 1e-9
+        assert cosine(gd[co[b]:co[b + 1]], g) >= 0.999, b
+
+
+def test_loss_only_matches_loss_grad(case):
+    c = case
+    K = c.K
+    Kcs, Vcs, tgt = select_fit_point(c, 0.1)
+    args = (c.Q, dev(np.concatenate(Kcs)), dev(np.concatenate(Vcs)),
+            dev(np.concatenate([t[0] for t in tgt])), dev(np.concatenate([t[1] for t in tgt])))
+    l1 = torch.empty(c.bt.B, device="cuda")
+    l2 = torch.empty(c.bt.B, device="cuda")
+    dK = torch.empty((c.batch.sum_c, c.wl.d), device="cuda")
+    K.kvs_loss_grad(c.batch, *args, 0.5, 2.0, l1, None, None, c.ws)
+    K.kvs_loss_grad(c.batch, *args, 0.5, 2.0, l2, None, dK, c.ws)
+    torch.cuda.synchronize()
+    np.testing.assert_array_equal(host(l1), host(l2))
+
+
+# ------------------------------------------------------------------ ridge fit
+
+def test_fit_values(case):
+    c = case
+    K = c.K
+    Kcs, _, tgt = select_fit_point(c, 0.2)
+    Y = dev(np.concatenate([t[0] for t in tgt]))
+    Vc = torch.zeros((c.batch.sum_c, c.wl.d), device="cuda")
+    status = torch.zeros(c.bt.B, dtype=torch.int32, device="cuda")
+    K.kvs_fit_values(c.batch, c.Q, dev(np.concatenate(Kcs)), Y, 1e-3, Vc, status, c.ws)
+    torch.cuda.synchronize()
+    gv = host(Vc)
+    assert not host(status).any()
+    co = c.batch.c_off_h
+    for b in range(c.bt.B):
+        Vo, st = O.ridge_fit(c.Qs[b], Kcs[b], tgt[b][0], 1e-3)
+        assert st == O.ST_OK
+        assert rel(gv[co[b]:co[b + 1]], Vo) < 1e-3, b
+
+
+def test_fit_not_pd_keeps_values():
+    c = Case(W.WORKLOADS["single_d64"], k=2)
+    K = c.K
+    Kc = np.stack([c.Zk[0][5], c.Zk[0][5]]).astype(np.float32)   # duplicate keys
+    Yo, _ = c.targets_oracle(0)
+    V0 = np.full((2, 64), 7.0, np.float32)
+    Vc = dev(V0)
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    K.kvs_fit_values(c.batch, c.Q, dev(Kc), dev(Yo.astype(np.float32)), -1e-3, Vc, status, c.ws)
+    torch.cuda.synchronize()
+    assert host(status)[0] & K.ST_NOT_PD
+    np.testing.assert_array_equal(host(Vc), V0)
+
+
+# ------------------------------------------------------------------ L-BFGS
+
+def test_lbfgs_first_step(case):
+    c = case
+    K = c.K
+    Kcs, Vcs, tgt = select_fit_point(c)
+    sched = K.Schedule(outer=1, steps=1)
+    Y = dev(np.concatenate([t[0] for t in tgt]))
+    lse = dev(np.concatenate([t[1] for t in tgt]))
+    Vc = dev(np.concatenate(Vcs))
+    Kc = dev(np.concatenate(Kcs))
+    state = K.alloc_state(c.batch, sched.history)
+    status = torch.zeros(c.bt.B, dtype=torch.int32, device="cuda")
+    fout = torch.empty(c.bt.B, device="cuda")
+    K.kvs_lbfgs_reset(c.batch, sched, c.Q, Y, lse, Vc, Kc, state, 1, c.ws)
+    K.kvs_lbfgs_step(c.batch, sched, c.Q, Y, lse, Vc, Kc, state, status, fout, c.ws)
+    torch.cuda.synchronize()
+    gk, gf = host(Kc), host(fout)
+    assert not host(status).any()
+    co = c.batch.c_off_h
+    d = c.wl.d
+    for b in range(c.bt.B):
+        Q, Yo, lo, V = c.Qs[b], tgt[b][0], tgt[b][1], Vcs[b]
+        f, g, _ = O.loss_grad(Q, Kcs[b], V, Yo, lo)
+        st = O.LBFGSState(x=Kcs[b].astype(np.float64).ravel(), f=f, g=g.ravel())
+        O.lbfgs_step(st, lambda x: O.loss_only(Q, x.reshape(-1, d), V, Yo, lo),
+                     lambda x: O.loss_grad(Q, x.reshape(-1, d), V, Yo, lo)[1].ravel())
+        assert abs(gf[b] - st.f) <= 1e-3 * st.f, b
+        step_gpu = gk[co[b]:co[b + 1]].astype(np.float64) - Kcs[b]
+        step_or = st.x.reshape(-1, d) - Kcs[b]
+        assert rel(step_gpu, step_or) < 2e-2, b
+
+
+def test_lbfgs_failed_search_flags():
+    c = Case(W.WORKLOADS["single_d64"])
+    K = c.K
+    Kcs, Vcs, tgt = select_fit_point(c)
+    Vbad = Vcs[0].copy()
+    Vbad[0, 0] = np.nan
+    sched = K.Schedule(max_bt=3)
+    Y, lse = dev(tgt[0][0]), dev(tgt[0][1])
+    Kc = dev(Kcs[0])
+    Vc = dev(Vbad)
+    state = K.alloc_state(c.batch, sched.history)
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    K.kvs_lbfgs_reset(c.batch, sched, c.Q, Y, lse, Vc, Kc, state, 1, c.ws)
+    K.kvs_lbfgs_step(c.batch, sched, c.Q, Y, lse, Vc, Kc, state, status, None, c.ws)
+    torch.cuda.synchronize()
+    assert host(status)[0] & K.ST_LS_FAIL
+    np.testing.assert_array_equal(host(Kc), Kcs[0])
+
+
+# ------------------------------------------------------------ whole schedule
+
+def run_compress(c, sched):
+    K = c.K
+    B = c.bt.B
+    Kc = torch.empty((c.batch.sum_c, c.wl.d), device="cuda")
+    Vc = torch.empty_like(Kc)
+    idx = torch.empty(c.batch.sum_c, dtype=torch.int32, device="cuda")
+    trace = torch.empty((B, sched.outer + 1), device="cuda")
+    parts = torch.empty((B, 2), device="cuda")
+    status = torch.empty(B, dtype=torch.int32, device="cuda")
+    state = K.alloc_state(c.batch, sched.history)
+    K.kvs_compress_batch(c.batch, sched, c.Q, c.Kz, c.Vz, Kc, Vc, idx, trace, parts, status,
+                         state, c.ws)
+    torch.cuda.synchronize()
+    return dict(Kc=host(Kc), Vc=host(Vc), idx=host(idx), trace=host(trace), parts=host(parts),
+                status=host(status))
+
+
+def check_topk_valid(gidx, Qb, Zk, Zv, k, tol=1e-4):
+    """The GPU's positions are a top-k of the oracle's importance up to tol."""
+    _, lo = O.targets(Qb, Zk, Zv)
+    imp = O.importance(Qb, Zk, lo)
+    sel = np.zeros(len(imp), bool)
+    sel[gidx] = True
+    assert sel.sum() == k and list(gidx) == sorted(gidx)
+    if k < len(imp):
+        assert imp[sel].min() >= imp[~sel].max() * (1 - tol)
+    return np.array_equal(gidx, O.topk_select(imp, k))
+
+
+@pytest.mark.parametrize("name", ["single_d64", "ragged", "small_d64"])
+def test_compress_small(name):
+    c = cases()[name]()
+    wl = c.wl
+    K = c.K
+    sched = K.Schedule(outer=wl.outer, steps=wl.steps)
+    r = run_compress(c, sched)
+    assert not r["status"].any()
+    co = c.batch.c_off_h
+    osched = O.Schedule(outer=wl.outer, steps=wl.steps)
+    for b in range(c.bt.B):
+        res = O.compress(c.Qs[b], c.Zk[b], c.Zv[b], int(c.k[b]), osched)
+        gi = r["idx"][co[b]:co[b + 1]]
+        check_topk_valid(gi, c.Qs[b], c.Zk[b], c.Zv[b], int(c.k[b]))
+        assert abs(r["trace"][b, 0] - res["trace"][0]) <= 1e-3 * res["trace"][0] + 1e-7, b
+        f_gpu, f_or = float(r["trace"][b, -1]), float(res["loss"])
+        assert f_gpu <= 1.05 * f_or + 1e-7, (b, f_gpu, f_or)
+        assert f_gpu <= r["trace"][b, 0]
+        assert abs(r["parts"][b, 0] * 1.0 + r["parts"][b, 1] - f_gpu) <= 1e-3 * f_gpu + 1e-7
+
+
+@pytest.mark.slow
+def test_compress_qwen_layer_head():
+    """One KV head of the Qwen-shaped layer, full 40 x 5 schedule."""
+    wl = W.WORKLOADS["qwen_layer"]
+    c = Case(wl, ids=[(0, 0, 1)])
+    sched = c.K.Schedule(outer=wl.outer, steps=wl.steps)
+    r = run_compress(c, sched)
+    assert not r["status"].any()
+    res = O.compress(c.Qs[0], c.Zk[0], c.Zv[0], wl.k, O.Schedule(outer=wl.outer, steps=wl.steps))
+    assert check_topk_valid(r["idx"], c.Qs[0], c.Zk[0], c.Zv[0], wl.k)
+    assert abs(r["trace"][0, 0] - res["trace"][0]) <= 1e-3 * res["trace"][0]
+    assert float(r["trace"][0, -1]) <= 1.05 * res["loss"]
