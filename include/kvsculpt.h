@@ -147,6 +147,30 @@ int kvs_loss_grad(const kvs_batch *batch, const float *Q, const float *Kc, const
                   float *loss, float *parts, float *dKc, void *ws, size_t ws_bytes,
                   void *stream);
 
+/* kvs_loss_grad for callers that cannot allocate device memory.  The paper
+ * has no counterpart to this call; it exists for deployment.  Some callers
+ * cannot call cudaMalloc to provide a workspace: a plug-in inside a host
+ * application that owns all device memory through its own pool and forbids
+ * side allocations, or a service that must fix its device footprint when the
+ * library loads.  This call computes exactly what kvs_loss_grad computes, with
+ * its scratch taken from one array compiled into the library: 32 MiB
+ * (KVS_STATIC_WS_BYTES in kvs_static.cu) of device memory on every GPU that
+ * loads the library, held until the process exits.  It allocates nothing.
+ * - Batches whose kvs_workspace_bytes() exceeds 32 MiB return KVS_EWORKSPACE
+ *   (e.g. one head-problem with n_q = 3840 and k = 960 does not fit; the d=64,
+ *   N=256 problem does).
+ * - The first call on a device looks up the array's device address with that
+ *   device current (cudaGetSymbolAddress) and caches it; make that first call
+ *   before any stream capture.
+ * - Every call on a device shares the one array and the array keeps the last
+ *   call's contents.  No part of it needs to start at zero for this call.
+ *   Calls whose work overlaps on the GPU (other streams, other host threads)
+ *   race on it: order them, e.g. on one stream.
+ * Arguments, outputs and errors are those of kvs_loss_grad. */
+int kvs_loss_grad_static(const kvs_batch *batch, const float *Q, const float *Kc,
+                         const float *Vc, const float *Y, const float *lse, float w_out,
+                         float w_lse, float *loss, float *parts, float *dKc, void *stream);
+
 /* Closed-form values (section 2 "Value Optimization"): with A = softmax(s Q Kc^T)
  * fixed, Vc = (A^T A + lambda I)^-1 A^T Y, by Cholesky.  A problem whose Gram
  * matrix is not positive definite gets KVS_ST_NOT_PD in status[b] (OR-ed in)

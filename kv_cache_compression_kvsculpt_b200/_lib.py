@@ -19,7 +19,7 @@ __all__ = [
     "KvsError", "KvsBatch", "Schedule", "QuerySpec", "LIB_PATH", "lib",
     "ST_NONFINITE", "ST_NOT_PD", "ST_LS_FAIL",
     "kvs_version", "kvs_launch_count", "kvs_workspace_bytes", "kvs_lbfgs_state_bytes", "kvs_build_queries",
-    "kvs_targets", "kvs_init_topk", "kvs_loss_grad", "kvs_fit_values", "kvs_lbfgs_reset",
+    "kvs_targets", "kvs_init_topk", "kvs_loss_grad", "kvs_loss_grad_static", "kvs_fit_values", "kvs_lbfgs_reset",
     "kvs_lbfgs_step", "kvs_compress_batch", "kvs_pilot_allocate",
     "alloc_workspace", "alloc_state",
 ]
@@ -64,6 +64,8 @@ _SIGS = {
     "kvs_init_topk": (ctypes.c_int, [_BP, _vp, _vp, _vp, _vp, _vp]),
     "kvs_loss_grad": (ctypes.c_int, [_BP, _vp, _vp, _vp, _vp, _vp, _f32, _f32, _vp, _vp, _vp,
                                      _vp, _sz, _vp]),
+    "kvs_loss_grad_static": (ctypes.c_int, [_BP, _vp, _vp, _vp, _vp, _vp, _f32, _f32, _vp, _vp,
+                                            _vp, _vp]),
     "kvs_fit_values": (ctypes.c_int, [_BP, _vp, _vp, _vp, _f32, _vp, _vp, _vp, _sz, _vp]),
     "kvs_lbfgs_reset": (ctypes.c_int, [_BP, _SP, _vp, _vp, _vp, _vp, _vp, _vp, _sz, _i32, _vp,
                                        _sz, _vp]),
@@ -258,6 +260,17 @@ def kvs_loss_grad(batch: KvsBatch, Q, Kc, Vc, Y, lse, w_out, w_lse, loss, parts,
         _ptr(Y, torch.float32), _ptr(lse, torch.float32), float(w_out), float(w_lse),
         _ptr(loss, torch.float32), _ptr(parts, torch.float32), _ptr(dKc, torch.float32),
         _ptr(ws), ws.numel(), _stream(stream)))
+
+
+def kvs_loss_grad_static(batch: KvsBatch, Q, Kc, Vc, Y, lse, w_out, w_lse, loss, parts, dKc,
+                         stream=None):
+    """kvs_loss_grad without a caller workspace, for callers that cannot allocate device
+    memory: scratch comes from a 32 MiB array inside the library (see the header)."""
+    _check("kvs_loss_grad_static", lib.kvs_loss_grad_static(
+        batch.ref, _ptr(Q, torch.float32), _ptr(Kc, torch.float32), _ptr(Vc, torch.float32),
+        _ptr(Y, torch.float32), _ptr(lse, torch.float32), float(w_out), float(w_lse),
+        _ptr(loss, torch.float32), _ptr(parts, torch.float32), _ptr(dKc, torch.float32),
+        _stream(stream)))
 
 
 def kvs_fit_values(batch: KvsBatch, Q, Kc, Y, lam, Vc, status, ws, stream=None):
