@@ -62,6 +62,7 @@ extern "C" {
 #define KVS_ST_NONFINITE 1  /* a loss, gradient or solve produced inf/nan */
 #define KVS_ST_NOT_PD    2  /* ridge Gram matrix not positive definite (Cholesky pivot <= 0) */
 #define KVS_ST_LS_FAIL   4  /* max_bt Armijo trials failed: x kept, history cleared */
+#define KVS_ST_TIMEOUT   8  /* a kernel's bounded wait expired (results of the call unreliable) */
 
 typedef struct kvs_batch {
   int32_t B;                 /* number of head-problems, >= 1 */

@@ -51,7 +51,9 @@ int geom_from_batch(const kvs_batch *b, HostGeom *g, bool need_c) {
   } else if (b->c_off_h) {
     if (check_offsets(b->c_off_h, b->B, &g->sum_c, &g->max_c, true)) return KVS_EINVAL;
   }
-  g->ld_s = align_up(std::max<int64_t>(std::max(g->max_z, g->max_c), 4), 4);
+  for (int bb = 0; bb < b->B; ++bb)
+    g->sum_qpad += align_up(b->q_off_h[bb + 1] - b->q_off_h[bb], 128);
+  g->ld_a = align_up(std::max(g->max_c, 1), 128);
   return KVS_OK;
 }
 
@@ -70,13 +72,22 @@ struct Carver {
 
 size_t carve_work(const HostGeom &g, void *base, Work *w) {
   Carver c{static_cast<char *>(base)};
-  w->S = c.take<float>(g.sum_q * g.ld_s);
-  w->Yh = c.take<float>(g.sum_q * g.d);
-  w->Go = c.take<float>(g.sum_q * g.d);
+  const int64_t kz = std::max(g.sum_z, g.sum_c);
+  w->qh = c.take<__nv_bfloat16>(g.sum_q * g.d);
+  w->ql = c.take<__nv_bfloat16>(g.sum_q * g.d);
+  w->kh = c.take<__nv_bfloat16>(kz * g.d);
+  w->kl = c.take<__nv_bfloat16>(kz * g.d);
+  w->vh = c.take<__nv_bfloat16>(kz * g.d);
+  w->vl = c.take<__nv_bfloat16>(kz * g.d);
+  w->go = c.take<__nv_bfloat16>(g.sum_q * g.d);
+  w->yh = c.take<__nv_bfloat16>(g.sum_q * g.d);
+  w->yl = c.take<__nv_bfloat16>(g.sum_q * g.d);
+  w->ahi = c.take<__nv_bfloat16>(g.sum_qpad * g.ld_a);
+  w->alo = c.take<__nv_bfloat16>(g.sum_qpad * g.ld_a);
   w->lse_h = c.take<float>(g.sum_q);
   w->delta = c.take<float>(g.sum_q);
-  w->row_out = c.take<float>(g.sum_q);
-  w->row_ls = c.take<float>(g.sum_q);
+  w->partials = c.take<float>((int64_t)g.B * ((g.max_q + 127) / 128) * 2);
+  w->a_pad_off = c.take<int64_t>(g.B + 1);
   w->gram = c.take<float>(g.sum_c * g.max_c);
   w->chol = c.take<double>(g.sum_c * g.max_c);
   w->xs = c.take<double>(g.sum_c * g.d);
@@ -86,6 +97,7 @@ size_t carve_work(const HostGeom &g, void *base, Work *w) {
   w->lset = c.take<float>(g.sum_q);
   w->imp = c.take<float>(g.sum_z);
   w->idx = c.take<int32_t>(g.sum_c);
+  w->err = c.take<int>(1);
   w->bytes = align_up((int64_t)c.off, 256);
   return w->bytes;
 }
@@ -117,6 +129,25 @@ static int prep(const kvs_batch *b, bool need_c, void *ws, size_t ws_bytes, void
   return KVS_OK;
 }
 
+// First device work of a call, after every argument check has passed.
+static int begin(const Batch &Bt, const Work &w) {
+  KVS_CUDA_TRY(cudaMemsetAsync(w.err, 0, sizeof(int), Bt.st));
+  return KVS_OK;
+}
+
+// status[b] |= KVS_ST_TIMEOUT when a kernel of the call gave up waiting.
+__global__ void k_fold_err(const int *err, int32_t *status, int B) {
+  const int b = blockIdx.x * blockDim.x + threadIdx.x;
+  if (b < B && *err) status[b] |= KVS_ST_TIMEOUT;
+}
+
+static int fold_err(const Batch &Bt, const Work &w, int32_t *status) {
+  if (!status) return KVS_OK;
+  k_fold_err<<<(Bt.g.B + 127) / 128, 128, 0, Bt.st>>>(w.err, status, Bt.g.B);
+  KVS_LAUNCH_CHECK("k_fold_err");
+  return KVS_OK;
+}
+
 static bool ok_ptr(const void *p) { return p && aligned(p, 16); }
 
 static bool ok_sched(const kvs_schedule *s) {
@@ -136,28 +167,30 @@ static const Filter ALL{nullptr, 0, 0};
 // Loss and gradient at Kc into (w.fbuf, s.gn), then the state reset.
 static int lbfgs_restart(const Batch &Bt, const kvs_schedule &sc, const float *Q, const float *Y,
                          const float *lse, const float *Vc, const float *Kc, const State &s,
-                         int clear, const Work &w) {
-  int rc = launch_forward(Bt, Q, Kc, Vc, Y, lse, sc.w_out, sc.w_lse, w.fbuf, nullptr, ALL, w);
+                         int clear, bool q_ready, const Work &w) {
+  int rc = launch_forward(Bt, Q, Kc, Vc, Y, lse, sc.w_out, sc.w_lse, w.fbuf, nullptr, ALL, q_ready,
+                          w);
   if (rc) return rc;
-  rc = launch_backward(Bt, Q, Vc, s.gn, ALL, w);
+  rc = launch_backward(Bt, s.gn, ALL, w);
   if (rc) return rc;
   return launch_lbfgs_reset(Bt, s, Kc, w.fbuf, s.gn, clear);
 }
 
 static int lbfgs_one_step(const Batch &Bt, const kvs_schedule &sc, const float *Q,
                           const float *Y, const float *lse, const float *Vc, float *Kc,
-                          const State &s, int32_t *status, float *f_out, const Work &w) {
+                          const State &s, int32_t *status, float *f_out, bool q_ready,
+                          const Work &w) {
   int rc = launch_lbfgs_direction(Bt, s, sc);
   if (rc) return rc;
   const Filter searching = phase_filter(s, PH_SEARCH);
   for (int t = 0; t < sc.max_bt; ++t) {
     if ((rc = launch_lbfgs_trial(Bt, s, Kc))) return rc;
     if ((rc = launch_forward(Bt, Q, Kc, Vc, Y, lse, sc.w_out, sc.w_lse, w.fbuf, nullptr,
-                             searching, w)))
+                             searching, q_ready || t > 0, w)))
       return rc;
     if ((rc = launch_lbfgs_armijo(Bt, s, sc, w.fbuf))) return rc;
   }
-  if ((rc = launch_backward(Bt, Q, Vc, s.gn, phase_filter(s, PH_ACCEPT), w))) return rc;
+  if ((rc = launch_backward(Bt, s.gn, phase_filter(s, PH_ACCEPT), w))) return rc;
   return launch_lbfgs_update(Bt, s, Kc, status, f_out);
 }
 
@@ -209,6 +242,7 @@ int kvs_targets(const kvs_batch *batch, const float *Q, const float *Kz, const f
   if (!ok_ptr(Q) || !ok_ptr(Kz) || !ok_ptr(Vz) || !ok_ptr(Y) || !ok_ptr(lse) ||
       (importance && !ok_ptr(importance)))
     return KVS_EINVAL;
+  if ((rc = begin(Bt, w))) return rc;
   return launch_targets(Bt, Q, Kz, Vz, Y, lse, importance, w);
 }
 
@@ -236,9 +270,10 @@ int kvs_loss_grad(const kvs_batch *batch, const float *Q, const float *Kc, const
   if (!ok_ptr(Q) || !ok_ptr(Kc) || !ok_ptr(Vc) || !ok_ptr(Y) || !ok_ptr(lse) || !ok_ptr(loss) ||
       (parts && !ok_ptr(parts)) || (dKc && !ok_ptr(dKc)))
     return KVS_EINVAL;
-  rc = launch_forward(Bt, Q, Kc, Vc, Y, lse, w_out, w_lse, loss, parts, ALL, w);
+  if ((rc = begin(Bt, w))) return rc;
+  rc = launch_forward(Bt, Q, Kc, Vc, Y, lse, w_out, w_lse, loss, parts, ALL, false, w);
   if (rc || !dKc) return rc;
-  return launch_backward(Bt, Q, Vc, dKc, ALL, w);
+  return launch_backward(Bt, dKc, ALL, w);
 }
 
 int kvs_fit_values(const kvs_batch *batch, const float *Q, const float *Kc, const float *Y,
@@ -251,7 +286,9 @@ int kvs_fit_values(const kvs_batch *batch, const float *Q, const float *Kc, cons
   if (!ok_ptr(Q) || !ok_ptr(Kc) || !ok_ptr(Y) || !ok_ptr(Vc) || !ok_ptr(status) ||
       !isfinite(lambda))
     return KVS_EINVAL;
-  return launch_fit(Bt, Q, Kc, Y, lambda, Vc, status, w);
+  if ((rc = begin(Bt, w))) return rc;
+  if ((rc = launch_fit(Bt, Q, Kc, Y, lambda, Vc, status, false, false, w))) return rc;
+  return fold_err(Bt, w, status);
 }
 
 static int prep_state(const Batch &Bt, const kvs_schedule *sched, void *state,
@@ -273,7 +310,8 @@ int kvs_lbfgs_reset(const kvs_batch *batch, const kvs_schedule *sched, const flo
   if (rc) return rc;
   if ((rc = prep_state(Bt, sched, state, state_bytes, &s))) return rc;
   if (!ok_ptr(Q) || !ok_ptr(Y) || !ok_ptr(lse) || !ok_ptr(Vc) || !ok_ptr(Kc)) return KVS_EINVAL;
-  return lbfgs_restart(Bt, *sched, Q, Y, lse, Vc, Kc, s, clear_history != 0, w);
+  if ((rc = begin(Bt, w))) return rc;
+  return lbfgs_restart(Bt, *sched, Q, Y, lse, Vc, Kc, s, clear_history != 0, false, w);
 }
 
 int kvs_lbfgs_step(const kvs_batch *batch, const kvs_schedule *sched, const float *Q,
@@ -289,7 +327,9 @@ int kvs_lbfgs_step(const kvs_batch *batch, const kvs_schedule *sched, const floa
   if (!ok_ptr(Q) || !ok_ptr(Y) || !ok_ptr(lse) || !ok_ptr(Vc) || !ok_ptr(Kc) ||
       (status && !ok_ptr(status)) || (f_out && !ok_ptr(f_out)))
     return KVS_EINVAL;
-  return lbfgs_one_step(Bt, *sched, Q, Y, lse, Vc, Kc, s, status, f_out, w);
+  if ((rc = begin(Bt, w))) return rc;
+  if ((rc = lbfgs_one_step(Bt, *sched, Q, Y, lse, Vc, Kc, s, status, f_out, false, w))) return rc;
+  return fold_err(Bt, w, status);
 }
 
 int kvs_compress_batch(const kvs_batch *batch, const kvs_schedule *sched, const float *Q,
@@ -312,25 +352,30 @@ int kvs_compress_batch(const kvs_batch *batch, const kvs_schedule *sched, const 
       return KVS_EINVAL;
   const kvs_schedule &sc = *sched;
   int32_t *ix = idx ? idx : w.idx;
+  if ((rc = begin(Bt, w))) return rc;
   KVS_CUDA_TRY(cudaMemsetAsync(status, 0, sizeof(int32_t) * Bt.g.B, Bt.st));
   if ((rc = launch_targets(Bt, Q, Kz, Vz, w.Yt, w.lset, w.imp, w))) return rc;
   if ((rc = launch_topk(Bt, w.imp, Kz, ix, Kc))) return rc;
-  if ((rc = launch_fit(Bt, Q, Kc, w.Yt, sc.lambda, Vc, status, w))) return rc;
-  if ((rc = lbfgs_restart(Bt, sc, Q, w.Yt, w.lset, Vc, Kc, s, 1, w))) return rc;
+  // from here on the bf16 splits of Q and of the targets Y stay in the workspace
+  if ((rc = launch_fit(Bt, Q, Kc, w.Yt, sc.lambda, Vc, status, true, true, w))) return rc;
+  if ((rc = lbfgs_restart(Bt, sc, Q, w.Yt, w.lset, Vc, Kc, s, 1, true, w))) return rc;
   const int64_t tstride = sc.outer + 1;
   if (loss_trace && (rc = launch_copy_f(Bt, s, loss_trace, tstride, 0))) return rc;
   for (int o = 0; o < sc.outer; ++o) {
     for (int t = 0; t < sc.steps; ++t)
-      if ((rc = lbfgs_one_step(Bt, sc, Q, w.Yt, w.lset, Vc, Kc, s, status, nullptr, w)))
+      if ((rc = lbfgs_one_step(Bt, sc, Q, w.Yt, w.lset, Vc, Kc, s, status, nullptr, true, w)))
         return rc;
-    if ((rc = launch_fit(Bt, Q, Kc, w.Yt, sc.lambda, Vc, status, w))) return rc;
-    if ((rc = lbfgs_restart(Bt, sc, Q, w.Yt, w.lset, Vc, Kc, s, sc.persist_history ? 0 : 1, w)))
+    if ((rc = launch_fit(Bt, Q, Kc, w.Yt, sc.lambda, Vc, status, true, true, w))) return rc;
+    if ((rc = lbfgs_restart(Bt, sc, Q, w.Yt, w.lset, Vc, Kc, s, sc.persist_history ? 0 : 1, true,
+                            w)))
       return rc;
     if (loss_trace && (rc = launch_copy_f(Bt, s, loss_trace, tstride, o + 1))) return rc;
   }
-  if (parts)
-    rc = launch_forward(Bt, Q, Kc, Vc, w.Yt, w.lset, sc.w_out, sc.w_lse, w.fbuf, parts, ALL, w);
-  return rc;
+  if (parts &&
+      (rc = launch_forward(Bt, Q, Kc, Vc, w.Yt, w.lset, sc.w_out, sc.w_lse, w.fbuf, parts, ALL,
+                           true, w)))
+    return rc;
+  return fold_err(Bt, w, status);
 }
 
 // Host-only budget allocation.  The real shares x_b(c) = clip(c w_b, k_min,

@@ -1,361 +1,327 @@
-// Attention contractions of the distillation solve: targets, loss forward,
-// dK_c backward and the ridge normal equations.
+// Host orchestration of the attention contractions: targets and importance,
+// loss forward, dK_c backward and the ridge normal equations, on the tcgen05
+// kernels (kvs_attn_fwd.cu, kvs_attn_bwd.cu, kvs_gemm3.cu).
 //
-// "KVSculpt: KV Cache Compression as Distillation", section 2 "Loss Function"
-// (output MSE + LSE matching), "Value Optimization" (ridge regression given
-// the attention weights) and "Initialization" (attention importance).
+// "KVSculpt: KV Cache Compression as Distillation", section 2 "Loss
+// Function", "Value Optimization" and "Initialization".
 //
-// This file holds the straightforward batched formulation on CUDA cores: the
-// score matrix of every problem is materialised in the workspace and each
-// contraction is a tiled fp32 GEMM with a small fused epilogue.
+// Operands enter the tensor cores as bf16 hi/lo pairs, every product taking
+// three MMAs (hi.hi + hi.lo + lo.hi, about 16 significant bits) except
+// dP = Go V^T, where Go is a single bf16 and delta is formed from the same
+// rounded Go, so that its rounding cancels exactly in dP - delta.
+#include <cudaTypedefs.h>
 #include <math.h>
 
-#include "kvs_internal.cuh"
+#include <algorithm>
+#include <mutex>
+
+#include "kvs_attn_tc.cuh"
 
 namespace kvs {
+
+// ------------------------------------------------------------ tensor maps
+
+static PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    cudaDriverEntryPointQueryResult q;
+    void *p = nullptr;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  });
+  return fn;
+}
+
+int make_map_bf16(CUtensorMap *m, const void *base, uint64_t rows, uint64_t cols,
+                  uint32_t box_rows) {
+  auto fn = encode_fn();
+  if (!fn) return KVS_ECUDA;
+  cuuint64_t dims[2] = {(cuuint64_t)cols, (cuuint64_t)(rows > 0 ? rows : 1)};
+  cuuint64_t strides[1] = {(cuuint64_t)cols * 2};
+  cuuint32_t box[2] = {64, box_rows};
+  cuuint32_t es[2] = {1, 1};
+  CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(base), dims, strides,
+                  box, es, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? KVS_OK : KVS_ECUDA;
+}
+
 namespace {
 
-enum { EPI_STORE = 0, EPI_GRAM = 1, EPI_DS = 2 };
+// ------------------------------------------------------ elementwise helpers
 
-struct GemmArgs {
-  Mat A, B, C;          // C is written through a const_cast
-  Dim M, N, K;
-  float alpha, lam;
-  Mat rowvec;           // EPI_DS: delta per row (ld = 1)
-  Filter flt;
-};
-
-constexpr int TM = 64, TN = 64, TK = 16;
-
-// C = alpha * op(A) op(B) with op(A) = A (row-major M x K) or A^T (A stored K x M),
-// op(B) = B^T (B stored N x K) or B (stored K x N).  One 64 x 64 tile per CTA.
-template <bool TA, bool TB, int EPI>
-__global__ void __launch_bounds__(256) k_gemm(GemmArgs a) {
-  const int b = blockIdx.z;
-  if (a.flt.skip(b)) return;
-  const int M = a.M.of(b), N = a.N.of(b), K = a.K.of(b);
-  const int m0 = blockIdx.y * TM, n0 = blockIdx.x * TN;
-  if (m0 >= M || n0 >= N) return;
-  const float *A = a.A.at(b);
-  const float *Bm = a.B.at(b);
-  float *C = const_cast<float *>(a.C.at(b));
-  __shared__ float As[TK][TM + 4];
-  __shared__ float Bs[TK][TN + 4];
-  float acc[4][4];
+// x -> (hi, lo) bf16 with hi = rn(x), lo = rn(x - hi); lo may be null (hi only).
+__global__ void k_split(const float *__restrict__ x, __nv_bfloat16 *__restrict__ hi,
+                        __nv_bfloat16 *__restrict__ lo, int64_t n4) {
+  for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < n4;
+       i += (int64_t)gridDim.x * blockDim.x) {
+    const float4 v = reinterpret_cast<const float4 *>(x)[i];
+    const float e[4] = {v.x, v.y, v.z, v.w};
+    __nv_bfloat16 h[4], l[4];
 #pragma unroll
-  for (int i = 0; i < 4; ++i)
-#pragma unroll
-    for (int j = 0; j < 4; ++j) acc[i][j] = 0.f;
-  const int t = threadIdx.x, tx = t & 15, ty = t >> 4;
-  for (int k0 = 0; k0 < K; k0 += TK) {
-#pragma unroll
-    for (int e = t; e < TM * TK; e += 256) {
-      int m, kk;
-      if (!TA) { m = e >> 4; kk = e & 15; } else { kk = e >> 6; m = e & 63; }
-      const int gm = m0 + m, gk = k0 + kk;
-      float v = 0.f;
-      if (gm < M && gk < K)
-        v = TA ? A[(int64_t)gk * a.A.ld + gm] : A[(int64_t)gm * a.A.ld + gk];
-      As[kk][m] = v;
-    }
-#pragma unroll
-    for (int e = t; e < TN * TK; e += 256) {
-      int n, kk;
-      if (TB) { n = e >> 4; kk = e & 15; } else { kk = e >> 6; n = e & 63; }
-      const int gn = n0 + n, gk = k0 + kk;
-      float v = 0.f;
-      if (gn < N && gk < K)
-        v = TB ? Bm[(int64_t)gn * a.B.ld + gk] : Bm[(int64_t)gk * a.B.ld + gn];
-      Bs[kk][n] = v;
-    }
-    __syncthreads();
-#pragma unroll
-    for (int kk = 0; kk < TK; ++kk) {
-      float av[4], bv[4];
-#pragma unroll
-      for (int i = 0; i < 4; ++i) av[i] = As[kk][ty * 4 + i];
-#pragma unroll
-      for (int j = 0; j < 4; ++j) bv[j] = Bs[kk][tx * 4 + j];
-#pragma unroll
-      for (int i = 0; i < 4; ++i)
-#pragma unroll
-        for (int j = 0; j < 4; ++j) acc[i][j] = fmaf(av[i], bv[j], acc[i][j]);
-    }
-    __syncthreads();
-  }
-  const float *dl = (EPI == EPI_DS) ? a.rowvec.at(b) : nullptr;
-#pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    const int gm = m0 + ty * 4 + i;
-    if (gm >= M) continue;
-#pragma unroll
-    for (int j = 0; j < 4; ++j) {
-      const int gn = n0 + tx * 4 + j;
-      if (gn >= N) continue;
-      float v = a.alpha * acc[i][j];
-      float *c = C + (int64_t)gm * a.C.ld + gn;
-      if (EPI == EPI_STORE) *c = v;
-      else if (EPI == EPI_GRAM) *c = v + (gm == gn ? a.lam : 0.f);
-      else *c = *c * (v - dl[gm]);
+    for (int u = 0; u < 4; ++u) tc::split_bf16(e[u], h[u], l[u]);
+    uint2 hv, lv;
+    hv.x = (uint32_t)__bfloat16_as_ushort(h[0]) | ((uint32_t)__bfloat16_as_ushort(h[1]) << 16);
+    hv.y = (uint32_t)__bfloat16_as_ushort(h[2]) | ((uint32_t)__bfloat16_as_ushort(h[3]) << 16);
+    reinterpret_cast<uint2 *>(hi)[i] = hv;
+    if (lo) {
+      lv.x = (uint32_t)__bfloat16_as_ushort(l[0]) | ((uint32_t)__bfloat16_as_ushort(l[1]) << 16);
+      lv.y = (uint32_t)__bfloat16_as_ushort(l[2]) | ((uint32_t)__bfloat16_as_ushort(l[3]) << 16);
+      reinterpret_cast<uint2 *>(lo)[i] = lv;
     }
   }
 }
 
-template <bool TA, bool TB, int EPI>
-int gemm(const Batch &Bt, const GemmArgs &a, int max_m, int max_n) {
-  if (max_m <= 0 || max_n <= 0) return KVS_OK;
-  dim3 grid((max_n + TN - 1) / TN, (max_m + TM - 1) / TM, Bt.g.B);
-  k_gemm<TA, TB, EPI><<<grid, 256, 0, Bt.st>>>(a);
-  KVS_LAUNCH_CHECK("k_gemm");
+int split(const float *x, __nv_bfloat16 *hi, __nv_bfloat16 *lo, int64_t n, cudaStream_t st) {
+  const int64_t n4 = n / 4;  // row length d is a multiple of 4
+  if (n4 == 0) return KVS_OK;
+  const int blocks = (int)std::min<int64_t>((n4 + 255) / 256, 148 * 16);
+  k_split<<<blocks, 256, 0, st>>>(x, hi, lo, n4);
+  KVS_LAUNCH_CHECK("k_split");
   return KVS_OK;
 }
 
-// Row softmax in place: S[i, :n] <- exp(S - lse_i); lse_i = log sum_j exp(S_ij).
-__global__ void __launch_bounds__(256) k_softmax_rows(Mat S, Dim rows, Dim cols, Mat lse,
-                                                      Filter flt) {
-  const int b = blockIdx.y;
-  if (flt.skip(b)) return;
-  const int r = blockIdx.x;
-  if (r >= rows.of(b)) return;
-  const int n = cols.of(b);
-  float *s = const_cast<float *>(S.at(b)) + (int64_t)r * S.ld;
-  __shared__ float red[32];
-  float mx = -INFINITY;
-  for (int j = threadIdx.x; j < n; j += blockDim.x) mx = fmaxf(mx, s[j]);
-  mx = block_max(mx, red);
-  float sum = 0.f;
-  for (int j = threadIdx.x; j < n; j += blockDim.x) sum += expf(s[j] - mx);
-  sum = block_sum(sum, red);
-  const float l = mx + logf(sum);
-  for (int j = threadIdx.x; j < n; j += blockDim.x) s[j] = expf(s[j] - l);
-  if (threadIdx.x == 0) const_cast<float *>(lse.at(b))[r] = l;
-}
-
-// Per-row residual of the loss: one warp per training query.
-//   Go = c_o (Yh - Y), delta = Go . Yh - c_l (lh - l), row_out = |Yh - Y|^2,
-//   row_ls = (lh - l)^2, with c_o = 2 w_out / (n_q d) and c_l = 2 w_lse / n_q.
-__global__ void __launch_bounds__(256) k_residual(Mat Yh, Mat Y, Mat lh, Mat l, Mat Go,
-                                                  Mat delta, Mat row_out, Mat row_ls, Dim rows,
-                                                  int d, float w_out, float w_lse,
-                                                  Filter flt) {
-  const int b = blockIdx.y;
-  if (flt.skip(b)) return;
-  const int nq = rows.of(b);
-  const int r = blockIdx.x * 8 + (threadIdx.x >> 5);
-  const int lane = threadIdx.x & 31;
-  if (r >= nq) return;
-  const float co = 2.f * w_out / ((float)nq * (float)d);
-  const float cl = 2.f * w_lse / (float)nq;
-  const float *yh = Yh.at(b) + (int64_t)r * d;
-  const float *y = Y.at(b) + (int64_t)r * d;
-  float *go = const_cast<float *>(Go.at(b)) + (int64_t)r * d;
-  float se = 0.f, gy = 0.f;
-  for (int c = lane; c < d; c += 32) {
-    const float e = yh[c] - y[c];
-    se = fmaf(e, e, se);
-    const float gv = co * e;
-    go[c] = gv;
-    gy = fmaf(gv, yh[c], gy);
-  }
-  se = warp_sum(se);
-  gy = warp_sum(gy);
-  if (lane == 0) {
-    const float el = lh.at(b)[r] - l.at(b)[r];
-    const_cast<float *>(delta.at(b))[r] = gy - cl * el;
-    const_cast<float *>(row_out.at(b))[r] = se;
-    const_cast<float *>(row_ls.at(b))[r] = el * el;
-  }
-}
-
-// loss[b] = w_out/(n_q d) sum row_out + w_lse/n_q sum row_ls (fixed-order block sums).
-__global__ void __launch_bounds__(256) k_loss_reduce(Mat row_out, Mat row_ls, Dim rows, int d,
-                                                     float w_out, float w_lse, float *loss,
-                                                     float *parts, Filter flt) {
-  const int b = blockIdx.x;
-  if (flt.skip(b)) return;
-  const int nq = rows.of(b);
-  __shared__ double red[32];
-  const float *ro = row_out.at(b), *rl = row_ls.at(b);
-  double so = 0.0, sl = 0.0;
-  for (int i = threadIdx.x; i < nq; i += blockDim.x) {
-    so += ro[i];
-    sl += rl[i];
-  }
-  so = block_sum_d(so, red);
-  sl = block_sum_d(sl, red);
-  if (threadIdx.x == 0) {
-    const double out = so / ((double)nq * d), ls = sl / (double)nq;
-    loss[b] = (float)(w_out * out + w_lse * ls);
-    if (parts) {
-      parts[2 * b] = (float)out;
-      parts[2 * b + 1] = (float)ls;
+// padded row offsets of the A buffer: pad[b] = sum_{b' < b} round_up(n_q_b', 128)
+__global__ void k_pad_offsets(const int64_t *q_off, int B, int64_t *pad) {
+  if (blockIdx.x == 0 && threadIdx.x == 0) {
+    int64_t s = 0;
+    pad[0] = 0;
+    for (int b = 0; b < B; ++b) {
+      const int64_t n = q_off[b + 1] - q_off[b];
+      s += (n + 127) / 128 * 128;
+      pad[b + 1] = s;
     }
   }
 }
 
-// importance[j] = sum_i A[i, j] over the problem's training queries.
-__global__ void __launch_bounds__(256) k_colsum(Mat A, Dim rows, Dim cols, Mat imp) {
-  const int b = blockIdx.y;
-  const int j = blockIdx.x * blockDim.x + threadIdx.x;
-  if (j >= cols.of(b)) return;
-  const int nq = rows.of(b);
-  const float *a = A.at(b) + j;
-  float s = 0.f;
-  for (int i = 0; i < nq; ++i) s += a[(int64_t)i * A.ld];
-  const_cast<float *>(imp.at(b))[j] = s;
+// loss[b] from the per-CTA partial sums of the loss forward (fixed order).
+__global__ void k_loss_reduce(const float *partials, int tiles, const int64_t *q_off, int d,
+                              float w_out, float w_lse, float *loss, float *parts, Filter flt,
+                              int B) {
+  const int b = blockIdx.x * blockDim.x + threadIdx.x;
+  if (b >= B || flt.skip(b)) return;
+  const int nq = (int)(q_off[b + 1] - q_off[b]);
+  const int nt = (nq + 127) / 128;
+  double so = 0.0, sl = 0.0;
+  for (int t = 0; t < nt; ++t) {
+    so += partials[((int64_t)b * tiles + t) * 2];
+    sl += partials[((int64_t)b * tiles + t) * 2 + 1];
+  }
+  const double out = so / ((double)nq * d), ls = sl / (double)nq;
+  loss[b] = (float)(w_out * out + w_lse * ls);
+  if (parts) {
+    parts[2 * b] = (float)out;
+    parts[2 * b + 1] = (float)ls;
+  }
 }
 
-Mat mat(const float *p, const int64_t *off, int64_t ld) { return Mat{p, off, 0, ld}; }
+int max_qtiles(const HostGeom &g) { return (g.max_q + 127) / 128; }
+
+template <int D>
+int targets_d(const Batch &Bt, const float *Q, const float *Kz, const float *Vz, float *Y,
+              float *lse, float *imp, const Work &w) {
+  const HostGeom &g = Bt.g;
+  int rc;
+  if ((rc = split(Q, w.qh, w.ql, g.sum_q * D, Bt.st))) return rc;
+  if ((rc = split(Kz, w.kh, w.kl, g.sum_z * D, Bt.st))) return rc;
+  if ((rc = split(Vz, w.vh, w.vl, g.sum_z * D, Bt.st))) return rc;
+  FwdMaps fm;
+  if ((rc = make_map_bf16(&fm.kh, w.kh, g.sum_z, D, 64)) ||
+      (rc = make_map_bf16(&fm.kl, w.kl, g.sum_z, D, 64)) ||
+      (rc = make_map_bf16(&fm.vh, w.vh, g.sum_z, D, 64)) ||
+      (rc = make_map_bf16(&fm.vl, w.vl, g.sum_z, D, 64)))
+    return rc;
+  FwdArgs a{};
+  a.q_off = Bt.b->q_off;
+  a.k_off = Bt.b->z_off;
+  a.q_hi = w.qh;
+  a.q_lo = w.ql;
+  a.flt = Filter{nullptr, 0, 0};
+  a.scale = 1.f / sqrtf((float)D);
+  a.y_out = Y;
+  a.y_hi = w.yh;
+  a.y_lo = w.yl;
+  a.lse_out = lse;
+  a.err = w.err;
+  if ((rc = launch_fwd_tc<D, FWD_TARGETS>(fm, a, max_qtiles(g), g.B, Bt.st))) return rc;
+  if (!imp) return KVS_OK;
+  BwdMaps bm;
+  if ((rc = make_map_bf16(&bm.kh, w.kh, g.sum_z, D, 128)) ||
+      (rc = make_map_bf16(&bm.kl, w.kl, g.sum_z, D, 128)) ||
+      (rc = make_map_bf16(&bm.qh, w.qh, g.sum_q, D, 64)) ||
+      (rc = make_map_bf16(&bm.ql, w.ql, g.sum_q, D, 64)))
+    return rc;
+  bm.g = bm.qh;
+  BwdArgs ba{};
+  ba.q_off = Bt.b->q_off;
+  ba.k_off = Bt.b->z_off;
+  ba.flt = Filter{nullptr, 0, 0};
+  ba.scale = a.scale;
+  ba.lse = lse;
+  ba.imp = imp;
+  ba.err = w.err;
+  return launch_bwd_tc<D, BWD_COLSUM>(bm, ba, (g.max_z + 127) / 128, g.B, Bt.st);
+}
+
+// bf16 hi/lo copies of the keys and values of the compressed pairs.
+template <int D>
+int prep_pairs(const Batch &Bt, const float *Kc, const float *Vc, const Work &w) {
+  int rc = split(Kc, w.kh, w.kl, Bt.g.sum_c * D, Bt.st);
+  if (rc || !Vc) return rc;
+  return split(Vc, w.vh, w.vl, Bt.g.sum_c * D, Bt.st);
+}
+
+template <int D>
+int forward_d(const Batch &Bt, const float *Q, const float *Kc, const float *Vc, const float *Y,
+              const float *lse, float w_out, float w_lse, float *loss, float *parts, Filter flt,
+              bool q_ready, const Work &w) {
+  const HostGeom &g = Bt.g;
+  int rc;
+  if (!q_ready && (rc = split(Q, w.qh, w.ql, g.sum_q * D, Bt.st))) return rc;
+  if ((rc = prep_pairs<D>(Bt, Kc, Vc, w))) return rc;
+  FwdMaps fm;
+  if ((rc = make_map_bf16(&fm.kh, w.kh, g.sum_c, D, 64)) ||
+      (rc = make_map_bf16(&fm.kl, w.kl, g.sum_c, D, 64)) ||
+      (rc = make_map_bf16(&fm.vh, w.vh, g.sum_c, D, 64)) ||
+      (rc = make_map_bf16(&fm.vl, w.vl, g.sum_c, D, 64)))
+    return rc;
+  FwdArgs a{};
+  a.q_off = Bt.b->q_off;
+  a.k_off = Bt.b->c_off;
+  a.q_hi = w.qh;
+  a.q_lo = w.ql;
+  a.flt = flt;
+  a.scale = 1.f / sqrtf((float)D);
+  a.y_in = Y;
+  a.lse_in = lse;
+  a.lse_out = w.lse_h;
+  a.go = w.go;
+  a.delta = w.delta;
+  a.partials = w.partials;
+  a.tiles_per_problem = max_qtiles(g);
+  a.w_out = w_out;
+  a.w_lse = w_lse;
+  a.err = w.err;
+  if ((rc = launch_fwd_tc<D, FWD_LOSS>(fm, a, max_qtiles(g), g.B, Bt.st))) return rc;
+  k_loss_reduce<<<(g.B + 127) / 128, 128, 0, Bt.st>>>(w.partials, max_qtiles(g), Bt.b->q_off, D,
+                                                      w_out, w_lse, loss, parts, flt, g.B);
+  KVS_LAUNCH_CHECK("k_loss_reduce");
+  return KVS_OK;
+}
+
+template <int D>
+int backward_d(const Batch &Bt, float *dKc, Filter flt, const Work &w) {
+  const HostGeom &g = Bt.g;
+  int rc;
+  BwdMaps bm;
+  if ((rc = make_map_bf16(&bm.kh, w.kh, g.sum_c, D, 128)) ||
+      (rc = make_map_bf16(&bm.kl, w.kl, g.sum_c, D, 128)) ||
+      (rc = make_map_bf16(&bm.qh, w.qh, g.sum_q, D, 64)) ||
+      (rc = make_map_bf16(&bm.ql, w.ql, g.sum_q, D, 64)) ||
+      (rc = make_map_bf16(&bm.g, w.go, g.sum_q, D, 64)))
+    return rc;
+  BwdArgs ba{};
+  ba.q_off = Bt.b->q_off;
+  ba.k_off = Bt.b->c_off;
+  ba.flt = flt;
+  ba.scale = 1.f / sqrtf((float)D);
+  ba.lse = w.lse_h;
+  ba.delta = w.delta;
+  ba.v_hi = w.vh;
+  ba.v_lo = w.vl;
+  ba.dk = dKc;
+  ba.err = w.err;
+  return launch_bwd_tc<D, BWD_DK>(bm, ba, (g.max_c + 127) / 128, g.B, Bt.st);
+}
+
+template <int D>
+int fit_d(const Batch &Bt, const float *Q, const float *Kc, const float *Y, float lam, float *Vc,
+          int32_t *status, bool q_ready, bool y_ready, const Work &w) {
+  const HostGeom &g = Bt.g;
+  int rc;
+  if (!q_ready && (rc = split(Q, w.qh, w.ql, g.sum_q * D, Bt.st))) return rc;
+  if (!y_ready && (rc = split(Y, w.yh, w.yl, g.sum_q * D, Bt.st))) return rc;
+  if ((rc = prep_pairs<D>(Bt, Kc, nullptr, w))) return rc;
+  FwdMaps fm;
+  if ((rc = make_map_bf16(&fm.kh, w.kh, g.sum_c, D, 64)) ||
+      (rc = make_map_bf16(&fm.kl, w.kl, g.sum_c, D, 64)))
+    return rc;
+  fm.vh = fm.kh;
+  fm.vl = fm.kl;
+  FwdArgs a{};
+  a.q_off = Bt.b->q_off;
+  a.k_off = Bt.b->c_off;
+  a.q_hi = w.qh;
+  a.q_lo = w.ql;
+  a.flt = Filter{nullptr, 0, 0};
+  a.scale = 1.f / sqrtf((float)D);
+  a.lse_out = w.lse_h;
+  a.err = w.err;
+  if ((rc = launch_fwd_tc<D, FWD_STATS>(fm, a, max_qtiles(g), g.B, Bt.st))) return rc;
+  k_pad_offsets<<<1, 1, 0, Bt.st>>>(Bt.b->q_off, g.B, w.a_pad_off);
+  KVS_LAUNCH_CHECK("k_pad_offsets");
+  a.lse_in = w.lse_h;
+  a.a_hi = w.ahi;
+  a.a_lo = w.alo;
+  a.ld_a = g.ld_a;
+  a.a_pad_off = w.a_pad_off;
+  if ((rc = launch_fwd_tc<D, FWD_WRITE_A>(fm, a, max_qtiles(g), g.B, Bt.st))) return rc;
+  GemmMaps gm;
+  if ((rc = make_map_bf16(&gm.ah, w.ahi, g.sum_qpad, g.ld_a, 64)) ||
+      (rc = make_map_bf16(&gm.al, w.alo, g.sum_qpad, g.ld_a, 64)))
+    return rc;
+  gm.bh = gm.ah;
+  gm.bl = gm.al;
+  GemmArgs3 ga{};
+  ga.a_pad_off = w.a_pad_off;
+  ga.m_off = Bt.b->c_off;
+  ga.n_fixed = 0;
+  ga.b_row_off = w.a_pad_off;
+  ga.c = w.gram;
+  ga.ldc = g.max_c;
+  ga.diag = lam;
+  ga.err = w.err;
+  const int tm = (g.max_c + 127) / 128;
+  if ((rc = launch_gemm3_tc(gm, ga, tm, 1, g.B, Bt.st))) return rc;
+  if ((rc = make_map_bf16(&gm.bh, w.yh, g.sum_q, D, 64)) ||
+      (rc = make_map_bf16(&gm.bl, w.yl, g.sum_q, D, 64)))
+    return rc;
+  ga.n_fixed = D;
+  ga.b_row_off = Bt.b->q_off;
+  ga.c = w.R;
+  ga.ldc = D;
+  ga.diag = 0.f;
+  if ((rc = launch_gemm3_tc(gm, ga, tm, 0, g.B, Bt.st))) return rc;
+  return launch_chol_solve(Bt, Vc, status, w);
+}
 
 }  // namespace
 
 int launch_targets(const Batch &Bt, const float *Q, const float *Kz, const float *Vz, float *Y,
                    float *lse, float *imp, const Work &w) {
-  const HostGeom &g = Bt.g;
-  const kvs_batch *b = Bt.b;
-  const float s = 1.f / sqrtf((float)g.d);
-  GemmArgs a{};
-  a.A = mat(Q, b->q_off, g.d);
-  a.B = mat(Kz, b->z_off, g.d);
-  a.C = mat(w.S, b->q_off, g.ld_s);
-  a.M = Dim{b->q_off, 0};
-  a.N = Dim{b->z_off, 0};
-  a.K = Dim{nullptr, g.d};
-  a.alpha = s;
-  int rc = gemm<false, true, EPI_STORE>(Bt, a, g.max_q, g.max_z);
-  if (rc) return rc;
-  k_softmax_rows<<<dim3(g.max_q, g.B), 256, 0, Bt.st>>>(mat(w.S, b->q_off, g.ld_s), Dim{b->q_off, 0},
-                                                         Dim{b->z_off, 0}, mat(lse, b->q_off, 1),
-                                                         Filter{nullptr, 0, 0});
-  KVS_LAUNCH_CHECK("k_softmax_rows");
-  GemmArgs o{};
-  o.A = mat(w.S, b->q_off, g.ld_s);
-  o.B = mat(Vz, b->z_off, g.d);
-  o.C = mat(Y, b->q_off, g.d);
-  o.M = Dim{b->q_off, 0};
-  o.N = Dim{nullptr, g.d};
-  o.K = Dim{b->z_off, 0};
-  o.alpha = 1.f;
-  rc = gemm<false, false, EPI_STORE>(Bt, o, g.max_q, g.d);
-  if (rc) return rc;
-  if (imp) {
-    k_colsum<<<dim3((g.max_z + 255) / 256, g.B), 256, 0, Bt.st>>>(
-        mat(w.S, b->q_off, g.ld_s), Dim{b->q_off, 0}, Dim{b->z_off, 0}, mat(imp, b->z_off, 1));
-    KVS_LAUNCH_CHECK("k_colsum");
-  }
-  return KVS_OK;
-}
-
-static int scores_softmax(const Batch &Bt, const float *Q, const float *Kc, Filter flt,
-                          const Work &w) {
-  const HostGeom &g = Bt.g;
-  const kvs_batch *b = Bt.b;
-  GemmArgs a{};
-  a.A = mat(Q, b->q_off, g.d);
-  a.B = mat(Kc, b->c_off, g.d);
-  a.C = mat(w.S, b->q_off, g.ld_s);
-  a.M = Dim{b->q_off, 0};
-  a.N = Dim{b->c_off, 0};
-  a.K = Dim{nullptr, g.d};
-  a.alpha = 1.f / sqrtf((float)g.d);
-  a.flt = flt;
-  int rc = gemm<false, true, EPI_STORE>(Bt, a, g.max_q, g.max_c);
-  if (rc) return rc;
-  k_softmax_rows<<<dim3(g.max_q, g.B), 256, 0, Bt.st>>>(mat(w.S, b->q_off, g.ld_s), Dim{b->q_off, 0},
-                                                         Dim{b->c_off, 0},
-                                                         mat(w.lse_h, b->q_off, 1), flt);
-  KVS_LAUNCH_CHECK("k_softmax_rows");
-  return KVS_OK;
+  return Bt.g.d == 64 ? targets_d<64>(Bt, Q, Kz, Vz, Y, lse, imp, w)
+                      : targets_d<128>(Bt, Q, Kz, Vz, Y, lse, imp, w);
 }
 
 int launch_forward(const Batch &Bt, const float *Q, const float *Kc, const float *Vc,
                    const float *Y, const float *lse, float w_out, float w_lse, float *loss,
-                   float *parts, Filter flt, const Work &w) {
-  const HostGeom &g = Bt.g;
-  const kvs_batch *b = Bt.b;
-  int rc = scores_softmax(Bt, Q, Kc, flt, w);
-  if (rc) return rc;
-  GemmArgs o{};
-  o.A = mat(w.S, b->q_off, g.ld_s);
-  o.B = mat(Vc, b->c_off, g.d);
-  o.C = mat(w.Yh, b->q_off, g.d);
-  o.M = Dim{b->q_off, 0};
-  o.N = Dim{nullptr, g.d};
-  o.K = Dim{b->c_off, 0};
-  o.alpha = 1.f;
-  o.flt = flt;
-  rc = gemm<false, false, EPI_STORE>(Bt, o, g.max_q, g.d);
-  if (rc) return rc;
-  k_residual<<<dim3((g.max_q + 7) / 8, g.B), 256, 0, Bt.st>>>(
-      mat(w.Yh, b->q_off, g.d), mat(Y, b->q_off, g.d), mat(w.lse_h, b->q_off, 1),
-      mat(lse, b->q_off, 1), mat(w.Go, b->q_off, g.d), mat(w.delta, b->q_off, 1),
-      mat(w.row_out, b->q_off, 1), mat(w.row_ls, b->q_off, 1), Dim{b->q_off, 0}, g.d, w_out,
-      w_lse, flt);
-  KVS_LAUNCH_CHECK("k_residual");
-  k_loss_reduce<<<g.B, 256, 0, Bt.st>>>(mat(w.row_out, b->q_off, 1), mat(w.row_ls, b->q_off, 1),
-                                        Dim{b->q_off, 0}, g.d, w_out, w_lse, loss, parts, flt);
-  KVS_LAUNCH_CHECK("k_loss_reduce");
-  return KVS_OK;
+                   float *parts, Filter flt, bool q_ready, const Work &w) {
+  return Bt.g.d == 64
+             ? forward_d<64>(Bt, Q, Kc, Vc, Y, lse, w_out, w_lse, loss, parts, flt, q_ready, w)
+             : forward_d<128>(Bt, Q, Kc, Vc, Y, lse, w_out, w_lse, loss, parts, flt, q_ready, w);
 }
 
-int launch_backward(const Batch &Bt, const float *Q, const float *Vc, float *dKc,
-                    Filter flt, const Work &w) {
-  const HostGeom &g = Bt.g;
-  const kvs_batch *b = Bt.b;
-  // dS = A * (Go Vc^T - delta), in place over A.
-  GemmArgs p{};
-  p.A = mat(w.Go, b->q_off, g.d);
-  p.B = mat(Vc, b->c_off, g.d);
-  p.C = mat(w.S, b->q_off, g.ld_s);
-  p.M = Dim{b->q_off, 0};
-  p.N = Dim{b->c_off, 0};
-  p.K = Dim{nullptr, g.d};
-  p.alpha = 1.f;
-  p.rowvec = mat(w.delta, b->q_off, 1);
-  p.flt = flt;
-  int rc = gemm<false, true, EPI_DS>(Bt, p, g.max_q, g.max_c);
-  if (rc) return rc;
-  // dKc = s dS^T Q
-  GemmArgs k{};
-  k.A = mat(w.S, b->q_off, g.ld_s);
-  k.B = mat(Q, b->q_off, g.d);
-  k.C = mat(dKc, b->c_off, g.d);
-  k.M = Dim{b->c_off, 0};
-  k.N = Dim{nullptr, g.d};
-  k.K = Dim{b->q_off, 0};
-  k.alpha = 1.f / sqrtf((float)g.d);
-  k.flt = flt;
-  return gemm<true, false, EPI_STORE>(Bt, k, g.max_c, g.d);
+int launch_backward(const Batch &Bt, float *dKc, Filter flt, const Work &w) {
+  return Bt.g.d == 64 ? backward_d<64>(Bt, dKc, flt, w) : backward_d<128>(Bt, dKc, flt, w);
 }
 
 int launch_fit(const Batch &Bt, const float *Q, const float *Kc, const float *Y, float lam,
-               float *Vc, int32_t *status, const Work &w) {
-  const HostGeom &g = Bt.g;
-  const kvs_batch *b = Bt.b;
-  int rc = scores_softmax(Bt, Q, Kc, Filter{nullptr, 0, 0}, w);
-  if (rc) return rc;
-  GemmArgs G{};
-  G.A = mat(w.S, b->q_off, g.ld_s);
-  G.B = mat(w.S, b->q_off, g.ld_s);
-  G.C = mat(w.gram, b->c_off, g.max_c);
-  G.M = Dim{b->c_off, 0};
-  G.N = Dim{b->c_off, 0};
-  G.K = Dim{b->q_off, 0};
-  G.alpha = 1.f;
-  G.lam = lam;
-  rc = gemm<true, false, EPI_GRAM>(Bt, G, g.max_c, g.max_c);
-  if (rc) return rc;
-  GemmArgs R{};
-  R.A = mat(w.S, b->q_off, g.ld_s);
-  R.B = mat(Y, b->q_off, g.d);
-  R.C = mat(w.R, b->c_off, g.d);
-  R.M = Dim{b->c_off, 0};
-  R.N = Dim{nullptr, g.d};
-  R.K = Dim{b->q_off, 0};
-  R.alpha = 1.f;
-  rc = gemm<true, false, EPI_STORE>(Bt, R, g.max_c, g.d);
-  if (rc) return rc;
-  return launch_chol_solve(Bt, Vc, status, w);
+               float *Vc, int32_t *status, bool q_ready, bool y_ready, const Work &w) {
+  return Bt.g.d == 64 ? fit_d<64>(Bt, Q, Kc, Y, lam, Vc, status, q_ready, y_ready, w)
+                      : fit_d<128>(Bt, Q, Kc, Y, lam, Vc, status, q_ready, y_ready, w);
 }
 
 }  // namespace kvs

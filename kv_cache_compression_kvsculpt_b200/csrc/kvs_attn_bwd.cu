@@ -1,0 +1,329 @@
+// Key-tile attention kernel on tcgen05 tensor cores: the key gradient of the
+// distillation loss and the attention importance of each key.
+//
+// "KVSculpt: KV Cache Compression as Distillation", section 2 "Loss
+// Function" (gradient of output MSE + LSE matching with respect to the keys,
+// for L-BFGS in "Key Optimization") and "Initialization" (keys ranked by
+// attention importance).
+//
+// One CTA owns 128 keys of one problem and streams its training queries in
+// tiles of 64.  Per tile, with A = exp(S - l_row):
+//   S^T  = K Q^T                    K_hi Q_hi + K_lo Q_hi + K_hi Q_lo  (K in smem)
+//   DK:     dP^T = V Go^T           V_hi Go + V_lo Go  (V in TMEM, Go bf16; delta was
+//                                   formed from the same rounded Go)
+//           dS = A (dP - delta_row) written as bf16 hi/lo over the S buffer in TMEM
+//           dK += dS Q              dS_hi Q_hi + dS_hi Q_lo + dS_lo Q_hi
+//   COLSUM: importance += sum over the tile's queries of A
+// Near an optimum the key gradient is a small sum of large terms, so every
+// product keeps about 16 significant bits.
+// Tensor memory (512 columns): S buffers at 0 and 64, dP at 128 and 192,
+// dK at 256, V hi at 384, V lo at 384 + D/2.
+// Warp roles: warps 0-3 one thread per key row (TMEM lane), warp 4 TMA
+// producer (also stages l and delta of the tile), warp 5 MMA issuer.
+#include <math.h>
+
+#include "kvs_attn_tc.cuh"
+
+namespace kvs {
+namespace {
+
+using namespace tc;
+
+constexpr int BK = 128;  // keys per CTA
+constexpr int BQ = 64;   // queries per tile
+constexpr float L2E = 1.4426950408889634f;
+
+template <int D, int MODE>
+struct Bwd {
+  static constexpr int KD = D / 64;
+  static constexpr bool DK = (MODE == BWD_DK);
+  static constexpr int NS = 2;
+  static constexpr int K_BYTES = BK * D * 2;   // one copy of the key tile
+  static constexpr int Q_BYTES = BQ * D * 2;   // one copy of a query tile
+  static constexpr int STAGE = (DK ? 3 : 2) * Q_BYTES;  // Q hi, Q lo (, Go)
+  static constexpr int OFF_ST = 2 * K_BYTES;
+  static constexpr int BYTES = OFF_ST + NS * STAGE;
+  static constexpr int SMEM = BYTES + 1024;
+  static constexpr uint32_t TMEM_COLS = DK ? 512 : 128;
+  static constexpr uint32_t COL_DP = 128;
+  static constexpr uint32_t COL_DK = 256;
+  static constexpr uint32_t COL_V = 384;
+};
+
+struct BwdBars {
+  uint64_t k_full, v_full;
+  uint64_t q_full[2], q_empty[2];
+  uint64_t sd_full[2], sd_free[2];
+  uint64_t ds_full[2];
+  uint64_t done;
+  uint32_t tmem;
+  int abort;
+  float lse2[2][BQ];   // row lse in log2 units (+inf for rows outside the problem)
+  float del[2][BQ];
+};
+
+template <int D, int MODE>
+__global__ void __launch_bounds__(192, 1)
+    k_attn_bwd(const __grid_constant__ CUtensorMap mKh, const __grid_constant__ CUtensorMap mKl,
+               const __grid_constant__ CUtensorMap mQh, const __grid_constant__ CUtensorMap mQl,
+               const __grid_constant__ CUtensorMap mG, BwdArgs a) {
+  using C = Bwd<D, MODE>;
+  extern __shared__ unsigned char smraw[];
+  unsigned char *sm = (unsigned char *)(((uintptr_t)smraw + 1023) & ~(uintptr_t)1023);
+  __shared__ BwdBars bars;
+  const int b = blockIdx.y;
+  if (a.flt.skip(b)) return;
+  const int64_t k_begin = a.k_off[b];
+  const int nk = (int)(a.k_off[b + 1] - k_begin);
+  const int k0 = blockIdx.x * BK;
+  if (k0 >= nk) return;
+  const int64_t q_begin = a.q_off[b];
+  const int nq = (int)(a.q_off[b + 1] - q_begin);
+  const int nqt = (nq + BQ - 1) / BQ;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+
+  if (tid == 0) {
+    mbar_init(&bars.k_full, 1);
+    mbar_init(&bars.v_full, BK);
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&bars.q_full[i], 1);
+      mbar_init(&bars.q_empty[i], 1 + BK);
+      mbar_init(&bars.sd_full[i], 1);
+      mbar_init(&bars.sd_free[i], C::DK ? 1 : BK);
+      mbar_init(&bars.ds_full[i], BK);
+    }
+    mbar_init(&bars.done, 1);
+    bars.abort = 0;
+    fence_barrier_init();
+  }
+  if (warp == 5) tmem_alloc(&bars.tmem, C::TMEM_COLS);
+  fence_before_sync();
+  __syncthreads();
+  fence_after_sync();
+  const uint32_t tmem = bars.tmem;
+  volatile int *abort = &bars.abort;
+
+  if (warp == 4) {
+    // ------------------------------------------------------------ producer
+    if (lane == 0) {
+      const int krow = (int)(k_begin + k0);
+      mbar_arrive_expect_tx(&bars.k_full, 2 * C::K_BYTES);
+      for (int r = 0; r < C::KD; ++r) {
+        tma_load_2d(sm + r * BK * 128, &mKh, &bars.k_full, 64 * r, krow);
+        tma_load_2d(sm + C::K_BYTES + r * BK * 128, &mKl, &bars.k_full, 64 * r, krow);
+      }
+    }
+    int issued = 0;
+    for (int i = 0; i < nqt; ++i) {
+      const int st = i % C::NS;
+      if (i >= C::NS) {
+        const bool w = __all_sync(0xffffffffu,
+                                  mbar_wait(&bars.q_empty[st], ((i / C::NS) - 1) & 1, abort));
+        if (!w) {
+          *abort = 1;
+          break;
+        }
+      }
+      for (int e = lane; e < BQ; e += 32) {
+        const int q = i * BQ + e;
+        const bool v = q < nq;
+        bars.lse2[st][e] = v ? a.lse[q_begin + q] * L2E : INFINITY;
+        bars.del[st][e] = (v && C::DK) ? a.delta[q_begin + q] : 0.f;
+      }
+      __syncwarp();
+      if (lane == 0) {
+        issued = i + 1;
+        unsigned char *base = sm + C::OFF_ST + st * C::STAGE;
+        const int qrow = (int)(q_begin + i * BQ);
+        mbar_arrive_expect_tx(&bars.q_full[st], C::STAGE);
+        for (int r = 0; r < C::KD; ++r) {
+          tma_load_2d(base + r * BQ * 128, &mQh, &bars.q_full[st], 64 * r, qrow);
+          tma_load_2d(base + C::Q_BYTES + r * BQ * 128, &mQl, &bars.q_full[st], 64 * r, qrow);
+          if (C::DK)
+            tma_load_2d(base + 2 * C::Q_BYTES + r * BQ * 128, &mG, &bars.q_full[st], 64 * r, qrow);
+        }
+      }
+    }
+    if (lane == 0 && *abort) {  // let issued copies land before shared memory is released
+      mbar_wait(&bars.k_full, 0);
+      for (int i = (issued > C::NS ? issued - C::NS : 0); i < issued; ++i)
+        mbar_wait(&bars.q_full[i % C::NS], (i / C::NS) & 1);
+    }
+  } else if (warp == 5) {
+    // ------------------------------------------------------------- MMA issuer
+    if (lane == 0) {
+      const uint32_t id_s = idesc_bf16(BK, BQ, false, false);
+      const uint32_t id_dk = idesc_bf16(BK, D, false, true);
+      bool ok = mbar_wait(&bars.k_full, 0, abort);
+      if (C::DK) ok = ok && mbar_wait(&bars.v_full, 0, abort);
+      fence_after_sync();
+      const uint32_t aKh = smem_u32(sm), aKl = aKh + C::K_BYTES;
+      const uint32_t tv_hi = tmem + C::COL_V, tv_lo = tmem + C::COL_V + D / 2;
+      auto issue_dk = [&](int i) -> bool {
+        const int db = i & 1;
+        if (!mbar_wait(&bars.ds_full[db], (i >> 1) & 1, abort)) return false;
+        fence_after_sync();
+        const uint32_t qb = smem_u32(sm + C::OFF_ST + (i % C::NS) * C::STAGE);
+        const uint32_t tds = tmem + db * BQ;  // dS hi at +0, lo at +32 columns
+#pragma unroll
+        for (int kk = 0; kk < BQ / 16; ++kk) {
+          const uint64_t qh = sdesc(qb + kk * 2048, BQ * 128, 1024);
+          const uint64_t ql = sdesc(qb + C::Q_BYTES + kk * 2048, BQ * 128, 1024);
+          mma_bf16_ts(tmem + C::COL_DK, tds + kk * 8, qh, id_dk, (i > 0 || kk > 0) ? 1u : 0u);
+          mma_bf16_ts(tmem + C::COL_DK, tds + kk * 8, ql, id_dk, 1u);
+          mma_bf16_ts(tmem + C::COL_DK, tds + 32 + kk * 8, qh, id_dk, 1u);
+        }
+        mma_commit(&bars.q_empty[i % C::NS]);
+        mma_commit(&bars.sd_free[db]);
+        return true;
+      };
+      for (int i = 0; ok && i < nqt; ++i) {
+        const int st = i % C::NS, sb = i & 1;
+        if (!mbar_wait(&bars.q_full[st], (i / C::NS) & 1, abort)) { ok = false; break; }
+        if (i >= 2 && !mbar_wait(&bars.sd_free[sb], ((i >> 1) - 1) & 1, abort)) { ok = false; break; }
+        fence_after_sync();
+        const uint32_t qb = smem_u32(sm + C::OFF_ST + st * C::STAGE);
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint32_t ok_ = (kk >> 2) * (BK * 128) + (kk & 3) * 32;
+          const uint32_t oq = (kk >> 2) * (BQ * 128) + (kk & 3) * 32;
+          const uint64_t kh = sdesc(aKh + ok_, 16, 1024), kl = sdesc(aKl + ok_, 16, 1024);
+          const uint64_t qh = sdesc(qb + oq, 16, 1024), ql = sdesc(qb + C::Q_BYTES + oq, 16, 1024);
+          mma_bf16(tmem + sb * BQ, kh, qh, id_s, kk > 0 ? 1u : 0u);
+          mma_bf16(tmem + sb * BQ, kl, qh, id_s, 1u);
+          mma_bf16(tmem + sb * BQ, kh, ql, id_s, 1u);
+          if (C::DK) {
+            const uint64_t gd = sdesc(qb + 2 * C::Q_BYTES + oq, 16, 1024);
+            mma_bf16_ts(tmem + C::COL_DP + sb * BQ, tv_hi + kk * 8, gd, id_s, kk > 0 ? 1u : 0u);
+            mma_bf16_ts(tmem + C::COL_DP + sb * BQ, tv_lo + kk * 8, gd, id_s, 1u);
+          }
+        }
+        mma_commit(&bars.sd_full[sb]);
+        if (!C::DK) mma_commit(&bars.q_empty[st]);
+        if (C::DK && i >= 1 && !issue_dk(i - 1)) { ok = false; break; }
+      }
+      if (ok && C::DK && nqt > 0) ok = issue_dk(nqt - 1);
+      mma_commit(&bars.done);
+      if (!ok) *abort = 1;
+      mbar_wait(&bars.done, 0);  // every MMA of this CTA has completed
+    }
+  } else {
+    // --------------------------------------------------------- key rows
+    const int row = tid;
+    const int kr = k0 + row;
+    const bool kvalid = kr < nk;
+    const uint32_t lane_base = (uint32_t)(warp * 32) << 16;
+    if (C::DK) {
+      // the value row (hi, lo) into tensor memory as the A operand of dP^T = V Go^T
+      const uint4 *vh = reinterpret_cast<const uint4 *>(a.v_hi + (k_begin + kr) * D);
+      const uint4 *vl = reinterpret_cast<const uint4 *>(a.v_lo + (k_begin + kr) * D);
+#pragma unroll 1
+      for (int c0 = 0; c0 < D / 2; c0 += 32) {
+        uint32_t wh[32], wl[32];
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+          const uint4 h = kvalid ? vh[c0 / 4 + e] : make_uint4(0, 0, 0, 0);
+          const uint4 l = kvalid ? vl[c0 / 4 + e] : make_uint4(0, 0, 0, 0);
+          wh[4 * e] = h.x; wh[4 * e + 1] = h.y; wh[4 * e + 2] = h.z; wh[4 * e + 3] = h.w;
+          wl[4 * e] = l.x; wl[4 * e + 1] = l.y; wl[4 * e + 2] = l.z; wl[4 * e + 3] = l.w;
+        }
+        tmem_st32u(tmem + lane_base + C::COL_V + c0, wh);
+        tmem_st32u(tmem + lane_base + C::COL_V + D / 2 + c0, wl);
+      }
+      tmem_wait_st();
+      fence_before_sync();
+      mbar_arrive(&bars.v_full);
+    }
+    const float sl2 = a.scale * L2E;
+    float imp = 0.f;
+    bool ok = true;
+    for (int i = 0; i < nqt; ++i) {
+      const int sb = i & 1, st = i % C::NS;
+      ok = __all_sync(0xffffffffu, mbar_wait(&bars.sd_full[sb], (i >> 1) & 1, abort));
+      // the tile's l and delta were staged by the producer lanes: acquire them directly
+      ok = ok && __all_sync(0xffffffffu, mbar_wait(&bars.q_full[st], (i / C::NS) & 1, abort));
+      if (!ok) break;
+      fence_after_sync();
+      float s[BQ];
+      tmem_ld32(tmem + lane_base + sb * BQ, s);
+      tmem_ld32(tmem + lane_base + sb * BQ + 32, s + 32);
+      const int qvalid = nq - i * BQ;
+      if (!C::DK) {
+        fence_before_sync();
+        mbar_arrive(&bars.sd_free[sb]);
+#pragma unroll
+        for (int c = 0; c < BQ; ++c)
+          imp += (c < qvalid) ? exp2f(fmaf(s[c], sl2, -bars.lse2[st][c])) : 0.f;
+      } else {
+        float dp[BQ];
+        tmem_ld32(tmem + lane_base + C::COL_DP + sb * BQ, dp);
+        tmem_ld32(tmem + lane_base + C::COL_DP + sb * BQ + 32, dp + 32);
+        uint32_t hh[32], ll[32];
+#pragma unroll
+        for (int c2 = 0; c2 < 32; ++c2) {
+          float v[2];
+#pragma unroll
+          for (int u = 0; u < 2; ++u) {
+            const int c = 2 * c2 + u;
+            const float p = exp2f(fmaf(s[c], sl2, -bars.lse2[st][c]));
+            v[u] = (kvalid && c < qvalid) ? p * (dp[c] - bars.del[st][c]) : 0.f;
+          }
+          split_pack(v[0], v[1], hh[c2], ll[c2]);
+        }
+        // dS (hi, lo) over the S buffer: the A operand of dK += dS Q
+        tmem_st32u(tmem + lane_base + sb * BQ, hh);
+        tmem_st32u(tmem + lane_base + sb * BQ + 32, ll);
+        tmem_wait_st();
+        fence_before_sync();
+        mbar_arrive(&bars.ds_full[sb]);
+      }
+      mbar_arrive(&bars.q_empty[st]);
+    }
+    if (!ok) *abort = 1;
+    if (C::DK) {
+      if (!mbar_wait(&bars.done, 0, abort)) *abort = 1;
+      fence_after_sync();
+#pragma unroll 1
+      for (int c0 = 0; c0 < D; c0 += 32) {
+        float o[32];
+        tmem_ld32(tmem + lane_base + C::COL_DK + c0, o);
+        if (kvalid) {
+          float4 *dst = reinterpret_cast<float4 *>(a.dk + (k_begin + kr) * D + c0);
+#pragma unroll
+          for (int e = 0; e < 8; ++e)
+            dst[e] = make_float4(o[4 * e] * a.scale, o[4 * e + 1] * a.scale,
+                                 o[4 * e + 2] * a.scale, o[4 * e + 3] * a.scale);
+        }
+      }
+    } else if (kvalid) {
+      a.imp[k_begin + kr] = imp;
+    }
+  }
+  fence_before_sync();
+  __syncthreads();
+  if (warp == 5) {
+    fence_after_sync();
+    tmem_dealloc(tmem, C::TMEM_COLS);
+  }
+  if (tid == 0 && bars.abort && a.err) atomicOr(a.err, 1);
+}
+
+}  // namespace
+
+template <int D, int MODE>
+int launch_bwd_tc(const BwdMaps &m, const BwdArgs &a, int max_tiles, int B, cudaStream_t st) {
+  using C = Bwd<D, MODE>;
+  static_assert(C::SMEM + sizeof(BwdBars) <= 232448, "shared memory");
+  auto kern = k_attn_bwd<D, MODE>;
+  KVS_CUDA_TRY(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM));
+  kern<<<dim3(max_tiles, B), 192, C::SMEM, st>>>(m.kh, m.kl, m.qh, m.ql, m.g, a);
+  KVS_LAUNCH_CHECK("k_attn_bwd");
+  return KVS_OK;
+}
+
+template int launch_bwd_tc<64, BWD_DK>(const BwdMaps &, const BwdArgs &, int, int, cudaStream_t);
+template int launch_bwd_tc<128, BWD_DK>(const BwdMaps &, const BwdArgs &, int, int, cudaStream_t);
+template int launch_bwd_tc<64, BWD_COLSUM>(const BwdMaps &, const BwdArgs &, int, int, cudaStream_t);
+template int launch_bwd_tc<128, BWD_COLSUM>(const BwdMaps &, const BwdArgs &, int, int, cudaStream_t);
+
+}  // namespace kvs

@@ -1,0 +1,91 @@
+// Arguments and launchers of the tcgen05 attention kernels.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_bf16.h>
+
+#include "kvs_internal.cuh"
+#include "kvs_tc.cuh"
+
+namespace kvs {
+
+enum FwdMode : int { FWD_LOSS = 0, FWD_TARGETS = 1, FWD_STATS = 2, FWD_WRITE_A = 3 };
+enum BwdMode : int { BWD_DK = 0, BWD_COLSUM = 1 };
+
+// Tensor maps of the bf16 operands (2-D, [rows, d], box 64 columns x 64 rows).
+struct FwdMaps {
+  CUtensorMap kh, kl, vh, vl;
+};
+
+struct FwdArgs {
+  const int64_t *q_off;   // [B+1] query rows
+  const int64_t *k_off;   // [B+1] key rows (compress zone or compressed pairs)
+  Filter flt;
+  float scale;            // 1/sqrt(d)
+  const __nv_bfloat16 *q_hi, *q_lo;  // [sum_q, d] query split (loaded into tensor memory)
+  // LOSS
+  const float *y_in;      // [sum_q, d] targets
+  const float *lse_in;    // [sum_q] target lse (LOSS) or given row lse (WRITE_A)
+  float *lse_out;         // [sum_q] row lse of these keys
+  __nv_bfloat16 *go;      // [sum_q, d] dL/dY_hat, bf16
+  float *delta;           // [sum_q]
+  float *partials;        // [B, tiles_per_problem, 2]
+  int tiles_per_problem;
+  float w_out, w_lse;     // loss weights (means over n_q d and n_q)
+  // TARGETS
+  float *y_out;           // [sum_q, d]
+  __nv_bfloat16 *y_hi, *y_lo;
+  // WRITE_A
+  __nv_bfloat16 *a_hi, *a_lo;  // [sum padded q, ld_a]
+  int64_t ld_a;
+  const int64_t *a_pad_off;    // [B+1] padded query-row offsets of the A buffer
+  int *err;               // timeout flag
+};
+
+struct BwdMaps {
+  CUtensorMap kh, kl;     // key tile, box 64 columns x 128 rows
+  CUtensorMap qh, ql, g;  // query / Go tiles, box 64 columns x 64 rows
+};
+
+struct BwdArgs {
+  const int64_t *q_off;
+  const int64_t *k_off;
+  Filter flt;
+  float scale;
+  const float *lse;       // [sum_q] row lse used to form the probabilities
+  const float *delta;     // [sum_q] (DK)
+  const __nv_bfloat16 *v_hi, *v_lo;  // [sum_k, d] value split (DK; loaded into tensor memory)
+  float *dk;              // [sum_k, d] (DK): dL/dK
+  float *imp;             // [sum_k] (COLSUM): column sums of probabilities
+  int *err;
+};
+
+struct GemmMaps {
+  CUtensorMap ah, al, bh, bl;
+};
+
+struct GemmArgs3 {
+  const int64_t *a_pad_off;  // [B+1] padded K (query) row offsets of both operands' buffers
+  const int64_t *m_off;      // [B+1] M extents (keys)
+  int n_fixed;               // N extent when > 0 (e.g. d), else N = M extent (Gram)
+  const int64_t *b_row_off;  // [B+1] K-row offsets of the B operand (Gram: = a_pad_off)
+  float *c;                  // output rows at m_off[b], ld = ldc
+  int64_t ldc;
+  float diag;                // added on the diagonal (Gram: lambda)
+  int b_col_shift;           // Gram: 0 ; R: 0 (B columns start at 0)
+  int *err;
+};
+
+template <int D, int MODE>
+int launch_fwd_tc(const FwdMaps &m, const FwdArgs &a, int max_tiles, int B, cudaStream_t st);
+template <int D, int MODE>
+int launch_bwd_tc(const BwdMaps &m, const BwdArgs &a, int max_tiles, int B, cudaStream_t st);
+int launch_gemm3_tc(const GemmMaps &m, const GemmArgs3 &a, int tiles_m, int gram, int B,
+                    cudaStream_t st);
+
+// Host: a 2-D bf16 tensor map over [rows, cols] (row-major) with a
+// [box_rows, 64]-element box and 128-byte swizzle.
+int make_map_bf16(CUtensorMap *m, const void *base, uint64_t rows, uint64_t cols,
+                  uint32_t box_rows);
+
+}  // namespace kvs

@@ -68,7 +68,8 @@ struct HostGeom {
   int B = 0, d = 0;
   int64_t sum_q = 0, sum_z = 0, sum_c = 0;
   int max_q = 0, max_z = 0, max_c = 0;
-  int64_t ld_s = 0;      // leading dimension of the score buffer (>= max(max_z, max_c), mult of 4)
+  int64_t sum_qpad = 0;  // sum over problems of n_q rounded up to 128
+  int64_t ld_a = 0;      // columns of the attention-weight buffer (max_c rounded up to 128)
 };
 
 int geom_from_batch(const kvs_batch *b, HostGeom *g, bool need_c);

@@ -1,6 +1,8 @@
 // Internal launchers shared by the C-ABI layer (not part of the public ABI).
 #pragma once
 
+#include <cuda_bf16.h>
+
 #include "kvs_common.cuh"
 
 namespace kvs {
@@ -25,22 +27,26 @@ struct LbfgsScal {
 
 // Scratch buffers carved from the caller's workspace.
 struct Work {
-  float *S;        // [sum_q, ld_s]  scores / probabilities / dS
-  float *Yh;       // [sum_q, d]     compressed attention output
-  float *Go;       // [sum_q, d]     dloss/dYh
-  float *lse_h;    // [sum_q]
-  float *delta;    // [sum_q]
-  float *row_out;  // [sum_q]        per-row squared output error
-  float *row_ls;   // [sum_q]        per-row squared LSE error
-  float *gram;     // [sum_c, max_c] A^T A + lam I (float)
-  double *chol;    // [sum_c, max_c] Cholesky factor (double)
-  double *xs;      // [sum_c, d]     right-hand sides / solution (double)
-  float *R;        // [sum_c, d]     A^T Y
-  float *fbuf;     // [B]            loss scratch
-  float *Yt;       // [sum_q, d]     targets (kvs_compress_batch)
-  float *lset;     // [sum_q]        target log-sum-exp (kvs_compress_batch)
-  float *imp;      // [sum_z]        importance (kvs_compress_batch)
-  int32_t *idx;    // [sum_c]        top-k positions (kvs_compress_batch)
+  __nv_bfloat16 *qh, *ql;    // [sum_q, d]             training queries, hi/lo
+  __nv_bfloat16 *kh, *kl;    // [max(sum_z, sum_c), d] keys, hi/lo
+  __nv_bfloat16 *vh, *vl;    // [max(sum_z, sum_c), d] values, hi (and lo for targets)
+  __nv_bfloat16 *go;         // [sum_q, d]             dloss/dY_hat
+  __nv_bfloat16 *yh, *yl;    // [sum_q, d]             targets Y, hi/lo
+  __nv_bfloat16 *ahi, *alo;  // [sum_qpad, ld_a]       attention weights for the ridge fit
+  float *lse_h;              // [sum_q]                row lse of the compressed keys
+  float *delta;              // [sum_q]
+  float *partials;           // [B, max q tiles, 2]    per-CTA loss sums
+  int64_t *a_pad_off;        // [B+1]                  padded row offsets of ahi/alo
+  float *gram;               // [sum_c, max_c]         A^T A + lam I (float)
+  double *chol;              // [sum_c, max_c]         Cholesky factor (double)
+  double *xs;                // [sum_c, d]             right-hand sides / solution (double)
+  float *R;                  // [sum_c, d]             A^T Y
+  float *fbuf;               // [B]                    loss scratch
+  float *Yt;                 // [sum_q, d]             targets (kvs_compress_batch)
+  float *lset;               // [sum_q]                target log-sum-exp (kvs_compress_batch)
+  float *imp;                // [sum_z]                importance (kvs_compress_batch)
+  int32_t *idx;              // [sum_c]                top-k positions (kvs_compress_batch)
+  int *err;                  // [1]                    set when a kernel wait timed out
   size_t bytes;
 };
 
@@ -67,20 +73,22 @@ struct Batch {
 };
 
 // ---- attention contractions (kvs_attn.cu) ----
-// targets: Y, lse and (optionally) importance.
+// targets: Y, lse and (optionally) importance; leaves the Q split in w.qh/ql
+// and the Y split in w.yh/yl.
 int launch_targets(const Batch &B, const float *Q, const float *Kz, const float *Vz, float *Y,
                    float *lse, float *imp, const Work &w);
-// Forward over the compressed pairs for the problems selected by `flt`. Leaves A in w.S, lse_h, Yh, Go, delta and
-// writes loss[b] (and parts[2b..2b+1] if non-null).
+// Loss forward over the compressed pairs for the problems selected by `flt`:
+// writes loss[b] (and parts[2b..2b+1] if non-null) and leaves lse_h, go and
+// delta (plus the bf16 copies of Kc, Vc) for launch_backward.  q_ready: the
+// Q split in w.qh/ql is current.
 int launch_forward(const Batch &B, const float *Q, const float *Kc, const float *Vc,
                    const float *Y, const float *lse, float w_out, float w_lse, float *loss,
-                   float *parts, Filter flt, const Work &w);
-// Backward: dKc from the state left by launch_forward for the same problems.
-int launch_backward(const Batch &B, const float *Q, const float *Vc, float *dKc,
-                    Filter flt, const Work &w);
-// Ridge fit: Vc = (A^T A + lam I)^-1 A^T Y.
+                   float *parts, Filter flt, bool q_ready, const Work &w);
+// dKc from the state left by launch_forward for the same problems.
+int launch_backward(const Batch &B, float *dKc, Filter flt, const Work &w);
+// Ridge fit: Vc = (A^T A + lam I)^-1 A^T Y (y_ready: the Y split is current).
 int launch_fit(const Batch &B, const float *Q, const float *Kc, const float *Y, float lam,
-               float *Vc, int32_t *status, const Work &w);
+               float *Vc, int32_t *status, bool q_ready, bool y_ready, const Work &w);
 
 // ---- other kernels ----
 int launch_build_queries(const kvs_query_spec *sp, const float *q_retain, const float *q_ctx,

@@ -116,6 +116,23 @@ def test_topk_bit_exact(case):
 
 # ----------------------------------------------------------- loss and grad
 
+def grad_close(g_gpu, g_or, Q, lse):
+    """Gradient parity: cosine >= 0.999, i.e. |dg| <= 0.0447 |g|, with a floor.
+
+    The scores carry about 16 significant bits, so the GPU's l_hat may differ
+    from the float64 one by ~2^-16 max|l| per row; through dL/dl_hat =
+    2/n_q (l_hat - l) that moves the gradient by about
+    tau = s (2/n_q) 2^-16 max|l| sqrt(sum_i |q_i|^2) (root-mean-square
+    estimate).  Where the true gradient is that small (e.g. k = z with K_c = K_z)
+    the comparison is against tau instead."""
+    g_gpu = np.asarray(g_gpu, np.float64)
+    g_or = np.asarray(g_or, np.float64)
+    n_q, d = Q.shape
+    tau = (1 / np.sqrt(d)) * (2.0 / n_q) * 2.0 ** -16 * np.abs(lse).max() * np.sqrt(
+        (np.asarray(Q, np.float64) ** 2).sum())
+    return np.linalg.norm(g_gpu - g_or) <= max(0.0447 * np.linalg.norm(g_or), tau)
+
+
 def select_fit_point(c, perturb=0.0, seed=0):
     """K_c = top-k keys of the oracle's importance, V_c = oracle ridge fit (float32)."""
     r = np.random.default_rng(seed)
@@ -153,9 +170,14 @@ def test_loss_grad(case, perturb):
     for b in range(B):
         f, g, info = O.loss_grad(c.Qs[b], Kcs[b], Vcs[b], tgt[b][0], tgt[b][1])
         assert abs(gl[b] - f) <= 1e-3 * f, (b, gl[b], f)
-        assert abs(gp[b, 0] - info["out"]) <= 1e-3 * info["out"] + 1e-9
-        assert abs(gp[b, 1] - info["lse"]) <= 1e-3 * info["lse"] + 1e-9
-        assert cosine(gd[co[b]:co[b + 1]], g) >= 0.999, b
+        # Each term alone may be near zero (k = z): the products that set it keep
+        # 16 significant bits (three-term bf16 split), so allow an absolute floor of
+        # (2^-16 max|l|)^2 for the LSE term and (2^-16 rms|Y|)^2 for the output term.
+        floor_lse = (2.0 ** -16 * np.abs(tgt[b][1]).max()) ** 2
+        floor_out = (2.0 ** -16) ** 2 * float((tgt[b][0].astype(np.float64) ** 2).mean())
+        assert abs(gp[b, 0] - info["out"]) <= 1e-3 * info["out"] + floor_out
+        assert abs(gp[b, 1] - info["lse"]) <= 1e-3 * info["lse"] + floor_lse
+        assert grad_close(gd[co[b]:co[b + 1]], g, c.Qs[b], tgt[b][1]), b
 
 
 def test_loss_only_matches_loss_grad(case):
