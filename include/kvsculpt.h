@@ -158,8 +158,7 @@ int kvs_loss_grad(const kvs_batch *batch, const float *Q, const float *Kc, const
  * (KVS_STATIC_WS_BYTES in kvs_static.cu) of device memory on every GPU that
  * loads the library, held until the process exits.  It allocates nothing.
  * - Batches whose kvs_workspace_bytes() exceeds 32 MiB return KVS_EWORKSPACE
- *   (e.g. one head-problem with n_q = 3840 and k = 960 does not fit; the d=64,
- *   N=256 problem does).
+ *   (one head-problem with d = 128, n_q = 3840 and k = 960 fits; two do not).
  * - The first call on a device looks up the array's device address with that
  *   device current (cudaGetSymbolAddress) and caches it; make that first call
  *   before any stream capture.

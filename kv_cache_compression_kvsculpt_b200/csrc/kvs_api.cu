@@ -89,9 +89,9 @@ size_t carve_work(const HostGeom &g, void *base, Work *w) {
   w->partials = c.take<float>((int64_t)g.B * ((g.max_q + 127) / 128) * 2);
   w->a_pad_off = c.take<int64_t>(g.B + 1);
   w->gram = c.take<float>(g.sum_c * g.max_c);
-  w->chol = c.take<double>(g.sum_c * g.max_c);
-  w->xs = c.take<double>(g.sum_c * g.d);
   w->R = c.take<float>(g.sum_c * g.d);
+  w->chol_t = c.take<float>((int64_t)g.B * 64 * 64);
+  w->dead = c.take<int>(g.B);
   w->fbuf = c.take<float>(g.B);
   w->Yt = c.take<float>(g.sum_q * g.d);
   w->lset = c.take<float>(g.sum_q);

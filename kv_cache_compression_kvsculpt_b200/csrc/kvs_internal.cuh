@@ -37,10 +37,10 @@ struct Work {
   float *delta;              // [sum_q]
   float *partials;           // [B, max q tiles, 2]    per-CTA loss sums
   int64_t *a_pad_off;        // [B+1]                  padded row offsets of ahi/alo
-  float *gram;               // [sum_c, max_c]         A^T A + lam I (float)
-  double *chol;              // [sum_c, max_c]         Cholesky factor (double)
-  double *xs;                // [sum_c, d]             right-hand sides / solution (double)
-  float *R;                  // [sum_c, d]             A^T Y
+  float *gram;               // [sum_c, max_c]         A^T A + lam I, then its Cholesky factor
+  float *R;                  // [sum_c, d]             A^T Y, then the solution
+  float *chol_t;             // [B, 64, 64]            inverse of the current diagonal block
+  int *dead;                 // [B]                    factorisation failed
   float *fbuf;               // [B]                    loss scratch
   float *Yt;                 // [sum_q, d]             targets (kvs_compress_batch)
   float *lset;               // [sum_q]                target log-sum-exp (kvs_compress_batch)

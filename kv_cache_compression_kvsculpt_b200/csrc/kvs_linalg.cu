@@ -3,10 +3,18 @@
 // Distillation", section 2 "Value Optimization": values in closed form by
 // ridge regression).
 //
-// One CTA per problem; factor and solves run in float64 on the CUDA cores
-// (the Gram matrix of softmax weights reaches condition numbers of ~3e4 on
-// the synthetic Qwen-shaped workloads).  A pivot <= 0 (or non-finite) marks
-// the problem KVS_ST_NOT_PD and leaves its V_c untouched.
+// Right-looking blocked algorithm over panels of NB = 64 columns, float32,
+// every problem of the batch advancing together so that all SMs share the work:
+//   per panel j (one launch each):
+//     diag    factor the diagonal block G_jj = L_jj L_jj^T in shared memory,
+//             form T_j = L_jj^-1 and the forward-solved rows y_j = T_j r_j
+//     panel   L_ij = G_ij T_j^T for the rows below
+//     update  G_ik -= L_ij L_kj^T on the trailing lower triangle and
+//             r_i -= L_ij y_j on the right-hand sides (64 x 64 register tiles)
+//   then per panel from the last one: x_j = T_j^T y_j and y_i -= L_ji^T x_j.
+// The factor overwrites the Gram matrix, the solution the right-hand sides.
+// A pivot <= 0 (or non-finite) marks the problem KVS_ST_NOT_PD; its V_c is
+// left untouched and its remaining steps are skipped.
 #include <math.h>
 
 #include "kvs_internal.cuh"
@@ -14,175 +22,328 @@
 namespace kvs {
 namespace {
 
-constexpr int NB = 32;
+constexpr int NB = 64;
 
-__global__ void __launch_bounds__(1024) k_chol_solve(const float *__restrict__ gram,
-                                                     double *__restrict__ L,
-                                                     const float *__restrict__ R,
-                                                     double *__restrict__ X, float *Vc,
-                                                     int32_t *status, const int64_t *c_off,
-                                                     int64_t ld, int d) {
+struct CholArgs {
+  float *G;              // [sum_c, ld] Gram matrix -> factor (lower triangle)
+  float *R;              // [sum_c, d] right-hand sides -> solution
+  float *T;              // [B, NB, NB] inverse of the current diagonal block
+  int *dead;             // [B] set once a problem's factorisation failed
+  int32_t *status;
+  const int64_t *c_off;
+  int64_t ld;
+  int d;
+};
+
+__device__ __forceinline__ int kdim(const CholArgs &a, int b) {
+  return (int)(a.c_off[b + 1] - a.c_off[b]);
+}
+
+// Diagonal block of panel j0: factor, invert, and solve y = T r for its rows.
+__global__ void __launch_bounds__(256) k_chol_diag(CholArgs a, int j0) {
   const int b = blockIdx.x;
-  const int64_t r0 = c_off[b];
-  const int k = (int)(c_off[b + 1] - r0);
-  if (k <= 0) return;
-  const int tid = threadIdx.x, nt = blockDim.x;
-  const float *G = gram + r0 * ld;
-  double *Lb = L + r0 * ld;
-  __shared__ double D[NB][NB + 1];
-  __shared__ double Pi[NB][NB + 1];
-  __shared__ double Pj[NB][NB + 1];
+  const int k = kdim(a, b);
+  if (j0 >= k || a.dead[b]) return;
+  const int jb = min(NB, k - j0);
+  __shared__ float L[NB][NB + 1];
+  __shared__ float Ti[NB][NB + 1];
   __shared__ int bad;
+  float *G = a.G + (a.c_off[b] + j0) * a.ld + j0;
+  const int tid = threadIdx.x;
   if (tid == 0) bad = 0;
-  for (int64_t e = tid; e < (int64_t)k * k; e += nt) {
-    const int i = (int)(e / k), j = (int)(e % k);
-    if (j <= i) Lb[(int64_t)i * ld + j] = (double)G[(int64_t)i * ld + j];
+  for (int e = tid; e < NB * NB; e += blockDim.x) {
+    const int r = e / NB, c = e % NB;
+    L[r][c] = (r < jb && c <= r) ? G[(int64_t)r * a.ld + c] : 0.f;
+    Ti[r][c] = 0.f;
   }
   __syncthreads();
-  for (int j0 = 0; j0 < k; j0 += NB) {
-    const int jb = min(NB, k - j0);
-    // (1) diagonal block, unblocked, in shared memory by warp 0
-    for (int e = tid; e < NB * NB; e += nt) {
-      const int r = e / NB, c = e % NB;
-      D[r][c] = (r < jb && c <= r) ? Lb[(int64_t)(j0 + r) * ld + j0 + c] : 0.0;
+  for (int c = 0; c < jb; ++c) {
+    if (tid == 0) {
+      const float piv = L[c][c];
+      if (!(piv > 0.f) || !isfinite(piv)) bad = 1;
+      L[c][c] = sqrtf(fmaxf(piv, 1e-30f));
     }
     __syncthreads();
-    if (tid < 32) {
-      const int r = tid;
-      for (int c = 0; c < jb; ++c) {
-        if (r == c) {
-          const double piv = D[c][c];
-          if (!(piv > 0.0) || !isfinite(piv)) bad = 1;
-          D[c][c] = sqrt(fmax(piv, 1e-300));
-        }
-        __syncwarp();
-        if (r > c && r < jb) D[r][c] /= D[c][c];
-        __syncwarp();
-        if (r > c && r < jb)
-          for (int cc = c + 1; cc <= r; ++cc) D[r][cc] -= D[r][c] * D[cc][c];
-        __syncwarp();
-      }
-    }
+    const float inv = 1.f / L[c][c];
+    for (int i = c + 1 + tid; i < jb; i += blockDim.x) L[i][c] *= inv;
     __syncthreads();
-    if (bad) {
-      if (tid == 0) status[b] |= KVS_ST_NOT_PD;
-      return;
-    }
-    for (int e = tid; e < NB * NB; e += nt) {
-      const int r = e / NB, c = e % NB;
-      if (r < jb && c <= r) Lb[(int64_t)(j0 + r) * ld + j0 + c] = D[r][c];
-    }
-    // (2) panel below the diagonal block: L21 = A21 L11^-T, one row per thread
-    for (int i = j0 + jb + tid; i < k; i += nt) {
-      double *row = Lb + (int64_t)i * ld + j0;
-      double x[NB];
-#pragma unroll
-      for (int c = 0; c < NB; ++c) {
-        if (c < jb) {
-          double a = row[c];
-          for (int t = 0; t < c; ++t) a -= x[t] * D[c][t];
-          x[c] = a / D[c][c];
-          row[c] = x[c];
-        }
-      }
-    }
-    __syncthreads();
-    // (3) trailing update of the lower triangle: A22 -= L21 L21^T
-    const int s0 = j0 + jb;
-    const int n2 = k - s0;
-    const int nt2 = (n2 + NB - 1) / NB;
-    for (int ti = 0; ti < nt2; ++ti) {
-      for (int e = tid; e < NB * NB; e += nt) {
-        const int r = e / NB, c = e % NB;
-        const int i = s0 + ti * NB + r;
-        Pi[r][c] = (i < k && c < jb) ? Lb[(int64_t)i * ld + j0 + c] : 0.0;
-      }
-      for (int tj = 0; tj <= ti; ++tj) {
-        for (int e = tid; e < NB * NB; e += nt) {
-          const int r = e / NB, c = e % NB;
-          const int j = s0 + tj * NB + r;
-          Pj[r][c] = (j < k && c < jb) ? Lb[(int64_t)j * ld + j0 + c] : 0.0;
-        }
-        __syncthreads();
-        {
-          const int r = tid / NB, c = tid % NB;
-          const int i = s0 + ti * NB + r, j = s0 + tj * NB + c;
-          if (tid < NB * NB && i < k && j <= i) {
-            double acc = 0.0;
-#pragma unroll 8
-            for (int t = 0; t < NB; ++t) acc += Pi[r][t] * Pj[c][t];
-            Lb[(int64_t)i * ld + j] -= acc;
-          }
-        }
-        __syncthreads();
-      }
+    const int n = jb - c - 1;
+    for (int e = tid; e < n * n; e += blockDim.x) {
+      const int i = c + 1 + e / n, j = c + 1 + e % n;
+      if (j <= i) L[i][j] -= L[i][c] * L[j][c];
     }
     __syncthreads();
   }
-  // Solves: forward L y = R, backward L^T x = y; X holds the d right-hand sides.
-  double *Xb = X + r0 * d;
-  const float *Rb = R + r0 * d;
-  for (int64_t e = tid; e < (int64_t)k * d; e += nt) Xb[e] = (double)Rb[e];
-  __syncthreads();
-  for (int i0 = 0; i0 < k; i0 += NB) {
-    const int ib = min(NB, k - i0);
-    for (int e = tid; e < ib * d; e += nt) {
-      const int r = e / d, c = e % d;
-      const double *lr = Lb + (int64_t)(i0 + r) * ld;
-      double acc = 0.0;
-      for (int t = 0; t < i0; ++t) acc += lr[t] * Xb[(int64_t)t * d + c];
-      Xb[(int64_t)(i0 + r) * d + c] -= acc;
+  if (bad) {
+    if (tid == 0) {
+      a.status[b] |= KVS_ST_NOT_PD;
+      a.dead[b] = 1;
     }
-    __syncthreads();
-    for (int c = tid; c < d; c += nt) {
-      for (int r = 0; r < ib; ++r) {
-        const double *lr = Lb + (int64_t)(i0 + r) * ld + i0;
-        double a = Xb[(int64_t)(i0 + r) * d + c];
-        for (int t = 0; t < r; ++t) a -= lr[t] * Xb[(int64_t)(i0 + t) * d + c];
-        Xb[(int64_t)(i0 + r) * d + c] = a / lr[r];
-      }
-    }
-    __syncthreads();
-  }
-  const int nblk = (k + NB - 1) / NB;
-  for (int bi = nblk - 1; bi >= 0; --bi) {
-    const int i0 = bi * NB;
-    const int ib = min(NB, k - i0);
-    for (int e = tid; e < ib * d; e += nt) {
-      const int r = e / d, c = e % d;
-      const int i = i0 + r;
-      double acc = 0.0;
-      for (int t = i0 + ib; t < k; ++t) acc += Lb[(int64_t)t * ld + i] * Xb[(int64_t)t * d + c];
-      Xb[(int64_t)i * d + c] -= acc;
-    }
-    __syncthreads();
-    for (int c = tid; c < d; c += nt) {
-      for (int r = ib - 1; r >= 0; --r) {
-        const int i = i0 + r;
-        double a = Xb[(int64_t)i * d + c];
-        for (int t = r + 1; t < ib; ++t) a -= Lb[(int64_t)(i0 + t) * ld + i] * Xb[(int64_t)(i0 + t) * d + c];
-        Xb[(int64_t)i * d + c] = a / Lb[(int64_t)i * ld + i];
-      }
-    }
-    __syncthreads();
-  }
-  bool finite = true;
-  for (int64_t e = tid; e < (int64_t)k * d; e += nt) finite &= isfinite(Xb[e]);
-  finite = __syncthreads_and(finite);
-  if (!finite) {
-    if (tid == 0) status[b] |= KVS_ST_NONFINITE;
     return;
   }
-  float *V = Vc + r0 * d;
-  for (int64_t e = tid; e < (int64_t)k * d; e += nt) V[e] = (float)Xb[e];
+  // T = L^-1 (lower triangular), one column per thread
+  if (tid < jb) {
+    const int c = tid;
+    Ti[c][c] = 1.f / L[c][c];
+    for (int i = c + 1; i < jb; ++i) {
+      float s = 0.f;
+      for (int t = c; t < i; ++t) s = fmaf(L[i][t], Ti[t][c], s);
+      Ti[i][c] = -s / L[i][i];
+    }
+  }
+  __syncthreads();
+  for (int e = tid; e < NB * NB; e += blockDim.x) {
+    const int r = e / NB, c = e % NB;
+    if (r < jb && c <= r) G[(int64_t)r * a.ld + c] = L[r][c];
+    a.T[(int64_t)b * NB * NB + e] = Ti[r][c];
+  }
+  // forward solve of this block's right-hand sides: y = T r (columns of R independent)
+  float *R = a.R + (a.c_off[b] + j0) * a.d;
+  for (int c = tid; c < a.d; c += blockDim.x) {
+    float y[NB];
+#pragma unroll 8
+    for (int r = 0; r < NB; ++r) y[r] = (r < jb) ? R[(int64_t)r * a.d + c] : 0.f;
+    for (int r = jb - 1; r >= 0; --r) {
+      float s = 0.f;
+      for (int t = 0; t <= r; ++t) s = fmaf(Ti[r][t], y[t], s);
+      R[(int64_t)r * a.d + c] = s;
+    }
+  }
+}
+
+// L_ij = G_ij T^T for 64 rows of the panel below the diagonal block.
+__global__ void __launch_bounds__(256) k_chol_panel(CholArgs a, int j0) {
+  const int b = blockIdx.y;
+  const int k = kdim(a, b);
+  if (j0 >= k || a.dead[b]) return;
+  const int jb = min(NB, k - j0);
+  const int i0 = j0 + jb + blockIdx.x * NB;
+  if (i0 >= k) return;
+  const int ib = min(NB, k - i0);
+  __shared__ float Ti[NB][NB + 1];
+  __shared__ float Ar[NB][NB + 1];
+  const int tid = threadIdx.x;
+  float *P = a.G + (a.c_off[b] + i0) * a.ld + j0;
+  for (int e = tid; e < NB * NB; e += blockDim.x) {
+    const int r = e / NB, c = e % NB;
+    Ti[r][c] = a.T[(int64_t)b * NB * NB + e];
+    Ar[r][c] = (r < ib && c < jb) ? P[(int64_t)r * a.ld + c] : 0.f;
+  }
+  __syncthreads();
+  for (int e = tid; e < ib * jb; e += blockDim.x) {
+    const int r = e / jb, c = e % jb;
+    float s = 0.f;
+    for (int t = 0; t <= c; ++t) s = fmaf(Ar[r][t], Ti[c][t], s);
+    P[(int64_t)r * a.ld + c] = s;
+  }
+}
+
+// Trailing update: tiles (ti >= tj) of G_ik -= L_i L_k^T, and tiles of
+// r_i -= L_i y_j (columns of R in chunks of 64), 64 x 64 outputs per CTA.
+__global__ void __launch_bounds__(256) k_chol_update(CholArgs a, int j0, int ntile_max) {
+  const int b = blockIdx.y;
+  const int k = kdim(a, b);
+  if (j0 >= k || a.dead[b]) return;
+  const int jb = min(NB, k - j0);
+  const int s0 = j0 + jb;
+  const int n2 = k - s0;
+  if (n2 <= 0) return;
+  const int nt = (n2 + NB - 1) / NB;
+  const int ntri = nt * (nt + 1) / 2;
+  const int ndc = (a.d + NB - 1) / NB;
+  int t = blockIdx.x;
+  bool rhs = false;
+  int ti, tj;
+  if (t < ntri) {
+    ti = (int)((sqrtf(8.f * t + 1.f) - 1.f) * 0.5f);
+    while (ti * (ti + 1) / 2 > t) --ti;
+    while ((ti + 1) * (ti + 2) / 2 <= t) ++ti;
+    tj = t - ti * (ti + 1) / 2;
+  } else {
+    t -= ntri;
+    if (t >= nt * ndc) return;
+    rhs = true;
+    ti = t / ndc;
+    tj = t % ndc;
+  }
+  __shared__ float As[NB][NB + 4];  // L_i panel rows, [row][c]
+  __shared__ float Bs[NB][NB + 4];  // L_k panel rows or y_j, [row or col][c]
+  const int tid = threadIdx.x;
+  const int64_t row0 = a.c_off[b];
+  const int ri = s0 + ti * NB;
+  for (int e = tid; e < NB * NB; e += blockDim.x) {
+    const int r = e / NB, c = e % NB;
+    As[r][c] = (ri + r < k && c < jb) ? a.G[(row0 + ri + r) * a.ld + j0 + c] : 0.f;
+    if (!rhs) {
+      const int rk = s0 + tj * NB + r;
+      Bs[r][c] = (rk < k && c < jb) ? a.G[(row0 + rk) * a.ld + j0 + c] : 0.f;
+    } else {
+      // Bs[col][c] = y_j[c][col]
+      const int col = tj * NB + r;
+      Bs[r][c] = (col < a.d && c < jb) ? a.R[(row0 + j0 + c) * a.d + col] : 0.f;
+    }
+  }
+  __syncthreads();
+  const int tx = tid & 15, ty = tid >> 4;
+  float acc[4][4];
+#pragma unroll
+  for (int i = 0; i < 4; ++i)
+#pragma unroll
+    for (int j = 0; j < 4; ++j) acc[i][j] = 0.f;
+#pragma unroll 8
+  for (int c = 0; c < NB; ++c) {
+    float av[4], bv[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) av[i] = As[ty + 16 * i][c];
+#pragma unroll
+    for (int j = 0; j < 4; ++j) bv[j] = Bs[tx + 16 * j][c];
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+#pragma unroll
+      for (int j = 0; j < 4; ++j) acc[i][j] = fmaf(av[i], bv[j], acc[i][j]);
+  }
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const int r = ri + ty + 16 * i;
+    if (r >= k) continue;
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      if (!rhs) {
+        const int cc = s0 + tj * NB + tx + 16 * j;
+        if (cc < k && cc <= r) a.G[(row0 + r) * a.ld + cc] -= acc[i][j];
+      } else {
+        const int col = tj * NB + tx + 16 * j;
+        if (col < a.d) a.R[(row0 + r) * a.d + col] -= acc[i][j];
+      }
+    }
+  }
+}
+
+// Backward sweep, panel j0: x_j = L_jj^-T y_j (T recomputed from L_jj).
+__global__ void __launch_bounds__(256) k_chol_bdiag(CholArgs a, int j0) {
+  const int b = blockIdx.x;
+  const int k = kdim(a, b);
+  if (j0 >= k || a.dead[b]) return;
+  const int jb = min(NB, k - j0);
+  __shared__ float L[NB][NB + 1];
+  const float *G = a.G + (a.c_off[b] + j0) * a.ld + j0;
+  const int tid = threadIdx.x;
+  for (int e = tid; e < NB * NB; e += blockDim.x) {
+    const int r = e / NB, c = e % NB;
+    L[r][c] = (r < jb && c <= r) ? G[(int64_t)r * a.ld + c] : 0.f;
+  }
+  __syncthreads();
+  float *R = a.R + (a.c_off[b] + j0) * a.d;
+  for (int c = tid; c < a.d; c += blockDim.x) {
+    float x[NB];
+#pragma unroll 8
+    for (int r = 0; r < NB; ++r) x[r] = (r < jb) ? R[(int64_t)r * a.d + c] : 0.f;
+    for (int r = jb - 1; r >= 0; --r) {
+      float s = x[r];
+      for (int t = r + 1; t < jb; ++t) s = fmaf(-L[t][r], x[t], s);
+      x[r] = s / L[r][r];
+    }
+    for (int r = 0; r < jb; ++r) R[(int64_t)r * a.d + c] = x[r];
+  }
+}
+
+// Backward sweep update: y_i -= L_ji^T x_j for the rows i < j0 (64 x 64 tiles).
+__global__ void __launch_bounds__(256) k_chol_bupdate(CholArgs a, int j0) {
+  const int b = blockIdx.z;
+  const int k = kdim(a, b);
+  if (j0 >= k || a.dead[b]) return;
+  const int jb = min(NB, k - j0);
+  const int i0 = blockIdx.y * NB;
+  if (i0 >= j0) return;
+  const int c0 = blockIdx.x * NB;
+  if (c0 >= a.d) return;
+  __shared__ float As[NB][NB + 4];  // As[i][t] = L[j0 + t][i0 + i]
+  __shared__ float Bs[NB][NB + 4];  // Bs[col][t] = x[t][c0 + col]
+  const int tid = threadIdx.x;
+  const int64_t row0 = a.c_off[b];
+  for (int e = tid; e < NB * NB; e += blockDim.x) {
+    const int t = e / NB, u = e % NB;
+    As[u][t] = (t < jb && i0 + u < j0) ? a.G[(row0 + j0 + t) * a.ld + i0 + u] : 0.f;
+    Bs[u][t] = (t < jb && c0 + u < a.d) ? a.R[(row0 + j0 + t) * a.d + c0 + u] : 0.f;
+  }
+  __syncthreads();
+  const int tx = tid & 15, ty = tid >> 4;
+  float acc[4][4];
+#pragma unroll
+  for (int i = 0; i < 4; ++i)
+#pragma unroll
+    for (int j = 0; j < 4; ++j) acc[i][j] = 0.f;
+#pragma unroll 8
+  for (int t = 0; t < NB; ++t) {
+    float av[4], bv[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) av[i] = As[ty + 16 * i][t];
+#pragma unroll
+    for (int j = 0; j < 4; ++j) bv[j] = Bs[tx + 16 * j][t];
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+#pragma unroll
+      for (int j = 0; j < 4; ++j) acc[i][j] = fmaf(av[i], bv[j], acc[i][j]);
+  }
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const int r = i0 + ty + 16 * i;
+    if (r >= j0) continue;
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const int col = c0 + tx + 16 * j;
+      if (col < a.d) a.R[(row0 + r) * a.d + col] -= acc[i][j];
+    }
+  }
+}
+
+// V_c <- solution for the problems whose factorisation succeeded and is finite.
+__global__ void __launch_bounds__(256) k_chol_store(CholArgs a, float *Vc) {
+  const int b = blockIdx.x;
+  if (a.dead[b]) return;
+  const int64_t n = (int64_t)kdim(a, b) * a.d;
+  const float *X = a.R + a.c_off[b] * a.d;
+  bool finite = true;
+  for (int64_t e = threadIdx.x; e < n; e += blockDim.x) finite &= isfinite(X[e]);
+  finite = __syncthreads_and(finite);
+  if (!finite) {
+    if (threadIdx.x == 0) a.status[b] |= KVS_ST_NONFINITE;
+    return;
+  }
+  float *V = Vc + a.c_off[b] * a.d;
+  for (int64_t e = threadIdx.x; e < n; e += blockDim.x) V[e] = X[e];
 }
 
 }  // namespace
 
 int launch_chol_solve(const Batch &Bt, float *Vc, int32_t *status, const Work &w) {
-  k_chol_solve<<<Bt.g.B, 1024, 0, Bt.st>>>(w.gram, w.chol, w.R, w.xs, Vc, status, Bt.b->c_off,
-                                           Bt.g.max_c, Bt.g.d);
-  KVS_LAUNCH_CHECK("k_chol_solve");
+  const HostGeom &g = Bt.g;
+  CholArgs a{w.gram, w.R, w.chol_t, w.dead, status, Bt.b->c_off, (int64_t)g.max_c, g.d};
+  KVS_CUDA_TRY(cudaMemsetAsync(w.dead, 0, sizeof(int) * g.B, Bt.st));
+  const int npanel = (g.max_c + NB - 1) / NB;
+  const int ndc = (g.d + NB - 1) / NB;
+  for (int p = 0; p < npanel; ++p) {
+    const int j0 = p * NB;
+    k_chol_diag<<<g.B, 256, 0, Bt.st>>>(a, j0);
+    KVS_LAUNCH_CHECK("k_chol_diag");
+    const int n2 = g.max_c - j0 - NB;
+    if (n2 <= 0) continue;
+    const int nt = (n2 + NB - 1) / NB;
+    k_chol_panel<<<dim3(nt, g.B), 256, 0, Bt.st>>>(a, j0);
+    KVS_LAUNCH_CHECK("k_chol_panel");
+    k_chol_update<<<dim3(nt * (nt + 1) / 2 + nt * ndc, g.B), 256, 0, Bt.st>>>(a, j0, nt);
+    KVS_LAUNCH_CHECK("k_chol_update");
+  }
+  for (int p = npanel - 1; p >= 0; --p) {
+    const int j0 = p * NB;
+    k_chol_bdiag<<<g.B, 256, 0, Bt.st>>>(a, j0);
+    KVS_LAUNCH_CHECK("k_chol_bdiag");
+    if (j0 == 0) continue;
+    k_chol_bupdate<<<dim3(ndc, (j0 + NB - 1) / NB, g.B), 256, 0, Bt.st>>>(a, j0);
+    KVS_LAUNCH_CHECK("k_chol_bupdate");
+  }
+  k_chol_store<<<g.B, 256, 0, Bt.st>>>(a, Vc);
+  KVS_LAUNCH_CHECK("k_chol_store");
   return KVS_OK;
 }
 

@@ -62,7 +62,7 @@ def test_static_matches_workspace_call_twice(name):
 
 
 def test_static_rejects_batches_beyond_its_array():
-    c = Case(W.WORKLOADS["qwen_layer"], ids=[(0, 0, 0)])
+    c = Case(W.WORKLOADS["qwen_layer"])  # both KV heads of one layer
     K = c.K
     assert K.kvs_workspace_bytes(c.batch) > 32 << 20
     Kc = torch.zeros((c.batch.sum_c, c.wl.d), device="cuda")
