@@ -6,6 +6,8 @@
 
 #include <algorithm>
 #include <atomic>
+#include <map>
+#include <mutex>
 #include <cstddef>
 #include <vector>
 
@@ -17,6 +19,20 @@ static thread_local char g_err[256] = "no error";
 static std::atomic<uint64_t> g_launches{0};
 
 void count_launch() { g_launches.fetch_add(1, std::memory_order_relaxed); }
+
+cudaError_t set_smem_once_impl(const void *kern, int bytes) {
+  static std::mutex mu;
+  static std::map<std::pair<const void *, int>, int> done;  // (kernel, device) -> bytes set
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  std::lock_guard<std::mutex> lock(mu);
+  auto it = done.find({kern, dev});
+  if (it != done.end() && it->second >= bytes) return cudaSuccess;
+  e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+  if (e == cudaSuccess) done[{kern, dev}] = bytes;
+  return e;
+}
 
 void set_cuda_error(cudaError_t e, const char *where) {
   snprintf(g_err, sizeof g_err, "%s: %s (%s)", where, cudaGetErrorName(e), cudaGetErrorString(e));
@@ -90,7 +106,7 @@ size_t carve_work(const HostGeom &g, void *base, Work *w) {
   w->a_pad_off = c.take<int64_t>(g.B + 1);
   w->gram = c.take<float>(g.sum_c * g.max_c);
   w->R = c.take<float>(g.sum_c * g.d);
-  w->chol_t = c.take<float>((int64_t)g.B * 64 * 64);
+  w->chol_t = c.take<float>((int64_t)g.B * ((g.max_c + 63) / 64) * 64 * 64);
   w->dead = c.take<int>(g.B);
   w->fbuf = c.take<float>(g.B);
   w->Yt = c.take<float>(g.sum_q * g.d);
@@ -176,22 +192,118 @@ static int lbfgs_restart(const Batch &Bt, const kvs_schedule &sc, const float *Q
   return launch_lbfgs_reset(Bt, s, Kc, w.fbuf, s.gn, clear);
 }
 
+// One L-BFGS step in three parts: direction (and the bf16 split of the pairs),
+// the Armijo trial loop, then dK_c at the accepted points and the history update.
+static int step_head(const Batch &Bt, const kvs_schedule &sc, const float *Kc, const float *Vc,
+                     const State &s, const Work &w) {
+  int rc = launch_lbfgs_direction(Bt, s, sc);
+  if (rc) return rc;
+  return launch_split_pairs(Bt, Kc, Vc, w);  // V_c is fixed during the step
+}
+
+static int step_trial(const Batch &Bt, const kvs_schedule &sc, const float *Q, const float *Y,
+                      const float *lse, const float *Vc, float *Kc, const State &s,
+                      bool q_ready, const Work &w, const cudaGraphConditionalHandle *cond) {
+  int rc = launch_lbfgs_trial(Bt, s, Kc, w);
+  if (rc) return rc;
+  if ((rc = launch_forward(Bt, Q, Kc, Vc, Y, lse, sc.w_out, sc.w_lse, w.fbuf, nullptr,
+                           phase_filter(s, PH_SEARCH), q_ready, w, true, false)))
+    return rc;
+  return launch_lbfgs_armijo(Bt, s, sc, w, cond);
+}
+
+static int step_tail(const Batch &Bt, float *Kc, const State &s, int32_t *status, float *f_out,
+                     const Work &w) {
+  int rc = launch_backward(Bt, s.gn, phase_filter(s, PH_ACCEPT), w);
+  if (rc) return rc;
+  return launch_lbfgs_update(Bt, s, Kc, status, f_out);
+}
+
 static int lbfgs_one_step(const Batch &Bt, const kvs_schedule &sc, const float *Q,
                           const float *Y, const float *lse, const float *Vc, float *Kc,
                           const State &s, int32_t *status, float *f_out, bool q_ready,
                           const Work &w) {
-  int rc = launch_lbfgs_direction(Bt, s, sc);
+  int rc = step_head(Bt, sc, Kc, Vc, s, w);
   if (rc) return rc;
-  const Filter searching = phase_filter(s, PH_SEARCH);
-  for (int t = 0; t < sc.max_bt; ++t) {
-    if ((rc = launch_lbfgs_trial(Bt, s, Kc))) return rc;
-    if ((rc = launch_forward(Bt, Q, Kc, Vc, Y, lse, sc.w_out, sc.w_lse, w.fbuf, nullptr,
-                             searching, q_ready || t > 0, w)))
-      return rc;
-    if ((rc = launch_lbfgs_armijo(Bt, s, sc, w.fbuf))) return rc;
+  for (int t = 0; t < sc.max_bt; ++t)  // problems that have left the search skip each trial
+    if ((rc = step_trial(Bt, sc, Q, Y, lse, Vc, Kc, s, q_ready || t > 0, w, nullptr))) return rc;
+  return step_tail(Bt, Kc, s, status, f_out, w);
+}
+
+// One L-BFGS step as a CUDA graph whose trial loop is a conditional WHILE node:
+// trials run only while some problem is still searching (at most max_bt, since
+// every trial either accepts, backtracks or, at max_bt, fails the search).
+// The graph is recorded on two internal streams (the caller's stream may be the
+// legacy default stream, which cannot be captured) and launched on the caller's.
+struct StepGraph {
+  uint64_t kernels = 0;  // kernel nodes captured (the trial loop body counted once)
+  cudaGraph_t graph = nullptr;
+  cudaGraphExec_t exec = nullptr;
+  cudaStream_t cap = nullptr, side = nullptr;
+  ~StepGraph() {
+    if (exec) cudaGraphExecDestroy(exec);
+    if (graph) cudaGraphDestroy(graph);
+    if (side) cudaStreamDestroy(side);
+    if (cap) cudaStreamDestroy(cap);
   }
-  if ((rc = launch_backward(Bt, s.gn, phase_filter(s, PH_ACCEPT), w))) return rc;
-  return launch_lbfgs_update(Bt, s, Kc, status, f_out);
+};
+
+static int build_step_graph(const Batch &Bcaller, const kvs_schedule &sc, const float *Q,
+                            const float *Y, const float *lse, const float *Vc, float *Kc,
+                            const State &s, int32_t *status, const Work &w, StepGraph *sg) {
+  KVS_CUDA_TRY(cudaStreamCreateWithFlags(&sg->side, cudaStreamNonBlocking));
+  KVS_CUDA_TRY(cudaStreamCreateWithFlags(&sg->cap, cudaStreamNonBlocking));
+  Batch Bt = Bcaller;
+  Bt.st = sg->cap;
+  const uint64_t n0 = g_launches.load(std::memory_order_relaxed);
+  KVS_CUDA_TRY(cudaStreamBeginCapture(Bt.st, cudaStreamCaptureModeThreadLocal));
+  int rc = step_head(Bt, sc, Kc, Vc, s, w);
+  cudaStreamCaptureStatus cst;
+  cudaGraph_t g = nullptr;
+  const cudaGraphNode_t *deps = nullptr;
+  size_t ndeps = 0;
+  cudaGraphConditionalHandle cond{};
+  cudaGraphNode_t cnode = nullptr;
+  cudaGraphNodeParams cp = {};
+  cudaError_t e = cudaSuccess;
+  if (!rc) e = cudaStreamGetCaptureInfo(Bt.st, &cst, nullptr, &g, &deps, &ndeps);
+  if (!rc && e == cudaSuccess) e = cudaGraphConditionalHandleCreate(&cond, g, 1, cudaGraphCondAssignDefault);
+  if (!rc && e == cudaSuccess) {
+    cp.type = cudaGraphNodeTypeConditional;
+    cp.conditional.handle = cond;
+    cp.conditional.type = cudaGraphCondTypeWhile;
+    cp.conditional.size = 1;
+    e = cudaGraphAddNode(&cnode, g, deps, ndeps, &cp);
+  }
+  if (!rc && e == cudaSuccess)
+    e = cudaStreamUpdateCaptureDependencies(Bt.st, &cnode, 1, cudaStreamSetCaptureDependencies);
+  if (!rc && e == cudaSuccess) {
+    e = cudaStreamBeginCaptureToGraph(sg->side, cp.conditional.phGraph_out[0], nullptr, nullptr,
+                                      0, cudaStreamCaptureModeThreadLocal);
+    if (e == cudaSuccess) {
+      Batch side = Bt;
+      side.st = sg->side;
+      rc = step_trial(side, sc, Q, Y, lse, Vc, Kc, s, true, w, &cond);
+      cudaGraph_t body = nullptr;
+      const cudaError_t e2 = cudaStreamEndCapture(sg->side, &body);
+      if (e2 != cudaSuccess) e = e2;
+    }
+  }
+  if (!rc && e == cudaSuccess) rc = step_tail(Bt, Kc, s, status, nullptr, w);
+  cudaGraph_t graph = nullptr;
+  const cudaError_t e3 = cudaStreamEndCapture(Bt.st, &graph);
+  sg->graph = graph;
+  if (rc) return rc;
+  if (e != cudaSuccess) {
+    set_cuda_error(e, "building the L-BFGS step graph");
+    (void)cudaGetLastError();
+    return KVS_ECUDA;
+  }
+  KVS_CUDA_TRY(e3);
+  KVS_CUDA_TRY(cudaGraphInstantiate(&sg->exec, sg->graph, 0));
+  sg->kernels = g_launches.load(std::memory_order_relaxed) - n0;
+  g_launches.fetch_sub(sg->kernels, std::memory_order_relaxed);  // captured, not yet run
+  return KVS_OK;
 }
 
 }  // namespace kvs
@@ -361,10 +473,23 @@ int kvs_compress_batch(const kvs_batch *batch, const kvs_schedule *sched, const 
   if ((rc = lbfgs_restart(Bt, sc, Q, w.Yt, w.lset, Vc, Kc, s, 1, true, w))) return rc;
   const int64_t tstride = sc.outer + 1;
   if (loss_trace && (rc = launch_copy_f(Bt, s, loss_trace, tstride, 0))) return rc;
+  StepGraph sg;
+  bool have_graph = false;
   for (int o = 0; o < sc.outer; ++o) {
-    for (int t = 0; t < sc.steps; ++t)
-      if ((rc = lbfgs_one_step(Bt, sc, Q, w.Yt, w.lset, Vc, Kc, s, status, nullptr, true, w)))
+    for (int t = 0; t < sc.steps; ++t) {
+      if (!have_graph && o + t > 0) {
+        // every kernel has been launched once outside capture: record the step now
+        if ((rc = build_step_graph(Bt, sc, Q, w.Yt, w.lset, Vc, Kc, s, status, w, &sg))) return rc;
+        have_graph = true;
+      }
+      if (have_graph) {
+        KVS_CUDA_TRY(cudaGraphLaunch(sg.exec, Bt.st));
+        g_launches.fetch_add(sg.kernels, std::memory_order_relaxed);
+      } else if ((rc = lbfgs_one_step(Bt, sc, Q, w.Yt, w.lset, Vc, Kc, s, status, nullptr, true,
+                                      w))) {
         return rc;
+      }
+    }
     if ((rc = launch_fit(Bt, Q, Kc, w.Yt, sc.lambda, Vc, status, true, true, w))) return rc;
     if ((rc = lbfgs_restart(Bt, sc, Q, w.Yt, w.lset, Vc, Kc, s, sc.persist_history ? 0 : 1, true,
                             w)))

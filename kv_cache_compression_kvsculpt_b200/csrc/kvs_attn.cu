@@ -14,6 +14,7 @@
 
 #include <algorithm>
 #include <mutex>
+#include <unordered_map>
 
 #include "kvs_attn_tc.cuh"
 
@@ -35,8 +36,36 @@ static PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
   return fn;
 }
 
+namespace {
+struct MapKey {
+  const void *base;
+  uint64_t rows, cols;
+  uint32_t box;
+  bool operator==(const MapKey &o) const {
+    return base == o.base && rows == o.rows && cols == o.cols && box == o.box;
+  }
+};
+struct MapKeyHash {
+  size_t operator()(const MapKey &k) const {
+    return std::hash<const void *>()(k.base) ^ (k.rows * 0x9E3779B97F4A7C15ull) ^
+           (k.cols << 20) ^ ((uint64_t)k.box << 40);
+  }
+};
+std::mutex g_map_mu;
+std::unordered_map<MapKey, CUtensorMap, MapKeyHash> g_maps;  // encoded descriptors, reused
+}  // namespace
+
 int make_map_bf16(CUtensorMap *m, const void *base, uint64_t rows, uint64_t cols,
                   uint32_t box_rows) {
+  const MapKey key{base, rows, cols, box_rows};
+  {
+    std::lock_guard<std::mutex> lock(g_map_mu);
+    auto it = g_maps.find(key);
+    if (it != g_maps.end()) {
+      *m = it->second;
+      return KVS_OK;
+    }
+  }
   auto fn = encode_fn();
   if (!fn) return KVS_ECUDA;
   cuuint64_t dims[2] = {(cuuint64_t)cols, (cuuint64_t)(rows > 0 ? rows : 1)};
@@ -46,7 +75,11 @@ int make_map_bf16(CUtensorMap *m, const void *base, uint64_t rows, uint64_t cols
   CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(base), dims, strides,
                   box, es, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-  return r == CUDA_SUCCESS ? KVS_OK : KVS_ECUDA;
+  if (r != CUDA_SUCCESS) return KVS_ECUDA;
+  std::lock_guard<std::mutex> lock(g_map_mu);
+  if (g_maps.size() > 4096) g_maps.clear();
+  g_maps.emplace(key, *m);
+  return KVS_OK;
 }
 
 namespace {
@@ -177,11 +210,11 @@ int prep_pairs(const Batch &Bt, const float *Kc, const float *Vc, const Work &w)
 template <int D>
 int forward_d(const Batch &Bt, const float *Q, const float *Kc, const float *Vc, const float *Y,
               const float *lse, float w_out, float w_lse, float *loss, float *parts, Filter flt,
-              bool q_ready, const Work &w) {
+              bool q_ready, bool pairs_ready, bool reduce, const Work &w) {
   const HostGeom &g = Bt.g;
   int rc;
   if (!q_ready && (rc = split(Q, w.qh, w.ql, g.sum_q * D, Bt.st))) return rc;
-  if ((rc = prep_pairs<D>(Bt, Kc, Vc, w))) return rc;
+  if (!pairs_ready && (rc = prep_pairs<D>(Bt, Kc, Vc, w))) return rc;
   FwdMaps fm;
   if ((rc = make_map_bf16(&fm.kh, w.kh, g.sum_c, D, 64)) ||
       (rc = make_map_bf16(&fm.kl, w.kl, g.sum_c, D, 64)) ||
@@ -206,6 +239,7 @@ int forward_d(const Batch &Bt, const float *Q, const float *Kc, const float *Vc,
   a.w_lse = w_lse;
   a.err = w.err;
   if ((rc = launch_fwd_tc<D, FWD_LOSS>(fm, a, max_qtiles(g), g.B, Bt.st))) return rc;
+  if (!reduce) return KVS_OK;
   k_loss_reduce<<<(g.B + 127) / 128, 128, 0, Bt.st>>>(w.partials, max_qtiles(g), Bt.b->q_off, D,
                                                       w_out, w_lse, loss, parts, flt, g.B);
   KVS_LAUNCH_CHECK("k_loss_reduce");
@@ -308,10 +342,16 @@ int launch_targets(const Batch &Bt, const float *Q, const float *Kz, const float
 
 int launch_forward(const Batch &Bt, const float *Q, const float *Kc, const float *Vc,
                    const float *Y, const float *lse, float w_out, float w_lse, float *loss,
-                   float *parts, Filter flt, bool q_ready, const Work &w) {
-  return Bt.g.d == 64
-             ? forward_d<64>(Bt, Q, Kc, Vc, Y, lse, w_out, w_lse, loss, parts, flt, q_ready, w)
-             : forward_d<128>(Bt, Q, Kc, Vc, Y, lse, w_out, w_lse, loss, parts, flt, q_ready, w);
+                   float *parts, Filter flt, bool q_ready, const Work &w, bool pairs_ready,
+                   bool reduce) {
+  return Bt.g.d == 64 ? forward_d<64>(Bt, Q, Kc, Vc, Y, lse, w_out, w_lse, loss, parts, flt,
+                                      q_ready, pairs_ready, reduce, w)
+                      : forward_d<128>(Bt, Q, Kc, Vc, Y, lse, w_out, w_lse, loss, parts, flt,
+                                       q_ready, pairs_ready, reduce, w);
+}
+
+int launch_split_pairs(const Batch &Bt, const float *Kc, const float *Vc, const Work &w) {
+  return Bt.g.d == 64 ? prep_pairs<64>(Bt, Kc, Vc, w) : prep_pairs<128>(Bt, Kc, Vc, w);
 }
 
 int launch_backward(const Batch &Bt, float *dKc, Filter flt, const Work &w) {

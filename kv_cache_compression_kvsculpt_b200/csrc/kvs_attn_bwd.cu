@@ -315,7 +315,7 @@ int launch_bwd_tc(const BwdMaps &m, const BwdArgs &a, int max_tiles, int B, cuda
   using C = Bwd<D, MODE>;
   static_assert(C::SMEM + sizeof(BwdBars) <= 232448, "shared memory");
   auto kern = k_attn_bwd<D, MODE>;
-  KVS_CUDA_TRY(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM));
+  KVS_CUDA_TRY(set_smem_once(kern, C::SMEM));
   kern<<<dim3(max_tiles, B), 192, C::SMEM, st>>>(m.kh, m.kl, m.qh, m.ql, m.g, a);
   KVS_LAUNCH_CHECK("k_attn_bwd");
   return KVS_OK;

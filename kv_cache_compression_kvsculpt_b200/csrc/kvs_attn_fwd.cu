@@ -404,7 +404,7 @@ int launch_fwd_tc(const FwdMaps &m, const FwdArgs &a, int max_tiles, int B, cuda
   using C = Fwd<D, MODE>;
   static_assert(C::SMEM + sizeof(FwdBars) <= 232448, "shared memory");
   auto kern = k_attn_fwd<D, MODE>;
-  KVS_CUDA_TRY(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM));
+  KVS_CUDA_TRY(set_smem_once(kern, C::SMEM));
   kern<<<dim3(max_tiles, B), 192, C::SMEM, st>>>(m.kh, m.kl, m.vh, m.vl, a);
   KVS_LAUNCH_CHECK("k_attn_fwd");
   return KVS_OK;

@@ -18,6 +18,7 @@ void count_launch();
     cudaError_t _e = (expr);                                   \
     if (_e != cudaSuccess) {                                   \
       ::kvs::set_cuda_error(_e, #expr);                        \
+      (void)cudaGetLastError(); /* do not leak into later checks */ \
       return KVS_ECUDA;                                        \
     }                                                          \
   } while (0)
@@ -136,5 +137,12 @@ __device__ __forceinline__ float block_max(float v, float *red) {
 }
 
 inline int64_t align_up(int64_t x, int64_t a) { return (x + a - 1) / a * a; }
+
+// cudaFuncSetAttribute(MaxDynamicSharedMemorySize) once per kernel and device.
+cudaError_t set_smem_once_impl(const void *kern, int bytes);
+template <class F>
+cudaError_t set_smem_once(F *kern, int bytes) {
+  return set_smem_once_impl(reinterpret_cast<const void *>(kern), bytes);
+}
 
 }  // namespace kvs

@@ -169,7 +169,7 @@ __global__ void __launch_bounds__(192, 1)
 
 int launch_gemm3_tc(const GemmMaps &m, const GemmArgs3 &a, int tiles_m, int gram, int B,
                     cudaStream_t st) {
-  KVS_CUDA_TRY(cudaFuncSetAttribute(k_gemm3, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM));
+  KVS_CUDA_TRY(set_smem_once(k_gemm3, SMEM));
   const int tiles = gram ? tiles_m * (tiles_m + 1) / 2 : tiles_m;
   if (tiles <= 0) return KVS_OK;
   k_gemm3<<<dim3(tiles, B), 192, SMEM, st>>>(m.ah, m.al, m.bh, m.bl, a, gram);

@@ -39,7 +39,7 @@ struct Work {
   int64_t *a_pad_off;        // [B+1]                  padded row offsets of ahi/alo
   float *gram;               // [sum_c, max_c]         A^T A + lam I, then its Cholesky factor
   float *R;                  // [sum_c, d]             A^T Y, then the solution
-  float *chol_t;             // [B, 64, 64]            inverse of the current diagonal block
+  float *chol_t;             // [B, panels, 64, 64]    inverses of the diagonal blocks
   int *dead;                 // [B]                    factorisation failed
   float *fbuf;               // [B]                    loss scratch
   float *Yt;                 // [sum_q, d]             targets (kvs_compress_batch)
@@ -83,7 +83,10 @@ int launch_targets(const Batch &B, const float *Q, const float *Kz, const float 
 // Q split in w.qh/ql is current.
 int launch_forward(const Batch &B, const float *Q, const float *Kc, const float *Vc,
                    const float *Y, const float *lse, float w_out, float w_lse, float *loss,
-                   float *parts, Filter flt, bool q_ready, const Work &w);
+                   float *parts, Filter flt, bool q_ready, const Work &w,
+                   bool pairs_ready = false, bool reduce = true);
+// bf16 hi/lo copies of the compressed pairs (keys; values unless Vc is null).
+int launch_split_pairs(const Batch &B, const float *Kc, const float *Vc, const Work &w);
 // dKc from the state left by launch_forward for the same problems.
 int launch_backward(const Batch &B, float *dKc, Filter flt, const Work &w);
 // Ridge fit: Vc = (A^T A + lam I)^-1 A^T Y (y_ready: the Y split is current).
@@ -100,8 +103,12 @@ int launch_chol_solve(const Batch &B, float *Vc, int32_t *status, const Work &w)
 int launch_lbfgs_reset(const Batch &B, const State &s, const float *Kc, const float *f,
                        const float *g, int clear);
 int launch_lbfgs_direction(const Batch &B, const State &s, const kvs_schedule &sc);
-int launch_lbfgs_trial(const Batch &B, const State &s, float *Kc);
-int launch_lbfgs_armijo(const Batch &B, const State &s, const kvs_schedule &sc, const float *ft);
+// Kc = x + t d for searching problems, with its bf16 hi/lo split into w.kh/w.kl.
+int launch_lbfgs_trial(const Batch &B, const State &s, float *Kc, const Work &w);
+// Armijo test on the trial loss summed from the forward's per-CTA partials;
+// with `cond`, also sets that graph condition to "a problem is still searching".
+int launch_lbfgs_armijo(const Batch &B, const State &s, const kvs_schedule &sc, const Work &w,
+                        const cudaGraphConditionalHandle *cond = nullptr);
 int launch_lbfgs_update(const Batch &B, const State &s, float *Kc, int32_t *status,
                         float *f_out);
 int launch_copy_f(const Batch &B, const State &s, float *dst, int64_t stride, int64_t col);

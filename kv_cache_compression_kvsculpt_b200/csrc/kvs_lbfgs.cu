@@ -128,36 +128,63 @@ __global__ void __launch_bounds__(NT) k_direction(LbfgsScal *sc, const float *__
   }
 }
 
-// Kc = x + t d for problems still searching.
+// Kc = x + t d for problems still searching, with the bf16 hi/lo split of the
+// trial keys that the loss forward reads (pairs of elements: n is even).
 __global__ void k_trial(const LbfgsScal *sc, const float *__restrict__ x,
                         const float *__restrict__ dir, float *__restrict__ Kc,
+                        __nv_bfloat16 *__restrict__ kh, __nv_bfloat16 *__restrict__ kl,
                         const int64_t *c_off, int d) {
   const int b = blockIdx.y;
   if (sc[b].phase != PH_SEARCH) return;
   const int64_t o = seg0(c_off, b, d), n = c_off[b + 1] * (int64_t)d - o;
   const float t = sc[b].t;
-  for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < n;
-       i += (int64_t)gridDim.x * blockDim.x)
-    Kc[o + i] = fmaf(t, dir[o + i], x[o + i]);
+  for (int64_t i = 2 * (blockIdx.x * (int64_t)blockDim.x + threadIdx.x); i < n;
+       i += 2 * (int64_t)gridDim.x * blockDim.x) {
+    const float2 xv = *reinterpret_cast<const float2 *>(x + o + i);
+    const float2 dv = *reinterpret_cast<const float2 *>(dir + o + i);
+    const float k0 = fmaf(t, dv.x, xv.x), k1 = fmaf(t, dv.y, xv.y);
+    *reinterpret_cast<float2 *>(Kc + o + i) = make_float2(k0, k1);
+    const __nv_bfloat162 h = __floats2bfloat162_rn(k0, k1);
+    const float2 hf = __bfloat1622float2(h);
+    *reinterpret_cast<__nv_bfloat162 *>(kh + o + i) = h;
+    *reinterpret_cast<__nv_bfloat162 *>(kl + o + i) = __floats2bfloat162_rn(k0 - hf.x, k1 - hf.y);
+  }
 }
 
-// Armijo test of the trial loss: accept, or halve t, or give up after max_bt trials.
-__global__ void k_armijo(LbfgsScal *sc, int B, const float *ft, float c1, float backtrack,
-                         int max_bt) {
-  const int b = blockIdx.x * blockDim.x + threadIdx.x;
-  if (b >= B) return;
-  LbfgsScal &s = sc[b];
-  if (s.phase != PH_SEARCH) return;
-  const float f = ft[b];
-  s.trials += 1;
-  if (isfinite(f) && f <= s.f + c1 * s.t * s.gtd) {
-    s.ft = f;
-    s.phase = PH_ACCEPT;
-  } else if (s.trials >= max_bt) {
-    s.phase = PH_FAIL;
-  } else {
-    s.t *= backtrack;
+// Armijo test of the trial loss: accept, or halve t, or give up after max_bt
+// trials.  The loss is summed (fixed order, double) from the loss forward's
+// per-CTA partials of the output and LSE terms.  One CTA walks all problems;
+// inside a CUDA graph it also sets the trial loop's condition to "some
+// problem is still searching".
+__global__ void __launch_bounds__(256) k_armijo(LbfgsScal *sc, int B, const float *partials,
+                                                int tiles, const int64_t *q_off, int d,
+                                                float w_out, float w_lse, float c1,
+                                                float backtrack, int max_bt, int use_cond,
+                                                cudaGraphConditionalHandle cond) {
+  int still = 0;
+  for (int b = threadIdx.x; b < B; b += blockDim.x) {
+    LbfgsScal &s = sc[b];
+    if (s.phase != PH_SEARCH) continue;
+    const int nq = (int)(q_off[b + 1] - q_off[b]);
+    double so = 0.0, sl = 0.0;
+    for (int t = 0; t < (nq + 127) / 128; ++t) {
+      so += partials[((int64_t)b * tiles + t) * 2];
+      sl += partials[((int64_t)b * tiles + t) * 2 + 1];
+    }
+    const float f = (float)(w_out * (so / ((double)nq * d)) + w_lse * (sl / (double)nq));
+    s.trials += 1;
+    if (isfinite(f) && f <= s.f + c1 * s.t * s.gtd) {
+      s.ft = f;
+      s.phase = PH_ACCEPT;
+    } else if (s.trials >= max_bt) {
+      s.phase = PH_FAIL;
+    } else {
+      s.t *= backtrack;
+      still = 1;
+    }
   }
+  still = __syncthreads_or(still);
+  if (use_cond && threadIdx.x == 0) cudaGraphSetConditional(cond, still ? 1u : 0u);
 }
 
 // Accepted: store (s, y) in the scratch slot, keep it when s.y > 1e-10 y.y,
@@ -236,17 +263,21 @@ int launch_lbfgs_direction(const Batch &Bt, const State &s, const kvs_schedule &
   return KVS_OK;
 }
 
-int launch_lbfgs_trial(const Batch &Bt, const State &s, float *Kc) {
-  const int64_t n = (int64_t)Bt.g.max_c * Bt.g.d;
+int launch_lbfgs_trial(const Batch &Bt, const State &s, float *Kc, const Work &w) {
+  const int64_t n = (int64_t)Bt.g.max_c * Bt.g.d / 2;
   const int blocks = (int)std::min<int64_t>((n + 255) / 256, 64);
-  k_trial<<<dim3(blocks, Bt.g.B), 256, 0, Bt.st>>>(s.sc, s.x, s.dir, Kc, Bt.b->c_off, Bt.g.d);
+  k_trial<<<dim3(blocks, Bt.g.B), 256, 0, Bt.st>>>(s.sc, s.x, s.dir, Kc, w.kh, w.kl,
+                                                   Bt.b->c_off, Bt.g.d);
   KVS_LAUNCH_CHECK("k_trial");
   return KVS_OK;
 }
 
-int launch_lbfgs_armijo(const Batch &Bt, const State &s, const kvs_schedule &sc, const float *ft) {
-  k_armijo<<<(Bt.g.B + 127) / 128, 128, 0, Bt.st>>>(s.sc, Bt.g.B, ft, sc.c1, sc.backtrack,
-                                                    sc.max_bt);
+int launch_lbfgs_armijo(const Batch &Bt, const State &s, const kvs_schedule &sc, const Work &w,
+                        const cudaGraphConditionalHandle *cond) {
+  k_armijo<<<1, 256, 0, Bt.st>>>(s.sc, Bt.g.B, w.partials, (Bt.g.max_q + 127) / 128,
+                                 Bt.b->q_off, Bt.g.d, sc.w_out, sc.w_lse, sc.c1, sc.backtrack,
+                                 sc.max_bt, cond ? 1 : 0,
+                                 cond ? *cond : cudaGraphConditionalHandle{});
   KVS_LAUNCH_CHECK("k_armijo");
   return KVS_OK;
 }

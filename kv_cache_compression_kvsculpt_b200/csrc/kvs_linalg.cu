@@ -5,9 +5,10 @@
 //
 // Right-looking blocked algorithm over panels of NB = 64 columns, float32,
 // every problem of the batch advancing together so that all SMs share the work:
-//   per panel j (one launch each):
-//     diag    factor the diagonal block G_jj = L_jj L_jj^T in shared memory,
-//             form T_j = L_jj^-1 and the forward-solved rows y_j = T_j r_j
+//   per panel j:
+//     diag    factor the diagonal block G_jj = L_jj L_jj^T in shared memory and
+//             keep T_j = L_jj^-1
+//     tmul    forward-solved rows y_j = T_j r_j
 //     panel   L_ij = G_ij T_j^T for the rows below
 //     update  G_ik -= L_ij L_kj^T on the trailing lower triangle and
 //             r_i -= L_ij y_j on the right-hand sides (64 x 64 register tiles)
@@ -27,7 +28,8 @@ constexpr int NB = 64;
 struct CholArgs {
   float *G;              // [sum_c, ld] Gram matrix -> factor (lower triangle)
   float *R;              // [sum_c, d] right-hand sides -> solution
-  float *T;              // [B, NB, NB] inverse of the current diagonal block
+  float *T;              // [B, npanel, NB, NB] inverses of the diagonal blocks
+  int npanel;
   int *dead;             // [B] set once a problem's factorisation failed
   int32_t *status;
   const int64_t *c_off;
@@ -39,7 +41,7 @@ __device__ __forceinline__ int kdim(const CholArgs &a, int b) {
   return (int)(a.c_off[b + 1] - a.c_off[b]);
 }
 
-// Diagonal block of panel j0: factor, invert, and solve y = T r for its rows.
+// Diagonal block of panel j0: factor in shared memory and keep its inverse T_j.
 __global__ void __launch_bounds__(256) k_chol_diag(CholArgs a, int j0) {
   const int b = blockIdx.x;
   const int k = kdim(a, b);
@@ -92,21 +94,60 @@ __global__ void __launch_bounds__(256) k_chol_diag(CholArgs a, int j0) {
     }
   }
   __syncthreads();
+  float *Tg = a.T + ((int64_t)b * a.npanel + j0 / NB) * NB * NB;
   for (int e = tid; e < NB * NB; e += blockDim.x) {
     const int r = e / NB, c = e % NB;
     if (r < jb && c <= r) G[(int64_t)r * a.ld + c] = L[r][c];
-    a.T[(int64_t)b * NB * NB + e] = Ti[r][c];
+    Tg[e] = Ti[r][c];
   }
-  // forward solve of this block's right-hand sides: y = T r (columns of R independent)
-  float *R = a.R + (a.c_off[b] + j0) * a.d;
-  for (int c = tid; c < a.d; c += blockDim.x) {
-    float y[NB];
+}
+
+// Rows j0 .. j0+63 of the right-hand sides times T_j (forward sweep) or T_j^T
+// (backward sweep), in place; 64 columns of R per CTA, 4 x 4 register tiles.
+__global__ void __launch_bounds__(256) k_chol_tmul(CholArgs a, int j0, int transpose) {
+  const int b = blockIdx.y;
+  const int k = kdim(a, b);
+  if (j0 >= k || a.dead[b]) return;
+  const int jb = min(NB, k - j0);
+  const int c0 = blockIdx.x * NB;
+  if (c0 >= a.d) return;
+  __shared__ float Ts[NB][NB + 4];  // Ts[r][t] = M[r][t]
+  __shared__ float Xs[NB][NB + 4];  // Xs[col][t] = R[j0 + t][c0 + col]
+  const float *Tg = a.T + ((int64_t)b * a.npanel + j0 / NB) * NB * NB;
+  float *R = a.R + (a.c_off[b] + j0) * a.d + c0;
+  const int tid = threadIdx.x;
+  for (int e = tid; e < NB * NB; e += blockDim.x) {
+    const int r = e / NB, t = e % NB;
+    Ts[r][t] = transpose ? Tg[t * NB + r] : Tg[e];
+    Xs[t][r] = (r < jb && c0 + t < a.d) ? R[(int64_t)r * a.d + t] : 0.f;
+  }
+  __syncthreads();
+  const int tx = tid & 15, ty = tid >> 4;
+  float acc[4][4];
+#pragma unroll
+  for (int i = 0; i < 4; ++i)
+#pragma unroll
+    for (int j = 0; j < 4; ++j) acc[i][j] = 0.f;
 #pragma unroll 8
-    for (int r = 0; r < NB; ++r) y[r] = (r < jb) ? R[(int64_t)r * a.d + c] : 0.f;
-    for (int r = jb - 1; r >= 0; --r) {
-      float s = 0.f;
-      for (int t = 0; t <= r; ++t) s = fmaf(Ti[r][t], y[t], s);
-      R[(int64_t)r * a.d + c] = s;
+  for (int t = 0; t < NB; ++t) {
+    float av[4], bv[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) av[i] = Ts[ty + 16 * i][t];
+#pragma unroll
+    for (int j = 0; j < 4; ++j) bv[j] = Xs[tx + 16 * j][t];
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+#pragma unroll
+      for (int j = 0; j < 4; ++j) acc[i][j] = fmaf(av[i], bv[j], acc[i][j]);
+  }
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const int r = ty + 16 * i;
+    if (r >= jb) continue;
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const int col = tx + 16 * j;
+      if (c0 + col < a.d) R[(int64_t)r * a.d + col] = acc[i][j];
     }
   }
 }
@@ -126,7 +167,7 @@ __global__ void __launch_bounds__(256) k_chol_panel(CholArgs a, int j0) {
   float *P = a.G + (a.c_off[b] + i0) * a.ld + j0;
   for (int e = tid; e < NB * NB; e += blockDim.x) {
     const int r = e / NB, c = e % NB;
-    Ti[r][c] = a.T[(int64_t)b * NB * NB + e];
+    Ti[r][c] = a.T[((int64_t)b * a.npanel + j0 / NB) * NB * NB + e];
     Ar[r][c] = (r < ib && c < jb) ? P[(int64_t)r * a.ld + c] : 0.f;
   }
   __syncthreads();
@@ -219,34 +260,6 @@ __global__ void __launch_bounds__(256) k_chol_update(CholArgs a, int j0, int nti
   }
 }
 
-// Backward sweep, panel j0: x_j = L_jj^-T y_j (T recomputed from L_jj).
-__global__ void __launch_bounds__(256) k_chol_bdiag(CholArgs a, int j0) {
-  const int b = blockIdx.x;
-  const int k = kdim(a, b);
-  if (j0 >= k || a.dead[b]) return;
-  const int jb = min(NB, k - j0);
-  __shared__ float L[NB][NB + 1];
-  const float *G = a.G + (a.c_off[b] + j0) * a.ld + j0;
-  const int tid = threadIdx.x;
-  for (int e = tid; e < NB * NB; e += blockDim.x) {
-    const int r = e / NB, c = e % NB;
-    L[r][c] = (r < jb && c <= r) ? G[(int64_t)r * a.ld + c] : 0.f;
-  }
-  __syncthreads();
-  float *R = a.R + (a.c_off[b] + j0) * a.d;
-  for (int c = tid; c < a.d; c += blockDim.x) {
-    float x[NB];
-#pragma unroll 8
-    for (int r = 0; r < NB; ++r) x[r] = (r < jb) ? R[(int64_t)r * a.d + c] : 0.f;
-    for (int r = jb - 1; r >= 0; --r) {
-      float s = x[r];
-      for (int t = r + 1; t < jb; ++t) s = fmaf(-L[t][r], x[t], s);
-      x[r] = s / L[r][r];
-    }
-    for (int r = 0; r < jb; ++r) R[(int64_t)r * a.d + c] = x[r];
-  }
-}
-
 // Backward sweep update: y_i -= L_ji^T x_j for the rows i < j0 (64 x 64 tiles).
 __global__ void __launch_bounds__(256) k_chol_bupdate(CholArgs a, int j0) {
   const int b = blockIdx.z;
@@ -318,14 +331,16 @@ __global__ void __launch_bounds__(256) k_chol_store(CholArgs a, float *Vc) {
 
 int launch_chol_solve(const Batch &Bt, float *Vc, int32_t *status, const Work &w) {
   const HostGeom &g = Bt.g;
-  CholArgs a{w.gram, w.R, w.chol_t, w.dead, status, Bt.b->c_off, (int64_t)g.max_c, g.d};
-  KVS_CUDA_TRY(cudaMemsetAsync(w.dead, 0, sizeof(int) * g.B, Bt.st));
   const int npanel = (g.max_c + NB - 1) / NB;
+  CholArgs a{w.gram, w.R, w.chol_t, npanel, w.dead, status, Bt.b->c_off, (int64_t)g.max_c, g.d};
+  KVS_CUDA_TRY(cudaMemsetAsync(w.dead, 0, sizeof(int) * g.B, Bt.st));
   const int ndc = (g.d + NB - 1) / NB;
   for (int p = 0; p < npanel; ++p) {
     const int j0 = p * NB;
     k_chol_diag<<<g.B, 256, 0, Bt.st>>>(a, j0);
     KVS_LAUNCH_CHECK("k_chol_diag");
+    k_chol_tmul<<<dim3(ndc, g.B), 256, 0, Bt.st>>>(a, j0, 0);
+    KVS_LAUNCH_CHECK("k_chol_tmul");
     const int n2 = g.max_c - j0 - NB;
     if (n2 <= 0) continue;
     const int nt = (n2 + NB - 1) / NB;
@@ -336,8 +351,8 @@ int launch_chol_solve(const Batch &Bt, float *Vc, int32_t *status, const Work &w
   }
   for (int p = npanel - 1; p >= 0; --p) {
     const int j0 = p * NB;
-    k_chol_bdiag<<<g.B, 256, 0, Bt.st>>>(a, j0);
-    KVS_LAUNCH_CHECK("k_chol_bdiag");
+    k_chol_tmul<<<dim3(ndc, g.B), 256, 0, Bt.st>>>(a, j0, 1);
+    KVS_LAUNCH_CHECK("k_chol_tmul");
     if (j0 == 0) continue;
     k_chol_bupdate<<<dim3(ndc, (j0 + NB - 1) / NB, g.B), 256, 0, Bt.st>>>(a, j0);
     KVS_LAUNCH_CHECK("k_chol_bupdate");

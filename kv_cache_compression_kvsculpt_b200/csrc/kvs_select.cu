@@ -172,8 +172,7 @@ int launch_build_queries(const kvs_query_spec *sp, const float *q_retain, const 
 
 int launch_topk(const Batch &Bt, const float *imp, const float *Kz, int32_t *idx, float *Kc) {
   const size_t smem = (size_t)Bt.g.max_z * sizeof(uint32_t);
-  KVS_CUDA_TRY(cudaFuncSetAttribute(k_topk, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                    (int)smem));
+  KVS_CUDA_TRY(set_smem_once(k_topk, (int)smem));
   k_topk<<<Bt.g.B, 1024, smem, Bt.st>>>(imp, Bt.b->z_off, Bt.b->c_off, idx);
   KVS_LAUNCH_CHECK("k_topk");
   k_gather<<<dim3((Bt.g.max_c + 7) / 8, Bt.g.B), 256, 0, Bt.st>>>(Kz, Bt.b->z_off, Bt.b->c_off,
