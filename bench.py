@@ -385,9 +385,9 @@ def main():
     ap.add_argument("--outer", type=int, default=None, help="override the outer iterations")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-budget", type=float, default=20.0)
-    ap.add_argument("--bound", default="alu")
-    ap.add_argument("--peak-key", default="fp32_simt_tflops")
-    ap.add_argument("--dtype-label", default="f32")
+    ap.add_argument("--bound", default="tensor")
+    ap.add_argument("--peak-key", default="bf16_tflops")
+    ap.add_argument("--dtype-label", default="bf16x3-f32acc")
     args = ap.parse_args()
     if args.impl == "reference":
         run_reference(args)

@@ -18,8 +18,10 @@
 // product keeps about 16 significant bits.
 // Tensor memory (512 columns): S buffers at 0 and 64, dP at 128 and 192,
 // dK at 256, V hi at 384, V lo at 384 + D/2.
-// Warp roles: warps 0-3 one thread per key row (TMEM lane), warp 4 TMA
-// producer (also stages l and delta of the tile), warp 5 MMA issuer.
+// Two row warpgroups take alternate query tiles (each owns one of the two S /
+// dP buffers).  Warp roles: warps 0-7 one thread per key row (warp w <-> TMEM
+// lanes 32 (w % 4) ..), warp 8 TMA producer (also stages l and delta of the
+// tile), warp 9 MMA issuer.
 #include <math.h>
 
 #include "kvs_attn_tc.cuh"
@@ -31,13 +33,15 @@ using namespace tc;
 
 constexpr int BK = 128;  // keys per CTA
 constexpr int BQ = 64;   // queries per tile
+constexpr int NTHREADS = 320;
+constexpr int NSTAGE = 3;  // query-tile stages in flight
 constexpr float L2E = 1.4426950408889634f;
 
 template <int D, int MODE>
 struct Bwd {
   static constexpr int KD = D / 64;
   static constexpr bool DK = (MODE == BWD_DK);
-  static constexpr int NS = 2;
+  static constexpr int NS = NSTAGE;
   static constexpr int K_BYTES = BK * D * 2;   // one copy of the key tile
   static constexpr int Q_BYTES = BQ * D * 2;   // one copy of a query tile
   static constexpr int STAGE = (DK ? 3 : 2) * Q_BYTES;  // Q hi, Q lo (, Go)
@@ -52,18 +56,21 @@ struct Bwd {
 
 struct BwdBars {
   uint64_t k_full, v_full;
-  uint64_t q_full[2], q_empty[2];
+  uint64_t q_full[NSTAGE], q_empty[NSTAGE];
   uint64_t sd_full[2], sd_free[2];
   uint64_t ds_full[2];
   uint64_t done;
   uint32_t tmem;
   int abort;
-  float lse2[2][BQ];   // row lse in log2 units (+inf for rows outside the problem)
-  float del[2][BQ];
+  float lse2[NSTAGE][BQ];   // row lse in log2 units (+inf for rows outside the problem)
+  float del[NSTAGE][BQ];
+  float imp[BK];       // COLSUM: warpgroup 1's partial importance
 };
 
+__device__ __forceinline__ void rows_sync() { asm volatile("bar.sync 1, 256;" ::: "memory"); }
+
 template <int D, int MODE>
-__global__ void __launch_bounds__(192, 1)
+__global__ void __launch_bounds__(NTHREADS, 1)
     k_attn_bwd(const __grid_constant__ CUtensorMap mKh, const __grid_constant__ CUtensorMap mKl,
                const __grid_constant__ CUtensorMap mQh, const __grid_constant__ CUtensorMap mQl,
                const __grid_constant__ CUtensorMap mG, BwdArgs a) {
@@ -84,10 +91,12 @@ __global__ void __launch_bounds__(192, 1)
 
   if (tid == 0) {
     mbar_init(&bars.k_full, 1);
-    mbar_init(&bars.v_full, BK);
-    for (int i = 0; i < 2; ++i) {
+    mbar_init(&bars.v_full, 2 * BK);
+    for (int i = 0; i < NSTAGE; ++i) {
       mbar_init(&bars.q_full[i], 1);
       mbar_init(&bars.q_empty[i], 1 + BK);
+    }
+    for (int i = 0; i < 2; ++i) {
       mbar_init(&bars.sd_full[i], 1);
       mbar_init(&bars.sd_free[i], C::DK ? 1 : BK);
       mbar_init(&bars.ds_full[i], BK);
@@ -96,14 +105,14 @@ __global__ void __launch_bounds__(192, 1)
     bars.abort = 0;
     fence_barrier_init();
   }
-  if (warp == 5) tmem_alloc(&bars.tmem, C::TMEM_COLS);
+  if (warp == 9) tmem_alloc(&bars.tmem, C::TMEM_COLS);
   fence_before_sync();
   __syncthreads();
   fence_after_sync();
   const uint32_t tmem = bars.tmem;
   volatile int *abort = &bars.abort;
 
-  if (warp == 4) {
+  if (warp == 8) {
     // ------------------------------------------------------------ producer
     if (lane == 0) {
       const int krow = (int)(k_begin + k0);
@@ -149,7 +158,7 @@ __global__ void __launch_bounds__(192, 1)
       for (int i = (issued > C::NS ? issued - C::NS : 0); i < issued; ++i)
         mbar_wait(&bars.q_full[i % C::NS], (i / C::NS) & 1);
     }
-  } else if (warp == 5) {
+  } else if (warp == 9) {
     // ------------------------------------------------------------- MMA issuer
     if (lane == 0) {
       const uint32_t id_s = idesc_bf16(BK, BQ, false, false);
@@ -157,18 +166,19 @@ __global__ void __launch_bounds__(192, 1)
       bool ok = mbar_wait(&bars.k_full, 0, abort);
       if (C::DK) ok = ok && mbar_wait(&bars.v_full, 0, abort);
       fence_after_sync();
-      const uint32_t aKh = smem_u32(sm), aKl = aKh + C::K_BYTES;
+      const uint64_t kh0 = sdesc(smem_u32(sm), 16, 1024), kl0 = sdesc_add(kh0, C::K_BYTES);
       const uint32_t tv_hi = tmem + C::COL_V, tv_lo = tmem + C::COL_V + D / 2;
       auto issue_dk = [&](int i) -> bool {
         const int db = i & 1;
         if (!mbar_wait(&bars.ds_full[db], (i >> 1) & 1, abort)) return false;
         fence_after_sync();
-        const uint32_t qb = smem_u32(sm + C::OFF_ST + (i % C::NS) * C::STAGE);
+        const uint64_t qh0 = sdesc(smem_u32(sm + C::OFF_ST + (i % C::NS) * C::STAGE), BQ * 128,
+                                   1024);
+        const uint64_t ql0 = sdesc_add(qh0, C::Q_BYTES);
         const uint32_t tds = tmem + db * BQ;  // dS hi at +0, lo at +32 columns
 #pragma unroll
         for (int kk = 0; kk < BQ / 16; ++kk) {
-          const uint64_t qh = sdesc(qb + kk * 2048, BQ * 128, 1024);
-          const uint64_t ql = sdesc(qb + C::Q_BYTES + kk * 2048, BQ * 128, 1024);
+          const uint64_t qh = sdesc_add(qh0, kk * 2048), ql = sdesc_add(ql0, kk * 2048);
           mma_bf16_ts(tmem + C::COL_DK, tds + kk * 8, qh, id_dk, (i > 0 || kk > 0) ? 1u : 0u);
           mma_bf16_ts(tmem + C::COL_DK, tds + kk * 8, ql, id_dk, 1u);
           mma_bf16_ts(tmem + C::COL_DK, tds + 32 + kk * 8, qh, id_dk, 1u);
@@ -182,18 +192,19 @@ __global__ void __launch_bounds__(192, 1)
         if (!mbar_wait(&bars.q_full[st], (i / C::NS) & 1, abort)) { ok = false; break; }
         if (i >= 2 && !mbar_wait(&bars.sd_free[sb], ((i >> 1) - 1) & 1, abort)) { ok = false; break; }
         fence_after_sync();
-        const uint32_t qb = smem_u32(sm + C::OFF_ST + st * C::STAGE);
+        const uint64_t qh0 = sdesc(smem_u32(sm + C::OFF_ST + st * C::STAGE), 16, 1024);
+        const uint64_t ql0 = sdesc_add(qh0, C::Q_BYTES), gd0 = sdesc_add(qh0, 2 * C::Q_BYTES);
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
           const uint32_t ok_ = (kk >> 2) * (BK * 128) + (kk & 3) * 32;
           const uint32_t oq = (kk >> 2) * (BQ * 128) + (kk & 3) * 32;
-          const uint64_t kh = sdesc(aKh + ok_, 16, 1024), kl = sdesc(aKl + ok_, 16, 1024);
-          const uint64_t qh = sdesc(qb + oq, 16, 1024), ql = sdesc(qb + C::Q_BYTES + oq, 16, 1024);
+          const uint64_t kh = sdesc_add(kh0, ok_), kl = sdesc_add(kl0, ok_);
+          const uint64_t qh = sdesc_add(qh0, oq), ql = sdesc_add(ql0, oq);
           mma_bf16(tmem + sb * BQ, kh, qh, id_s, kk > 0 ? 1u : 0u);
           mma_bf16(tmem + sb * BQ, kl, qh, id_s, 1u);
           mma_bf16(tmem + sb * BQ, kh, ql, id_s, 1u);
           if (C::DK) {
-            const uint64_t gd = sdesc(qb + 2 * C::Q_BYTES + oq, 16, 1024);
+            const uint64_t gd = sdesc_add(gd0, oq);
             mma_bf16_ts(tmem + C::COL_DP + sb * BQ, tv_hi + kk * 8, gd, id_s, kk > 0 ? 1u : 0u);
             mma_bf16_ts(tmem + C::COL_DP + sb * BQ, tv_lo + kk * 8, gd, id_s, 1u);
           }
@@ -209,16 +220,18 @@ __global__ void __launch_bounds__(192, 1)
     }
   } else {
     // --------------------------------------------------------- key rows
-    const int row = tid;
+    const int wg = warp >> 2;  // warpgroup: query tiles i with i % 2 == wg
+    const int row = tid & (BK - 1);
     const int kr = k0 + row;
     const bool kvalid = kr < nk;
-    const uint32_t lane_base = (uint32_t)(warp * 32) << 16;
+    const uint32_t lane_base = (uint32_t)((warp & 3) * 32) << 16;
     if (C::DK) {
-      // the value row (hi, lo) into tensor memory as the A operand of dP^T = V Go^T
+      // this warpgroup's half of the value row (hi, lo) into tensor memory: the A
+      // operand of dP^T = V Go^T
       const uint4 *vh = reinterpret_cast<const uint4 *>(a.v_hi + (k_begin + kr) * D);
       const uint4 *vl = reinterpret_cast<const uint4 *>(a.v_lo + (k_begin + kr) * D);
 #pragma unroll 1
-      for (int c0 = 0; c0 < D / 2; c0 += 32) {
+      for (int c0 = wg * 32; c0 < D / 2; c0 += 64) {
         uint32_t wh[32], wl[32];
 #pragma unroll
         for (int e = 0; e < 8; ++e) {
@@ -237,7 +250,7 @@ __global__ void __launch_bounds__(192, 1)
     const float sl2 = a.scale * L2E;
     float imp = 0.f;
     bool ok = true;
-    for (int i = 0; i < nqt; ++i) {
+    for (int i = wg; i < nqt; i += 2) {
       const int sb = i & 1, st = i % C::NS;
       ok = __all_sync(0xffffffffu, mbar_wait(&bars.sd_full[sb], (i >> 1) & 1, abort));
       // the tile's l and delta were staged by the producer lanes: acquire them directly
@@ -284,7 +297,7 @@ __global__ void __launch_bounds__(192, 1)
       if (!mbar_wait(&bars.done, 0, abort)) *abort = 1;
       fence_after_sync();
 #pragma unroll 1
-      for (int c0 = 0; c0 < D; c0 += 32) {
+      for (int c0 = wg * (D / 2); c0 < (wg + 1) * (D / 2); c0 += 32) {
         float o[32];
         tmem_ld32(tmem + lane_base + C::COL_DK + c0, o);
         if (kvalid) {
@@ -295,13 +308,15 @@ __global__ void __launch_bounds__(192, 1)
                                  o[4 * e + 2] * a.scale, o[4 * e + 3] * a.scale);
         }
       }
-    } else if (kvalid) {
-      a.imp[k_begin + kr] = imp;
+    } else {
+      if (wg == 1) bars.imp[row] = imp;
+      rows_sync();
+      if (wg == 0 && kvalid) a.imp[k_begin + kr] = imp + bars.imp[row];
     }
   }
   fence_before_sync();
   __syncthreads();
-  if (warp == 5) {
+  if (warp == 9) {
     fence_after_sync();
     tmem_dealloc(tmem, C::TMEM_COLS);
   }
@@ -316,7 +331,7 @@ int launch_bwd_tc(const BwdMaps &m, const BwdArgs &a, int max_tiles, int B, cuda
   static_assert(C::SMEM + sizeof(BwdBars) <= 232448, "shared memory");
   auto kern = k_attn_bwd<D, MODE>;
   KVS_CUDA_TRY(set_smem_once(kern, C::SMEM));
-  kern<<<dim3(max_tiles, B), 192, C::SMEM, st>>>(m.kh, m.kl, m.qh, m.ql, m.g, a);
+  kern<<<dim3(max_tiles, B), NTHREADS, C::SMEM, st>>>(m.kh, m.kl, m.qh, m.ql, m.g, a);
   KVS_LAUNCH_CHECK("k_attn_bwd");
   return KVS_OK;
 }

@@ -8,17 +8,21 @@
 // problem's keys in tiles of 64.  Every product keeps about 16 significant
 // bits through a bf16 hi/lo split, with fp32 accumulation in tensor memory:
 //   S = Q K^T     Q_hi K_hi + Q_hi K_lo + Q_lo K_hi   (Q in TMEM, K in smem)
-//   online softmax, one thread per query row, lazy rescaling of O
+//   online softmax, one thread per query row and warpgroup, lazy rescaling
 //   O += P V      P_hi V_hi + P_hi V_lo + P_lo V_hi   (P in TMEM over S, V in smem)
-// Tensor memory (512 columns): S/P buffers at 0 and 64, O at 128, Q hi/lo at 256.
+// Two row warpgroups take alternate key tiles, each with its own running
+// max / sum and its own O accumulator; the two are merged at the end by their
+// log-sum-exp (the same identity that merges chunks of a cache).
+// Tensor memory (512 columns): S/P buffers at 0 and 64 (tile parity), O of
+// warpgroup g at 128 + g*D, Q hi/lo after them.
 // Modes:
 //   LOSS     keys K_c, values V_c: writes l_hat, Go = dL/dY_hat (bf16),
 //            delta = Go . Y_hat - dL/dl_hat (with the rounded Go), loss partials
 //   TARGETS  keys K_z, values V_z: writes Y (fp32 and bf16 hi/lo) and l
 //   STATS    row log-sum-exp only
 //   WRITE_A  given l_hat: writes A = exp(S - l_hat) as bf16 hi/lo
-// Warp roles: warps 0-3 softmax/epilogue (thread t <-> TMEM lane t <-> query
-// row t), warp 4 TMA producer, warp 5 TMEM allocator and MMA issuer.
+// Warp roles: warps 0-7 rows (warp w <-> TMEM lanes 32 (w % 4) ..), warp 8 TMA
+// producer, warp 9 TMEM allocator and MMA issuer.
 #include <math.h>
 
 #include "kvs_attn_tc.cuh"
@@ -30,6 +34,7 @@ using namespace tc;
 
 constexpr int BM = 128;          // queries per CTA
 constexpr int BN = 64;           // keys per tile
+constexpr int NTHREADS = 320;
 constexpr float kRescale = 8.f;  // lazy rescale threshold (log2 units)
 constexpr float L2E = 1.4426950408889634f;
 
@@ -44,8 +49,8 @@ struct Fwd {
   static constexpr int BYTES = NS * STAGE;
   static constexpr int SMEM = BYTES + 1024;
   static constexpr uint32_t TMEM_COLS = 512;
-  static constexpr uint32_t COL_O = 128;
-  static constexpr uint32_t COL_Q = 256;      // Q hi at +0, Q lo at +D/2
+  static constexpr uint32_t COL_O = 128;            // O of warpgroup g at COL_O + g * D
+  static constexpr uint32_t COL_Q = COL_O + 2 * D;  // Q hi at +0, Q lo at +D/2
 };
 
 struct FwdBars {
@@ -56,11 +61,15 @@ struct FwdBars {
   uint64_t o_done;
   uint32_t tmem;
   int abort;
-  float red[8];
+  float m2[2][BM], l[2][BM];  // per warpgroup running max (log2) and sum
+  float part[2][BM][2];       // per warpgroup half-row sums: |Yh - Y|^2, Go . Yh
+  float red[16];
 };
 
+__device__ __forceinline__ void rows_sync() { asm volatile("bar.sync 1, 256;" ::: "memory"); }
+
 template <int D, int MODE>
-__global__ void __launch_bounds__(192, 1)
+__global__ void __launch_bounds__(NTHREADS, 1)
     k_attn_fwd(const __grid_constant__ CUtensorMap mKh, const __grid_constant__ CUtensorMap mKl,
                const __grid_constant__ CUtensorMap mVh, const __grid_constant__ CUtensorMap mVl,
                FwdArgs a) {
@@ -80,7 +89,7 @@ __global__ void __launch_bounds__(192, 1)
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
 
   if (tid == 0) {
-    mbar_init(&bars.q_full, BM);
+    mbar_init(&bars.q_full, 2 * BM);
     for (int i = 0; i < C::NS; ++i) {
       mbar_init(&bars.kv_full[i], 1);
       mbar_init(&bars.kv_empty[i], 1);
@@ -94,14 +103,14 @@ __global__ void __launch_bounds__(192, 1)
     bars.abort = 0;
     fence_barrier_init();
   }
-  if (warp == 5) tmem_alloc(&bars.tmem, C::TMEM_COLS);
+  if (warp == 9) tmem_alloc(&bars.tmem, C::TMEM_COLS);
   fence_before_sync();
   __syncthreads();
   fence_after_sync();
   const uint32_t tmem = bars.tmem;
   volatile int *abort = &bars.abort;
 
-  if (warp == 4) {
+  if (warp == 8) {
     // ------------------------------------------------------------ TMA producer
     if (lane == 0) {
       tma_prefetch_map(&mKh);
@@ -129,7 +138,7 @@ __global__ void __launch_bounds__(192, 1)
         for (int j = (issued > C::NS ? issued - C::NS : 0); j < issued; ++j)
           mbar_wait(&bars.kv_full[j % C::NS], (j / C::NS) & 1);
     }
-  } else if (warp == 5) {
+  } else if (warp == 9) {
     // ------------------------------------------------------------- MMA issuer
     if (lane == 0) {
       const uint32_t id_s = idesc_bf16(BM, BN, false, false);
@@ -141,15 +150,17 @@ __global__ void __launch_bounds__(192, 1)
         const int pb = i & 1;
         if (!mbar_wait(&bars.p_full[pb], (i >> 1) & 1, abort)) return false;
         fence_after_sync();
-        const uint32_t vb = smem_u32(sm + (i % C::NS) * C::STAGE + 2 * C::T_BYTES);
-        const uint32_t tp = tmem + pb * BN;  // P hi at +0, P lo at +32 columns
+        const uint64_t vh0 = sdesc(smem_u32(sm + (i % C::NS) * C::STAGE + 2 * C::T_BYTES),
+                                   BN * 128, 1024);
+        const uint64_t vl0 = sdesc_add(vh0, C::T_BYTES);
+        const uint32_t tp = tmem + pb * BN;            // P hi at +0, P lo at +32 columns
+        const uint32_t to = tmem + C::COL_O + pb * D;  // O of the tile's warpgroup
 #pragma unroll
         for (int kk = 0; kk < BN / 16; ++kk) {
-          const uint64_t vh = sdesc(vb + kk * 2048, BN * 128, 1024);
-          const uint64_t vl = sdesc(vb + C::T_BYTES + kk * 2048, BN * 128, 1024);
-          mma_bf16_ts(tmem + C::COL_O, tp + kk * 8, vh, id_pv, (i > 0 || kk > 0) ? 1u : 0u);
-          mma_bf16_ts(tmem + C::COL_O, tp + kk * 8, vl, id_pv, 1u);
-          mma_bf16_ts(tmem + C::COL_O, tp + 32 + kk * 8, vh, id_pv, 1u);
+          const uint64_t vh = sdesc_add(vh0, kk * 2048), vl = sdesc_add(vl0, kk * 2048);
+          mma_bf16_ts(to, tp + kk * 8, vh, id_pv, (i > 1 || kk > 0) ? 1u : 0u);
+          mma_bf16_ts(to, tp + kk * 8, vl, id_pv, 1u);
+          mma_bf16_ts(to, tp + 32 + kk * 8, vh, id_pv, 1u);
         }
         mma_commit(&bars.kv_empty[i % C::NS]);
         mma_commit(&bars.s_free[pb]);
@@ -160,12 +171,12 @@ __global__ void __launch_bounds__(192, 1)
         if (!mbar_wait(&bars.kv_full[st], (j / C::NS) & 1, abort)) { ok = false; break; }
         if (j >= 2 && !mbar_wait(&bars.s_free[sb], ((j >> 1) - 1) & 1, abort)) { ok = false; break; }
         fence_after_sync();
-        const uint32_t kb = smem_u32(sm + st * C::STAGE);
+        const uint64_t kh0 = sdesc(smem_u32(sm + st * C::STAGE), 16, 1024);
+        const uint64_t kl0 = sdesc_add(kh0, C::T_BYTES);
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
           const uint32_t off_k = (kk >> 2) * (BN * 128) + (kk & 3) * 32;
-          const uint64_t kh = sdesc(kb + off_k, 16, 1024);
-          const uint64_t kl = sdesc(kb + C::T_BYTES + off_k, 16, 1024);
+          const uint64_t kh = sdesc_add(kh0, off_k), kl = sdesc_add(kl0, off_k);
           mma_bf16_ts(tmem + sb * BN, tq_hi + kk * 8, kh, id_s, kk > 0 ? 1u : 0u);
           mma_bf16_ts(tmem + sb * BN, tq_hi + kk * 8, kl, id_s, 1u);
           mma_bf16_ts(tmem + sb * BN, tq_lo + kk * 8, kh, id_s, 1u);
@@ -180,17 +191,19 @@ __global__ void __launch_bounds__(192, 1)
       mbar_wait(&bars.o_done, 0);  // every MMA of this CTA has completed
     }
   } else {
-    // ------------------------------------------------- softmax / epilogue rows
-    const int row = tid;  // 0..127
+    // ------------------------------------------------------------ row warps
+    const int wg = warp >> 2;  // warpgroup: tiles j with j % 2 == wg
+    const int row = tid & (BM - 1);
     const int q = q0 + row;
     const bool valid = q < nq;
-    const uint32_t lane_base = (uint32_t)(warp * 32) << 16;
-    // the query row (hi, lo) into tensor memory as the A operand of S = Q K^T
+    const uint32_t lane_base = (uint32_t)((warp & 3) * 32) << 16;
     {
+      // this warpgroup's half of the query row (hi, lo) into tensor memory:
+      // the A operand of S = Q K^T
       const uint4 *qh = reinterpret_cast<const uint4 *>(a.q_hi + (q_begin + q) * D);
       const uint4 *ql = reinterpret_cast<const uint4 *>(a.q_lo + (q_begin + q) * D);
 #pragma unroll 1
-      for (int c0 = 0; c0 < D / 2; c0 += 32) {
+      for (int c0 = wg * 32; c0 < D / 2; c0 += 64) {
         uint32_t vh[32], vl[32];
 #pragma unroll
         for (int e = 0; e < 8; ++e) {
@@ -211,7 +224,7 @@ __global__ void __launch_bounds__(192, 1)
     if (MODE == FWD_WRITE_A && valid) lrow2 = a.lse_in[q_begin + q] * L2E;
     float mref = -INFINITY, lsum = 0.f;
     bool ok = true;
-    for (int j = 0; j < ntiles; ++j) {
+    for (int j = wg; j < ntiles; j += 2) {
       const int sb = j & 1;
       ok = __all_sync(0xffffffffu, mbar_wait(&bars.s_full[sb], (j >> 1) & 1, abort));
       if (!ok) break;
@@ -220,14 +233,16 @@ __global__ void __launch_bounds__(192, 1)
       tmem_ld32(tmem + lane_base + sb * BN, s);
       tmem_ld32(tmem + lane_base + sb * BN + 32, s + 32);
       const int kvalid = nk - j * BN;
+      if (kvalid < BN) {
 #pragma unroll
-      for (int c = 0; c < BN; ++c) s[c] = (c < kvalid) ? s[c] * sl2 : -INFINITY;
+        for (int c = 0; c < BN; ++c) s[c] = (c < kvalid) ? s[c] : -INFINITY;
+      }
       if (!C::PV) {
         fence_before_sync();
         mbar_arrive(&bars.s_free[sb]);
       }
       if (MODE == FWD_WRITE_A) {
-        // A = exp2(t - lse2), split into bf16 hi / lo, into the padded A buffer
+        // A = exp2(s sl2 - lse2), split into bf16 hi / lo, into the padded A buffer
         const int64_t arow = a.a_pad_off[b] + q0 + row;
         uint4 *dh = reinterpret_cast<uint4 *>(a.a_hi + arow * a.ld_a + j * BN);
         uint4 *dl = reinterpret_cast<uint4 *>(a.a_lo + arow * a.ld_a + j * BN);
@@ -236,8 +251,8 @@ __global__ void __launch_bounds__(192, 1)
           uint32_t h[4], l[4];
 #pragma unroll
           for (int e = 0; e < 4; ++e) {
-            const float p0 = valid ? exp2f(s[ch * 8 + 2 * e] - lrow2) : 0.f;
-            const float p1 = valid ? exp2f(s[ch * 8 + 2 * e + 1] - lrow2) : 0.f;
+            const float p0 = valid ? exp2f(fmaf(s[ch * 8 + 2 * e], sl2, -lrow2)) : 0.f;
+            const float p1 = valid ? exp2f(fmaf(s[ch * 8 + 2 * e + 1], sl2, -lrow2)) : 0.f;
             split_pack(p0, p1, h[e], l[e]);
           }
           dh[ch] = make_uint4(h[0], h[1], h[2], h[3]);
@@ -248,6 +263,7 @@ __global__ void __launch_bounds__(192, 1)
       float mt = -INFINITY;
 #pragma unroll
       for (int c = 0; c < BN; ++c) mt = fmaxf(mt, s[c]);
+      mt *= sl2;
       float alpha = 1.f;
       bool rescale = false;
       if (mt > mref + kRescale || mref == -INFINITY) {
@@ -261,31 +277,29 @@ __global__ void __launch_bounds__(192, 1)
       float ts = 0.f;
 #pragma unroll
       for (int c = 0; c < BN; ++c) {
-        s[c] = exp2f(s[c] - mref);
+        s[c] = exp2f(fmaf(s[c], sl2, -mref));
         ts += s[c];
       }
       lsum = lsum * alpha + ts;
       if (C::PV) {
-        // P (hi, lo) over the S buffer: the A operand of O += P V
+        // P (hi, lo) over the S buffer: the A operand of O_wg += P V
         uint32_t ph[32], pl[32];
 #pragma unroll
         for (int c = 0; c < 32; ++c) split_pack(s[2 * c], s[2 * c + 1], ph[c], pl[c]);
         tmem_st32u(tmem + lane_base + sb * BN, ph);
         tmem_st32u(tmem + lane_base + sb * BN + 32, pl);
         if (__any_sync(0xffffffffu, rescale)) {
-          // O *= alpha once PV of tile j-1 has landed (PV of tile j waits for p_full);
-          // the TMEM access is warp-wide, rows without a new max use alpha = 1.
-          const int pj = j - 1;
-          ok = __all_sync(0xffffffffu, mbar_wait(&bars.s_free[pj & 1], (pj >> 1) & 1, abort));
-          if (!ok) break;
-          fence_after_sync();
+          // O_wg *= alpha.  Its last update, PV of tile j-2, was issued before S of
+          // tile j, whose completion this warp has observed, so O_wg is settled.
+          // The TMEM access is warp-wide: rows without a new max use alpha = 1.
+          const uint32_t to = tmem + lane_base + C::COL_O + wg * D;
 #pragma unroll 1
           for (int c0 = 0; c0 < D; c0 += 32) {
             float o[32];
-            tmem_ld32(tmem + lane_base + C::COL_O + c0, o);
+            tmem_ld32(to + c0, o);
 #pragma unroll
             for (int e = 0; e < 32; ++e) o[e] *= alpha;
-            tmem_st32(tmem + lane_base + C::COL_O + c0, o);
+            tmem_st32(to + c0, o);
           }
         }
         tmem_wait_st();
@@ -296,24 +310,37 @@ __global__ void __launch_bounds__(192, 1)
     if (!ok) *abort = 1;
     // ------------------------------------------------------------ epilogue
     if (MODE != FWD_WRITE_A) {
-      const float lse = (mref + log2f(lsum)) * 0.6931471805599453f;
+      // merge the two warpgroups' statistics: m = max(m0, m1), l = sum l_g 2^(m_g - m)
+      bars.m2[wg][row] = mref;
+      bars.l[wg][row] = lsum;
+      rows_sync();
+      const float m0 = bars.m2[0][row], m1 = bars.m2[1][row];
+      const float mm = fmaxf(m0, m1);
+      const float e0 = (m0 == -INFINITY) ? 0.f : exp2f(m0 - mm);
+      const float e1 = (m1 == -INFINITY) ? 0.f : exp2f(m1 - mm);
+      const float ltot = bars.l[0][row] * e0 + bars.l[1][row] * e1;
+      const float lse = (mm + log2f(ltot)) * 0.6931471805599453f;
       if (C::PV) {
         if (!mbar_wait(&bars.o_done, 0, abort)) *abort = 1;
         fence_after_sync();
       }
-      const float inv = 1.f / lsum;
+      const float inv = 1.f / ltot;
+      const float w0 = e0 * inv, w1 = e1 * inv;  // weights of O_0 and O_1
+      const bool has1 = ntiles > 1;              // O_1 holds data
       const float c_out = 2.f * a.w_out / ((float)nq * (float)D);
       const float c_lse = 2.f * a.w_lse / (float)nq;
       const int64_t grow = q_begin + q;
-      float se = 0.f, ls = 0.f, gy = 0.f;
+      float se = 0.f, gy = 0.f;
       if (C::PV) {
+        // this warpgroup's half of the row's columns
 #pragma unroll 1
-        for (int c0 = 0; c0 < D; c0 += 32) {
-          float o[32];
+        for (int c0 = wg * (D / 2); c0 < (wg + 1) * (D / 2); c0 += 32) {
+          float o[32], o1[32];
           tmem_ld32(tmem + lane_base + C::COL_O + c0, o);
+          tmem_ld32(tmem + lane_base + C::COL_O + D + c0, o1);
           if (!valid) continue;
 #pragma unroll
-          for (int e = 0; e < 32; ++e) o[e] *= inv;
+          for (int e = 0; e < 32; ++e) o[e] = o[e] * w0 + (has1 ? o1[e] * w1 : 0.f);
           if (MODE == FWD_TARGETS) {
             float4 *y4 = reinterpret_cast<float4 *>(a.y_out + grow * D + c0);
 #pragma unroll
@@ -363,34 +390,44 @@ __global__ void __launch_bounds__(192, 1)
           }
         }
       }
-      if (valid) {
-        a.lse_out[grow] = lse;
-        if (MODE == FWD_LOSS) {
-          const float el = lse - a.lse_in[grow];
-          ls = el * el;
-          a.delta[grow] = gy - c_lse * el;
-        }
-      }
       if (MODE == FWD_LOSS) {
-        // deterministic per-CTA partial sums of the two loss terms
-        se = warp_sum(se);
-        ls = warp_sum(ls);
-        if (lane == 0) {
-          bars.red[warp] = se;
-          bars.red[4 + warp] = ls;
+        bars.part[wg][row][0] = se;
+        bars.part[wg][row][1] = gy;
+        rows_sync();
+        if (wg == 0) {
+          float ls = 0.f;
+          se = bars.part[0][row][0] + bars.part[1][row][0];
+          gy = bars.part[0][row][1] + bars.part[1][row][1];
+          if (valid) {
+            const float el = lse - a.lse_in[grow];
+            ls = el * el;
+            a.lse_out[grow] = lse;
+            a.delta[grow] = gy - c_lse * el;
+          } else {
+            se = 0.f;
+          }
+          // deterministic per-CTA partial sums of the two loss terms
+          se = warp_sum(se);
+          ls = warp_sum(ls);
+          if (lane == 0) {
+            bars.red[warp] = se;
+            bars.red[4 + warp] = ls;
+          }
         }
-        asm volatile("bar.sync 1, 128;" ::: "memory");
-        if (row == 0) {
+        rows_sync();
+        if (tid == 0) {
           float *part = a.partials + ((int64_t)b * a.tiles_per_problem + blockIdx.x) * 2;
           part[0] = (bars.red[0] + bars.red[1]) + (bars.red[2] + bars.red[3]);
           part[1] = (bars.red[4] + bars.red[5]) + (bars.red[6] + bars.red[7]);
         }
+      } else if (wg == 0 && valid) {  // TARGETS, STATS
+        a.lse_out[grow] = lse;
       }
     }
   }
   fence_before_sync();
   __syncthreads();
-  if (warp == 5) {
+  if (warp == 9) {
     fence_after_sync();
     tmem_dealloc(tmem, C::TMEM_COLS);
   }
@@ -405,7 +442,7 @@ int launch_fwd_tc(const FwdMaps &m, const FwdArgs &a, int max_tiles, int B, cuda
   static_assert(C::SMEM + sizeof(FwdBars) <= 232448, "shared memory");
   auto kern = k_attn_fwd<D, MODE>;
   KVS_CUDA_TRY(set_smem_once(kern, C::SMEM));
-  kern<<<dim3(max_tiles, B), 192, C::SMEM, st>>>(m.kh, m.kl, m.vh, m.vl, a);
+  kern<<<dim3(max_tiles, B), NTHREADS, C::SMEM, st>>>(m.kh, m.kl, m.vh, m.vl, a);
   KVS_LAUNCH_CHECK("k_attn_fwd");
   return KVS_OK;
 }

@@ -115,14 +115,13 @@ __global__ void __launch_bounds__(192, 1)
         const int st = i % NS;
         if (!mbar_wait(&bars.full[st], (i / NS) & 1, abort)) { ok = false; break; }
         fence_after_sync();
-        const uint32_t base = smem_u32(sm + st * STAGE);
+        const uint64_t d0 = sdesc(smem_u32(sm + st * STAGE), TKQ * 128, 1024);
 #pragma unroll
         for (int kk = 0; kk < TKQ / 16; ++kk) {
-          const uint32_t o = kk * 2048;
-          const uint64_t ah = sdesc(base + o, TKQ * 128, 1024);
-          const uint64_t al = sdesc(base + OP_BYTES + o, TKQ * 128, 1024);
-          const uint64_t bh = sdesc(base + 2 * OP_BYTES + o, TKQ * 128, 1024);
-          const uint64_t bl = sdesc(base + 3 * OP_BYTES + o, TKQ * 128, 1024);
+          const uint64_t ah = sdesc_add(d0, kk * 2048);
+          const uint64_t al = sdesc_add(ah, OP_BYTES);
+          const uint64_t bh = sdesc_add(ah, 2 * OP_BYTES);
+          const uint64_t bl = sdesc_add(ah, 3 * OP_BYTES);
           mma_bf16(tmem, ah, bh, id, (i > 0 || kk > 0) ? 1u : 0u);
           mma_bf16(tmem, ah, bl, id, 1u);
           mma_bf16(tmem, al, bh, id, 1u);

@@ -168,6 +168,12 @@ __device__ __forceinline__ uint64_t sdesc(uint32_t saddr, uint32_t lbo, uint32_t
   return d;
 }
 
+// Descriptor of the same tile `bytes` further on (shared addresses are below
+// 256 KB, so the 14-bit address field never carries into the next field).
+__device__ __forceinline__ uint64_t sdesc_add(uint64_t desc, uint32_t bytes) {
+  return desc + (uint64_t)(bytes >> 4);
+}
+
 // Instruction descriptor: bf16 x bf16 -> f32, dense, shape M x N.
 __host__ __device__ constexpr uint32_t idesc_bf16(int M, int N, bool a_mn, bool b_mn) {
   return (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)a_mn << 15) | ((uint32_t)b_mn << 16) |
@@ -236,13 +242,15 @@ __device__ __forceinline__ void split_bf16(float x, __nv_bfloat16 &hi, __nv_bflo
   lo = __float2bfloat16_rn(x - __bfloat162float(hi));
 }
 
-// Packed hi and lo words of the pair (a, b): a in the low half.
+// Packed hi and lo words of the pair (a, b): a in the low half; hi = rn(x),
+// lo = rn(x - hi) with packed conversions.
 __device__ __forceinline__ void split_pack(float a, float b, uint32_t &hi, uint32_t &lo) {
-  __nv_bfloat16 ha, la, hb, lb;
-  split_bf16(a, ha, la);
-  split_bf16(b, hb, lb);
-  hi = (uint32_t)__bfloat16_as_ushort(ha) | ((uint32_t)__bfloat16_as_ushort(hb) << 16);
-  lo = (uint32_t)__bfloat16_as_ushort(la) | ((uint32_t)__bfloat16_as_ushort(lb) << 16);
+  const __nv_bfloat162 h = __floats2bfloat162_rn(a, b);
+  const uint32_t hw = *reinterpret_cast<const uint32_t *>(&h);
+  const float ha = __uint_as_float(hw << 16), hb = __uint_as_float(hw & 0xffff0000u);
+  const __nv_bfloat162 l = __floats2bfloat162_rn(a - ha, b - hb);
+  hi = hw;
+  lo = *reinterpret_cast<const uint32_t *>(&l);
 }
 
 // Byte offset of 16-byte chunk `chunk` of row `row` in a 128-byte-swizzled tile.
