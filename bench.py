@@ -111,13 +111,18 @@ class ClockSampler:
 
 # ---------------------------------------------------------------- GPU arm
 
+def group_size(group):
+    import torch.distributed as dist
+    return dist.get_world_size(group)
+
+
 class Job:
     """Device buffers of one rank's batch and the calls of one step."""
 
-    def __init__(self, wl, seq, dev):
+    def __init__(self, wl, seq, dev, group=None):
         import torch
         import kv_cache_compression_kvsculpt_b200 as K
-        self.K, self.torch, self.wl = K, torch, wl
+        self.K, self.torch, self.wl, self.group = K, torch, wl, group
         ids = [(seq, l, h) for l in range(wl.n_layers) for h in range(wl.n_kv_heads)]
         self.bt = W.make_batch(wl, 0, ids)
         B = self.bt.B
@@ -134,6 +139,8 @@ class Job:
         self.spec = K.QuerySpec(B, wl.d, wl.g, wl.m_q, wl.n_syn, wl.N, wl.rope_base)
         self.sched = K.Schedule(outer=wl.outer, steps=wl.steps, history=wl.history, lam=wl.lam,
                                 w_out=wl.w_out, w_lse=wl.w_lse)
+        self.pilot = K.Schedule(outer=wl.pilot_outer, steps=wl.pilot_steps, history=wl.history,
+                                lam=wl.lam, w_out=wl.w_out, w_lse=wl.w_lse)
         self.Q = torch.empty((self.batch.sum_q, wl.d), device=dev)
         self.Kc = torch.empty((self.batch.sum_c, wl.d), device=dev)
         self.Vc = torch.empty_like(self.Kc)
@@ -142,6 +149,7 @@ class Job:
         self.status = torch.empty(B, dtype=torch.int32, device=dev)
         self.ws = K.alloc_workspace(self.batch, device=dev)
         self.state = K.alloc_state(self.batch, wl.history, device=dev)
+        self.total = wl.k * B * (1 if group is None else group_size(group))
         self.out_host = {"Kc": torch.empty(self.Kc.shape).pin_memory(),
                          "Vc": torch.empty(self.Vc.shape).pin_memory()}
 
@@ -149,6 +157,17 @@ class Job:
         K = self.K
         d = d or self.dev
         K.kvs_build_queries(self.spec, d["q_retain"], d["q_ctx"], d["pos"], self.Q)
+        if self.wl.adaptive:
+            # pilot at uniform k, pooled allocation (one all-gather over ranks), full solve
+            from kv_cache_compression_kvsculpt_b200 import adaptive
+            r = adaptive.compress_adaptive(self.wl.d, self.bt.q_off, self.bt.z_off, self.Q,
+                                           d["Kz"], d["Vz"], self.total, self.sched, self.pilot,
+                                           group=self.group)
+            self.Kc, self.Vc, self.trace, self.parts, self.status = (
+                r["Kc"], r["Vc"], r["trace"], r["parts"], r["status"])
+            self.batch = K.KvsBatch(self.wl.d, self.bt.q_off, self.bt.z_off, r["c_off"])
+            self.k_alloc = r["k"]
+            return
         K.kvs_compress_batch(self.batch, self.sched, self.Q, d["Kz"], d["Vz"], self.Kc, self.Vc,
                              None, self.trace, self.parts, self.status, self.state, self.ws)
 
@@ -193,12 +212,14 @@ def loss_grad_roofline(job, peaks, reps=20):
     B = job.batch.B
     Y = torch.empty_like(job.Q)
     lse = torch.empty(job.batch.sum_q, device=job.Q.device)
-    K.kvs_targets(job.batch, job.Q, job.dev["Kz"], job.dev["Vz"], Y, lse, None, job.ws)
+    K.kvs_targets(job.batch, job.Q, job.dev["Kz"], job.dev["Vz"], Y, lse, None,
+                  K.alloc_workspace(job.batch))
     loss = torch.empty(B, device=job.Q.device)
     dK = torch.empty_like(job.Kc)
+    ws = K.alloc_workspace(job.batch)  # sized for the batch's (possibly allocated) k
 
     def ev():
-        K.kvs_loss_grad(job.batch, job.Q, job.Kc, job.Vc, Y, lse, 1.0, 1.0, loss, None, dK, job.ws)
+        K.kvs_loss_grad(job.batch, job.Q, job.Kc, job.Vc, Y, lse, 1.0, 1.0, loss, None, dK, ws)
 
     for _ in range(3):
         ev()
@@ -225,7 +246,7 @@ def run_gpu(args):
     wl = W.WORKLOADS[args.workload]
     if args.outer is not None:
         wl = wl.with_(outer=args.outer)
-    job = Job(wl, seq=rank, dev="cuda")
+    job = Job(wl, seq=rank, dev="cuda", group=dist.group.WORLD if dist else None)
     for _ in range(args.warmup):
         job.step()
     torch.cuda.synchronize()
@@ -326,6 +347,10 @@ def oracle_sample(wl, budget_s, pid=(0, 0, 0)):
     sample = (f"1 problem {pid} of {wl.name}: query build, targets, top-k, first fit, then "
               f"{done} of {wl.outer} outer iterations ({wl.steps} L-BFGS steps + re-fit each) "
               f"timed; per-problem time extrapolated to the full schedule")
+    if wl.adaptive:
+        # the pilot repeats the setup and runs pilot_outer outer iterations at uniform k
+        total += t_setup + t_outer * wl.pilot_outer * wl.pilot_steps / wl.steps
+        sample += f", plus a {wl.pilot_outer}x{wl.pilot_steps} pilot extrapolated the same way"
     return total, sample
 
 

@@ -204,7 +204,11 @@ int kvs_lbfgs_step(const kvs_batch *batch, const kvs_schedule *sched, const floa
  * sched->outer times { sched->steps L-BFGS steps; ridge re-fit }.
  * Outputs Kc, Vc [sum k_b, d]; idx (nullable) [sum k_b] the top-k positions;
  * loss_trace (nullable) [B, outer+1] the loss after every fit; parts
- * (nullable) [B, 2] final unweighted output-MSE and LSE-MSE; status [B]. */
+ * (nullable) [B, 2] final unweighted output-MSE and LSE-MSE; status [B].
+ * After its first step each L-BFGS step runs as one CUDA graph whose trial
+ * loop is a conditional node; with the environment variable
+ * KVS_STEP_GRAPHS=0 (read once per process) the same kernels are launched
+ * one by one instead, for kernel-level profilers. */
 int kvs_compress_batch(const kvs_batch *batch, const kvs_schedule *sched, const float *Q,
                        const float *Kz, const float *Vz, float *Kc, float *Vc, int32_t *idx,
                        float *loss_trace, float *parts, int32_t *status,

@@ -1,5 +1,6 @@
 // C ABI of the KVSculpt library: argument validation, workspace layout and
 // the orchestration of the kernels for each call (see include/kvsculpt.h).
+#include <stdlib.h>
 #include <math.h>
 #include <stdio.h>
 #include <string.h>
@@ -70,6 +71,7 @@ int geom_from_batch(const kvs_batch *b, HostGeom *g, bool need_c) {
   for (int bb = 0; bb < b->B; ++bb)
     g->sum_qpad += align_up(b->q_off_h[bb + 1] - b->q_off_h[bb], 128);
   g->ld_a = align_up(std::max(g->max_c, 1), 128);
+  g->ld_g = align_up(std::max(g->max_c, 1), 4);
   return KVS_OK;
 }
 
@@ -104,8 +106,9 @@ size_t carve_work(const HostGeom &g, void *base, Work *w) {
   w->delta = c.take<float>(g.sum_q);
   w->partials = c.take<float>((int64_t)g.B * ((g.max_q + 127) / 128) * 2);
   w->a_pad_off = c.take<int64_t>(g.B + 1);
-  w->gram = c.take<float>(g.sum_c * g.max_c);
+  w->gram = c.take<float>(g.sum_c * g.ld_g);
   w->R = c.take<float>(g.sum_c * g.d);
+  w->X = c.take<float>(g.sum_c * g.d);
   w->chol_t = c.take<float>((int64_t)g.B * ((g.max_c + 63) / 64) * 64 * 64);
   w->dead = c.take<int>(g.B);
   w->fbuf = c.take<float>(g.B);
@@ -122,6 +125,11 @@ size_t carve_state(const HostGeom &g, int h, void *base, State *s) {
   Carver c{static_cast<char *>(base)};
   const int64_t n = g.sum_c * g.d;
   s->sc = c.take<LbfgsScal>(g.B);
+  s->gram = c.take<LbfgsGram>(g.B);
+  s->dc = c.take<DirCoef>(g.B);
+  s->cmax = (int)(((int64_t)g.max_c * g.d + LBFGS_CHUNK - 1) / LBFGS_CHUNK);
+  s->part = c.take<float>((int64_t)g.B * s->cmax * LBFGS_NDOT);
+  s->ticket = c.take<int>(g.B);
   s->x = c.take<float>(n);
   s->g = c.take<float>(n);
   s->dir = c.take<float>(n);
@@ -475,9 +483,15 @@ int kvs_compress_batch(const kvs_batch *batch, const kvs_schedule *sched, const 
   if (loss_trace && (rc = launch_copy_f(Bt, s, loss_trace, tstride, 0))) return rc;
   StepGraph sg;
   bool have_graph = false;
+  // KVS_STEP_GRAPHS=0 launches every kernel of a step individually (the same
+  // arithmetic; kernel profilers do not look inside graphs with conditional nodes)
+  static const bool use_graphs = [] {
+    const char *e = getenv("KVS_STEP_GRAPHS");
+    return !(e && e[0] == '0');
+  }();
   for (int o = 0; o < sc.outer; ++o) {
     for (int t = 0; t < sc.steps; ++t) {
-      if (!have_graph && o + t > 0) {
+      if (use_graphs && !have_graph && o + t > 0) {
         // every kernel has been launched once outside capture: record the step now
         if ((rc = build_step_graph(Bt, sc, Q, w.Yt, w.lset, Vc, Kc, s, status, w, &sg))) return rc;
         have_graph = true;

@@ -315,7 +315,7 @@ int fit_d(const Batch &Bt, const float *Q, const float *Kc, const float *Y, floa
   ga.n_fixed = 0;
   ga.b_row_off = w.a_pad_off;
   ga.c = w.gram;
-  ga.ldc = g.max_c;
+  ga.ldc = g.ld_g;
   ga.diag = lam;
   ga.err = w.err;
   const int tm = (g.max_c + 127) / 128;

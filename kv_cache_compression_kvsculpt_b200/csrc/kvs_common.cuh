@@ -71,6 +71,7 @@ struct HostGeom {
   int max_q = 0, max_z = 0, max_c = 0;
   int64_t sum_qpad = 0;  // sum over problems of n_q rounded up to 128
   int64_t ld_a = 0;      // columns of the attention-weight buffer (max_c rounded up to 128)
+  int64_t ld_g = 0;      // columns of the Gram / factor buffer (max_c rounded up to 4)
 };
 
 int geom_from_batch(const kvs_batch *b, HostGeom *g, bool need_c);

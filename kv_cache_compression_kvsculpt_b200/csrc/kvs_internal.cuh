@@ -37,8 +37,9 @@ struct Work {
   float *delta;              // [sum_q]
   float *partials;           // [B, max q tiles, 2]    per-CTA loss sums
   int64_t *a_pad_off;        // [B+1]                  padded row offsets of ahi/alo
-  float *gram;               // [sum_c, max_c]         A^T A + lam I, then its Cholesky factor
-  float *R;                  // [sum_c, d]             A^T Y, then the solution
+  float *gram;               // [sum_c, ld_g]          A^T A + lam I, then its Cholesky factor
+  float *R;                  // [sum_c, d]             A^T Y, then the forward-solved rows
+  float *X;                  // [sum_c, d]             solution of the ridge system
   float *chol_t;             // [B, panels, 64, 64]    inverses of the diagonal blocks
   int *dead;                 // [B]                    factorisation failed
   float *fbuf;               // [B]                    loss scratch
@@ -51,8 +52,31 @@ struct Work {
 };
 
 // Persistent L-BFGS state carved from the caller's state buffer.
+// Inner products of the stored pairs, indexed by ring slot: sy[i][j] = s_i . y_j
+// (filled for s older than y and on the diagonal), yy[i][j] = y_i . y_j.
+struct LbfgsGram {
+  double sy[16][16];
+  double yy[16][16];
+};
+
+// The next search direction as a combination d = cg g + sum_p (cy[p] y_p + cs[p] s_p)
+// over the cnt newest pairs (p = 0 newest), with g . d and the first trial step.
+struct DirCoef {
+  float cg, gtd, t0;
+  int cnt;
+  float cy[16], cs[16];
+};
+
+constexpr int LBFGS_CHUNK = 2048;  // elements of a problem's vector per CTA
+constexpr int LBFGS_NDOT = 65;     // inner products one CTA reports (h <= 15)
+
 struct State {
   LbfgsScal *sc;   // [B]
+  LbfgsGram *gram; // [B]
+  DirCoef *dc;     // [B]
+  float *part;     // [B][cmax][LBFGS_NDOT] per-CTA partial inner products
+  int *ticket;     // [B] CTAs of the current pass that have finished
+  int cmax;        // chunks of the longest problem
   float *x;        // [sum_c*d] accepted keys
   float *g;        // [sum_c*d] gradient at x
   float *dir;      // [sum_c*d] search direction

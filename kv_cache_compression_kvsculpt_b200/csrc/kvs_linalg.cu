@@ -6,16 +6,18 @@
 // Right-looking blocked algorithm over panels of NB = 64 columns, float32,
 // every problem of the batch advancing together so that all SMs share the work:
 //   per panel j:
-//     diag    factor the diagonal block G_jj = L_jj L_jj^T in shared memory and
-//             keep T_j = L_jj^-1
-//     tmul    forward-solved rows y_j = T_j r_j
+//     diag    factor the diagonal block G_jj = L_jj L_jj^T in shared memory,
+//             keep T_j = L_jj^-1 and forward-solve its rows y_j = T_j r_j
 //     panel   L_ij = G_ij T_j^T for the rows below
 //     update  G_ik -= L_ij L_kj^T on the trailing lower triangle and
-//             r_i -= L_ij y_j on the right-hand sides (64 x 64 register tiles)
-//   then per panel from the last one: x_j = T_j^T y_j and y_i -= L_ji^T x_j.
-// The factor overwrites the Gram matrix, the solution the right-hand sides.
-// A pivot <= 0 (or non-finite) marks the problem KVS_ST_NOT_PD; its V_c is
-// left untouched and its remaining steps are skipped.
+//             r_i -= L_ij y_j on the right-hand sides
+//   then per panel from the last one: x_j = T_j^T y_j, y_i -= L_ji^T x_j.
+// Every 64 x 64 product runs from shared memory with 4 x 4 register tiles and
+// 128-bit shared loads.  The factor overwrites the Gram matrix, the forward
+// sweep the right-hand sides; the solution goes to a separate buffer and is
+// copied to V_c only when finite.  A pivot <= 0 (or non-finite) marks the
+// problem KVS_ST_NOT_PD; its V_c is left untouched and its remaining steps
+// are skipped.
 #include <math.h>
 
 #include "kvs_internal.cuh"
@@ -24,73 +26,163 @@ namespace kvs {
 namespace {
 
 constexpr int NB = 64;
+constexpr int SP = NB + 4;  // shared row stride (floats): 16-byte rows, conflict-free columns
+constexpr int DEAD_NOT_PD = 1, DEAD_NONFINITE = 2;
 
 struct CholArgs {
   float *G;              // [sum_c, ld] Gram matrix -> factor (lower triangle)
-  float *R;              // [sum_c, d] right-hand sides -> solution
+  float *R;              // [sum_c, d] right-hand sides -> forward-solved rows
+  float *X;              // [sum_c, d] solution
   float *T;              // [B, npanel, NB, NB] inverses of the diagonal blocks
   int npanel;
-  int *dead;             // [B] set once a problem's factorisation failed
+  int *dead;             // [B] DEAD_* bits
   int32_t *status;
   const int64_t *c_off;
-  int64_t ld;
-  int d;
+  int64_t ld;            // multiple of 4
+  int d;                 // 64 or 128
 };
 
 __device__ __forceinline__ int kdim(const CholArgs &a, int b) {
   return (int)(a.c_off[b + 1] - a.c_off[b]);
 }
 
-// Diagonal block of panel j0: factor in shared memory and keep its inverse T_j.
+__device__ __forceinline__ float4 ld4(const float *p) { return *reinterpret_cast<const float4 *>(p); }
+
+// S[r][c] = M[r0 + r][c0 + c] for r0 + r < rmax, c0 + c < cmax, else 0
+// (M row-major with ld a multiple of 4 and c0 a multiple of 4).
+__device__ __forceinline__ void load_tile(float (*S)[SP], const float *M, int64_t ld, int r0,
+                                          int rmax, int c0, int cmax) {
+  for (int e = threadIdx.x; e < NB * NB / 4; e += blockDim.x) {
+    const int r = e >> 4, c = (e & 15) * 4;
+    float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
+    if (r0 + r < rmax && c0 + c < cmax) {
+      v = ld4(M + (int64_t)(r0 + r) * ld + c0 + c);
+      const int m = cmax - c0 - c;  // valid lanes of the vector
+      if (m < 4) {
+        v.w = 0.f;
+        if (m < 3) v.z = 0.f;
+        if (m < 2) v.y = 0.f;
+      }
+    }
+    *reinterpret_cast<float4 *>(&S[r][c]) = v;
+  }
+}
+
+// Transposed: S[c][r] = M[r0 + r][c0 + c], same bounds.
+__device__ __forceinline__ void load_tile_t(float (*S)[SP], const float *M, int64_t ld, int r0,
+                                            int rmax, int c0, int cmax) {
+  for (int e = threadIdx.x; e < NB * NB / 4; e += blockDim.x) {
+    const int r = e >> 4, c = (e & 15) * 4;
+    float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
+    if (r0 + r < rmax && c0 + c < cmax) v = ld4(M + (int64_t)(r0 + r) * ld + c0 + c);
+    const int m = cmax - c0 - c;
+    S[c][r] = m > 0 ? v.x : 0.f;
+    S[c + 1][r] = m > 1 ? v.y : 0.f;
+    S[c + 2][r] = m > 2 ? v.z : 0.f;
+    S[c + 3][r] = m > 3 ? v.w : 0.f;
+  }
+}
+
+// acc[i][j] += sum_t A[ty + 16 i][t] * B[tx + 16 j][t], t ascending
+__device__ __forceinline__ void mm64(const float (*A)[SP], const float (*B)[SP], float acc[4][4],
+                                     int tx, int ty) {
+#pragma unroll 2
+  for (int t = 0; t < NB; t += 4) {
+    float4 av[4], bv[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) av[i] = *reinterpret_cast<const float4 *>(&A[ty + 16 * i][t]);
+#pragma unroll
+    for (int j = 0; j < 4; ++j) bv[j] = *reinterpret_cast<const float4 *>(&B[tx + 16 * j][t]);
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        float s = acc[i][j];
+        s = fmaf(av[i].x, bv[j].x, s);
+        s = fmaf(av[i].y, bv[j].y, s);
+        s = fmaf(av[i].z, bv[j].z, s);
+        acc[i][j] = fmaf(av[i].w, bv[j].w, s);
+      }
+  }
+}
+
+__device__ __forceinline__ void zero_acc(float acc[4][4]) {
+#pragma unroll
+  for (int i = 0; i < 4; ++i)
+#pragma unroll
+    for (int j = 0; j < 4; ++j) acc[i][j] = 0.f;
+}
+
+// Diagonal block of panel j0: factor in shared memory, keep T_j = L_jj^-1 and
+// forward-solve the block's rows of the right-hand sides, y_j = T_j r_j.
 __global__ void __launch_bounds__(256) k_chol_diag(CholArgs a, int j0) {
   const int b = blockIdx.x;
   const int k = kdim(a, b);
   if (j0 >= k || a.dead[b]) return;
   const int jb = min(NB, k - j0);
-  __shared__ float L[NB][NB + 1];
-  __shared__ float Ti[NB][NB + 1];
+  __shared__ __align__(16) float L[NB][SP];   // the block; later the right-hand side tile
+  __shared__ __align__(16) float Ts[NB][SP];  // T_j
+  __shared__ float dsq[NB];
   __shared__ int bad;
   float *G = a.G + (a.c_off[b] + j0) * a.ld + j0;
   const int tid = threadIdx.x;
   if (tid == 0) bad = 0;
-  for (int e = tid; e < NB * NB; e += blockDim.x) {
-    const int r = e / NB, c = e % NB;
-    L[r][c] = (r < jb && c <= r) ? G[(int64_t)r * a.ld + c] : 0.f;
-    Ti[r][c] = 0.f;
+  load_tile(L, G, a.ld, 0, jb, 0, jb);
+  for (int e = tid; e < NB * SP; e += blockDim.x) (&Ts[0][0])[e] = 0.f;
+  __syncthreads();
+  // Unnormalised elimination: after step c, column c holds l_ic * sqrt(p_c) and
+  // L[c][c] = p_c, the pivot; the trailing block loses l_i l_j^T = L_ic L_jc / p_c.
+  // Thread (i, q) owns row i = tid / 4 at the columns j = q + 4 m.
+  {
+    const int i = tid >> 2, q = tid & 3;
+    for (int c = 0; c < jb - 1; ++c) {
+      if (i > c && i < jb) {
+        const float lic = L[i][c] / L[c][c];
+        const int m0 = (c + 1 - q + 3) >> 2;  // first m with q + 4 m > c
+#pragma unroll 4
+        for (int m = m0; m < 16; ++m) {
+          const int j = q + 4 * m;
+          if (j > i) break;
+          L[i][j] = fmaf(-lic, L[j][c], L[i][j]);
+        }
+      }
+      __syncthreads();
+    }
+  }
+  if (tid < jb) {
+    const float p = L[tid][tid];
+    if (!(p > 0.f) || !isfinite(p)) atomicOr(&bad, 1);
+    dsq[tid] = sqrtf(fmaxf(p, 1e-30f));
   }
   __syncthreads();
-  for (int c = 0; c < jb; ++c) {
-    if (tid == 0) {
-      const float piv = L[c][c];
-      if (!(piv > 0.f) || !isfinite(piv)) bad = 1;
-      L[c][c] = sqrtf(fmaxf(piv, 1e-30f));
-    }
-    __syncthreads();
-    const float inv = 1.f / L[c][c];
-    for (int i = c + 1 + tid; i < jb; i += blockDim.x) L[i][c] *= inv;
-    __syncthreads();
-    const int n = jb - c - 1;
-    for (int e = tid; e < n * n; e += blockDim.x) {
-      const int i = c + 1 + e / n, j = c + 1 + e % n;
-      if (j <= i) L[i][j] -= L[i][c] * L[j][c];
-    }
-    __syncthreads();
-  }
   if (bad) {
     if (tid == 0) {
       a.status[b] |= KVS_ST_NOT_PD;
-      a.dead[b] = 1;
+      a.dead[b] = DEAD_NOT_PD;
     }
     return;
   }
-  // T = L^-1 (lower triangular), one column per thread
-  if (tid < jb) {
-    const int c = tid;
-    Ti[c][c] = 1.f / L[c][c];
-    for (int i = c + 1; i < jb; ++i) {
+  for (int e = tid; e < jb * jb; e += blockDim.x) {
+    const int r = e / jb, c = e % jb;
+    if (c < r) L[r][c] /= dsq[c];
+    else if (c == r) L[r][c] = dsq[c];
+  }
+  __syncthreads();
+  // T = L^-1 column by column: warp w owns columns 8w .. 8w+7, four lanes per
+  // column split each row's dot product; T[i][cc] = -(sum_t L[i][t] T[t][cc]) / L[i][i].
+  if (tid < jb) Ts[tid][tid] = 1.f / L[tid][tid];
+  __syncthreads();
+  {
+    const int warp = tid >> 5, lane = tid & 31;
+    const int cc = warp * 8 + (lane >> 2), q = lane & 3;
+    for (int i = 1; i < jb; ++i) {
       float s = 0.f;
-      for (int t = c; t < i; ++t) s = fmaf(L[i][t], Ti[t][c], s);
-      Ti[i][c] = -s / L[i][i];
+      if (i > cc)
+        for (int t = cc + q; t < i; t += 4) s = fmaf(L[i][t], Ts[t][cc], s);
+      s += __shfl_xor_sync(0xffffffffu, s, 1);
+      s += __shfl_xor_sync(0xffffffffu, s, 2);
+      if (i > cc && q == 0) Ts[i][cc] = -s * Ts[i][i];
+      __syncwarp();
     }
   }
   __syncthreads();
@@ -98,61 +190,30 @@ __global__ void __launch_bounds__(256) k_chol_diag(CholArgs a, int j0) {
   for (int e = tid; e < NB * NB; e += blockDim.x) {
     const int r = e / NB, c = e % NB;
     if (r < jb && c <= r) G[(int64_t)r * a.ld + c] = L[r][c];
-    Tg[e] = Ti[r][c];
-  }
-}
-
-// Rows j0 .. j0+63 of the right-hand sides times T_j (forward sweep) or T_j^T
-// (backward sweep), in place; 64 columns of R per CTA, 4 x 4 register tiles.
-__global__ void __launch_bounds__(256) k_chol_tmul(CholArgs a, int j0, int transpose) {
-  const int b = blockIdx.y;
-  const int k = kdim(a, b);
-  if (j0 >= k || a.dead[b]) return;
-  const int jb = min(NB, k - j0);
-  const int c0 = blockIdx.x * NB;
-  if (c0 >= a.d) return;
-  __shared__ float Ts[NB][NB + 4];  // Ts[r][t] = M[r][t]
-  __shared__ float Xs[NB][NB + 4];  // Xs[col][t] = R[j0 + t][c0 + col]
-  const float *Tg = a.T + ((int64_t)b * a.npanel + j0 / NB) * NB * NB;
-  float *R = a.R + (a.c_off[b] + j0) * a.d + c0;
-  const int tid = threadIdx.x;
-  for (int e = tid; e < NB * NB; e += blockDim.x) {
-    const int r = e / NB, t = e % NB;
-    Ts[r][t] = transpose ? Tg[t * NB + r] : Tg[e];
-    Xs[t][r] = (r < jb && c0 + t < a.d) ? R[(int64_t)r * a.d + t] : 0.f;
+    Tg[e] = Ts[r][c];
   }
   __syncthreads();
+  // y_j = T_j r_j, 64 right-hand-side columns at a time (the tile reuses L)
   const int tx = tid & 15, ty = tid >> 4;
-  float acc[4][4];
+  float *R = a.R + (a.c_off[b] + j0) * a.d;
+  for (int c0 = 0; c0 < a.d; c0 += NB) {
+    load_tile_t(L, R, a.d, 0, jb, c0, a.d);  // L[col][t] = r[t][c0 + col]
+    __syncthreads();
+    float acc[4][4];
+    zero_acc(acc);
+    mm64(Ts, L, acc, tx, ty);
 #pragma unroll
-  for (int i = 0; i < 4; ++i)
+    for (int i = 0; i < 4; ++i) {
+      const int r = ty + 16 * i;
+      if (r >= jb) continue;
 #pragma unroll
-    for (int j = 0; j < 4; ++j) acc[i][j] = 0.f;
-#pragma unroll 8
-  for (int t = 0; t < NB; ++t) {
-    float av[4], bv[4];
-#pragma unroll
-    for (int i = 0; i < 4; ++i) av[i] = Ts[ty + 16 * i][t];
-#pragma unroll
-    for (int j = 0; j < 4; ++j) bv[j] = Xs[tx + 16 * j][t];
-#pragma unroll
-    for (int i = 0; i < 4; ++i)
-#pragma unroll
-      for (int j = 0; j < 4; ++j) acc[i][j] = fmaf(av[i], bv[j], acc[i][j]);
-  }
-#pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    const int r = ty + 16 * i;
-    if (r >= jb) continue;
-#pragma unroll
-    for (int j = 0; j < 4; ++j) {
-      const int col = tx + 16 * j;
-      if (c0 + col < a.d) R[(int64_t)r * a.d + col] = acc[i][j];
+      for (int j = 0; j < 4; ++j) R[(int64_t)r * a.d + c0 + tx + 16 * j] = acc[i][j];
     }
+    __syncthreads();
   }
 }
 
-// L_ij = G_ij T^T for 64 rows of the panel below the diagonal block.
+// L_ij = G_ij T_j^T for 64 rows of the panel below the diagonal block.
 __global__ void __launch_bounds__(256) k_chol_panel(CholArgs a, int j0) {
   const int b = blockIdx.y;
   const int k = kdim(a, b);
@@ -160,28 +221,36 @@ __global__ void __launch_bounds__(256) k_chol_panel(CholArgs a, int j0) {
   const int jb = min(NB, k - j0);
   const int i0 = j0 + jb + blockIdx.x * NB;
   if (i0 >= k) return;
-  const int ib = min(NB, k - i0);
-  __shared__ float Ti[NB][NB + 1];
-  __shared__ float Ar[NB][NB + 1];
+  __shared__ __align__(16) float Ar[NB][SP];
+  __shared__ __align__(16) float Ts[NB][SP];
   const int tid = threadIdx.x;
-  float *P = a.G + (a.c_off[b] + i0) * a.ld + j0;
-  for (int e = tid; e < NB * NB; e += blockDim.x) {
-    const int r = e / NB, c = e % NB;
-    Ti[r][c] = a.T[((int64_t)b * a.npanel + j0 / NB) * NB * NB + e];
-    Ar[r][c] = (r < ib && c < jb) ? P[(int64_t)r * a.ld + c] : 0.f;
+  const int64_t row0 = a.c_off[b];
+  load_tile(Ar, a.G + row0 * a.ld, a.ld, i0, k, j0, j0 + jb);
+  const float *Tg = a.T + ((int64_t)b * a.npanel + j0 / NB) * NB * NB;
+  for (int e = tid; e < NB * NB / 4; e += blockDim.x) {
+    const int r = e >> 4, c = (e & 15) * 4;
+    *reinterpret_cast<float4 *>(&Ts[r][c]) = ld4(Tg + r * NB + c);
   }
   __syncthreads();
-  for (int e = tid; e < ib * jb; e += blockDim.x) {
-    const int r = e / jb, c = e % jb;
-    float s = 0.f;
-    for (int t = 0; t <= c; ++t) s = fmaf(Ar[r][t], Ti[c][t], s);
-    P[(int64_t)r * a.ld + c] = s;
+  const int tx = tid & 15, ty = tid >> 4;
+  float acc[4][4];
+  zero_acc(acc);
+  mm64(Ar, Ts, acc, tx, ty);  // sum_t G[r][t] T[col][t]
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const int r = i0 + ty + 16 * i;
+    if (r >= k) continue;
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const int c = tx + 16 * j;
+      if (c < jb) a.G[(row0 + r) * a.ld + j0 + c] = acc[i][j];
+    }
   }
 }
 
 // Trailing update: tiles (ti >= tj) of G_ik -= L_i L_k^T, and tiles of
 // r_i -= L_i y_j (columns of R in chunks of 64), 64 x 64 outputs per CTA.
-__global__ void __launch_bounds__(256) k_chol_update(CholArgs a, int j0, int ntile_max) {
+__global__ void __launch_bounds__(256) k_chol_update(CholArgs a, int j0) {
   const int b = blockIdx.y;
   const int k = kdim(a, b);
   if (j0 >= k || a.dead[b]) return;
@@ -191,7 +260,7 @@ __global__ void __launch_bounds__(256) k_chol_update(CholArgs a, int j0, int nti
   if (n2 <= 0) return;
   const int nt = (n2 + NB - 1) / NB;
   const int ntri = nt * (nt + 1) / 2;
-  const int ndc = (a.d + NB - 1) / NB;
+  const int ndc = a.d / NB;
   int t = blockIdx.x;
   bool rhs = false;
   int ti, tj;
@@ -207,42 +276,38 @@ __global__ void __launch_bounds__(256) k_chol_update(CholArgs a, int j0, int nti
     ti = t / ndc;
     tj = t % ndc;
   }
-  __shared__ float As[NB][NB + 4];  // L_i panel rows, [row][c]
-  __shared__ float Bs[NB][NB + 4];  // L_k panel rows or y_j, [row or col][c]
+  __shared__ __align__(16) float As[NB][SP];  // L_i panel rows, [row][c]
+  __shared__ __align__(16) float Bs[NB][SP];  // L_k panel rows [row][c], or y_j as [col][c]
   const int tid = threadIdx.x;
+  const int tx = tid & 15, ty = tid >> 4;
   const int64_t row0 = a.c_off[b];
   const int ri = s0 + ti * NB;
-  for (int e = tid; e < NB * NB; e += blockDim.x) {
-    const int r = e / NB, c = e % NB;
-    As[r][c] = (ri + r < k && c < jb) ? a.G[(row0 + ri + r) * a.ld + j0 + c] : 0.f;
-    if (!rhs) {
-      const int rk = s0 + tj * NB + r;
-      Bs[r][c] = (rk < k && c < jb) ? a.G[(row0 + rk) * a.ld + j0 + c] : 0.f;
-    } else {
-      // Bs[col][c] = y_j[c][col]
-      const int col = tj * NB + r;
-      Bs[r][c] = (col < a.d && c < jb) ? a.R[(row0 + j0 + c) * a.d + col] : 0.f;
+  // the outputs' current values first: their loads overlap the tile loads
+  float cur[4][4];
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const int r = ri + ty + 16 * i;
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      cur[i][j] = 0.f;
+      if (r >= k) continue;
+      if (!rhs) {
+        const int cc = s0 + tj * NB + tx + 16 * j;
+        if (cc <= r) cur[i][j] = a.G[(row0 + r) * a.ld + cc];
+      } else {
+        cur[i][j] = a.R[(row0 + r) * a.d + tj * NB + tx + 16 * j];
+      }
     }
   }
+  load_tile(As, a.G + row0 * a.ld, a.ld, ri, k, j0, j0 + jb);
+  if (!rhs)
+    load_tile(Bs, a.G + row0 * a.ld, a.ld, s0 + tj * NB, k, j0, j0 + jb);
+  else
+    load_tile_t(Bs, a.R + row0 * a.d, a.d, j0, j0 + jb, tj * NB, a.d);
   __syncthreads();
-  const int tx = tid & 15, ty = tid >> 4;
   float acc[4][4];
-#pragma unroll
-  for (int i = 0; i < 4; ++i)
-#pragma unroll
-    for (int j = 0; j < 4; ++j) acc[i][j] = 0.f;
-#pragma unroll 8
-  for (int c = 0; c < NB; ++c) {
-    float av[4], bv[4];
-#pragma unroll
-    for (int i = 0; i < 4; ++i) av[i] = As[ty + 16 * i][c];
-#pragma unroll
-    for (int j = 0; j < 4; ++j) bv[j] = Bs[tx + 16 * j][c];
-#pragma unroll
-    for (int i = 0; i < 4; ++i)
-#pragma unroll
-      for (int j = 0; j < 4; ++j) acc[i][j] = fmaf(av[i], bv[j], acc[i][j]);
-  }
+  zero_acc(acc);
+  mm64(As, Bs, acc, tx, ty);
 #pragma unroll
   for (int i = 0; i < 4; ++i) {
     const int r = ri + ty + 16 * i;
@@ -251,80 +316,96 @@ __global__ void __launch_bounds__(256) k_chol_update(CholArgs a, int j0, int nti
     for (int j = 0; j < 4; ++j) {
       if (!rhs) {
         const int cc = s0 + tj * NB + tx + 16 * j;
-        if (cc < k && cc <= r) a.G[(row0 + r) * a.ld + cc] -= acc[i][j];
+        if (cc <= r) a.G[(row0 + r) * a.ld + cc] = cur[i][j] - acc[i][j];
       } else {
-        const int col = tj * NB + tx + 16 * j;
-        if (col < a.d) a.R[(row0 + r) * a.d + col] -= acc[i][j];
+        a.R[(row0 + r) * a.d + tj * NB + tx + 16 * j] = cur[i][j] - acc[i][j];
       }
     }
   }
 }
 
-// Backward sweep update: y_i -= L_ji^T x_j for the rows i < j0 (64 x 64 tiles).
-__global__ void __launch_bounds__(256) k_chol_bupdate(CholArgs a, int j0) {
+// Backward sweep at panel j0: x_j = T_j^T y_j (each CTA forms it for its 64
+// right-hand-side columns; the CTAs of row block 0 store it and check it is
+// finite), then y_i -= L_ji^T x_j for the row block i < j0 of this CTA.
+__global__ void __launch_bounds__(256) k_chol_bsolve(CholArgs a, int j0) {
   const int b = blockIdx.z;
   const int k = kdim(a, b);
   if (j0 >= k || a.dead[b]) return;
   const int jb = min(NB, k - j0);
   const int i0 = blockIdx.y * NB;
-  if (i0 >= j0) return;
+  if (i0 > 0 && i0 >= j0) return;
   const int c0 = blockIdx.x * NB;
-  if (c0 >= a.d) return;
-  __shared__ float As[NB][NB + 4];  // As[i][t] = L[j0 + t][i0 + i]
-  __shared__ float Bs[NB][NB + 4];  // Bs[col][t] = x[t][c0 + col]
+  __shared__ __align__(16) float As[NB][SP];
+  __shared__ __align__(16) float Bs[NB][SP];
   const int tid = threadIdx.x;
-  const int64_t row0 = a.c_off[b];
-  for (int e = tid; e < NB * NB; e += blockDim.x) {
-    const int t = e / NB, u = e % NB;
-    As[u][t] = (t < jb && i0 + u < j0) ? a.G[(row0 + j0 + t) * a.ld + i0 + u] : 0.f;
-    Bs[u][t] = (t < jb && c0 + u < a.d) ? a.R[(row0 + j0 + t) * a.d + c0 + u] : 0.f;
-  }
-  __syncthreads();
   const int tx = tid & 15, ty = tid >> 4;
+  const int64_t row0 = a.c_off[b];
+  const float *Tg = a.T + ((int64_t)b * a.npanel + j0 / NB) * NB * NB;
+  load_tile_t(As, Tg, NB, 0, NB, 0, NB);                         // As[r][t] = T[t][r]
+  load_tile_t(Bs, a.R + row0 * a.d, a.d, j0, j0 + jb, c0, a.d);  // Bs[col][t] = y[t][col]
+  __syncthreads();
   float acc[4][4];
+  zero_acc(acc);
+  mm64(As, Bs, acc, tx, ty);  // x[r][col]
+  if (blockIdx.y == 0) {
+    bool fin = true;
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const int r = ty + 16 * i;
+      if (r >= jb) continue;
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        a.X[(row0 + j0 + r) * a.d + c0 + tx + 16 * j] = acc[i][j];
+        fin &= isfinite(acc[i][j]);
+      }
+    }
+    if (!fin) atomicOr(&a.dead[b], DEAD_NONFINITE);
+  }
+  if (j0 == 0) return;
+  __syncthreads();
+  // Bs[col][t] = x[t][col]; As[r][t] = L[j0 + t][i0 + r]
 #pragma unroll
   for (int i = 0; i < 4; ++i)
 #pragma unroll
-    for (int j = 0; j < 4; ++j) acc[i][j] = 0.f;
-#pragma unroll 8
-  for (int t = 0; t < NB; ++t) {
-    float av[4], bv[4];
+    for (int j = 0; j < 4; ++j) Bs[tx + 16 * j][ty + 16 * i] = acc[i][j];
+  load_tile_t(As, a.G + row0 * a.ld, a.ld, j0, j0 + jb, i0, j0);
+  float cur[4][4];
 #pragma unroll
-    for (int i = 0; i < 4; ++i) av[i] = As[ty + 16 * i][t];
+  for (int i = 0; i < 4; ++i)
 #pragma unroll
-    for (int j = 0; j < 4; ++j) bv[j] = Bs[tx + 16 * j][t];
-#pragma unroll
-    for (int i = 0; i < 4; ++i)
-#pragma unroll
-      for (int j = 0; j < 4; ++j) acc[i][j] = fmaf(av[i], bv[j], acc[i][j]);
-  }
+    for (int j = 0; j < 4; ++j) {
+      const int r = i0 + ty + 16 * i;
+      cur[i][j] = r < j0 ? a.R[(row0 + r) * a.d + c0 + tx + 16 * j] : 0.f;
+    }
+  __syncthreads();
+  zero_acc(acc);
+  mm64(As, Bs, acc, tx, ty);
 #pragma unroll
   for (int i = 0; i < 4; ++i) {
     const int r = i0 + ty + 16 * i;
     if (r >= j0) continue;
 #pragma unroll
-    for (int j = 0; j < 4; ++j) {
-      const int col = c0 + tx + 16 * j;
-      if (col < a.d) a.R[(row0 + r) * a.d + col] -= acc[i][j];
-    }
+    for (int j = 0; j < 4; ++j)
+      a.R[(row0 + r) * a.d + c0 + tx + 16 * j] = cur[i][j] - acc[i][j];
   }
 }
 
-// V_c <- solution for the problems whose factorisation succeeded and is finite.
+// V_c <- solution for the problems whose factorisation succeeded and whose
+// solution is finite; the others keep V_c and get their status bit.
 __global__ void __launch_bounds__(256) k_chol_store(CholArgs a, float *Vc) {
-  const int b = blockIdx.x;
-  if (a.dead[b]) return;
-  const int64_t n = (int64_t)kdim(a, b) * a.d;
-  const float *X = a.R + a.c_off[b] * a.d;
-  bool finite = true;
-  for (int64_t e = threadIdx.x; e < n; e += blockDim.x) finite &= isfinite(X[e]);
-  finite = __syncthreads_and(finite);
-  if (!finite) {
-    if (threadIdx.x == 0) a.status[b] |= KVS_ST_NONFINITE;
+  const int b = blockIdx.y;
+  const int dead = a.dead[b];
+  if (dead) {
+    if (blockIdx.x == 0 && threadIdx.x == 0 && (dead & DEAD_NONFINITE))
+      a.status[b] |= KVS_ST_NONFINITE;
     return;
   }
-  float *V = Vc + a.c_off[b] * a.d;
-  for (int64_t e = threadIdx.x; e < n; e += blockDim.x) V[e] = X[e];
+  const int64_t n4 = (int64_t)kdim(a, b) * a.d / 4;
+  const float4 *X = reinterpret_cast<const float4 *>(a.X + a.c_off[b] * a.d);
+  float4 *V = reinterpret_cast<float4 *>(Vc + a.c_off[b] * a.d);
+  for (int64_t e = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; e < n4;
+       e += (int64_t)gridDim.x * blockDim.x)
+    V[e] = X[e];
 }
 
 }  // namespace
@@ -332,32 +413,28 @@ __global__ void __launch_bounds__(256) k_chol_store(CholArgs a, float *Vc) {
 int launch_chol_solve(const Batch &Bt, float *Vc, int32_t *status, const Work &w) {
   const HostGeom &g = Bt.g;
   const int npanel = (g.max_c + NB - 1) / NB;
-  CholArgs a{w.gram, w.R, w.chol_t, npanel, w.dead, status, Bt.b->c_off, (int64_t)g.max_c, g.d};
+  CholArgs a{w.gram, w.R, w.X, w.chol_t, npanel, w.dead, status, Bt.b->c_off, g.ld_g, g.d};
   KVS_CUDA_TRY(cudaMemsetAsync(w.dead, 0, sizeof(int) * g.B, Bt.st));
-  const int ndc = (g.d + NB - 1) / NB;
+  const int ndc = g.d / NB;
   for (int p = 0; p < npanel; ++p) {
     const int j0 = p * NB;
     k_chol_diag<<<g.B, 256, 0, Bt.st>>>(a, j0);
     KVS_LAUNCH_CHECK("k_chol_diag");
-    k_chol_tmul<<<dim3(ndc, g.B), 256, 0, Bt.st>>>(a, j0, 0);
-    KVS_LAUNCH_CHECK("k_chol_tmul");
     const int n2 = g.max_c - j0 - NB;
     if (n2 <= 0) continue;
     const int nt = (n2 + NB - 1) / NB;
     k_chol_panel<<<dim3(nt, g.B), 256, 0, Bt.st>>>(a, j0);
     KVS_LAUNCH_CHECK("k_chol_panel");
-    k_chol_update<<<dim3(nt * (nt + 1) / 2 + nt * ndc, g.B), 256, 0, Bt.st>>>(a, j0, nt);
+    k_chol_update<<<dim3(nt * (nt + 1) / 2 + nt * ndc, g.B), 256, 0, Bt.st>>>(a, j0);
     KVS_LAUNCH_CHECK("k_chol_update");
   }
   for (int p = npanel - 1; p >= 0; --p) {
-    const int j0 = p * NB;
-    k_chol_tmul<<<dim3(ndc, g.B), 256, 0, Bt.st>>>(a, j0, 1);
-    KVS_LAUNCH_CHECK("k_chol_tmul");
-    if (j0 == 0) continue;
-    k_chol_bupdate<<<dim3(ndc, (j0 + NB - 1) / NB, g.B), 256, 0, Bt.st>>>(a, j0);
-    KVS_LAUNCH_CHECK("k_chol_bupdate");
+    k_chol_bsolve<<<dim3(ndc, std::max(p, 1), g.B), 256, 0, Bt.st>>>(a, p * NB);
+    KVS_LAUNCH_CHECK("k_chol_bsolve");
   }
-  k_chol_store<<<g.B, 256, 0, Bt.st>>>(a, Vc);
+  const int64_t n4 = (int64_t)g.max_c * g.d / 4;
+  const int blocks = (int)std::min<int64_t>((n4 + 255) / 256, 64);
+  k_chol_store<<<dim3(blocks, g.B), 256, 0, Bt.st>>>(a, Vc);
   KVS_LAUNCH_CHECK("k_chol_store");
   return KVS_OK;
 }
