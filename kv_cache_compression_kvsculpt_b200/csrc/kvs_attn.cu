@@ -162,10 +162,10 @@ int targets_d(const Batch &Bt, const float *Q, const float *Kz, const float *Vz,
   if ((rc = split(Kz, w.kh, w.kl, g.sum_z * D, Bt.st))) return rc;
   if ((rc = split(Vz, w.vh, w.vl, g.sum_z * D, Bt.st))) return rc;
   FwdMaps fm;
-  if ((rc = make_map_bf16(&fm.kh, w.kh, g.sum_z, D, 64)) ||
-      (rc = make_map_bf16(&fm.kl, w.kl, g.sum_z, D, 64)) ||
-      (rc = make_map_bf16(&fm.vh, w.vh, g.sum_z, D, 64)) ||
-      (rc = make_map_bf16(&fm.vl, w.vl, g.sum_z, D, 64)))
+  if ((rc = make_map_bf16(&fm.kh, w.kh, g.sum_z, D, FWD_BN)) ||
+      (rc = make_map_bf16(&fm.kl, w.kl, g.sum_z, D, FWD_BN)) ||
+      (rc = make_map_bf16(&fm.vh, w.vh, g.sum_z, D, FWD_BN)) ||
+      (rc = make_map_bf16(&fm.vl, w.vl, g.sum_z, D, FWD_BN)))
     return rc;
   FwdArgs a{};
   a.q_off = Bt.b->q_off;
@@ -184,8 +184,8 @@ int targets_d(const Batch &Bt, const float *Q, const float *Kz, const float *Vz,
   BwdMaps bm;
   if ((rc = make_map_bf16(&bm.kh, w.kh, g.sum_z, D, 128)) ||
       (rc = make_map_bf16(&bm.kl, w.kl, g.sum_z, D, 128)) ||
-      (rc = make_map_bf16(&bm.qh, w.qh, g.sum_q, D, 64)) ||
-      (rc = make_map_bf16(&bm.ql, w.ql, g.sum_q, D, 64)))
+      (rc = make_map_bf16(&bm.qh, w.qh, g.sum_q, D, BWD_BQ)) ||
+      (rc = make_map_bf16(&bm.ql, w.ql, g.sum_q, D, BWD_BQ)))
     return rc;
   bm.g = bm.qh;
   BwdArgs ba{};
@@ -216,10 +216,10 @@ int forward_d(const Batch &Bt, const float *Q, const float *Kc, const float *Vc,
   if (!q_ready && (rc = split(Q, w.qh, w.ql, g.sum_q * D, Bt.st))) return rc;
   if (!pairs_ready && (rc = prep_pairs<D>(Bt, Kc, Vc, w))) return rc;
   FwdMaps fm;
-  if ((rc = make_map_bf16(&fm.kh, w.kh, g.sum_c, D, 64)) ||
-      (rc = make_map_bf16(&fm.kl, w.kl, g.sum_c, D, 64)) ||
-      (rc = make_map_bf16(&fm.vh, w.vh, g.sum_c, D, 64)) ||
-      (rc = make_map_bf16(&fm.vl, w.vl, g.sum_c, D, 64)))
+  if ((rc = make_map_bf16(&fm.kh, w.kh, g.sum_c, D, FWD_BN)) ||
+      (rc = make_map_bf16(&fm.kl, w.kl, g.sum_c, D, FWD_BN)) ||
+      (rc = make_map_bf16(&fm.vh, w.vh, g.sum_c, D, FWD_BN)) ||
+      (rc = make_map_bf16(&fm.vl, w.vl, g.sum_c, D, FWD_BN)))
     return rc;
   FwdArgs a{};
   a.q_off = Bt.b->q_off;
@@ -253,9 +253,9 @@ int backward_d(const Batch &Bt, float *dKc, Filter flt, const Work &w) {
   BwdMaps bm;
   if ((rc = make_map_bf16(&bm.kh, w.kh, g.sum_c, D, 128)) ||
       (rc = make_map_bf16(&bm.kl, w.kl, g.sum_c, D, 128)) ||
-      (rc = make_map_bf16(&bm.qh, w.qh, g.sum_q, D, 64)) ||
-      (rc = make_map_bf16(&bm.ql, w.ql, g.sum_q, D, 64)) ||
-      (rc = make_map_bf16(&bm.g, w.go, g.sum_q, D, 64)))
+      (rc = make_map_bf16(&bm.qh, w.qh, g.sum_q, D, BWD_BQ)) ||
+      (rc = make_map_bf16(&bm.ql, w.ql, g.sum_q, D, BWD_BQ)) ||
+      (rc = make_map_bf16(&bm.g, w.go, g.sum_q, D, BWD_BQ)))
     return rc;
   BwdArgs ba{};
   ba.q_off = Bt.b->q_off;
@@ -280,8 +280,8 @@ int fit_d(const Batch &Bt, const float *Q, const float *Kc, const float *Y, floa
   if (!y_ready && (rc = split(Y, w.yh, w.yl, g.sum_q * D, Bt.st))) return rc;
   if ((rc = prep_pairs<D>(Bt, Kc, nullptr, w))) return rc;
   FwdMaps fm;
-  if ((rc = make_map_bf16(&fm.kh, w.kh, g.sum_c, D, 64)) ||
-      (rc = make_map_bf16(&fm.kl, w.kl, g.sum_c, D, 64)))
+  if ((rc = make_map_bf16(&fm.kh, w.kh, g.sum_c, D, FWD_BN)) ||
+      (rc = make_map_bf16(&fm.kl, w.kl, g.sum_c, D, FWD_BN)))
     return rc;
   fm.vh = fm.kh;
   fm.vl = fm.kl;

@@ -12,7 +12,14 @@ namespace kvs {
 enum FwdMode : int { FWD_LOSS = 0, FWD_TARGETS = 1, FWD_STATS = 2, FWD_WRITE_A = 3 };
 enum BwdMode : int { BWD_DK = 0, BWD_COLSUM = 1 };
 
-// Tensor maps of the bf16 operands (2-D, [rows, d], box 64 columns x 64 rows).
+// Rows of one key / value tile of the query-tile kernel (the TMA box height of
+// its key and value maps).
+constexpr int FWD_BN = 128;
+// Queries of one tile of the key-tile kernel (the TMA box height of its query
+// and Go maps).
+constexpr int BWD_BQ = 128;
+
+// Tensor maps of the bf16 operands (2-D, [rows, d], box 64 columns x FWD_BN rows).
 struct FwdMaps {
   CUtensorMap kh, kl, vh, vl;
 };
@@ -44,7 +51,7 @@ struct FwdArgs {
 
 struct BwdMaps {
   CUtensorMap kh, kl;     // key tile, box 64 columns x 128 rows
-  CUtensorMap qh, ql, g;  // query / Go tiles, box 64 columns x 64 rows
+  CUtensorMap qh, ql, g;  // query / Go tiles, box 64 columns x BWD_BQ rows
 };
 
 struct BwdArgs {
