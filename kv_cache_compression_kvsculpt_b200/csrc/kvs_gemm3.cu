@@ -8,8 +8,10 @@
 // with fp32 accumulation in TMEM, which keeps about 16 significant bits of
 // each operand.  Both operands are read MN-major (keys / value columns
 // contiguous), the contraction runs over training queries in tiles of 64.
-// One CTA owns one 128 x 128 output tile: the Gram matrix is formed on its
-// lower block triangle only (the Cholesky reads the lower triangle).
+// One CTA owns one 128-row output tile, as wide as the product allows: a
+// tcgen05.mma instruction costs about the same for any N up to 256, so Gram
+// tiles are 128 x 256 (only those that reach the lower triangle, which the
+// Cholesky reads) and A^T Y tiles are 128 x d.
 #include <math.h>
 
 #include "kvs_attn_tc.cuh"
@@ -19,22 +21,56 @@ namespace {
 
 using namespace tc;
 
-constexpr int TM = 128, TN = 128, TKQ = 64, NS = 3;
-constexpr int OP_BYTES = TKQ * TM * 2;        // one 64-row x 128-column bf16 operand tile
-constexpr int STAGE = 4 * OP_BYTES;           // A hi, A lo, B hi, B lo
-constexpr int SMEM = NS * STAGE + 1024;
+constexpr int TM = 128, TKQ = 64;
+constexpr int A_BYTES = TKQ * TM * 2;  // one 64-row x 128-column bf16 operand tile
+
+template <int TN>
+struct G3 {
+  static constexpr int B_BYTES = TKQ * TN * 2;            // one 64-row x TN-column tile
+  static constexpr int STAGE = 2 * A_BYTES + 2 * B_BYTES;  // A hi, A lo, B hi, B lo
+  static constexpr int NS = TN > 128 ? 2 : 3;
+  static constexpr int SMEM = NS * STAGE + 1024;
+  static constexpr uint32_t TMEM_COLS = TN < 32 ? 32 : TN;
+};
+constexpr int NSMAX = 3;
+
+// Gram tile t of a problem with T row tiles: the t-th (row, column) pair in
+// row-major order among the 128 x TN tiles that reach the lower triangle.
+template <int TN>
+__device__ __forceinline__ bool gram_tile(int t, int T, int *ti, int *tj) {
+  for (int i = 0; i < T; ++i) {
+    const int n = (i * TM + TM - 1) / TN + 1;  // column tiles of row tile i
+    if (t < n) {
+      *ti = i;
+      *tj = t;
+      return true;
+    }
+    t -= n;
+  }
+  return false;
+}
+
+template <int TN>
+__host__ __device__ constexpr int gram_tiles(int T) {
+  int n = 0;
+  for (int i = 0; i < T; ++i) n += (i * TM + TM - 1) / TN + 1;
+  return n;
+}
 
 struct GBars {
-  uint64_t full[NS], empty[NS];
+  uint64_t full[NSMAX], empty[NSMAX];
   uint64_t done;
   uint32_t tmem;
   int abort;
 };
 
+template <int TN>
 __global__ void __launch_bounds__(192, 1)
     k_gemm3(const __grid_constant__ CUtensorMap mAh, const __grid_constant__ CUtensorMap mAl,
             const __grid_constant__ CUtensorMap mBh, const __grid_constant__ CUtensorMap mBl,
             GemmArgs3 a, int gram) {
+  using C = G3<TN>;
+  constexpr int NS = C::NS;
   extern __shared__ unsigned char smraw[];
   unsigned char *sm = (unsigned char *)(((uintptr_t)smraw + 1023) & ~(uintptr_t)1023);
   __shared__ GBars bars;
@@ -45,17 +81,13 @@ __global__ void __launch_bounds__(192, 1)
   int ti, tj;
   const int t = blockIdx.x;
   if (gram) {
-    if (t >= T * (T + 1) / 2) return;
-    ti = (int)((sqrtf(8.f * t + 1.f) - 1.f) * 0.5f);
-    while (ti * (ti + 1) / 2 > t) --ti;
-    while ((ti + 1) * (ti + 2) / 2 <= t) ++ti;
-    tj = t - ti * (ti + 1) / 2;
+    if (!gram_tile<TN>(t, T, &ti, &tj)) return;
   } else {
     if (t >= T) return;
     ti = t;
     tj = 0;
   }
-  const int N = gram ? TN : a.n_fixed;          // MMA N
+  const int N = TN;                             // MMA N (A^T Y: TN = d)
   const int ncols = gram ? nk : a.n_fixed;      // valid output columns
   const int64_t ka0 = a.a_pad_off[b];
   const int kq = (int)(a.a_pad_off[b + 1] - ka0);  // padded query rows (multiple of 128)
@@ -72,14 +104,14 @@ __global__ void __launch_bounds__(192, 1)
     bars.abort = 0;
     fence_barrier_init();
   }
-  if (warp == 5) tmem_alloc(&bars.tmem, 128);
+  if (warp == 5) tmem_alloc(&bars.tmem, C::TMEM_COLS);
   fence_before_sync();
   __syncthreads();
   fence_after_sync();
   const uint32_t tmem = bars.tmem;
   volatile int *abort = &bars.abort;
   const int nb_boxes = N / 64;
-  const uint32_t stage_tx = 2 * OP_BYTES + 2 * (uint32_t)(nb_boxes * 64 * TKQ * 2);
+  const uint32_t stage_tx = C::STAGE;
 
   if (warp == 4) {
     if (lane == 0) {
@@ -91,16 +123,17 @@ __global__ void __launch_bounds__(192, 1)
           break;
         }
         issued = i + 1;
-        unsigned char *base = sm + st * STAGE;
+        unsigned char *base = sm + st * C::STAGE;
         mbar_arrive_expect_tx(&bars.full[st], stage_tx);
         const int ya = (int)(ka0 + i * TKQ), yb = (int)(kb0 + i * TKQ);
         for (int r = 0; r < 2; ++r) {
           tma_load_2d(base + r * TKQ * 128, &mAh, &bars.full[st], ti * TM + 64 * r, ya);
-          tma_load_2d(base + OP_BYTES + r * TKQ * 128, &mAl, &bars.full[st], ti * TM + 64 * r, ya);
+          tma_load_2d(base + A_BYTES + r * TKQ * 128, &mAl, &bars.full[st], ti * TM + 64 * r, ya);
         }
         for (int r = 0; r < nb_boxes; ++r) {
-          tma_load_2d(base + 2 * OP_BYTES + r * TKQ * 128, &mBh, &bars.full[st], tj * TN + 64 * r, yb);
-          tma_load_2d(base + 3 * OP_BYTES + r * TKQ * 128, &mBl, &bars.full[st], tj * TN + 64 * r, yb);
+          tma_load_2d(base + 2 * A_BYTES + r * TKQ * 128, &mBh, &bars.full[st], tj * TN + 64 * r, yb);
+          tma_load_2d(base + 2 * A_BYTES + C::B_BYTES + r * TKQ * 128, &mBl, &bars.full[st],
+                      tj * TN + 64 * r, yb);
         }
       }
       if (*abort)
@@ -115,13 +148,13 @@ __global__ void __launch_bounds__(192, 1)
         const int st = i % NS;
         if (!mbar_wait(&bars.full[st], (i / NS) & 1, abort)) { ok = false; break; }
         fence_after_sync();
-        const uint64_t d0 = sdesc(smem_u32(sm + st * STAGE), TKQ * 128, 1024);
+        const uint64_t d0 = sdesc(smem_u32(sm + st * C::STAGE), TKQ * 128, 1024);
 #pragma unroll
         for (int kk = 0; kk < TKQ / 16; ++kk) {
           const uint64_t ah = sdesc_add(d0, kk * 2048);
-          const uint64_t al = sdesc_add(ah, OP_BYTES);
-          const uint64_t bh = sdesc_add(ah, 2 * OP_BYTES);
-          const uint64_t bl = sdesc_add(ah, 3 * OP_BYTES);
+          const uint64_t al = sdesc_add(ah, A_BYTES);
+          const uint64_t bh = sdesc_add(ah, 2 * A_BYTES);
+          const uint64_t bl = sdesc_add(ah, 2 * A_BYTES + C::B_BYTES);
           mma_bf16(tmem, ah, bh, id, (i > 0 || kk > 0) ? 1u : 0u);
           mma_bf16(tmem, ah, bl, id, 1u);
           mma_bf16(tmem, al, bh, id, 1u);
@@ -159,21 +192,29 @@ __global__ void __launch_bounds__(192, 1)
   __syncthreads();
   if (warp == 5) {
     fence_after_sync();
-    tmem_dealloc(tmem, 128);
+    tmem_dealloc(tmem, C::TMEM_COLS);
   }
   if (tid == 0 && bars.abort && a.err) atomicOr(a.err, 1);
 }
 
 }  // namespace
 
-int launch_gemm3_tc(const GemmMaps &m, const GemmArgs3 &a, int tiles_m, int gram, int B,
-                    cudaStream_t st) {
-  KVS_CUDA_TRY(set_smem_once(k_gemm3, SMEM));
-  const int tiles = gram ? tiles_m * (tiles_m + 1) / 2 : tiles_m;
+template <int TN>
+int launch_tn(const GemmMaps &m, const GemmArgs3 &a, int tiles, int gram, int B,
+              cudaStream_t st) {
+  KVS_CUDA_TRY(set_smem_once(k_gemm3<TN>, G3<TN>::SMEM));
   if (tiles <= 0) return KVS_OK;
-  k_gemm3<<<dim3(tiles, B), 192, SMEM, st>>>(m.ah, m.al, m.bh, m.bl, a, gram);
+  k_gemm3<TN><<<dim3(tiles, B), 192, G3<TN>::SMEM, st>>>(m.ah, m.al, m.bh, m.bl, a, gram);
   KVS_LAUNCH_CHECK("k_gemm3");
   return KVS_OK;
+}
+
+int launch_gemm3_tc(const GemmMaps &m, const GemmArgs3 &a, int tiles_m, int gram, int B,
+                    cudaStream_t st) {
+  if (gram) return launch_tn<256>(m, a, gram_tiles<256>(tiles_m), 1, B, st);
+  if (a.n_fixed == 128) return launch_tn<128>(m, a, tiles_m, 0, B, st);
+  if (a.n_fixed == 64) return launch_tn<64>(m, a, tiles_m, 0, B, st);
+  return KVS_ENOTSUP;
 }
 
 }  // namespace kvs
