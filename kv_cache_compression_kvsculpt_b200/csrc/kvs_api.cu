@@ -109,6 +109,7 @@ size_t carve_work(const HostGeom &g, void *base, Work *w) {
   w->gram = c.take<float>(g.sum_c * g.ld_g);
   w->R = c.take<float>(g.sum_c * g.d);
   w->X = c.take<float>(g.sum_c * g.d);
+  w->dkp = c.take<float>(4 * g.sum_c * g.d);
   w->chol_t = c.take<float>((int64_t)g.B * ((g.max_c + 63) / 64) * 64 * 64);
   w->dead = c.take<int>(g.B);
   w->fbuf = c.take<float>(g.B);
@@ -187,6 +188,14 @@ static Filter phase_filter(const State &s, int want) {
 }
 
 static const Filter ALL{nullptr, 0, 0};
+
+// Problems whose last L-BFGS search failed: the loss forward left l_hat of a
+// rejected trial in the workspace, so the ridge fit recomputes theirs.
+static Filter stale_filter(const State &s) {
+  return Filter{reinterpret_cast<const int *>(reinterpret_cast<const char *>(s.sc) +
+                                              offsetof(LbfgsScal, lse_stale)),
+                (int)(sizeof(LbfgsScal) / sizeof(int)), 1};
+}
 
 // Loss and gradient at Kc into (w.fbuf, s.gn), then the state reset.
 static int lbfgs_restart(const Batch &Bt, const kvs_schedule &sc, const float *Q, const float *Y,
@@ -504,7 +513,11 @@ int kvs_compress_batch(const kvs_batch *batch, const kvs_schedule *sched, const 
         return rc;
       }
     }
-    if ((rc = launch_fit(Bt, Q, Kc, w.Yt, sc.lambda, Vc, status, true, true, w))) return rc;
+    // every problem's l_hat at Kc is in the workspace from its accepted trial's
+    // loss forward, except after a failed search
+    if ((rc = launch_fit(Bt, Q, Kc, w.Yt, sc.lambda, Vc, status, true, true, w,
+                         sc.steps > 0 ? stale_filter(s) : ALL)))
+      return rc;
     if ((rc = lbfgs_restart(Bt, sc, Q, w.Yt, w.lset, Vc, Kc, s, sc.persist_history ? 0 : 1, true,
                             w)))
       return rc;

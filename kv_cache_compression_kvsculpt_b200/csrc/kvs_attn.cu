@@ -153,6 +153,56 @@ __global__ void k_loss_reduce(const float *partials, int tiles, const int64_t *q
 
 int max_qtiles(const HostGeom &g) { return (g.max_q + 127) / 128; }
 
+int sm_count() {
+  static int n[64] = {0};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 148;
+  if (!n[dev] && cudaDeviceGetAttribute(&n[dev], cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+    n[dev] = 148;
+  return n[dev];
+}
+
+// Query-range splits of the key-gradient kernel: the one whose last wave of
+// CTAs wastes least, with a small charge per split for the extra prologue,
+// epilogue and partial-sum traffic, and at least 8 query tiles per split.
+int bwd_split(int ctas, int nqt_max) {
+  const int nsm = sm_count();
+  int best = 1;
+  double bc = 1e30;
+  for (int sp = 1; sp <= 4; ++sp) {
+    if (sp > 1 && nqt_max / sp < 8) break;
+    const double cost = std::ceil((double)ctas * sp / nsm) / sp + 0.05 * sp;
+    if (cost < bc - 1e-9) {
+      bc = cost;
+      best = sp;
+    }
+  }
+  return best;
+}
+
+// dK = sum of the splits' partial sums, in split order, for the problems the
+// filter selects.
+__global__ void k_dk_reduce(const float *__restrict__ part, int ns, int64_t stride,
+                            const int64_t *c_off, int d, Filter flt, float *__restrict__ dk) {
+  const int b = blockIdx.y;
+  if (flt.skip(b)) return;
+  const int64_t o = c_off[b] * d / 4, n = c_off[b + 1] * d / 4 - o;
+  const float4 *p4 = reinterpret_cast<const float4 *>(part);
+  float4 *d4 = reinterpret_cast<float4 *>(dk);
+  for (int64_t e = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; e < n;
+       e += (int64_t)gridDim.x * blockDim.x) {
+    float4 acc = p4[o + e];
+    for (int z = 1; z < ns; ++z) {
+      const float4 v = p4[z * (stride / 4) + o + e];
+      acc.x += v.x;
+      acc.y += v.y;
+      acc.z += v.z;
+      acc.w += v.w;
+    }
+    d4[o + e] = acc;
+  }
+}
+
 template <int D>
 int targets_d(const Batch &Bt, const float *Q, const float *Kz, const float *Vz, float *Y,
               float *lse, float *imp, const Work &w) {
@@ -196,6 +246,7 @@ int targets_d(const Batch &Bt, const float *Q, const float *Kz, const float *Vz,
   ba.lse = lse;
   ba.imp = imp;
   ba.err = w.err;
+  ba.nsplit = 1;
   return launch_bwd_tc<D, BWD_COLSUM>(bm, ba, (g.max_z + 127) / 128, g.B, Bt.st);
 }
 
@@ -268,12 +319,26 @@ int backward_d(const Batch &Bt, float *dKc, Filter flt, const Work &w) {
   ba.v_lo = w.vl;
   ba.dk = dKc;
   ba.err = w.err;
-  return launch_bwd_tc<D, BWD_DK>(bm, ba, (g.max_c + 127) / 128, g.B, Bt.st);
+  ba.nsplit = 1;
+  const int ktiles = (g.max_c + 127) / 128;
+  const int ns = bwd_split(ktiles * g.B, (g.max_q + 63) / 64);
+  if (ns > 1) {
+    // partial sums of ns query ranges, then their fixed-order sum
+    ba.nsplit = ns;
+    ba.dk = w.dkp;
+    ba.dk_stride = g.sum_c * D;
+  }
+  if ((rc = launch_bwd_tc<D, BWD_DK>(bm, ba, ktiles, g.B, Bt.st))) return rc;
+  if (ns == 1) return KVS_OK;
+  k_dk_reduce<<<dim3(std::min<int64_t>(((int64_t)g.max_c * D / 4 + 255) / 256, 32), g.B), 256, 0,
+                Bt.st>>>(w.dkp, ns, g.sum_c * D, Bt.b->c_off, D, flt, dKc);
+  KVS_LAUNCH_CHECK("k_dk_reduce");
+  return KVS_OK;
 }
 
 template <int D>
 int fit_d(const Batch &Bt, const float *Q, const float *Kc, const float *Y, float lam, float *Vc,
-          int32_t *status, bool q_ready, bool y_ready, const Work &w) {
+          int32_t *status, bool q_ready, bool y_ready, Filter stats, const Work &w) {
   const HostGeom &g = Bt.g;
   int rc;
   if (!q_ready && (rc = split(Q, w.qh, w.ql, g.sum_q * D, Bt.st))) return rc;
@@ -290,11 +355,12 @@ int fit_d(const Batch &Bt, const float *Q, const float *Kc, const float *Y, floa
   a.k_off = Bt.b->c_off;
   a.q_hi = w.qh;
   a.q_lo = w.ql;
-  a.flt = Filter{nullptr, 0, 0};
+  a.flt = stats;  // problems whose l_hat in the workspace is not that of Kc
   a.scale = 1.f / sqrtf((float)D);
   a.lse_out = w.lse_h;
   a.err = w.err;
   if ((rc = launch_fwd_tc<D, FWD_STATS>(fm, a, max_qtiles(g), g.B, Bt.st))) return rc;
+  a.flt = Filter{nullptr, 0, 0};
   k_pad_offsets<<<1, 1, 0, Bt.st>>>(Bt.b->q_off, g.B, w.a_pad_off);
   KVS_LAUNCH_CHECK("k_pad_offsets");
   a.lse_in = w.lse_h;
@@ -359,9 +425,10 @@ int launch_backward(const Batch &Bt, float *dKc, Filter flt, const Work &w) {
 }
 
 int launch_fit(const Batch &Bt, const float *Q, const float *Kc, const float *Y, float lam,
-               float *Vc, int32_t *status, bool q_ready, bool y_ready, const Work &w) {
-  return Bt.g.d == 64 ? fit_d<64>(Bt, Q, Kc, Y, lam, Vc, status, q_ready, y_ready, w)
-                      : fit_d<128>(Bt, Q, Kc, Y, lam, Vc, status, q_ready, y_ready, w);
+               float *Vc, int32_t *status, bool q_ready, bool y_ready, const Work &w,
+               Filter stats) {
+  return Bt.g.d == 64 ? fit_d<64>(Bt, Q, Kc, Y, lam, Vc, status, q_ready, y_ready, stats, w)
+                      : fit_d<128>(Bt, Q, Kc, Y, lam, Vc, status, q_ready, y_ready, stats, w);
 }
 
 }  // namespace kvs

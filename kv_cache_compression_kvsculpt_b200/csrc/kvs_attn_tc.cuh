@@ -17,7 +17,7 @@ enum BwdMode : int { BWD_DK = 0, BWD_COLSUM = 1 };
 constexpr int FWD_BN = 128;
 // Queries of one tile of the key-tile kernel (the TMA box height of its query
 // and Go maps).
-constexpr int BWD_BQ = 128;
+constexpr int BWD_BQ = 64;
 
 // Tensor maps of the bf16 operands (2-D, [rows, d], box 64 columns x FWD_BN rows).
 struct FwdMaps {
@@ -62,9 +62,11 @@ struct BwdArgs {
   const float *lse;       // [sum_q] row lse used to form the probabilities
   const float *delta;     // [sum_q] (DK)
   const __nv_bfloat16 *v_hi, *v_lo;  // [sum_k, d] value split (DK; loaded into tensor memory)
-  float *dk;              // [sum_k, d] (DK): dL/dK
+  float *dk;              // [sum_k, d] (DK): dL/dK, or nsplit partial sums dk_stride apart
   float *imp;             // [sum_k] (COLSUM): column sums of probabilities
   int *err;
+  int nsplit;             // query tiles of a problem split over this many CTAs (COLSUM: 1)
+  int64_t dk_stride;      // floats between the partial sums of two splits
 };
 
 struct GemmMaps {

@@ -22,7 +22,8 @@ struct LbfgsScal {
   int head;       // next ring slot to write
   int phase;      // Phase
   int trials;     // trials of the current search
-  int pad[3];
+  int lse_stale;  // 1: the workspace l_hat is not that of the accepted keys (failed search)
+  int pad[2];
 };
 
 // Scratch buffers carved from the caller's workspace.
@@ -40,6 +41,7 @@ struct Work {
   float *gram;               // [sum_c, ld_g]          A^T A + lam I, then its Cholesky factor
   float *R;                  // [sum_c, d]             A^T Y, then the forward-solved rows
   float *X;                  // [sum_c, d]             solution of the ridge system
+  float *dkp;                // [4, sum_c, d]          key-gradient partial sums of query splits
   float *chol_t;             // [B, panels, 64, 64]    inverses of the diagonal blocks
   int *dead;                 // [B]                    factorisation failed
   float *fbuf;               // [B]                    loss scratch
@@ -113,9 +115,12 @@ int launch_forward(const Batch &B, const float *Q, const float *Kc, const float 
 int launch_split_pairs(const Batch &B, const float *Kc, const float *Vc, const Work &w);
 // dKc from the state left by launch_forward for the same problems.
 int launch_backward(const Batch &B, float *dKc, Filter flt, const Work &w);
-// Ridge fit: Vc = (A^T A + lam I)^-1 A^T Y (y_ready: the Y split is current).
+// Ridge fit: Vc = (A^T A + lam I)^-1 A^T Y (y_ready: the Y split is current).  The
+// row log-sum-exp of Kc is recomputed for the problems `stats` selects; the others
+// take the one the last loss forward left in the workspace.
 int launch_fit(const Batch &B, const float *Q, const float *Kc, const float *Y, float lam,
-               float *Vc, int32_t *status, bool q_ready, bool y_ready, const Work &w);
+               float *Vc, int32_t *status, bool q_ready, bool y_ready, const Work &w,
+               Filter stats = Filter{nullptr, 0, 0});
 
 // ---- other kernels ----
 int launch_build_queries(const kvs_query_spec *sp, const float *q_retain, const float *q_ctx,

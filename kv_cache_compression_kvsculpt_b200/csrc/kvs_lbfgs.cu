@@ -245,11 +245,13 @@ __global__ void __launch_bounds__(PT) k_pairs(PairArgs a) {
       if (a.status) a.status[b] |= KVS_ST_LS_FAIL;
     }
     s.phase = PH_IDLE;
+    s.lse_stale = phase == PH_FAIL;  // the last loss forward ran at a rejected trial
     if (a.f_out) a.f_out[b] = s.f;
   } else {
     s.f = a.f[b];
     s.phase = PH_IDLE;
     s.trials = 0;
+    s.lse_stale = 0;
     if (a.clear) {
       count = 0;
       head = 0;

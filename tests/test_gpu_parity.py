@@ -36,10 +36,14 @@ def cases():
         "qwen_layer": lambda: Case(W.WORKLOADS["qwen_layer"]),
         "ragged": lambda: Case(RAGGED, k=RAGGED_K, n_q=RAGGED_NQ),
         "small_d64": lambda: Case(SMALL64, k=[50, 7, 160, 33]),
+        # one long and one short query set: the key-gradient kernel splits the long
+        # problem's query tiles over several CTAs and some splits of the short one are empty
+        "uneven": lambda: Case(W.WORKLOADS["qwen_layer"], k=[960, 200], n_q=[3840, 100]),
     }
 
 
-@pytest.fixture(scope="module", params=["single_d64", "qwen_layer", "ragged", "small_d64"])
+@pytest.fixture(scope="module", params=["single_d64", "qwen_layer", "ragged", "small_d64",
+                                        "uneven"])
 def case(request):
     return cases()[request.param]()
 
@@ -347,3 +351,33 @@ def test_compress_qwen_layer_head():
     assert check_topk_valid(r["idx"], c.Qs[0], c.Zk[0], c.Zv[0], wl.k)
     assert abs(r["trace"][0, 0] - res["trace"][0]) <= 1e-3 * res["trace"][0]
     assert float(r["trace"][0, -1]) <= 1.05 * res["loss"]
+
+
+@pytest.mark.slow
+def test_longctx_head_targets_fit_loss_grad():
+    """One head-problem at the long-context size (N = 8192, m = 256, n_q = 7680,
+    z = 7936, k = 2381): targets, the ridge fit at the top-k keys and loss and
+    gradient at a perturbed Select+Fit point, each against the oracle."""
+    wl = W.WORKLOADS["longctx"]
+    c = Case(wl, ids=[(0, 0, 0)])
+    K = c.K
+    Y, lse, imp = run_targets(c)
+    Yo, lo = c.targets_oracle(0)
+    assert rel(Y, Yo) < 1e-4
+    assert np.max(np.abs(lse - lo) / (1 + np.abs(lo))) < 1e-5
+    assert rel(imp, O.importance(c.Qs[0], c.Zk[0], lo)) < 1e-4
+    Kcs, Vcs, tgt = select_fit_point(c, 0.2)
+    Vc = torch.zeros((c.batch.sum_c, wl.d), device="cuda")
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    K.kvs_fit_values(c.batch, c.Q, dev(Kcs[0]), dev(tgt[0][0]), 1e-3, Vc, status, c.ws)
+    torch.cuda.synchronize()
+    assert not host(status).any()
+    assert rel(host(Vc), Vcs[0]) < 1e-3
+    loss = torch.empty(1, device="cuda")
+    dK = torch.empty((c.batch.sum_c, wl.d), device="cuda")
+    K.kvs_loss_grad(c.batch, c.Q, dev(Kcs[0]), dev(Vcs[0]), dev(tgt[0][0]), dev(tgt[0][1]),
+                    1.0, 1.0, loss, None, dK, c.ws)
+    torch.cuda.synchronize()
+    f, g, _ = O.loss_grad(c.Qs[0], Kcs[0], Vcs[0], tgt[0][0], tgt[0][1])
+    assert abs(host(loss)[0] - f) <= 1e-3 * f
+    assert grad_close(host(dK), g, c.Qs[0], tgt[0][1])
