@@ -217,6 +217,9 @@ int targets_d(const Batch &Bt, const float *Q, const float *Kz, const float *Vz,
       (rc = make_map_bf16(&fm.vh, w.vh, g.sum_z, D, FWD_BN)) ||
       (rc = make_map_bf16(&fm.vl, w.vl, g.sum_z, D, FWD_BN)))
     return rc;
+  if ((rc = make_map_bf16(&fm.qh, w.qh, g.sum_q, D, FWD_BN)) ||
+      (rc = make_map_bf16(&fm.ql, w.ql, g.sum_q, D, FWD_BN)))
+    return rc;
   FwdArgs a{};
   a.q_off = Bt.b->q_off;
   a.k_off = Bt.b->z_off;
@@ -271,6 +274,9 @@ int forward_d(const Batch &Bt, const float *Q, const float *Kc, const float *Vc,
       (rc = make_map_bf16(&fm.kl, w.kl, g.sum_c, D, FWD_BN)) ||
       (rc = make_map_bf16(&fm.vh, w.vh, g.sum_c, D, FWD_BN)) ||
       (rc = make_map_bf16(&fm.vl, w.vl, g.sum_c, D, FWD_BN)))
+    return rc;
+  if ((rc = make_map_bf16(&fm.qh, w.qh, g.sum_q, D, FWD_BN)) ||
+      (rc = make_map_bf16(&fm.ql, w.ql, g.sum_q, D, FWD_BN)))
     return rc;
   FwdArgs a{};
   a.q_off = Bt.b->q_off;
@@ -347,6 +353,9 @@ int fit_d(const Batch &Bt, const float *Q, const float *Kc, const float *Y, floa
   FwdMaps fm;
   if ((rc = make_map_bf16(&fm.kh, w.kh, g.sum_c, D, FWD_BN)) ||
       (rc = make_map_bf16(&fm.kl, w.kl, g.sum_c, D, FWD_BN)))
+    return rc;
+  if ((rc = make_map_bf16(&fm.qh, w.qh, g.sum_q, D, FWD_BN)) ||
+      (rc = make_map_bf16(&fm.ql, w.ql, g.sum_q, D, FWD_BN)))
     return rc;
   fm.vh = fm.kh;
   fm.vl = fm.kl;

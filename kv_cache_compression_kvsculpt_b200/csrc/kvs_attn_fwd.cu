@@ -7,14 +7,16 @@
 // One CTA owns 128 training queries of one head-problem and streams the
 // problem's keys in tiles of 128.  Every product keeps about 16 significant
 // bits through a bf16 hi/lo split, with fp32 accumulation in tensor memory:
-//   S = Q K^T     Q_hi K_hi + Q_hi K_lo + Q_lo K_hi   (Q in TMEM, K in smem; N = 128)
+//   S = Q K^T     Q_hi K_hi + Q_hi K_lo + Q_lo K_hi   (Q and K in smem; N = 128)
 //   online softmax, one thread per query row, lazy rescaling of O
-//   O += P V      P_hi V_hi + P_hi V_lo + P_lo V_hi   (P in TMEM over S, V in smem)
-// Each tcgen05.mma instruction costs about the same up to N = 256, so the key
-// tile is as wide as tensor memory allows (two S buffers of 128 columns).
+//   O += P V      P_hi [V_hi | V_lo] + P_lo [V_hi | V_lo]  (P in TMEM over S; N = 2d)
+// Each tcgen05.mma instruction costs about the same for any N up to 256, so
+// the key tile is 128 wide and the value product takes V_hi and V_lo side by
+// side: two instructions per 16 keys instead of three, into two output halves
+// O_a = P V_hi, O_b = P V_lo (plus the negligible P_lo V_lo) summed at the end.
 // Keys and values have separate shared-memory rings: the next key tile loads
 // while P V of the previous tile runs, the value tile while S of the next runs.
-// Tensor memory (512 columns): S/P buffers at 0 and 128, O at 256, Q hi/lo after.
+// Tensor memory (512 columns): S/P buffers at 0 and 128, O_a | O_b at 256.
 // Modes:
 //   LOSS     keys K_c, values V_c: writes l_hat, Go = dL/dY_hat (bf16),
 //            delta = Go . Y_hat - dL/dl_hat (with the rounded Go), loss partials
@@ -22,7 +24,8 @@
 //   STATS    row log-sum-exp only
 //   WRITE_A  given l_hat: writes A = exp(S - l_hat) as bf16 hi/lo
 // Warp roles: warps 0-3 softmax/epilogue (thread t <-> TMEM lane t <-> query
-// row t), warp 4 TMA producer, warp 5 TMEM allocator and MMA issuer.
+// row t), warp 4 TMA producer (Q once, then keys and values), warp 5 TMEM
+// allocator and MMA issuer.
 #include <math.h>
 
 #include "kvs_attn_tc.cuh"
@@ -43,16 +46,17 @@ struct Fwd {
   static constexpr int KD = D / 64;
   static constexpr bool PV = (MODE == FWD_LOSS || MODE == FWD_TARGETS);
   static constexpr int T_BYTES = BN * D * 2;   // one 128-row bf16 tile (hi or lo)
-  static constexpr int NSK = PV ? 2 : 3;       // key stages (K hi + K lo each)
+  static constexpr int NSK = PV ? 1 : 2;       // key stages (K hi + K lo each)
   static constexpr int NSV = PV ? 1 : 0;       // value stages (V hi + V lo each)
   static constexpr int NSVI = PV ? NSV : 1;     // ring index modulus (unused without values)
-  static constexpr int OFF_V = NSK * 2 * T_BYTES;
-  static constexpr int BYTES = (NSK + NSV) * 2 * T_BYTES;
+  static constexpr int OFF_K = 2 * T_BYTES;    // after Q hi, Q lo (BM = BN rows)
+  static constexpr int OFF_V = OFF_K + NSK * 2 * T_BYTES;
+  static constexpr int BYTES = OFF_V + NSV * 2 * T_BYTES;
   static constexpr int SMEM = BYTES + 1024;
   static constexpr uint32_t TMEM_COLS = 512;
-  static constexpr uint32_t COL_O = 2 * BN;
-  static constexpr uint32_t COL_Q = COL_O + D;  // Q hi at +0, Q lo at +D/2
+  static constexpr uint32_t COL_O = 2 * BN;     // O_a at +0, O_b at +D
 };
+static_assert(BM == BN, "the Q tile shares the key tile's layout");
 
 struct FwdBars {
   uint64_t q_full;
@@ -70,6 +74,7 @@ template <int D, int MODE>
 __global__ void __launch_bounds__(192, 1)
     k_attn_fwd(const __grid_constant__ CUtensorMap mKh, const __grid_constant__ CUtensorMap mKl,
                const __grid_constant__ CUtensorMap mVh, const __grid_constant__ CUtensorMap mVl,
+               const __grid_constant__ CUtensorMap mQh, const __grid_constant__ CUtensorMap mQl,
                FwdArgs a) {
   using C = Fwd<D, MODE>;
   extern __shared__ unsigned char smraw[];
@@ -87,7 +92,7 @@ __global__ void __launch_bounds__(192, 1)
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
 
   if (tid == 0) {
-    mbar_init(&bars.q_full, BM);
+    mbar_init(&bars.q_full, 1);
     for (int i = 0; i < C::NSK; ++i) {
       mbar_init(&bars.k_full[i], 1);
       mbar_init(&bars.k_empty[i], 1);
@@ -116,13 +121,20 @@ __global__ void __launch_bounds__(192, 1)
     // ------------------------------------------------------------ TMA producer
     if (lane == 0) {
       tma_prefetch_map(&mKh);
+      // the CTA's query tile, hi and lo
+      const int qrow = (int)(q_begin + q0);
+      mbar_arrive_expect_tx(&bars.q_full, 2 * C::T_BYTES);
+      for (int r = 0; r < C::KD; ++r) {
+        tma_load_2d(sm + r * BM * 128, &mQh, &bars.q_full, 64 * r, qrow);
+        tma_load_2d(sm + C::T_BYTES + r * BM * 128, &mQl, &bars.q_full, 64 * r, qrow);
+      }
       int k_issued = 0, v_issued = 0;
       auto load_k = [&](int j) -> bool {
         const int st = j % C::NSK;
         if (j >= C::NSK && !mbar_wait(&bars.k_empty[st], ((j / C::NSK) - 1) & 1, abort))
           return false;
         k_issued = j + 1;
-        unsigned char *base = sm + st * 2 * C::T_BYTES;
+        unsigned char *base = sm + C::OFF_K + st * 2 * C::T_BYTES;
         const int krow = (int)(k_begin + j * BN);
         mbar_arrive_expect_tx(&bars.k_full[st], 2 * C::T_BYTES);
         for (int r = 0; r < C::KD; ++r) {
@@ -159,6 +171,7 @@ __global__ void __launch_bounds__(192, 1)
       }
       if (!ok) *abort = 1;
       if (*abort) {  // let issued copies land before shared memory is released
+        mbar_wait(&bars.q_full, 0);
         for (int j = (k_issued > C::NSK ? k_issued - C::NSK : 0); j < k_issued; ++j)
           mbar_wait(&bars.k_full[j % C::NSK], (j / C::NSK) & 1);
         for (int j = (v_issued > C::NSVI ? v_issued - C::NSVI : 0); j < v_issued; ++j)
@@ -170,26 +183,25 @@ __global__ void __launch_bounds__(192, 1)
     if (lane == 0) {
       const uint32_t id_s128 = idesc_bf16(BM, BN, false, false);
       const uint32_t id_s64 = idesc_bf16(BM, 64, false, false);
-      const uint32_t id_pv = idesc_bf16(BM, D, false, true);
-      const uint32_t tq_hi = tmem + C::COL_Q, tq_lo = tmem + C::COL_Q + D / 2;
+      const uint32_t id_pv = idesc_bf16(BM, 2 * D, false, true);  // N = [V_hi | V_lo]
       bool ok = mbar_wait(&bars.q_full, 0, abort);
       fence_after_sync();
+      const uint64_t qh0 = sdesc(smem_u32(sm), 16, 1024), ql0 = sdesc_add(qh0, C::T_BYTES);
       auto issue_pv = [&](int i) -> bool {
         const int pb = i & 1;
         if (!mbar_wait(&bars.p_full[pb], (i >> 1) & 1, abort)) return false;
         if (!mbar_wait(&bars.v_full[i % C::NSVI], (i / C::NSVI) & 1, abort)) return false;
         fence_after_sync();
-        const uint64_t vh0 = sdesc(smem_u32(sm + C::OFF_V + (i % C::NSVI) * 2 * C::T_BYTES),
-                                   BN * 128, 1024);
-        const uint64_t vl0 = sdesc_add(vh0, C::T_BYTES);
+        // V_hi and V_lo boxes sit back to back with one stride: one N = 2d operand
+        const uint64_t v0 = sdesc(smem_u32(sm + C::OFF_V + (i % C::NSVI) * 2 * C::T_BYTES),
+                                  BN * 128, 1024);
         const uint32_t tp = tmem + pb * BN;  // P hi at +0, P lo at +BN/2 columns
         const int kv = min(nk - i * BN, BN);
         const int nks = (kv + 15) / 16;      // key steps that hold valid keys
         for (int kk = 0; kk < nks; ++kk) {
-          const uint64_t vh = sdesc_add(vh0, kk * 2048), vl = sdesc_add(vl0, kk * 2048);
-          mma_bf16_ts(tmem + C::COL_O, tp + kk * 8, vh, id_pv, (i > 0 || kk > 0) ? 1u : 0u);
-          mma_bf16_ts(tmem + C::COL_O, tp + kk * 8, vl, id_pv, 1u);
-          mma_bf16_ts(tmem + C::COL_O, tp + BN / 2 + kk * 8, vh, id_pv, 1u);
+          const uint64_t v = sdesc_add(v0, kk * 2048);
+          mma_bf16_ts(tmem + C::COL_O, tp + kk * 8, v, id_pv, (i > 0 || kk > 0) ? 1u : 0u);
+          mma_bf16_ts(tmem + C::COL_O, tp + BN / 2 + kk * 8, v, id_pv, 1u);
         }
         mma_commit(&bars.v_empty[i % C::NSVI]);
         mma_commit(&bars.s_free[pb]);
@@ -202,15 +214,16 @@ __global__ void __launch_bounds__(192, 1)
         fence_after_sync();
         // a last tile with at most 64 keys takes the narrower product
         const uint32_t id_s = (nk - j * BN) > 64 ? id_s128 : id_s64;
-        const uint64_t kh0 = sdesc(smem_u32(sm + st * 2 * C::T_BYTES), 16, 1024);
+        const uint64_t kh0 = sdesc(smem_u32(sm + C::OFF_K + st * 2 * C::T_BYTES), 16, 1024);
         const uint64_t kl0 = sdesc_add(kh0, C::T_BYTES);
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
-          const uint32_t off_k = (kk >> 2) * (BN * 128) + (kk & 3) * 32;
-          const uint64_t kh = sdesc_add(kh0, off_k), kl = sdesc_add(kl0, off_k);
-          mma_bf16_ts(tmem + sb * BN, tq_hi + kk * 8, kh, id_s, kk > 0 ? 1u : 0u);
-          mma_bf16_ts(tmem + sb * BN, tq_hi + kk * 8, kl, id_s, 1u);
-          mma_bf16_ts(tmem + sb * BN, tq_lo + kk * 8, kh, id_s, 1u);
+          const uint32_t off = (kk >> 2) * (BN * 128) + (kk & 3) * 32;  // same for Q and K
+          const uint64_t kh = sdesc_add(kh0, off), kl = sdesc_add(kl0, off);
+          const uint64_t qh = sdesc_add(qh0, off), ql = sdesc_add(ql0, off);
+          mma_bf16(tmem + sb * BN, qh, kh, id_s, kk > 0 ? 1u : 0u);
+          mma_bf16(tmem + sb * BN, qh, kl, id_s, 1u);
+          mma_bf16(tmem + sb * BN, ql, kh, id_s, 1u);
         }
         mma_commit(&bars.s_full[sb]);
         mma_commit(&bars.k_empty[st]);
@@ -227,27 +240,6 @@ __global__ void __launch_bounds__(192, 1)
     const int q = q0 + row;
     const bool valid = q < nq;
     const uint32_t lane_base = (uint32_t)(warp * 32) << 16;
-    // the query row (hi, lo) into tensor memory as the A operand of S = Q K^T
-    {
-      const uint4 *qh = reinterpret_cast<const uint4 *>(a.q_hi + (q_begin + q) * D);
-      const uint4 *ql = reinterpret_cast<const uint4 *>(a.q_lo + (q_begin + q) * D);
-#pragma unroll 1
-      for (int c0 = 0; c0 < D / 2; c0 += 32) {
-        uint32_t vh[32], vl[32];
-#pragma unroll
-        for (int e = 0; e < 8; ++e) {
-          const uint4 h = valid ? qh[c0 / 4 + e] : make_uint4(0, 0, 0, 0);
-          const uint4 l = valid ? ql[c0 / 4 + e] : make_uint4(0, 0, 0, 0);
-          vh[4 * e] = h.x; vh[4 * e + 1] = h.y; vh[4 * e + 2] = h.z; vh[4 * e + 3] = h.w;
-          vl[4 * e] = l.x; vl[4 * e + 1] = l.y; vl[4 * e + 2] = l.z; vl[4 * e + 3] = l.w;
-        }
-        tmem_st32u(tmem + lane_base + C::COL_Q + c0, vh);
-        tmem_st32u(tmem + lane_base + C::COL_Q + D / 2 + c0, vl);
-      }
-      tmem_wait_st();
-      fence_before_sync();
-      mbar_arrive(&bars.q_full);
-    }
     const float sl2 = a.scale * L2E;  // score scale in log2 units
     float lrow2 = 0.f;                // WRITE_A: the given lse in log2 units
     if (MODE == FWD_WRITE_A && valid) lrow2 = a.lse_in[q_begin + q] * L2E;
@@ -326,7 +318,7 @@ __global__ void __launch_bounds__(192, 1)
           if (!ok) break;
           fence_after_sync();
 #pragma unroll 1
-          for (int c0 = 0; c0 < D; c0 += 32) {
+          for (int c0 = 0; c0 < 2 * D; c0 += 32) {  // both output halves
             float o[32];
             tmem_ld32(tmem + lane_base + C::COL_O + c0, o);
 #pragma unroll
@@ -355,11 +347,12 @@ __global__ void __launch_bounds__(192, 1)
       if (C::PV) {
 #pragma unroll 1
         for (int c0 = 0; c0 < D; c0 += 32) {
-          float o[32];
+          float o[32], ob[32];
           tmem_ld32(tmem + lane_base + C::COL_O + c0, o);
+          tmem_ld32(tmem + lane_base + C::COL_O + D + c0, ob);
           if (!valid) continue;
 #pragma unroll
-          for (int e = 0; e < 32; ++e) o[e] *= inv;
+          for (int e = 0; e < 32; ++e) o[e] = (o[e] + ob[e]) * inv;  // O = O_a + O_b
           if (MODE == FWD_TARGETS) {
             float4 *y4 = reinterpret_cast<float4 *>(a.y_out + grow * D + c0);
 #pragma unroll
@@ -451,7 +444,7 @@ int launch_fwd_tc(const FwdMaps &m, const FwdArgs &a, int max_tiles, int B, cuda
   static_assert(C::SMEM + sizeof(FwdBars) <= 232448, "shared memory");
   auto kern = k_attn_fwd<D, MODE>;
   KVS_CUDA_TRY(set_smem_once(kern, C::SMEM));
-  kern<<<dim3(max_tiles, B), 192, C::SMEM, st>>>(m.kh, m.kl, m.vh, m.vl, a);
+  kern<<<dim3(max_tiles, B), 192, C::SMEM, st>>>(m.kh, m.kl, m.vh, m.vl, m.qh, m.ql, a);
   KVS_LAUNCH_CHECK("k_attn_fwd");
   return KVS_OK;
 }

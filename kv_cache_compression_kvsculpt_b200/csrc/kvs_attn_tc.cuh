@@ -22,6 +22,7 @@ constexpr int BWD_BQ = 64;
 // Tensor maps of the bf16 operands (2-D, [rows, d], box 64 columns x FWD_BN rows).
 struct FwdMaps {
   CUtensorMap kh, kl, vh, vl;
+  CUtensorMap qh, ql;     // query tiles (box 64 columns x FWD_BN rows)
 };
 
 struct FwdArgs {
