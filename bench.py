@@ -16,6 +16,7 @@ oracle on a bounded sample of the same workload instead.
 from __future__ import annotations
 
 import argparse
+import hashlib
 import json
 import math
 import os
@@ -36,6 +37,37 @@ METRIC = "head-problems compressed/sec at N=2048,r=0.5"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 # CUDA-core fp32 FMA peak from unit counts and clock: 148 SMs x 128 lanes x 2 flop x 1.965 GHz
 DERIVED_PEAKS = {"fp32_simt_tflops": 148 * 128 * 2 * 1.965e9 / 1e12}
+
+
+# Sources of the loss/gradient kernels: the DRAM traffic recorded under profiles/
+# holds only while these files are unchanged.
+TRAFFIC_SOURCES = ["kvs_attn_fwd.cu", "kvs_attn_bwd.cu", "kvs_attn_tc.cuh", "kvs_tc.cuh"]
+TRAFFIC_FILE = os.path.join(ROOT, "profiles", "loss_grad_traffic_qwen_cache_r05.md")
+
+
+def kernel_source_hash():
+    h = hashlib.sha256()
+    for f in TRAFFIC_SOURCES:
+        with open(os.path.join(ROOT, "kv_cache_compression_kvsculpt_b200", "csrc", f), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()
+
+
+def recorded_traffic(workload):
+    """DRAM bytes of one loss/gradient evaluation (forward + key gradient) from the
+    committed ncu summary, or None when the summary is missing, is for another
+    workload, or predates the current kernel sources."""
+    try:
+        with open(TRAFFIC_FILE) as fh:
+            kv = dict(line.strip("- \n").split(": ", 1) for line in fh if ": " in line)
+    except OSError:
+        return None
+    if kv.get("workload") != workload or kv.get("source_sha256") != kernel_source_hash():
+        return None
+    try:
+        return int(kv["dram_bytes_per_launch"])
+    except (KeyError, ValueError):
+        return None
 
 
 def load_peaks():
@@ -293,7 +325,10 @@ def run_gpu(args):
         "roofline": {"kernel": "kvs_loss_grad (forward + dKc backward, whole batch)",
                      "bound": args.bound, "achieved": round(lg_tflops, 3), "peak": peak,
                      "unit": "TFLOP/s", "frac": round(lg_tflops / peak, 4),
-                     "traffic": None, "peak_source": f"{peak_src} {args.peak_key}",
+                     "traffic": recorded_traffic(wl.name),
+                     "traffic_source": "ncu dram__bytes_read.sum + dram__bytes_write.sum of "
+                                       "k_attn_fwd LOSS + k_attn_bwd DK, one launch each",
+                     "peak_source": f"{peak_src} {args.peak_key}",
                      "ms_per_launch": round(lg_ms, 4),
                      "algorithmic_flops_per_launch": lg_flops},
         "gpu_launches": int(launches),

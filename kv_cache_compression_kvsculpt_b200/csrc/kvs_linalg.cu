@@ -48,12 +48,11 @@ __device__ __forceinline__ int kdim(const CholArgs &a, int b) {
 
 __device__ __forceinline__ float4 ld4(const float *p) { return *reinterpret_cast<const float4 *>(p); }
 
-// S[r][c] = M[r0 + r][c0 + c] for r < ROWS, c < 64, r0 + r < rmax, c0 + c < cmax,
-// else 0 (M row-major with ld a multiple of 4 and c0 a multiple of 4).
-template <int ROWS = NB>
+// S[r][c] = M[r0 + r][c0 + c] for r0 + r < rmax, c0 + c < cmax, else 0
+// (M row-major with ld a multiple of 4 and c0 a multiple of 4).
 __device__ __forceinline__ void load_tile(float (*S)[SP], const float *M, int64_t ld, int r0,
                                           int rmax, int c0, int cmax) {
-  for (int e = threadIdx.x; e < ROWS * NB / 4; e += blockDim.x) {
+  for (int e = threadIdx.x; e < NB * NB / 4; e += blockDim.x) {
     const int r = e >> 4, c = (e & 15) * 4;
     float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
     if (r0 + r < rmax && c0 + c < cmax) {
@@ -69,12 +68,11 @@ __device__ __forceinline__ void load_tile(float (*S)[SP], const float *M, int64_
   }
 }
 
-// Transposed: S[c][r] = M[r0 + r][c0 + c] for r < 64, c < 4 COLS4, same bounds.
-template <int COLS4 = NB / 4>
+// Transposed: S[c][r] = M[r0 + r][c0 + c], same bounds.
 __device__ __forceinline__ void load_tile_t(float (*S)[SP], const float *M, int64_t ld, int r0,
                                             int rmax, int c0, int cmax) {
-  for (int e = threadIdx.x; e < NB * COLS4; e += blockDim.x) {
-    const int r = e / COLS4, c = (e % COLS4) * 4;
+  for (int e = threadIdx.x; e < NB * NB / 4; e += blockDim.x) {
+    const int r = e >> 4, c = (e & 15) * 4;
     float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
     if (r0 + r < rmax && c0 + c < cmax) v = ld4(M + (int64_t)(r0 + r) * ld + c0 + c);
     const int m = cmax - c0 - c;
@@ -99,29 +97,6 @@ __device__ __forceinline__ void mm64(const float (*A)[SP], const float (*B)[SP],
     for (int i = 0; i < 4; ++i)
 #pragma unroll
       for (int j = 0; j < 4; ++j) {
-        float s = acc[i][j];
-        s = fmaf(av[i].x, bv[j].x, s);
-        s = fmaf(av[i].y, bv[j].y, s);
-        s = fmaf(av[i].z, bv[j].z, s);
-        acc[i][j] = fmaf(av[i].w, bv[j].w, s);
-      }
-  }
-}
-
-// acc[i][j] += sum_t A[ty + 16 i][t] * B[tx + 16 j][t] over 128 x 128 outputs
-__device__ __forceinline__ void mm128(const float (*A)[SP], const float (*B)[SP],
-                                      float acc[8][8], int tx, int ty) {
-#pragma unroll 1
-  for (int t = 0; t < NB; t += 4) {
-    float4 av[8], bv[8];
-#pragma unroll
-    for (int i = 0; i < 8; ++i) av[i] = *reinterpret_cast<const float4 *>(&A[ty + 16 * i][t]);
-#pragma unroll
-    for (int j = 0; j < 8; ++j) bv[j] = *reinterpret_cast<const float4 *>(&B[tx + 16 * j][t]);
-#pragma unroll
-    for (int i = 0; i < 8; ++i)
-#pragma unroll
-      for (int j = 0; j < 8; ++j) {
         float s = acc[i][j];
         s = fmaf(av[i].x, bv[j].x, s);
         s = fmaf(av[i].y, bv[j].y, s);
@@ -273,15 +248,9 @@ __global__ void __launch_bounds__(256) k_chol_panel(CholArgs a, int j0) {
   }
 }
 
-// Trailing update: 128 x 128 tiles (ti >= tj) of G_ik -= L_i L_k^T, and tiles
-// of r_i -= L_i y_j (all d columns of R in one tile), 8 x 8 outputs per thread.
-constexpr int UT = 128;
-constexpr int UPD_SMEM = 2 * UT * SP * 4;
-
+// Trailing update: tiles (ti >= tj) of G_ik -= L_i L_k^T, and tiles of
+// r_i -= L_i y_j (columns of R in chunks of 64), 64 x 64 outputs per CTA.
 __global__ void __launch_bounds__(256) k_chol_update(CholArgs a, int j0) {
-  extern __shared__ __align__(16) float usm[];
-  float (*As)[SP] = reinterpret_cast<float (*)[SP]>(usm);           // L_i panel rows [row][c]
-  float (*Bs)[SP] = reinterpret_cast<float (*)[SP]>(usm + UT * SP);  // L_k rows, or y_j [col][c]
   const int b = blockIdx.y;
   const int k = kdim(a, b);
   if (j0 >= k || a.dead[b]) return;
@@ -289,51 +258,67 @@ __global__ void __launch_bounds__(256) k_chol_update(CholArgs a, int j0) {
   const int s0 = j0 + jb;
   const int n2 = k - s0;
   if (n2 <= 0) return;
-  const int nt = (n2 + UT - 1) / UT;
+  const int nt = (n2 + NB - 1) / NB;
   const int ntri = nt * (nt + 1) / 2;
+  const int ndc = a.d / NB;
   int t = blockIdx.x;
   bool rhs = false;
-  int ti, tj = 0;
+  int ti, tj;
   if (t < ntri) {
     ti = (int)((sqrtf(8.f * t + 1.f) - 1.f) * 0.5f);
     while (ti * (ti + 1) / 2 > t) --ti;
     while ((ti + 1) * (ti + 2) / 2 <= t) ++ti;
     tj = t - ti * (ti + 1) / 2;
   } else {
-    ti = t - ntri;
-    if (ti >= nt) return;
+    t -= ntri;
+    if (t >= nt * ndc) return;
     rhs = true;
+    ti = t / ndc;
+    tj = t % ndc;
   }
+  __shared__ __align__(16) float As[NB][SP];  // L_i panel rows, [row][c]
+  __shared__ __align__(16) float Bs[NB][SP];  // L_k panel rows [row][c], or y_j as [col][c]
   const int tid = threadIdx.x;
   const int tx = tid & 15, ty = tid >> 4;
   const int64_t row0 = a.c_off[b];
-  const int ri = s0 + ti * UT;
-  load_tile<UT>(As, a.G + row0 * a.ld, a.ld, ri, k, j0, j0 + jb);
-  if (!rhs) {
-    load_tile<UT>(Bs, a.G + row0 * a.ld, a.ld, s0 + tj * UT, k, j0, j0 + jb);
-  } else {
-    // Bs[col][t] = y_j[t][col] for the d columns; rows d .. 127 stay unused
-    load_tile_t<UT / 4>(Bs, a.R + row0 * a.d, a.d, j0, j0 + jb, 0, a.d);
+  const int ri = s0 + ti * NB;
+  // the outputs' current values first: their loads overlap the tile loads
+  float cur[4][4];
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const int r = ri + ty + 16 * i;
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      cur[i][j] = 0.f;
+      if (r >= k) continue;
+      if (!rhs) {
+        const int cc = s0 + tj * NB + tx + 16 * j;
+        if (cc <= r) cur[i][j] = a.G[(row0 + r) * a.ld + cc];
+      } else {
+        cur[i][j] = a.R[(row0 + r) * a.d + tj * NB + tx + 16 * j];
+      }
+    }
   }
+  load_tile(As, a.G + row0 * a.ld, a.ld, ri, k, j0, j0 + jb);
+  if (!rhs)
+    load_tile(Bs, a.G + row0 * a.ld, a.ld, s0 + tj * NB, k, j0, j0 + jb);
+  else
+    load_tile_t(Bs, a.R + row0 * a.d, a.d, j0, j0 + jb, tj * NB, a.d);
   __syncthreads();
-  float acc[8][8];
+  float acc[4][4];
+  zero_acc(acc);
+  mm64(As, Bs, acc, tx, ty);
 #pragma unroll
-  for (int i = 0; i < 8; ++i)
-#pragma unroll
-    for (int j = 0; j < 8; ++j) acc[i][j] = 0.f;
-  mm128(As, Bs, acc, tx, ty);
-#pragma unroll
-  for (int i = 0; i < 8; ++i) {
+  for (int i = 0; i < 4; ++i) {
     const int r = ri + ty + 16 * i;
     if (r >= k) continue;
 #pragma unroll
-    for (int j = 0; j < 8; ++j) {
+    for (int j = 0; j < 4; ++j) {
       if (!rhs) {
-        const int cc = s0 + tj * UT + tx + 16 * j;
-        if (cc <= r) a.G[(row0 + r) * a.ld + cc] -= acc[i][j];
+        const int cc = s0 + tj * NB + tx + 16 * j;
+        if (cc <= r) a.G[(row0 + r) * a.ld + cc] = cur[i][j] - acc[i][j];
       } else {
-        const int col = tx + 16 * j;
-        if (col < a.d) a.R[(row0 + r) * a.d + col] -= acc[i][j];
+        a.R[(row0 + r) * a.d + tj * NB + tx + 16 * j] = cur[i][j] - acc[i][j];
       }
     }
   }
@@ -429,7 +414,6 @@ int launch_chol_solve(const Batch &Bt, float *Vc, int32_t *status, const Work &w
   const HostGeom &g = Bt.g;
   const int npanel = (g.max_c + NB - 1) / NB;
   CholArgs a{w.gram, w.R, w.X, w.chol_t, npanel, w.dead, status, Bt.b->c_off, g.ld_g, g.d};
-  KVS_CUDA_TRY(set_smem_once(k_chol_update, UPD_SMEM));
   KVS_CUDA_TRY(cudaMemsetAsync(w.dead, 0, sizeof(int) * g.B, Bt.st));
   const int ndc = g.d / NB;
   for (int p = 0; p < npanel; ++p) {
@@ -441,8 +425,7 @@ int launch_chol_solve(const Batch &Bt, float *Vc, int32_t *status, const Work &w
     const int nt = (n2 + NB - 1) / NB;
     k_chol_panel<<<dim3(nt, g.B), 256, 0, Bt.st>>>(a, j0);
     KVS_LAUNCH_CHECK("k_chol_panel");
-    const int nt2 = (n2 + UT - 1) / UT;
-    k_chol_update<<<dim3(nt2 * (nt2 + 1) / 2 + nt2, g.B), 256, UPD_SMEM, Bt.st>>>(a, j0);
+    k_chol_update<<<dim3(nt * (nt + 1) / 2 + nt * ndc, g.B), 256, 0, Bt.st>>>(a, j0);
     KVS_LAUNCH_CHECK("k_chol_update");
   }
   for (int p = npanel - 1; p >= 0; --p) {
