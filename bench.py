@@ -151,11 +151,11 @@ def group_size(group):
 class Job:
     """Device buffers of one rank's batch and the calls of one step."""
 
-    def __init__(self, wl, seq, dev, group=None):
+    def __init__(self, wl, seqs, dev, group=None):
         import torch
         import kv_cache_compression_kvsculpt_b200 as K
         self.K, self.torch, self.wl, self.group = K, torch, wl, group
-        ids = [(seq, l, h) for l in range(wl.n_layers) for h in range(wl.n_kv_heads)]
+        ids = [(s, l, h) for s in seqs for l in range(wl.n_layers) for h in range(wl.n_kv_heads)]
         self.bt = W.make_batch(wl, 0, ids)
         B = self.bt.B
         self.host = {
@@ -215,6 +215,18 @@ class Job:
 
     def d2h_bytes(self):
         return sum(v.numel() * v.element_size() for v in self.out_host.values())
+
+
+def rank_sequences(wl, rank, world):
+    """Sequences (each n_layers x n_kv_heads head-problems) this rank compresses.
+    A workload of several sequences is partitioned over the ranks (the total is
+    fixed: strong scaling; the rank count must divide it); a one-sequence
+    workload gives every rank a sequence of its own (weak scaling)."""
+    if wl.n_seq > 1:
+        if wl.n_seq % world:
+            raise SystemExit(f"{wl.name}: {wl.n_seq} sequences do not split over {world} ranks")
+        return list(range(rank, wl.n_seq, world)), "strong"
+    return [rank], "weak"
 
 
 def time_region(torch, fn, n, dist=None):
@@ -278,7 +290,8 @@ def run_gpu(args):
     wl = W.WORKLOADS[args.workload]
     if args.outer is not None:
         wl = wl.with_(outer=args.outer)
-    job = Job(wl, seq=rank, dev="cuda", group=dist.group.WORLD if dist else None)
+    seqs, scaling = rank_sequences(wl, rank, world)
+    job = Job(wl, seqs, dev="cuda", group=dist.group.WORLD if dist else None)
     for _ in range(args.warmup):
         job.step()
     torch.cuda.synchronize()
@@ -289,7 +302,7 @@ def run_gpu(args):
     launches = K.kvs_launch_count() - n0
     status = job.status.cpu().numpy()
     ms_step = ms / args.steps
-    problems = wl.B * world
+    problems = job.batch.B * world  # every rank holds the same number of problems
     value = problems / (ms_step * 1e-3)
     # e2e through host buffers
     job.step_e2e()
@@ -312,11 +325,11 @@ def run_gpu(args):
         "warmup": args.warmup,
         "ms_per_step": round(ms_step, 3),
         "higher_is_better": True,
-        "scaling": "weak",
+        "scaling": scaling,
         "vs_baseline": None,
         "dtype": args.dtype_label,
         "data": "synthetic (seeded generator; stands in for Qwen2.5-1.5B-Instruct KV caches)",
-        "config": {"workload": describe(wl), "problems_per_gpu": wl.B,
+        "config": {"workload": describe(wl), "problems_per_gpu": job.batch.B,
                    "l2": "inputs and per-step working set larger than L2 (126 MB)",
                    "parallelism": f"problem-sharded x{world}, no collective"},
         "e2e": {"value": round(e2e_value, 4), "unit": "head-problems/s",

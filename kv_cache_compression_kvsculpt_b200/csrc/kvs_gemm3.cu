@@ -30,7 +30,11 @@ struct G3 {
   static constexpr int STAGE = 2 * A_BYTES + 2 * B_BYTES;  // A hi, A lo, B hi, B lo
   static constexpr int NS = TN > 128 ? 2 : 3;
   static constexpr int SMEM = NS * STAGE + 1024;
-  static constexpr uint32_t TMEM_COLS = TN < 32 ? 32 : TN;
+  // tiles up to 128 wide take B_hi and B_lo side by side as one operand of N = 2 TN
+  // (two instructions per 16-row step instead of three), into two summed halves
+  static constexpr bool CAT = TN <= 128;
+  static constexpr int MMA_N = CAT ? 2 * TN : TN;
+  static constexpr uint32_t TMEM_COLS = MMA_N < 32 ? 32 : MMA_N;
 };
 constexpr int NSMAX = 3;
 
@@ -142,7 +146,7 @@ __global__ void __launch_bounds__(192, 1)
     }
   } else if (warp == 5) {
     if (lane == 0) {
-      const uint32_t id = idesc_bf16(TM, N, true, true);
+      const uint32_t id = idesc_bf16(TM, C::MMA_N, true, true);
       bool ok = true;
       for (int i = 0; i < nkt; ++i) {
         const int st = i % NS;
@@ -155,9 +159,14 @@ __global__ void __launch_bounds__(192, 1)
           const uint64_t al = sdesc_add(ah, A_BYTES);
           const uint64_t bh = sdesc_add(ah, 2 * A_BYTES);
           const uint64_t bl = sdesc_add(ah, 2 * A_BYTES + C::B_BYTES);
-          mma_bf16(tmem, ah, bh, id, (i > 0 || kk > 0) ? 1u : 0u);
-          mma_bf16(tmem, ah, bl, id, 1u);
-          mma_bf16(tmem, al, bh, id, 1u);
+          if (C::CAT) {  // A_hi [B_hi | B_lo] + A_lo [B_hi | B_lo]
+            mma_bf16(tmem, ah, bh, id, (i > 0 || kk > 0) ? 1u : 0u);
+            mma_bf16(tmem, al, bh, id, 1u);
+          } else {
+            mma_bf16(tmem, ah, bh, id, (i > 0 || kk > 0) ? 1u : 0u);
+            mma_bf16(tmem, ah, bl, id, 1u);
+            mma_bf16(tmem, al, bh, id, 1u);
+          }
         }
         mma_commit(&bars.empty[st]);
       }
@@ -176,6 +185,12 @@ __global__ void __launch_bounds__(192, 1)
     for (int c0 = 0; c0 < N; c0 += 32) {
       float v[32];
       tmem_ld32(tmem + lane_base + c0, v);
+      if (C::CAT) {
+        float v2[32];
+        tmem_ld32(tmem + lane_base + TN + c0, v2);
+#pragma unroll
+        for (int e = 0; e < 32; ++e) v[e] += v2[e];
+      }
       if (gi < nk && nkt > 0) {
 #pragma unroll
         for (int e = 0; e < 32; ++e) {
