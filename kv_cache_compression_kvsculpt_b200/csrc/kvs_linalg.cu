@@ -11,7 +11,8 @@
 //     panel   L_ij = G_ij T_j^T for the rows below
 //     update  G_ik -= L_ij L_kj^T on the trailing lower triangle and
 //             r_i -= L_ij y_j on the right-hand sides
-//   then per panel from the last one: x_j = T_j^T y_j, y_i -= L_ji^T x_j.
+//   then one kernel sweeps the panels from the last one: x_j = T_j^T y_j,
+//   y_i -= L_ji^T x_j.
 // Every 64 x 64 product runs from shared memory with 4 x 4 register tiles and
 // 128-bit shared loads.  The factor overwrites the Gram matrix, the forward
 // sweep the right-hand sides; the solution goes to a separate buffer and is
@@ -324,69 +325,93 @@ __global__ void __launch_bounds__(256) k_chol_update(CholArgs a, int j0) {
   }
 }
 
-// Backward sweep at panel j0: x_j = T_j^T y_j (each CTA forms it for its 64
-// right-hand-side columns; the CTAs of row block 0 store it and check it is
-// finite), then y_i -= L_ji^T x_j for the row block i < j0 of this CTA.
-__global__ void __launch_bounds__(256) k_chol_bsolve(CholArgs a, int j0) {
-  const int b = blockIdx.z;
+// The whole backward sweep for 64 right-hand-side columns of one problem, from
+// the last panel to the first: x_j = T_j^T y_j (stored, checked finite), then
+// y_i -= L_ji^T x_j for every i < j.  The next L_ji tile is fetched into
+// registers while the current one is multiplied (two shared tiles in turn).
+constexpr int BWD_SMEM = 3 * NB * SP * 4;
+
+__global__ void __launch_bounds__(256) k_chol_backward(CholArgs a) {
+  extern __shared__ __align__(16) float bsm[];
+  float (*Xs)[SP] = reinterpret_cast<float (*)[SP]>(bsm);
+  float (*At[2])[SP] = {reinterpret_cast<float (*)[SP]>(bsm + NB * SP),
+                        reinterpret_cast<float (*)[SP]>(bsm + 2 * NB * SP)};
+  const int b = blockIdx.y;
   const int k = kdim(a, b);
-  if (j0 >= k || a.dead[b]) return;
-  const int jb = min(NB, k - j0);
-  const int i0 = blockIdx.y * NB;
-  if (i0 > 0 && i0 >= j0) return;
+  if (a.dead[b]) return;
   const int c0 = blockIdx.x * NB;
-  __shared__ __align__(16) float As[NB][SP];
-  __shared__ __align__(16) float Bs[NB][SP];
+  const int np = (k + NB - 1) / NB;
   const int tid = threadIdx.x;
   const int tx = tid & 15, ty = tid >> 4;
   const int64_t row0 = a.c_off[b];
-  const float *Tg = a.T + ((int64_t)b * a.npanel + j0 / NB) * NB * NB;
-  load_tile_t(As, Tg, NB, 0, NB, 0, NB);                         // As[r][t] = T[t][r]
-  load_tile_t(Bs, a.R + row0 * a.d, a.d, j0, j0 + jb, c0, a.d);  // Bs[col][t] = y[t][col]
-  __syncthreads();
-  float acc[4][4];
-  zero_acc(acc);
-  mm64(As, Bs, acc, tx, ty);  // x[r][col]
-  if (blockIdx.y == 0) {
+  const float *G = a.G + row0 * a.ld;
+  float *R = a.R + row0 * a.d;
+  for (int p = np - 1; p >= 0; --p) {
+    const int j0 = p * NB, jb = min(NB, k - j0);
+    const float *Tg = a.T + ((int64_t)b * a.npanel + p) * NB * NB;
+    load_tile_t(At[0], Tg, NB, 0, NB, 0, NB);           // At[r][t] = T[t][r]
+    load_tile_t(Xs, R, a.d, j0, j0 + jb, c0, a.d);      // Xs[col][t] = y[j0 + t][c0 + col]
+    __syncthreads();
+    float acc[4][4];
+    zero_acc(acc);
+    mm64(At[0], Xs, acc, tx, ty);                       // x[r][col]
+    __syncthreads();
     bool fin = true;
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
       const int r = ty + 16 * i;
-      if (r >= jb) continue;
 #pragma unroll
       for (int j = 0; j < 4; ++j) {
-        a.X[(row0 + j0 + r) * a.d + c0 + tx + 16 * j] = acc[i][j];
-        fin &= isfinite(acc[i][j]);
+        Xs[tx + 16 * j][r] = acc[i][j];  // as the B operand of the updates
+        if (r < jb) {
+          a.X[(row0 + j0 + r) * a.d + c0 + tx + 16 * j] = acc[i][j];
+          fin &= isfinite(acc[i][j]);
+        }
       }
     }
     if (!fin) atomicOr(&a.dead[b], DEAD_NONFINITE);
-  }
-  if (j0 == 0) return;
-  __syncthreads();
-  // Bs[col][t] = x[t][col]; As[r][t] = L[j0 + t][i0 + r]
+    if (p == 0) break;
+    // y_i -= L_ji^T x_j, with At[r][t] = L[j0 + t][64 i + r]
+    float4 pf[4];
+    auto fetch = [&](int i) {
 #pragma unroll
-  for (int i = 0; i < 4; ++i)
+      for (int u = 0; u < 4; ++u) {
+        const int e = tid + 256 * u, r = e >> 4, c = (e & 15) * 4;
+        pf[u] = r < jb ? ld4(G + (int64_t)(j0 + r) * a.ld + NB * i + c)
+                       : make_float4(0.f, 0.f, 0.f, 0.f);
+      }
+    };
+    auto place = [&](float (*S)[SP]) {
 #pragma unroll
-    for (int j = 0; j < 4; ++j) Bs[tx + 16 * j][ty + 16 * i] = acc[i][j];
-  load_tile_t(As, a.G + row0 * a.ld, a.ld, j0, j0 + jb, i0, j0);
-  float cur[4][4];
+      for (int u = 0; u < 4; ++u) {
+        const int e = tid + 256 * u, r = e >> 4, c = (e & 15) * 4;
+        S[c][r] = pf[u].x;
+        S[c + 1][r] = pf[u].y;
+        S[c + 2][r] = pf[u].z;
+        S[c + 3][r] = pf[u].w;
+      }
+    };
+    fetch(0);
+    place(At[0]);
+    __syncthreads();
+    for (int i = 0; i < p; ++i) {
+      float cur[4][4];
 #pragma unroll
-  for (int i = 0; i < 4; ++i)
+      for (int ii = 0; ii < 4; ++ii)
 #pragma unroll
-    for (int j = 0; j < 4; ++j) {
-      const int r = i0 + ty + 16 * i;
-      cur[i][j] = r < j0 ? a.R[(row0 + r) * a.d + c0 + tx + 16 * j] : 0.f;
+        for (int jj = 0; jj < 4; ++jj)
+          cur[ii][jj] = R[(int64_t)(NB * i + ty + 16 * ii) * a.d + c0 + tx + 16 * jj];
+      if (i + 1 < p) fetch(i + 1);
+      zero_acc(acc);
+      mm64(At[i & 1], Xs, acc, tx, ty);
+#pragma unroll
+      for (int ii = 0; ii < 4; ++ii)
+#pragma unroll
+        for (int jj = 0; jj < 4; ++jj)
+          R[(int64_t)(NB * i + ty + 16 * ii) * a.d + c0 + tx + 16 * jj] = cur[ii][jj] - acc[ii][jj];
+      if (i + 1 < p) place(At[(i + 1) & 1]);
+      __syncthreads();
     }
-  __syncthreads();
-  zero_acc(acc);
-  mm64(As, Bs, acc, tx, ty);
-#pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    const int r = i0 + ty + 16 * i;
-    if (r >= j0) continue;
-#pragma unroll
-    for (int j = 0; j < 4; ++j)
-      a.R[(row0 + r) * a.d + c0 + tx + 16 * j] = cur[i][j] - acc[i][j];
   }
 }
 
@@ -414,6 +439,7 @@ int launch_chol_solve(const Batch &Bt, float *Vc, int32_t *status, const Work &w
   const HostGeom &g = Bt.g;
   const int npanel = (g.max_c + NB - 1) / NB;
   CholArgs a{w.gram, w.R, w.X, w.chol_t, npanel, w.dead, status, Bt.b->c_off, g.ld_g, g.d};
+  KVS_CUDA_TRY(set_smem_once(k_chol_backward, BWD_SMEM));
   KVS_CUDA_TRY(cudaMemsetAsync(w.dead, 0, sizeof(int) * g.B, Bt.st));
   const int ndc = g.d / NB;
   for (int p = 0; p < npanel; ++p) {
@@ -428,10 +454,8 @@ int launch_chol_solve(const Batch &Bt, float *Vc, int32_t *status, const Work &w
     k_chol_update<<<dim3(nt * (nt + 1) / 2 + nt * ndc, g.B), 256, 0, Bt.st>>>(a, j0);
     KVS_LAUNCH_CHECK("k_chol_update");
   }
-  for (int p = npanel - 1; p >= 0; --p) {
-    k_chol_bsolve<<<dim3(ndc, std::max(p, 1), g.B), 256, 0, Bt.st>>>(a, p * NB);
-    KVS_LAUNCH_CHECK("k_chol_bsolve");
-  }
+  k_chol_backward<<<dim3(ndc, g.B), 256, BWD_SMEM, Bt.st>>>(a);
+  KVS_LAUNCH_CHECK("k_chol_backward");
   const int64_t n4 = (int64_t)g.max_c * g.d / 4;
   const int blocks = (int)std::min<int64_t>((n4 + 255) / 256, 64);
   k_chol_store<<<dim3(blocks, g.B), 256, 0, Bt.st>>>(a, Vc);
