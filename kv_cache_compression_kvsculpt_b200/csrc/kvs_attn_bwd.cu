@@ -264,13 +264,12 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       float s[BQ];
       tmem_ld32(tmem + lane_base + sb * BQ, s);
       tmem_ld32(tmem + lane_base + sb * BQ + 32, s + 32);
-      const int qvalid = nq - (t0 + i) * BQ;
       if (!C::DK) {
         fence_before_sync();
         mbar_arrive(&bars.sd_free[sb]);
 #pragma unroll
         for (int c = 0; c < BQ; ++c)
-          imp += (c < qvalid) ? exp2f(fmaf(s[c], sl2, -bars.lse2[st][c])) : 0.f;
+          imp += ex2(fmaf(s[c], sl2, -bars.lse2[st][c]));  // l = +inf past the problem
       } else {
         float dp[BQ];
         tmem_ld32(tmem + lane_base + C::COL_DP + sb * BQ, dp);
@@ -282,8 +281,10 @@ __global__ void __launch_bounds__(NTHREADS, 1)
 #pragma unroll
           for (int u = 0; u < 2; ++u) {
             const int c = 2 * c2 + u;
-            const float p = exp2f(fmaf(s[c], sl2, -bars.lse2[st][c]));
-            v[u] = (kvalid && c < qvalid) ? p * (dp[c] - bars.del[st][c]) : 0.f;
+            // queries past the problem have l = +inf (p = 0) and delta = 0; rows of keys
+            // past it only feed their own dK rows, which are not stored
+            const float p = ex2(fmaf(s[c], sl2, -bars.lse2[st][c]));
+            v[u] = p * (dp[c] - bars.del[st][c]);
           }
           split_pack(v[0], v[1], hh[c2], ll[c2]);
         }

@@ -253,9 +253,11 @@ __global__ void __launch_bounds__(192, 1)
       float s[BN];
 #pragma unroll
       for (int c0 = 0; c0 < BN; c0 += 32) tmem_ld32(tmem + lane_base + sb * BN + c0, s + c0);
-      const int kvalid = nk - j * BN;
+      const int kvalid = nk - j * BN;  // raw scores; keys past the problem get -inf
+      if (kvalid < BN) {
 #pragma unroll
-      for (int c = 0; c < BN; ++c) s[c] = (c < kvalid) ? s[c] * sl2 : -INFINITY;
+        for (int c = 0; c < BN; ++c) s[c] = (c < kvalid) ? s[c] : -INFINITY;
+      }
       if (!C::PV) {
         fence_before_sync();
         mbar_arrive(&bars.s_free[sb]);
@@ -270,8 +272,8 @@ __global__ void __launch_bounds__(192, 1)
           uint32_t h[4], l[4];
 #pragma unroll
           for (int e = 0; e < 4; ++e) {
-            const float p0 = valid ? exp2f(s[ch * 8 + 2 * e] - lrow2) : 0.f;
-            const float p1 = valid ? exp2f(s[ch * 8 + 2 * e + 1] - lrow2) : 0.f;
+            const float p0 = valid ? ex2(fmaf(s[ch * 8 + 2 * e], sl2, -lrow2)) : 0.f;
+            const float p1 = valid ? ex2(fmaf(s[ch * 8 + 2 * e + 1], sl2, -lrow2)) : 0.f;
             split_pack(p0, p1, h[e], l[e]);
           }
           dh[ch] = make_uint4(h[0], h[1], h[2], h[3]);
@@ -282,12 +284,13 @@ __global__ void __launch_bounds__(192, 1)
       float mt = -INFINITY;
 #pragma unroll
       for (int c = 0; c < BN; ++c) mt = fmaxf(mt, s[c]);
+      mt *= sl2;  // the scale is positive: the max of the scaled scores
       float alpha = 1.f;
       bool rescale = false;
       if (mt > mref + kRescale || mref == -INFINITY) {
         const float mnew = fmaxf(mt, mref);
         if (mref != -INFINITY) {
-          alpha = exp2f(mref - mnew);
+          alpha = ex2(mref - mnew);
           rescale = true;
         }
         mref = mnew;
@@ -295,7 +298,7 @@ __global__ void __launch_bounds__(192, 1)
       float ts = 0.f;
 #pragma unroll
       for (int c = 0; c < BN; ++c) {
-        s[c] = exp2f(s[c] - mref);
+        s[c] = ex2(fmaf(s[c], sl2, -mref));
         ts += s[c];
       }
       lsum = lsum * alpha + ts;
