@@ -62,8 +62,8 @@ struct BwdBars {
   uint64_t done;
   uint32_t tmem;
   int abort;
-  float lse2[NSTAGE][BQ];   // row lse in log2 units (+inf for rows outside the problem)
-  float del[NSTAGE][BQ];
+  __align__(16) float lse2[NSTAGE][BQ];  // row lse in log2 units (+inf past the problem)
+  __align__(16) float del[NSTAGE][BQ];
   float imp[BK];       // COLSUM: warpgroup 1's partial importance
 };
 
@@ -267,26 +267,32 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       if (!C::DK) {
         fence_before_sync();
         mbar_arrive(&bars.sd_free[sb]);
+        const float4 *l4 = reinterpret_cast<const float4 *>(bars.lse2[st]);
 #pragma unroll
-        for (int c = 0; c < BQ; ++c)
-          imp += ex2(fmaf(s[c], sl2, -bars.lse2[st][c]));  // l = +inf past the problem
+        for (int c4 = 0; c4 < BQ / 4; ++c4) {  // l = +inf past the problem
+          const float4 l = l4[c4];
+          imp += ex2(fmaf(s[4 * c4], sl2, -l.x)) + ex2(fmaf(s[4 * c4 + 1], sl2, -l.y)) +
+                 ex2(fmaf(s[4 * c4 + 2], sl2, -l.z)) + ex2(fmaf(s[4 * c4 + 3], sl2, -l.w));
+        }
       } else {
         float dp[BQ];
         tmem_ld32(tmem + lane_base + C::COL_DP + sb * BQ, dp);
         tmem_ld32(tmem + lane_base + C::COL_DP + sb * BQ + 32, dp + 32);
         uint32_t hh[32], ll[32];
+        const float4 *l4 = reinterpret_cast<const float4 *>(bars.lse2[st]);
+        const float4 *d4 = reinterpret_cast<const float4 *>(bars.del[st]);
 #pragma unroll
-        for (int c2 = 0; c2 < 32; ++c2) {
-          float v[2];
-#pragma unroll
-          for (int u = 0; u < 2; ++u) {
-            const int c = 2 * c2 + u;
-            // queries past the problem have l = +inf (p = 0) and delta = 0; rows of keys
-            // past it only feed their own dK rows, which are not stored
-            const float p = ex2(fmaf(s[c], sl2, -bars.lse2[st][c]));
-            v[u] = p * (dp[c] - bars.del[st][c]);
-          }
-          split_pack(v[0], v[1], hh[c2], ll[c2]);
+        for (int c4 = 0; c4 < BQ / 4; ++c4) {
+          // queries past the problem have l = +inf (p = 0) and delta = 0; rows of keys
+          // past it only feed their own dK rows, which are not stored
+          const float4 l = l4[c4], dl = d4[c4];
+          const int c = 4 * c4;
+          const float v0 = ex2(fmaf(s[c], sl2, -l.x)) * (dp[c] - dl.x);
+          const float v1 = ex2(fmaf(s[c + 1], sl2, -l.y)) * (dp[c + 1] - dl.y);
+          const float v2 = ex2(fmaf(s[c + 2], sl2, -l.z)) * (dp[c + 2] - dl.z);
+          const float v3 = ex2(fmaf(s[c + 3], sl2, -l.w)) * (dp[c + 3] - dl.w);
+          split_pack(v0, v1, hh[2 * c4], ll[2 * c4]);
+          split_pack(v2, v3, hh[2 * c4 + 1], ll[2 * c4 + 1]);
         }
         // dS (hi, lo) over the S buffer: the A operand of dK += dS Q
         tmem_st32u(tmem + lane_base + sb * BQ, hh);

@@ -23,9 +23,12 @@
 //   TARGETS  keys K_z, values V_z: writes Y (fp32 and bf16 hi/lo) and l
 //   STATS    row log-sum-exp only
 //   WRITE_A  given l_hat: writes A = exp(S - l_hat) as bf16 hi/lo
-// Warp roles: warps 0-3 softmax/epilogue (thread t <-> TMEM lane t <-> query
-// row t), warp 4 TMA producer (Q once, then keys and values), warp 5 TMEM
-// allocator and MMA issuer.
+// Two row warpgroups split every key tile: warpgroup g takes keys 64g .. 64g+63
+// of each tile for all 128 query rows (the row maximum is exchanged through
+// shared memory once per tile), and output columns g*d/2 .. in the epilogue.
+// Warp roles: warps 0-7 softmax/epilogue (warp w <-> TMEM lanes 32 (w % 4) ..,
+// thread t <-> query row t % 128), warp 8 TMA producer (Q once, then keys and
+// values), warp 9 TMEM allocator and MMA issuer.
 #include <math.h>
 
 #include "kvs_attn_tc.cuh"
@@ -37,6 +40,8 @@ using namespace tc;
 
 constexpr int BM = 128;          // queries per CTA
 constexpr int BN = FWD_BN;       // keys per tile
+constexpr int HB = BN / 2;       // keys of a tile per row warpgroup
+constexpr int NTHREADS = 320;
 constexpr float kRescale = 8.f;  // lazy rescale threshold (log2 units)
 constexpr float L2E = 1.4426950408889634f;
 static_assert(BN == 128, "tensor-memory layout assumes 128-key tiles");
@@ -68,10 +73,30 @@ struct FwdBars {
   uint32_t tmem;
   int abort;
   float red[8];
+  float mx[2][BM];       // per warpgroup row maximum of the current tile (raw scores)
+  float ls[2][BM];       // per warpgroup running sums
+  float part[2][BM][2];  // per warpgroup half-row sums: |Yh - Y|^2, Go . Yh
 };
 
+__device__ __forceinline__ void rows_sync() { asm volatile("bar.sync 1, 256;" ::: "memory"); }
+
+// Barrier of the 256 row threads that also ANDs a predicate over them: every
+// row thread leaves the tile loop at the same tile.
+__device__ __forceinline__ bool rows_all(bool p) {
+  uint32_t r;
+  asm volatile(
+      "{\n\t.reg .pred p, q;\n\t"
+      "setp.ne.u32 p, %1, 0;\n\t"
+      "bar.red.and.pred q, 1, 256, p;\n\t"
+      "selp.u32 %0, 1, 0, q;\n\t}"
+      : "=r"(r)
+      : "r"((uint32_t)p)
+      : "memory");
+  return r != 0;
+}
+
 template <int D, int MODE>
-__global__ void __launch_bounds__(192, 1)
+__global__ void __launch_bounds__(NTHREADS, 1)
     k_attn_fwd(const __grid_constant__ CUtensorMap mKh, const __grid_constant__ CUtensorMap mKl,
                const __grid_constant__ CUtensorMap mVh, const __grid_constant__ CUtensorMap mVl,
                const __grid_constant__ CUtensorMap mQh, const __grid_constant__ CUtensorMap mQl,
@@ -103,21 +128,21 @@ __global__ void __launch_bounds__(192, 1)
     }
     for (int i = 0; i < 2; ++i) {
       mbar_init(&bars.s_full[i], 1);
-      mbar_init(&bars.s_free[i], C::PV ? 1 : BM);
-      mbar_init(&bars.p_full[i], BM);
+      mbar_init(&bars.s_free[i], C::PV ? 1 : 2 * BM);
+      mbar_init(&bars.p_full[i], 2 * BM);
     }
     mbar_init(&bars.o_done, 1);
     bars.abort = 0;
     fence_barrier_init();
   }
-  if (warp == 5) tmem_alloc(&bars.tmem, C::TMEM_COLS);
+  if (warp == 9) tmem_alloc(&bars.tmem, C::TMEM_COLS);
   fence_before_sync();
   __syncthreads();
   fence_after_sync();
   const uint32_t tmem = bars.tmem;
   volatile int *abort = &bars.abort;
 
-  if (warp == 4) {
+  if (warp == 8) {
     // ------------------------------------------------------------ TMA producer
     if (lane == 0) {
       tma_prefetch_map(&mKh);
@@ -178,7 +203,7 @@ __global__ void __launch_bounds__(192, 1)
           mbar_wait(&bars.v_full[j % C::NSVI], (j / C::NSVI) & 1);
       }
     }
-  } else if (warp == 5) {
+  } else if (warp == 9) {
     // ------------------------------------------------------------- MMA issuer
     if (lane == 0) {
       const uint32_t id_s128 = idesc_bf16(BM, BN, false, false);
@@ -236,27 +261,34 @@ __global__ void __launch_bounds__(192, 1)
     }
   } else {
     // ------------------------------------------------- softmax / epilogue rows
-    const int row = tid;  // 0..127
+    const int wg = warp >> 2;          // keys 64 wg .. of every tile
+    const int row = tid & (BM - 1);    // query row
+    const int cb = wg * HB;            // first key (S column) of this warpgroup
     const int q = q0 + row;
     const bool valid = q < nq;
-    const uint32_t lane_base = (uint32_t)(warp * 32) << 16;
+    const uint32_t lane_base = (uint32_t)((warp & 3) * 32) << 16;
     const float sl2 = a.scale * L2E;  // score scale in log2 units
     float lrow2 = 0.f;                // WRITE_A: the given lse in log2 units
     if (MODE == FWD_WRITE_A && valid) lrow2 = a.lse_in[q_begin + q] * L2E;
-    float mref = -INFINITY, lsum = 0.f;
+    float mref = -INFINITY, lsum = 0.f;  // mref is the same in both warpgroups
     bool ok = true;
     for (int j = 0; j < ntiles; ++j) {
       const int sb = j & 1;
-      ok = __all_sync(0xffffffffu, mbar_wait(&bars.s_full[sb], (j >> 1) & 1, abort));
-      if (!ok) break;
-      fence_after_sync();
-      float s[BN];
+      ok = ok && __all_sync(0xffffffffu, mbar_wait(&bars.s_full[sb], (j >> 1) & 1, abort));
+      if (MODE == FWD_WRITE_A && !ok) break;  // no barrier below in this mode
+      float s[HB];
+      if (ok) {
+        fence_after_sync();
+        tmem_ld32(tmem + lane_base + sb * BN + cb, s);
+        tmem_ld32(tmem + lane_base + sb * BN + cb + 32, s + 32);
+      } else {
 #pragma unroll
-      for (int c0 = 0; c0 < BN; c0 += 32) tmem_ld32(tmem + lane_base + sb * BN + c0, s + c0);
-      const int kvalid = nk - j * BN;  // raw scores; keys past the problem get -inf
-      if (kvalid < BN) {
+        for (int c = 0; c < HB; ++c) s[c] = -INFINITY;
+      }
+      const int kvalid = nk - j * BN - cb;  // raw scores; keys past the problem get -inf
+      if (kvalid < HB) {
 #pragma unroll
-        for (int c = 0; c < BN; ++c) s[c] = (c < kvalid) ? s[c] : -INFINITY;
+        for (int c = 0; c < HB; ++c) s[c] = (c < kvalid) ? s[c] : -INFINITY;
       }
       if (!C::PV) {
         fence_before_sync();
@@ -265,10 +297,10 @@ __global__ void __launch_bounds__(192, 1)
       if (MODE == FWD_WRITE_A) {
         // A = exp2(t - lse2), split into bf16 hi / lo, into the padded A buffer
         const int64_t arow = a.a_pad_off[b] + q0 + row;
-        uint4 *dh = reinterpret_cast<uint4 *>(a.a_hi + arow * a.ld_a + j * BN);
-        uint4 *dl = reinterpret_cast<uint4 *>(a.a_lo + arow * a.ld_a + j * BN);
+        uint4 *dh = reinterpret_cast<uint4 *>(a.a_hi + arow * a.ld_a + j * BN + cb);
+        uint4 *dl = reinterpret_cast<uint4 *>(a.a_lo + arow * a.ld_a + j * BN + cb);
 #pragma unroll
-        for (int ch = 0; ch < BN / 8; ++ch) {
+        for (int ch = 0; ch < HB / 8; ++ch) {
           uint32_t h[4], l[4];
 #pragma unroll
           for (int e = 0; e < 4; ++e) {
@@ -283,8 +315,13 @@ __global__ void __launch_bounds__(192, 1)
       }
       float mt = -INFINITY;
 #pragma unroll
-      for (int c = 0; c < BN; ++c) mt = fmaxf(mt, s[c]);
-      mt *= sl2;  // the scale is positive: the max of the scaled scores
+      for (int c = 0; c < HB; ++c) mt = fmaxf(mt, s[c]);
+      // the tile's row maximum over both halves; the barrier also orders both
+      // warpgroups' S loads before either writes P over the buffer
+      bars.mx[wg][row] = mt;
+      ok = rows_all(ok);  // a wait that gave up anywhere ends the loop for every row
+      if (!ok) break;
+      mt = fmaxf(bars.mx[0][row], bars.mx[1][row]) * sl2;  // the scale is positive
       float alpha = 1.f;
       bool rescale = false;
       if (mt > mref + kRescale || mref == -INFINITY) {
@@ -297,36 +334,37 @@ __global__ void __launch_bounds__(192, 1)
       }
       float ts = 0.f;
 #pragma unroll
-      for (int c = 0; c < BN; ++c) {
+      for (int c = 0; c < HB; ++c) {
         s[c] = ex2(fmaf(s[c], sl2, -mref));
         ts += s[c];
       }
       lsum = lsum * alpha + ts;
       if (C::PV) {
-        // P (hi, lo) over the S buffer: the A operand of O += P V
-#pragma unroll
-        for (int h = 0; h < 2; ++h) {
+        // P (hi, lo) of this warpgroup's keys over the S buffer: the A operand of O += P V
+        {
           uint32_t ph[32], pl[32];
 #pragma unroll
-          for (int c = 0; c < 32; ++c)
-            split_pack(s[64 * h + 2 * c], s[64 * h + 2 * c + 1], ph[c], pl[c]);
-          tmem_st32u(tmem + lane_base + sb * BN + 32 * h, ph);
-          tmem_st32u(tmem + lane_base + sb * BN + BN / 2 + 32 * h, pl);
+          for (int c = 0; c < 32; ++c) split_pack(s[2 * c], s[2 * c + 1], ph[c], pl[c]);
+          tmem_st32u(tmem + lane_base + sb * BN + cb / 2, ph);
+          tmem_st32u(tmem + lane_base + sb * BN + BN / 2 + cb / 2, pl);
         }
         if (__any_sync(0xffffffffu, rescale)) {
           // O *= alpha once PV of tile j-1 has landed (PV of tile j waits for p_full);
-          // the TMEM access is warp-wide, rows without a new max use alpha = 1.
+          // the TMEM access is warp-wide, rows without a new max use alpha = 1.  The
+          // rows' rescale decisions are the same in both warpgroups; each scales
+          // one output half.
           const int pj = j - 1;
           ok = __all_sync(0xffffffffu, mbar_wait(&bars.s_free[pj & 1], (pj >> 1) & 1, abort));
-          if (!ok) break;
-          fence_after_sync();
+          if (ok) {  // a failed wait ends the loop at the next tile's row barrier
+            fence_after_sync();
 #pragma unroll 1
-          for (int c0 = 0; c0 < 2 * D; c0 += 32) {  // both output halves
-            float o[32];
-            tmem_ld32(tmem + lane_base + C::COL_O + c0, o);
+            for (int c0 = wg * D; c0 < (wg + 1) * D; c0 += 32) {
+              float o[32];
+              tmem_ld32(tmem + lane_base + C::COL_O + c0, o);
 #pragma unroll
-            for (int e = 0; e < 32; ++e) o[e] *= alpha;
-            tmem_st32(tmem + lane_base + C::COL_O + c0, o);
+              for (int e = 0; e < 32; ++e) o[e] *= alpha;
+              tmem_st32(tmem + lane_base + C::COL_O + c0, o);
+            }
           }
         }
         tmem_wait_st();
@@ -337,6 +375,9 @@ __global__ void __launch_bounds__(192, 1)
     if (!ok) *abort = 1;
     // ------------------------------------------------------------ epilogue
     if (MODE != FWD_WRITE_A) {
+      bars.ls[wg][row] = lsum;
+      rows_sync();
+      lsum = bars.ls[0][row] + bars.ls[1][row];
       const float lse = (mref + log2f(lsum)) * 0.6931471805599453f;
       if (C::PV) {
         if (!mbar_wait(&bars.o_done, 0, abort)) *abort = 1;
@@ -348,8 +389,9 @@ __global__ void __launch_bounds__(192, 1)
       const int64_t grow = q_begin + q;
       float se = 0.f, ls = 0.f, gy = 0.f;
       if (C::PV) {
+        // this warpgroup's half of the row's output columns
 #pragma unroll 1
-        for (int c0 = 0; c0 < D; c0 += 32) {
+        for (int c0 = wg * (D / 2); c0 < (wg + 1) * (D / 2); c0 += 32) {
           float o[32], ob[32];
           tmem_ld32(tmem + lane_base + C::COL_O + c0, o);
           tmem_ld32(tmem + lane_base + C::COL_O + D + c0, ob);
@@ -405,34 +447,43 @@ __global__ void __launch_bounds__(192, 1)
           }
         }
       }
-      if (valid) {
-        a.lse_out[grow] = lse;
-        if (MODE == FWD_LOSS) {
-          const float el = lse - a.lse_in[grow];
-          ls = el * el;
-          a.delta[grow] = gy - c_lse * el;
-        }
-      }
       if (MODE == FWD_LOSS) {
-        // deterministic per-CTA partial sums of the two loss terms
-        se = warp_sum(se);
-        ls = warp_sum(ls);
-        if (lane == 0) {
-          bars.red[warp] = se;
-          bars.red[4 + warp] = ls;
+        bars.part[wg][row][0] = se;
+        bars.part[wg][row][1] = gy;
+        rows_sync();
+        if (wg == 0) {
+          se = bars.part[0][row][0] + bars.part[1][row][0];
+          gy = bars.part[0][row][1] + bars.part[1][row][1];
+          if (valid) {
+            const float el = lse - a.lse_in[grow];
+            ls = el * el;
+            a.lse_out[grow] = lse;
+            a.delta[grow] = gy - c_lse * el;
+          } else {
+            se = 0.f;
+          }
+          // deterministic per-CTA partial sums of the two loss terms
+          se = warp_sum(se);
+          ls = warp_sum(ls);
+          if (lane == 0) {
+            bars.red[warp] = se;
+            bars.red[4 + warp] = ls;
+          }
         }
-        asm volatile("bar.sync 1, 128;" ::: "memory");
-        if (row == 0) {
+        rows_sync();
+        if (tid == 0) {
           float *part = a.partials + ((int64_t)b * a.tiles_per_problem + blockIdx.x) * 2;
           part[0] = (bars.red[0] + bars.red[1]) + (bars.red[2] + bars.red[3]);
           part[1] = (bars.red[4] + bars.red[5]) + (bars.red[6] + bars.red[7]);
         }
+      } else if (wg == 0 && valid) {  // TARGETS, STATS
+        a.lse_out[grow] = lse;
       }
     }
   }
   fence_before_sync();
   __syncthreads();
-  if (warp == 5) {
+  if (warp == 9) {
     fence_after_sync();
     tmem_dealloc(tmem, C::TMEM_COLS);
   }
@@ -447,7 +498,7 @@ int launch_fwd_tc(const FwdMaps &m, const FwdArgs &a, int max_tiles, int B, cuda
   static_assert(C::SMEM + sizeof(FwdBars) <= 232448, "shared memory");
   auto kern = k_attn_fwd<D, MODE>;
   KVS_CUDA_TRY(set_smem_once(kern, C::SMEM));
-  kern<<<dim3(max_tiles, B), 192, C::SMEM, st>>>(m.kh, m.kl, m.vh, m.vl, m.qh, m.ql, a);
+  kern<<<dim3(max_tiles, B), NTHREADS, C::SMEM, st>>>(m.kh, m.kl, m.vh, m.vl, m.qh, m.ql, a);
   KVS_LAUNCH_CHECK("k_attn_fwd");
   return KVS_OK;
 }

@@ -253,7 +253,6 @@ __device__ __forceinline__ void split_pack(float a, float b, uint32_t &hi, uint3
   lo = *reinterpret_cast<const uint32_t *>(&l);
 }
 
-// Byte offset of 16-byte chunk `chunk` of row `row` in a 128-byte-swizzled tile.
 // 2^x on the special-function unit; subnormal results flush to zero (softmax
 // weights that small do not change any sum they enter).
 __device__ __forceinline__ float ex2(float x) {
@@ -361,6 +360,7 @@ __device__ __forceinline__ void mma_commit_pair(uint64_t *bar) {
       : "memory");
 }
 
+// Byte offset of 16-byte chunk `chunk` of row `row` in a 128-byte-swizzled tile.
 __device__ __forceinline__ uint32_t sw128_offset(int row, int chunk) {
   return (uint32_t)(row >> 3) * 1024u + (uint32_t)(row & 7) * 128u +
          (uint32_t)((chunk ^ (row & 7)) << 4);
