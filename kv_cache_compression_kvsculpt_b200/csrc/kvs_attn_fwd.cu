@@ -51,12 +51,15 @@ struct Fwd {
   static constexpr int KD = D / 64;
   static constexpr bool PV = (MODE == FWD_LOSS || MODE == FWD_TARGETS);
   static constexpr int T_BYTES = BN * D * 2;   // one 128-row bf16 tile (hi or lo)
-  static constexpr int NSK = PV ? 1 : 2;       // key stages (K hi + K lo each)
+  static constexpr bool WA = MODE == FWD_WRITE_A;
+  static constexpr int NSK = (PV || WA) ? 1 : 2;  // key stages (K hi + K lo each)
   static constexpr int NSV = PV ? 1 : 0;       // value stages (V hi + V lo each)
   static constexpr int NSVI = PV ? NSV : 1;     // ring index modulus (unused without values)
   static constexpr int OFF_K = 2 * T_BYTES;    // after Q hi, Q lo (BM = BN rows)
   static constexpr int OFF_V = OFF_K + NSK * 2 * T_BYTES;
-  static constexpr int BYTES = OFF_V + NSV * 2 * T_BYTES;
+  static constexpr int OFF_STG = OFF_V + NSV * 2 * T_BYTES;
+  static constexpr int STG_WARP = 2 * 32 * HB * 2;  // WRITE_A: a row warp's 32 x 64 A hi and lo
+  static constexpr int BYTES = OFF_STG + (WA ? 8 * STG_WARP : 0);
   static constexpr int SMEM = BYTES + 1024;
   static constexpr uint32_t TMEM_COLS = 512;
   static constexpr uint32_t COL_O = 2 * BN;     // O_a at +0, O_b at +D
@@ -295,10 +298,10 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         mbar_arrive(&bars.s_free[sb]);
       }
       if (MODE == FWD_WRITE_A) {
-        // A = exp2(t - lse2), split into bf16 hi / lo, into the padded A buffer
-        const int64_t arow = a.a_pad_off[b] + q0 + row;
-        uint4 *dh = reinterpret_cast<uint4 *>(a.a_hi + arow * a.ld_a + j * BN + cb);
-        uint4 *dl = reinterpret_cast<uint4 *>(a.a_lo + arow * a.ld_a + j * BN + cb);
+        // A = exp2(t - lse2), split into bf16 hi / lo.  The warp stages its 32 rows
+        // x 64 keys in shared memory (16-byte chunks XOR-swizzled by row), then
+        // writes them out as whole 128-byte row segments of the padded A buffer.
+        uint4 *stg = reinterpret_cast<uint4 *>(sm + C::OFF_STG + warp * C::STG_WARP);
 #pragma unroll
         for (int ch = 0; ch < HB / 8; ++ch) {
           uint32_t h[4], l[4];
@@ -308,9 +311,22 @@ __global__ void __launch_bounds__(NTHREADS, 1)
             const float p1 = valid ? ex2(fmaf(s[ch * 8 + 2 * e + 1], sl2, -lrow2)) : 0.f;
             split_pack(p0, p1, h[e], l[e]);
           }
-          dh[ch] = make_uint4(h[0], h[1], h[2], h[3]);
-          dl[ch] = make_uint4(l[0], l[1], l[2], l[3]);
+          const int slot = lane * 8 + (ch ^ (lane & 7));
+          stg[slot] = make_uint4(h[0], h[1], h[2], h[3]);
+          stg[256 + slot] = make_uint4(l[0], l[1], l[2], l[3]);
         }
+        __syncwarp();
+        const int64_t arow0 = a.a_pad_off[b] + q0 + (warp & 3) * 32;
+        const int cc = lane & 7;
+#pragma unroll
+        for (int it = 0; it < 8; ++it) {
+          const int rr = it * 4 + (lane >> 3);
+          const int slot = rr * 8 + (cc ^ (rr & 7));
+          const int64_t off = (arow0 + rr) * a.ld_a + j * BN + cb + cc * 8;
+          *reinterpret_cast<uint4 *>(a.a_hi + off) = stg[slot];
+          *reinterpret_cast<uint4 *>(a.a_lo + off) = stg[256 + slot];
+        }
+        __syncwarp();  // the staging is reused by the next tile
         continue;
       }
       float mt = -INFINITY;

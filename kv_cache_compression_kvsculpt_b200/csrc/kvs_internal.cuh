@@ -42,7 +42,7 @@ struct Work {
   float *R;                  // [sum_c, d]             A^T Y, then the forward-solved rows
   float *X;                  // [sum_c, d]             solution of the ridge system
   float *dkp;                // [4, sum_c, d]          key-gradient partial sums of query splits
-  float *chol_t;             // [B, panels, 64, 64]    inverses of the diagonal blocks
+  float *chol_t;             // [B, panels, 64, 64]    transposed inverses of the diagonal blocks
   int *dead;                 // [B]                    factorisation failed
   float *fbuf;               // [B]                    loss scratch
   float *Yt;                 // [sum_q, d]             targets (kvs_compress_batch)

@@ -13,12 +13,17 @@
 //             r_i -= L_ij y_j on the right-hand sides
 //   then one kernel sweeps the panels from the last one: x_j = T_j^T y_j,
 //   y_i -= L_ji^T x_j.
-// Every 64 x 64 product runs from shared memory with 4 x 4 register tiles and
-// 128-bit shared loads.  The factor overwrites the Gram matrix, the forward
-// sweep the right-hand sides; the solution goes to a separate buffer and is
-// copied to V_c only when finite.  A pivot <= 0 (or non-finite) marks the
-// problem KVS_ST_NOT_PD; its V_c is left untouched and its remaining steps
-// are skipped.
+// Every 64 x 64 x 64 product runs from shared memory with both operands stored
+// contraction-index-major (S[t][row]): each thread owns a 4 x 4 output block
+// and forms a rank-1 update from two 128-bit loads per t.  The diagonal block
+// is factored 16 columns at a time: one warp factors and inverts the 16 x 16
+// pivot block in registers, then all threads apply it to the rows below and to
+// the trailing block, and T_j is assembled from the four 16 x 16 inverses.  The
+// factor overwrites the Gram matrix (lower triangle; the upper one is scratch),
+// the forward sweep the right-hand sides; the solution goes to a separate
+// buffer and is copied to V_c only when finite.  A pivot <= 0 (or non-finite)
+// marks the problem KVS_ST_NOT_PD; its V_c is left untouched and its remaining
+// steps are skipped.
 #include <math.h>
 
 #include "kvs_internal.cuh"
@@ -27,14 +32,15 @@ namespace kvs {
 namespace {
 
 constexpr int NB = 64;
-constexpr int SP = NB + 4;  // shared row stride (floats): 16-byte rows, conflict-free columns
+constexpr int SP = NB + 4;  // shared row stride (floats): 16-byte rows, offset banks
 constexpr int DEAD_NOT_PD = 1, DEAD_NONFINITE = 2;
+constexpr unsigned FULL = 0xffffffffu;
 
 struct CholArgs {
   float *G;              // [sum_c, ld] Gram matrix -> factor (lower triangle)
   float *R;              // [sum_c, d] right-hand sides -> forward-solved rows
   float *X;              // [sum_c, d] solution
-  float *T;              // [B, npanel, NB, NB] inverses of the diagonal blocks
+  float *Tt;             // [B, npanel, NB, NB] transposes of the diagonal-block inverses
   int npanel;
   int *dead;             // [B] DEAD_* bits
   int32_t *status;
@@ -48,62 +54,60 @@ __device__ __forceinline__ int kdim(const CholArgs &a, int b) {
 }
 
 __device__ __forceinline__ float4 ld4(const float *p) { return *reinterpret_cast<const float4 *>(p); }
+__device__ __forceinline__ void st4(float *p, float4 v) { *reinterpret_cast<float4 *>(p) = v; }
 
-// S[r][c] = M[r0 + r][c0 + c] for r0 + r < rmax, c0 + c < cmax, else 0
-// (M row-major with ld a multiple of 4 and c0 a multiple of 4).
-__device__ __forceinline__ void load_tile(float (*S)[SP], const float *M, int64_t ld, int r0,
-                                          int rmax, int c0, int cmax) {
+// M[r][c0 + c .. c0 + c + 3] with the lanes at or past cmax zeroed (c0 + c < cmax;
+// M row-major with ld a multiple of 4 and c0 + c a multiple of 4).
+__device__ __forceinline__ float4 ld4m(const float *M, int64_t ld, int r, int c, int cmax) {
+  float4 v = ld4(M + (int64_t)r * ld + c);
+  const int m = cmax - c;
+  if (m < 4) {
+    v.w = 0.f;
+    if (m < 3) v.z = 0.f;
+    if (m < 2) v.y = 0.f;
+  }
+  return v;
+}
+
+// S[r][c] = M[r0 + r][c0 + c] for r0 + r < rmax, c0 + c < cmax, else 0.
+__device__ __forceinline__ void load_d(float (*S)[SP], const float *M, int64_t ld, int r0,
+                                       int rmax, int c0, int cmax) {
   for (int e = threadIdx.x; e < NB * NB / 4; e += blockDim.x) {
     const int r = e >> 4, c = (e & 15) * 4;
     float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
-    if (r0 + r < rmax && c0 + c < cmax) {
-      v = ld4(M + (int64_t)(r0 + r) * ld + c0 + c);
-      const int m = cmax - c0 - c;  // valid lanes of the vector
-      if (m < 4) {
-        v.w = 0.f;
-        if (m < 3) v.z = 0.f;
-        if (m < 2) v.y = 0.f;
-      }
-    }
-    *reinterpret_cast<float4 *>(&S[r][c]) = v;
+    if (r0 + r < rmax && c0 + c < cmax) v = ld4m(M, ld, r0 + r, c0 + c, cmax);
+    st4(&S[r][c], v);
   }
 }
 
-// Transposed: S[c][r] = M[r0 + r][c0 + c], same bounds.
-__device__ __forceinline__ void load_tile_t(float (*S)[SP], const float *M, int64_t ld, int r0,
-                                            int rmax, int c0, int cmax) {
+// Transposed: S[c][r] = M[r0 + r][c0 + c], same bounds.  Lanes take consecutive
+// rows, so the shared-memory stores of a warp hit 32 consecutive words.
+__device__ __forceinline__ void load_t(float (*S)[SP], const float *M, int64_t ld, int r0,
+                                       int rmax, int c0, int cmax) {
   for (int e = threadIdx.x; e < NB * NB / 4; e += blockDim.x) {
-    const int r = e >> 4, c = (e & 15) * 4;
+    const int r = e & (NB - 1), c = (e >> 6) * 4;
     float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
-    if (r0 + r < rmax && c0 + c < cmax) v = ld4(M + (int64_t)(r0 + r) * ld + c0 + c);
-    const int m = cmax - c0 - c;
-    S[c][r] = m > 0 ? v.x : 0.f;
-    S[c + 1][r] = m > 1 ? v.y : 0.f;
-    S[c + 2][r] = m > 2 ? v.z : 0.f;
-    S[c + 3][r] = m > 3 ? v.w : 0.f;
+    if (r0 + r < rmax && c0 + c < cmax) v = ld4m(M, ld, r0 + r, c0 + c, cmax);
+    S[c][r] = v.x;
+    S[c + 1][r] = v.y;
+    S[c + 2][r] = v.z;
+    S[c + 3][r] = v.w;
   }
 }
 
-// acc[i][j] += sum_t A[ty + 16 i][t] * B[tx + 16 j][t], t ascending
-__device__ __forceinline__ void mm64(const float (*A)[SP], const float (*B)[SP], float acc[4][4],
-                                     int tx, int ty) {
-#pragma unroll 2
-  for (int t = 0; t < NB; t += 4) {
-    float4 av[4], bv[4];
-#pragma unroll
-    for (int i = 0; i < 4; ++i) av[i] = *reinterpret_cast<const float4 *>(&A[ty + 16 * i][t]);
-#pragma unroll
-    for (int j = 0; j < 4; ++j) bv[j] = *reinterpret_cast<const float4 *>(&B[tx + 16 * j][t]);
+// acc[i][j] += sum_t A[t][4 ty + i] * B[t][4 tx + j], t ascending
+__device__ __forceinline__ void mmk(const float (*A)[SP], const float (*B)[SP], float acc[4][4],
+                                    int tx, int ty) {
+#pragma unroll 8
+  for (int t = 0; t < NB; ++t) {
+    const float4 av = ld4(&A[t][4 * ty]);
+    const float4 bv = ld4(&B[t][4 * tx]);
+    const float ai[4] = {av.x, av.y, av.z, av.w};
+    const float bj[4] = {bv.x, bv.y, bv.z, bv.w};
 #pragma unroll
     for (int i = 0; i < 4; ++i)
 #pragma unroll
-      for (int j = 0; j < 4; ++j) {
-        float s = acc[i][j];
-        s = fmaf(av[i].x, bv[j].x, s);
-        s = fmaf(av[i].y, bv[j].y, s);
-        s = fmaf(av[i].z, bv[j].z, s);
-        acc[i][j] = fmaf(av[i].w, bv[j].w, s);
-      }
+      for (int j = 0; j < 4; ++j) acc[i][j] = fmaf(ai[i], bj[j], acc[i][j]);
   }
 }
 
@@ -114,48 +118,152 @@ __device__ __forceinline__ void zero_acc(float acc[4][4]) {
     for (int j = 0; j < 4; ++j) acc[i][j] = 0.f;
 }
 
-// Diagonal block of panel j0: factor in shared memory, keep T_j = L_jj^-1 and
-// forward-solve the block's rows of the right-hand sides, y_j = T_j r_j.
+// Warp step of the diagonal-block factorisation: lane r (and its mirror r + 16)
+// holds row r of the 16 x 16 pivot block at (c0, c0) (rows of the padding past jb
+// read as identity rows), factors it, inverts the factor and writes both back.
+// Returns true when a pivot was not positive and finite.
+__device__ __forceinline__ bool factor16(float (*L)[SP], float (*Ts)[SP], int c0, int jb,
+                                         int lane) {
+  const int r = lane & 15, gr = c0 + r;
+  float av[16];
+#pragma unroll
+  for (int j = 0; j < 16; ++j) {
+    float v = j <= r ? L[gr][c0 + j] : 0.f;
+    if (gr >= jb) v = j == r ? 1.f : 0.f;
+    av[j] = v;
+  }
+  // unblocked Cholesky, column c: pivot from lane c, scale, rank-1 update
+  bool bad = false;
+  float invd = 1.f;
+#pragma unroll
+  for (int c = 0; c < 16; ++c) {
+    const float p = __shfl_sync(FULL, av[c], c);
+    bad |= !(p > 0.f) || !isfinite(p);
+    const float dc = sqrtf(fmaxf(p, 1e-30f));
+    const float inv = 1.f / dc;
+    const float l = r == c ? dc : av[c] * inv;
+    if (r == c) invd = inv;
+    av[c] = l;
+#pragma unroll
+    for (int j = c + 1; j < 16; ++j) av[j] = fmaf(-l, __shfl_sync(FULL, l, j), av[j]);
+  }
+  // T = L^-1 row by row: lane r accumulates -sum_u L[r][u] T[u][j] over the rows
+  // u < r as lane u finalises them, then scales by 1 / L[r][r]
+  float tv[16];
+#pragma unroll
+  for (int j = 0; j < 16; ++j) tv[j] = 0.f;
+#pragma unroll
+  for (int u = 0; u < 16; ++u) {
+    if (r == u) {
+#pragma unroll
+      for (int j = 0; j < u; ++j) tv[j] *= invd;
+      tv[u] = invd;
+    }
+#pragma unroll
+    for (int j = 0; j <= u; ++j) {
+      const float tu = __shfl_sync(FULL, tv[j], u);
+      if (r > u) tv[j] = fmaf(-av[u], tu, tv[j]);
+    }
+  }
+  if (lane < 16) {
+#pragma unroll
+    for (int j = 0; j < 16; ++j)
+      if (j <= r) {
+        L[gr][c0 + j] = av[j];
+        Ts[gr][c0 + j] = tv[j];
+      }
+  }
+  return bad;
+}
+
+// Diagonal block of panel j0: factor in shared memory, keep T_j = L_jj^-1 (stored
+// transposed) and forward-solve the block's rows of the right-hand sides, y_j = T_j r_j.
+// Rows past jb (the last panel of a problem whose k is not a multiple of 64) are
+// factored as identity rows, so T_j is the identity there.
 __global__ void __launch_bounds__(256) k_chol_diag(CholArgs a, int j0) {
   const int b = blockIdx.x;
   const int k = kdim(a, b);
   if (j0 >= k || a.dead[b]) return;
   const int jb = min(NB, k - j0);
-  __shared__ __align__(16) float L[NB][SP];   // the block; later the right-hand side tile
-  __shared__ __align__(16) float Ts[NB][SP];  // T_j
-  __shared__ float dsq[NB];
+  __shared__ __align__(16) float L[NB][SP];   // the block; then T_j^T
+  __shared__ __align__(16) float Ts[NB][SP];  // T_j; then right-hand-side tiles
   __shared__ int bad;
   float *G = a.G + (a.c_off[b] + j0) * a.ld + j0;
-  const int tid = threadIdx.x;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   if (tid == 0) bad = 0;
-  load_tile(L, G, a.ld, 0, jb, 0, jb);
+  load_d(L, G, a.ld, 0, jb, 0, jb);
   for (int e = tid; e < NB * SP; e += blockDim.x) (&Ts[0][0])[e] = 0.f;
   __syncthreads();
-  // Unnormalised elimination: after step c, column c holds l_ic * sqrt(p_c) and
-  // L[c][c] = p_c, the pivot; the trailing block loses l_i l_j^T = L_ic L_jc / p_c.
-  // Thread (i, q) owns row i = tid / 4 at the columns j = q + 4 m.
-  {
-    const int i = tid >> 2, q = tid & 3;
-    for (int c = 0; c < jb - 1; ++c) {
-      if (i > c && i < jb) {
-        const float lic = L[i][c] / L[c][c];
-        const int m0 = (c + 1 - q + 3) >> 2;  // first m with q + 4 m > c
-#pragma unroll 4
-        for (int m = m0; m < 16; ++m) {
-          const int j = q + 4 * m;
-          if (j > i) break;
-          L[i][j] = fmaf(-lic, L[j][c], L[i][j]);
+#pragma unroll 1
+  for (int c0 = 0; c0 < NB; c0 += 16) {
+    if (warp == 0 && factor16(L, Ts, c0, jb, lane) && lane == 0) bad = 1;
+    __syncthreads();
+    const int m = NB - c0 - 16;  // rows below the pivot block
+    if (m == 0) break;
+    // L[i][c0 ..] = A[i][c0 ..] T_kk^T for the rows below: four threads per row
+    // (one warp holds all four), four columns each
+    {
+      const int i = c0 + 16 + (tid >> 2), q = tid & 3;
+      const bool act = (tid >> 2) < m;
+      float4 ar[4];
+      if (act)
+#pragma unroll
+        for (int u = 0; u < 4; ++u) ar[u] = ld4(&L[i][c0 + 4 * u]);
+      __syncwarp();
+      if (act) {
+        float o[4];
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const float *tr = &Ts[c0 + 4 * q + e][c0];  // row of T_kk (zero past the diagonal)
+          float s = 0.f;
+#pragma unroll
+          for (int u = 0; u < 4; ++u) {
+            const float4 t4 = ld4(tr + 4 * u);
+            s = fmaf(ar[u].x, t4.x, s);
+            s = fmaf(ar[u].y, t4.y, s);
+            s = fmaf(ar[u].z, t4.z, s);
+            s = fmaf(ar[u].w, t4.w, s);
+          }
+          o[e] = s;
         }
+        st4(&L[i][c0 + 4 * q], make_float4(o[0], o[1], o[2], o[3]));
       }
-      __syncthreads();
     }
+    __syncthreads();
+    // trailing block: A[i][j] -= sum_t L[i][c0 + t] L[j][c0 + t], c0 + 16 <= j <= i,
+    // in groups of four columns
+    {
+      const int ng = m / 4, s0 = c0 + 16;
+      for (int e = tid; e < m * ng; e += blockDim.x) {
+        const int i = s0 + e / ng, j4 = s0 + (e % ng) * 4;
+        if (j4 > i) continue;
+        float4 li[4];
+#pragma unroll
+        for (int u = 0; u < 4; ++u) li[u] = ld4(&L[i][c0 + 4 * u]);
+        float acc[4];
+#pragma unroll
+        for (int jj = 0; jj < 4; ++jj) {
+          float s = 0.f;
+#pragma unroll
+          for (int u = 0; u < 4; ++u) {
+            const float4 lj = ld4(&L[j4 + jj][c0 + 4 * u]);
+            s = fmaf(li[u].x, lj.x, s);
+            s = fmaf(li[u].y, lj.y, s);
+            s = fmaf(li[u].z, lj.z, s);
+            s = fmaf(li[u].w, lj.w, s);
+          }
+          acc[jj] = s;
+        }
+        float4 v = ld4(&L[i][j4]);
+        v.x -= acc[0];
+        v.y -= acc[1];
+        v.z -= acc[2];
+        v.w -= acc[3];
+        st4(&L[i][j4], v);
+      }
+    }
+    __syncthreads();
   }
-  if (tid < jb) {
-    const float p = L[tid][tid];
-    if (!(p > 0.f) || !isfinite(p)) atomicOr(&bad, 1);
-    dsq[tid] = sqrtf(fmaxf(p, 1e-30f));
-  }
-  __syncthreads();
   if (bad) {
     if (tid == 0) {
       a.status[b] |= KVS_ST_NOT_PD;
@@ -163,52 +271,100 @@ __global__ void __launch_bounds__(256) k_chol_diag(CholArgs a, int j0) {
     }
     return;
   }
-  for (int e = tid; e < jb * jb; e += blockDim.x) {
-    const int r = e / jb, c = e % jb;
-    if (c < r) L[r][c] /= dsq[c];
-    else if (c == r) L[r][c] = dsq[c];
-  }
-  __syncthreads();
-  // T = L^-1 column by column: warp w owns columns 8w .. 8w+7, four lanes per
-  // column split each row's dot product; T[i][cc] = -(sum_t L[i][t] T[t][cc]) / L[i][i].
-  if (tid < jb) Ts[tid][tid] = 1.f / L[tid][tid];
-  __syncthreads();
+  // T_j from the four 16 x 16 inverses T_k on its diagonal, by 2 x 2 blocks:
+  // [[T1, 0], [L21, L22]]^-1 has lower-left block -T2 L21 T1.  Products go
+  // through the upper-right quadrant of Ts (zero in T_j) as scratch.
   {
-    const int warp = tid >> 5, lane = tid & 31;
-    const int cc = warp * 8 + (lane >> 2), q = lane & 3;
-    for (int i = 1; i < jb; ++i) {
-      float s = 0.f;
-      if (i > cc)
-        for (int t = cc + q; t < i; t += 4) s = fmaf(L[i][t], Ts[t][cc], s);
-      s += __shfl_xor_sync(0xffffffffu, s, 1);
-      s += __shfl_xor_sync(0xffffffffu, s, 2);
-      if (i > cc && q == 0) Ts[i][cc] = -s * Ts[i][i];
-      __syncwarp();
+    // 16 x 16 level, both 32 x 32 halves q: W_q = L[32q+16 ..][32q ..] T_2q
+    const int q = tid >> 7, i = (tid >> 3) & 15, j2 = (tid & 7) * 2;
+    const int o = 32 * q;
+    float *W = &Ts[16 * q][32 + 16 * q];  // 16 x 16 scratch, row stride SP
+    {
+      float s0 = 0.f, s1 = 0.f;
+#pragma unroll
+      for (int t = 0; t < 16; ++t) {
+        const float l = L[o + 16 + i][o + t];
+        s0 = fmaf(l, Ts[o + t][o + j2], s0);
+        s1 = fmaf(l, Ts[o + t][o + j2 + 1], s1);
+      }
+      W[i * SP + j2] = s0;
+      W[i * SP + j2 + 1] = s1;
     }
+    __syncthreads();
+    {
+      float s0 = 0.f, s1 = 0.f;
+#pragma unroll
+      for (int t = 0; t < 16; ++t) {
+        const float tt = Ts[o + 16 + i][o + 16 + t];
+        s0 = fmaf(tt, W[t * SP + j2], s0);
+        s1 = fmaf(tt, W[t * SP + j2 + 1], s1);
+      }
+      Ts[o + 16 + i][o + j2] = -s0;
+      Ts[o + 16 + i][o + j2 + 1] = -s1;
+    }
+    __syncthreads();
+    // 32 x 32 level: W = L[32 ..][0 .. 32) T1 into the upper-right quadrant, then
+    // the lower-left quadrant = -T2 W
+    const int i2 = tid >> 3, j4 = (tid & 7) * 4;
+    {
+      float s[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll 8
+      for (int t = 0; t < 32; ++t) {
+        const float l = L[32 + i2][t];
+        const float4 tt = ld4(&Ts[t][j4]);
+        s[0] = fmaf(l, tt.x, s[0]);
+        s[1] = fmaf(l, tt.y, s[1]);
+        s[2] = fmaf(l, tt.z, s[2]);
+        s[3] = fmaf(l, tt.w, s[3]);
+      }
+      st4(&Ts[i2][32 + j4], make_float4(s[0], s[1], s[2], s[3]));
+    }
+    __syncthreads();
+    {
+      float s[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll 8
+      for (int t = 0; t < 32; ++t) {
+        const float tt = Ts[32 + i2][32 + t];
+        const float4 w = ld4(&Ts[t][32 + j4]);
+        s[0] = fmaf(tt, w.x, s[0]);
+        s[1] = fmaf(tt, w.y, s[1]);
+        s[2] = fmaf(tt, w.z, s[2]);
+        s[3] = fmaf(tt, w.w, s[3]);
+      }
+      st4(&Ts[32 + i2][j4], make_float4(-s[0], -s[1], -s[2], -s[3]));
+    }
+    __syncthreads();
+    st4(&Ts[i2][32 + j4], make_float4(0.f, 0.f, 0.f, 0.f));
   }
-  __syncthreads();
-  float *Tg = a.T + ((int64_t)b * a.npanel + j0 / NB) * NB * NB;
+  // the factor's lower triangle back to G
   for (int e = tid; e < NB * NB; e += blockDim.x) {
-    const int r = e / NB, c = e % NB;
+    const int r = e >> 6, c = e & (NB - 1);
     if (r < jb && c <= r) G[(int64_t)r * a.ld + c] = L[r][c];
-    Tg[e] = Ts[r][c];
   }
   __syncthreads();
-  // y_j = T_j r_j, 64 right-hand-side columns at a time (the tile reuses L)
+  // T_j^T to global and into L (the A operand of the forward solve)
+  float *Tg = a.Tt + ((int64_t)b * a.npanel + j0 / NB) * NB * NB;
+  for (int e = tid; e < NB * NB; e += blockDim.x) {
+    const int c = e >> 6, r = e & (NB - 1);
+    const float v = Ts[r][c];
+    Tg[e] = v;
+    L[c][r] = v;
+  }
+  __syncthreads();
+  // y_j = T_j r_j, 64 right-hand-side columns at a time (the tile reuses Ts)
   const int tx = tid & 15, ty = tid >> 4;
   float *R = a.R + (a.c_off[b] + j0) * a.d;
   for (int c0 = 0; c0 < a.d; c0 += NB) {
-    load_tile_t(L, R, a.d, 0, jb, c0, a.d);  // L[col][t] = r[t][c0 + col]
+    load_d(Ts, R, a.d, 0, jb, c0, a.d);
     __syncthreads();
     float acc[4][4];
     zero_acc(acc);
-    mm64(Ts, L, acc, tx, ty);
+    mmk(L, Ts, acc, tx, ty);
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
-      const int r = ty + 16 * i;
-      if (r >= jb) continue;
-#pragma unroll
-      for (int j = 0; j < 4; ++j) R[(int64_t)r * a.d + c0 + tx + 16 * j] = acc[i][j];
+      const int r = 4 * ty + i;
+      if (r < jb)
+        st4(R + (int64_t)r * a.d + c0 + 4 * tx, make_float4(acc[i][0], acc[i][1], acc[i][2], acc[i][3]));
     }
     __syncthreads();
   }
@@ -218,39 +374,32 @@ __global__ void __launch_bounds__(256) k_chol_diag(CholArgs a, int j0) {
 __global__ void __launch_bounds__(256) k_chol_panel(CholArgs a, int j0) {
   const int b = blockIdx.y;
   const int k = kdim(a, b);
-  if (j0 >= k || a.dead[b]) return;
-  const int jb = min(NB, k - j0);
-  const int i0 = j0 + jb + blockIdx.x * NB;
+  if (j0 + NB >= k || a.dead[b]) return;  // rows below exist only after a full block
+  const int i0 = j0 + NB + blockIdx.x * NB;
   if (i0 >= k) return;
-  __shared__ __align__(16) float Ar[NB][SP];
-  __shared__ __align__(16) float Ts[NB][SP];
+  __shared__ __align__(16) float As[NB][SP];  // As[t][r] = G[i0 + r][j0 + t]
+  __shared__ __align__(16) float Bs[NB][SP];  // Bs[t][c] = T[c][t]
   const int tid = threadIdx.x;
   const int64_t row0 = a.c_off[b];
-  load_tile(Ar, a.G + row0 * a.ld, a.ld, i0, k, j0, j0 + jb);
-  const float *Tg = a.T + ((int64_t)b * a.npanel + j0 / NB) * NB * NB;
-  for (int e = tid; e < NB * NB / 4; e += blockDim.x) {
-    const int r = e >> 4, c = (e & 15) * 4;
-    *reinterpret_cast<float4 *>(&Ts[r][c]) = ld4(Tg + r * NB + c);
-  }
+  load_t(As, a.G + row0 * a.ld, a.ld, i0, k, j0, j0 + NB);
+  load_d(Bs, a.Tt + ((int64_t)b * a.npanel + j0 / NB) * NB * NB, NB, 0, NB, 0, NB);
   __syncthreads();
   const int tx = tid & 15, ty = tid >> 4;
   float acc[4][4];
   zero_acc(acc);
-  mm64(Ar, Ts, acc, tx, ty);  // sum_t G[r][t] T[col][t]
+  mmk(As, Bs, acc, tx, ty);
 #pragma unroll
   for (int i = 0; i < 4; ++i) {
-    const int r = i0 + ty + 16 * i;
-    if (r >= k) continue;
-#pragma unroll
-    for (int j = 0; j < 4; ++j) {
-      const int c = tx + 16 * j;
-      if (c < jb) a.G[(row0 + r) * a.ld + j0 + c] = acc[i][j];
-    }
+    const int r = i0 + 4 * ty + i;
+    if (r < k)
+      st4(a.G + (row0 + r) * a.ld + j0 + 4 * tx,
+          make_float4(acc[i][0], acc[i][1], acc[i][2], acc[i][3]));
   }
 }
 
 // Trailing update: tiles (ti >= tj) of G_ik -= L_i L_k^T, and tiles of
-// r_i -= L_i y_j (columns of R in chunks of 64), 64 x 64 outputs per CTA.
+// r_i -= L_i y_j (columns of R in chunks of 64), 64 x 64 outputs per CTA.  The
+// diagonal tiles are written whole: their upper triangle is scratch.
 __global__ void __launch_bounds__(256) k_chol_update(CholArgs a, int j0) {
   const int b = blockIdx.y;
   const int k = kdim(a, b);
@@ -277,50 +426,54 @@ __global__ void __launch_bounds__(256) k_chol_update(CholArgs a, int j0) {
     ti = t / ndc;
     tj = t % ndc;
   }
-  __shared__ __align__(16) float As[NB][SP];  // L_i panel rows, [row][c]
-  __shared__ __align__(16) float Bs[NB][SP];  // L_k panel rows [row][c], or y_j as [col][c]
+  __shared__ __align__(16) float As[NB][SP];  // As[t][r] = L[ri + r][j0 + t]
+  __shared__ __align__(16) float Bs[NB][SP];  // Bs[t][c] = L[rk + c][j0 + t], or y[j0 + t][c]
   const int tid = threadIdx.x;
   const int tx = tid & 15, ty = tid >> 4;
   const int64_t row0 = a.c_off[b];
   const int ri = s0 + ti * NB;
+  float *out;
+  int64_t ldo;
+  int cmax;
+  if (!rhs) {
+    out = a.G + row0 * a.ld + s0 + tj * NB + 4 * tx;
+    ldo = a.ld;
+    cmax = k - (s0 + tj * NB + 4 * tx);  // valid columns from this thread's first
+  } else {
+    out = a.R + row0 * a.d + tj * NB + 4 * tx;
+    ldo = a.d;
+    cmax = 4;
+  }
   // the outputs' current values first: their loads overlap the tile loads
-  float cur[4][4];
+  float4 cur[4];
 #pragma unroll
   for (int i = 0; i < 4; ++i) {
-    const int r = ri + ty + 16 * i;
-#pragma unroll
-    for (int j = 0; j < 4; ++j) {
-      cur[i][j] = 0.f;
-      if (r >= k) continue;
-      if (!rhs) {
-        const int cc = s0 + tj * NB + tx + 16 * j;
-        if (cc <= r) cur[i][j] = a.G[(row0 + r) * a.ld + cc];
-      } else {
-        cur[i][j] = a.R[(row0 + r) * a.d + tj * NB + tx + 16 * j];
-      }
-    }
+    const int r = ri + 4 * ty + i;
+    cur[i] = make_float4(0.f, 0.f, 0.f, 0.f);
+    if (r < k && cmax > 0) cur[i] = ld4m(out, ldo, r, 0, cmax);
   }
-  load_tile(As, a.G + row0 * a.ld, a.ld, ri, k, j0, j0 + jb);
+  load_t(As, a.G + row0 * a.ld, a.ld, ri, k, j0, j0 + jb);
   if (!rhs)
-    load_tile(Bs, a.G + row0 * a.ld, a.ld, s0 + tj * NB, k, j0, j0 + jb);
+    load_t(Bs, a.G + row0 * a.ld, a.ld, s0 + tj * NB, k, j0, j0 + jb);
   else
-    load_tile_t(Bs, a.R + row0 * a.d, a.d, j0, j0 + jb, tj * NB, a.d);
+    load_d(Bs, a.R + row0 * a.d, a.d, j0, j0 + jb, tj * NB, a.d);
   __syncthreads();
   float acc[4][4];
   zero_acc(acc);
-  mm64(As, Bs, acc, tx, ty);
+  mmk(As, Bs, acc, tx, ty);
 #pragma unroll
   for (int i = 0; i < 4; ++i) {
-    const int r = ri + ty + 16 * i;
-    if (r >= k) continue;
-#pragma unroll
-    for (int j = 0; j < 4; ++j) {
-      if (!rhs) {
-        const int cc = s0 + tj * NB + tx + 16 * j;
-        if (cc <= r) a.G[(row0 + r) * a.ld + cc] = cur[i][j] - acc[i][j];
-      } else {
-        a.R[(row0 + r) * a.d + tj * NB + tx + 16 * j] = cur[i][j] - acc[i][j];
-      }
+    const int r = ri + 4 * ty + i;
+    if (r >= k || cmax <= 0) continue;
+    const float4 v = make_float4(cur[i].x - acc[i][0], cur[i].y - acc[i][1],
+                                 cur[i].z - acc[i][2], cur[i].w - acc[i][3]);
+    float *p = out + (int64_t)r * ldo;
+    if (cmax >= 4) {
+      st4(p, v);
+    } else {
+      p[0] = v.x;
+      if (cmax > 1) p[1] = v.y;
+      if (cmax > 2) p[2] = v.z;
     }
   }
 }
@@ -348,30 +501,28 @@ __global__ void __launch_bounds__(256) k_chol_backward(CholArgs a) {
   float *R = a.R + row0 * a.d;
   for (int p = np - 1; p >= 0; --p) {
     const int j0 = p * NB, jb = min(NB, k - j0);
-    const float *Tg = a.T + ((int64_t)b * a.npanel + p) * NB * NB;
-    load_tile_t(At[0], Tg, NB, 0, NB, 0, NB);           // At[r][t] = T[t][r]
-    load_tile_t(Xs, R, a.d, j0, j0 + jb, c0, a.d);      // Xs[col][t] = y[j0 + t][c0 + col]
+    const float *Tg = a.Tt + ((int64_t)b * a.npanel + p) * NB * NB;
+    load_t(At[0], Tg, NB, 0, NB, 0, NB);          // At[t][r] = T[t][r]
+    load_d(Xs, R, a.d, j0, j0 + jb, c0, a.d);     // Xs[t][col] = y[j0 + t][c0 + col]
     __syncthreads();
     float acc[4][4];
     zero_acc(acc);
-    mm64(At[0], Xs, acc, tx, ty);                       // x[r][col]
+    mmk(At[0], Xs, acc, tx, ty);                  // x[r][col]
     __syncthreads();
     bool fin = true;
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
-      const int r = ty + 16 * i;
-#pragma unroll
-      for (int j = 0; j < 4; ++j) {
-        Xs[tx + 16 * j][r] = acc[i][j];  // as the B operand of the updates
-        if (r < jb) {
-          a.X[(row0 + j0 + r) * a.d + c0 + tx + 16 * j] = acc[i][j];
-          fin &= isfinite(acc[i][j]);
-        }
+      const int r = 4 * ty + i;
+      const float4 v = make_float4(acc[i][0], acc[i][1], acc[i][2], acc[i][3]);
+      st4(&Xs[r][4 * tx], v);  // as the B operand of the updates
+      if (r < jb) {
+        st4(a.X + (row0 + j0 + r) * a.d + c0 + 4 * tx, v);
+        fin &= isfinite(v.x) && isfinite(v.y) && isfinite(v.z) && isfinite(v.w);
       }
     }
     if (!fin) atomicOr(&a.dead[b], DEAD_NONFINITE);
     if (p == 0) break;
-    // y_i -= L_ji^T x_j, with At[r][t] = L[j0 + t][64 i + r]
+    // y_i -= L_ji^T x_j, with At[t][r] = L[j0 + t][64 i + r]
     float4 pf[4];
     auto fetch = [&](int i) {
 #pragma unroll
@@ -385,30 +536,25 @@ __global__ void __launch_bounds__(256) k_chol_backward(CholArgs a) {
 #pragma unroll
       for (int u = 0; u < 4; ++u) {
         const int e = tid + 256 * u, r = e >> 4, c = (e & 15) * 4;
-        S[c][r] = pf[u].x;
-        S[c + 1][r] = pf[u].y;
-        S[c + 2][r] = pf[u].z;
-        S[c + 3][r] = pf[u].w;
+        st4(&S[r][c], pf[u]);
       }
     };
     fetch(0);
     place(At[0]);
     __syncthreads();
     for (int i = 0; i < p; ++i) {
-      float cur[4][4];
+      float4 cur[4];
 #pragma unroll
       for (int ii = 0; ii < 4; ++ii)
-#pragma unroll
-        for (int jj = 0; jj < 4; ++jj)
-          cur[ii][jj] = R[(int64_t)(NB * i + ty + 16 * ii) * a.d + c0 + tx + 16 * jj];
+        cur[ii] = ld4(R + (int64_t)(NB * i + 4 * ty + ii) * a.d + c0 + 4 * tx);
       if (i + 1 < p) fetch(i + 1);
       zero_acc(acc);
-      mm64(At[i & 1], Xs, acc, tx, ty);
+      mmk(At[i & 1], Xs, acc, tx, ty);
 #pragma unroll
       for (int ii = 0; ii < 4; ++ii)
-#pragma unroll
-        for (int jj = 0; jj < 4; ++jj)
-          R[(int64_t)(NB * i + ty + 16 * ii) * a.d + c0 + tx + 16 * jj] = cur[ii][jj] - acc[ii][jj];
+        st4(R + (int64_t)(NB * i + 4 * ty + ii) * a.d + c0 + 4 * tx,
+            make_float4(cur[ii].x - acc[ii][0], cur[ii].y - acc[ii][1], cur[ii].z - acc[ii][2],
+                        cur[ii].w - acc[ii][3]));
       if (i + 1 < p) place(At[(i + 1) & 1]);
       __syncthreads();
     }
