@@ -262,9 +262,8 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       if (!ok) break;
       fence_after_sync();
       float s[BQ];
-      tmem_ld32(tmem + lane_base + sb * BQ, s);
-      tmem_ld32(tmem + lane_base + sb * BQ + 32, s + 32);
       if (!C::DK) {
+        tmem_ld64(tmem + lane_base + sb * BQ, s);
         fence_before_sync();
         mbar_arrive(&bars.sd_free[sb]);
         const float4 *l4 = reinterpret_cast<const float4 *>(bars.lse2[st]);
@@ -276,8 +275,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         }
       } else {
         float dp[BQ];
-        tmem_ld32(tmem + lane_base + C::COL_DP + sb * BQ, dp);
-        tmem_ld32(tmem + lane_base + C::COL_DP + sb * BQ + 32, dp + 32);
+        tmem_ld64x2(tmem + lane_base + sb * BQ, s, tmem + lane_base + C::COL_DP + sb * BQ, dp);
         uint32_t hh[32], ll[32];
         const float4 *l4 = reinterpret_cast<const float4 *>(bars.lse2[st]);
         const float4 *d4 = reinterpret_cast<const float4 *>(bars.del[st]);

@@ -282,8 +282,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       float s[HB];
       if (ok) {
         fence_after_sync();
-        tmem_ld32(tmem + lane_base + sb * BN + cb, s);
-        tmem_ld32(tmem + lane_base + sb * BN + cb + 32, s + 32);
+        tmem_ld64(tmem + lane_base + sb * BN + cb, s);
       } else {
 #pragma unroll
         for (int c = 0; c < HB; ++c) s[c] = -INFINITY;
