@@ -173,20 +173,38 @@ __global__ void __launch_bounds__(PT) k_pairs(PairArgs a) {
     const float v = warp_sum(acc[k]);
     if (lane == 0) wsum[warp][k] = v;
   }
-  // one read of each stored pair: y_new . s_j, y_new . y_j, g . s_j, g . y_j
-  for (int p = 0; p < nvalid; ++p) {
+  // one read of each stored pair: y_new . s_j, y_new . y_j, g . s_j, g . y_j; the
+  // next pair's loads are issued before this pair's warp sums
+  float4 sj[V4], yj[V4];
+  auto fetch = [&](int p, float4 *sd, float4 *yd) {
     const int sl = ring_slot(head0, p, slots);
     const float *rs = a.ring_s + sl * a.rstride, *ry = a.ring_y + sl * a.rstride;
-    float c4[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
     for (int u = 0; u < V4; ++u) {
       const int e = (u * PT + threadIdx.x) * 4;
-      if (e >= lim) continue;
-      const float4 sj = ld4(rs + base + e), yj = ld4(ry + base + e);
-      c4[0] = dot4(yv[u], sj, c4[0]);
-      c4[1] = dot4(yv[u], yj, c4[1]);
-      c4[2] = dot4(gv[u], sj, c4[2]);
-      c4[3] = dot4(gv[u], yj, c4[3]);
+      sd[u] = yd[u] = z4;
+      if (e < lim) {
+        sd[u] = ld4(rs + base + e);
+        yd[u] = ld4(ry + base + e);
+      }
+    }
+  };
+  if (nvalid > 0) fetch(0, sj, yj);
+  for (int p = 0; p < nvalid; ++p) {
+    float4 sn[V4], yn[V4];
+    if (p + 1 < nvalid) fetch(p + 1, sn, yn);
+    float c4[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+    for (int u = 0; u < V4; ++u) {
+      c4[0] = dot4(yv[u], sj[u], c4[0]);
+      c4[1] = dot4(yv[u], yj[u], c4[1]);
+      c4[2] = dot4(gv[u], sj[u], c4[2]);
+      c4[3] = dot4(gv[u], yj[u], c4[3]);
+    }
+#pragma unroll
+    for (int u = 0; u < V4; ++u) {
+      sj[u] = sn[u];
+      yj[u] = yn[u];
     }
 #pragma unroll
     for (int k = 0; k < 4; ++k) {

@@ -13,6 +13,9 @@
 //             r_i -= L_ij y_j on the right-hand sides
 //   then one kernel sweeps the panels from the last one: x_j = T_j^T y_j,
 //   y_i -= L_ji^T x_j.
+// Look-ahead: the update is split into the next panel's column and the rest, and
+// the next diagonal block and panel are computed on a second stream while the
+// rest of the update runs.
 // Every 64 x 64 x 64 product runs from shared memory with both operands stored
 // contraction-index-major (S[t][row]): each thread owns a 4 x 4 output block
 // and forms a rank-1 update from two 128-bit loads per t.  The diagonal block
@@ -399,8 +402,13 @@ __global__ void __launch_bounds__(256) k_chol_panel(CholArgs a, int j0) {
 
 // Trailing update: tiles (ti >= tj) of G_ik -= L_i L_k^T, and tiles of
 // r_i -= L_i y_j (columns of R in chunks of 64), 64 x 64 outputs per CTA.  The
-// diagonal tiles are written whole: their upper triangle is scratch.
-__global__ void __launch_bounds__(256) k_chol_update(CholArgs a, int j0) {
+// diagonal tiles are written whole: their upper triangle is scratch.  The tiles
+// come in two parts so that the next panel can start early:
+//   part 1: the next panel's column (ti = 0 .. nt-1, tj = 0), then the right-hand
+//           sides of the next diagonal block (ti = 0)
+//   part 2: the other lower-triangle tiles (1 <= tj <= ti), then the other
+//           right-hand-side rows (ti >= 1)
+__global__ void __launch_bounds__(256) k_chol_update(CholArgs a, int j0, int part) {
   const int b = blockIdx.y;
   const int k = kdim(a, b);
   if (j0 >= k || a.dead[b]) return;
@@ -409,22 +417,35 @@ __global__ void __launch_bounds__(256) k_chol_update(CholArgs a, int j0) {
   const int n2 = k - s0;
   if (n2 <= 0) return;
   const int nt = (n2 + NB - 1) / NB;
-  const int ntri = nt * (nt + 1) / 2;
   const int ndc = a.d / NB;
   int t = blockIdx.x;
   bool rhs = false;
   int ti, tj;
-  if (t < ntri) {
-    ti = (int)((sqrtf(8.f * t + 1.f) - 1.f) * 0.5f);
-    while (ti * (ti + 1) / 2 > t) --ti;
-    while ((ti + 1) * (ti + 2) / 2 <= t) ++ti;
-    tj = t - ti * (ti + 1) / 2;
+  if (part == 1) {
+    if (t >= nt + ndc) return;
+    if (t < nt) {
+      ti = t;
+      tj = 0;
+    } else {
+      rhs = true;
+      ti = 0;
+      tj = t - nt;
+    }
   } else {
-    t -= ntri;
-    if (t >= nt * ndc) return;
-    rhs = true;
-    ti = t / ndc;
-    tj = t % ndc;
+    const int ntri1 = nt * (nt - 1) / 2;  // the triangle 1 <= tj <= ti < nt
+    if (t < ntri1) {
+      int r = (int)((sqrtf(8.f * t + 1.f) - 1.f) * 0.5f);
+      while (r * (r + 1) / 2 > t) --r;
+      while ((r + 1) * (r + 2) / 2 <= t) ++r;
+      ti = r + 1;
+      tj = t - r * (r + 1) / 2 + 1;
+    } else {
+      t -= ntri1;
+      if (t >= (nt - 1) * ndc) return;
+      rhs = true;
+      ti = 1 + t / ndc;
+      tj = t % ndc;
+    }
   }
   __shared__ __align__(16) float As[NB][SP];  // As[t][r] = L[ri + r][j0 + t]
   __shared__ __align__(16) float Bs[NB][SP];  // Bs[t][c] = L[rk + c][j0 + t], or y[j0 + t][c]
@@ -581,24 +602,74 @@ __global__ void __launch_bounds__(256) k_chol_store(CholArgs a, float *Vc) {
 
 }  // namespace
 
+// A side stream (highest priority) and two events per host thread and device: the
+// next panel's diagonal block and panel run on the side stream while the caller's
+// stream finishes the current trailing update (disjoint tiles).  Per-thread objects
+// keep concurrent callers from sharing events.
+struct Lookahead {
+  cudaStream_t side = nullptr;
+  cudaEvent_t fork = nullptr, join = nullptr;
+};
+
+static cudaError_t lookahead(Lookahead **out) {
+  constexpr int kMaxDev = 64;
+  static thread_local Lookahead la[kMaxDev];
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev < 0 || dev >= kMaxDev) return cudaErrorInvalidDevice;
+  Lookahead &l = la[dev];
+  if (!l.side) {
+    // the highest priority: the next panel's few CTAs take SMs as soon as update
+    // CTAs retire instead of queueing behind all of them
+    int least = 0, greatest = 0;
+    if ((e = cudaDeviceGetStreamPriorityRange(&least, &greatest)) != cudaSuccess ||
+        (e = cudaStreamCreateWithPriority(&l.side, cudaStreamNonBlocking, greatest)) != cudaSuccess ||
+        (e = cudaEventCreateWithFlags(&l.fork, cudaEventDisableTiming)) != cudaSuccess ||
+        (e = cudaEventCreateWithFlags(&l.join, cudaEventDisableTiming)) != cudaSuccess)
+      return e;
+  }
+  *out = &l;
+  return cudaSuccess;
+}
+
 int launch_chol_solve(const Batch &Bt, float *Vc, int32_t *status, const Work &w) {
   const HostGeom &g = Bt.g;
   const int npanel = (g.max_c + NB - 1) / NB;
   CholArgs a{w.gram, w.R, w.X, w.chol_t, npanel, w.dead, status, Bt.b->c_off, g.ld_g, g.d};
   KVS_CUDA_TRY(set_smem_once(k_chol_backward, BWD_SMEM));
+  Lookahead *la = nullptr;
+  KVS_CUDA_TRY(lookahead(&la));
   KVS_CUDA_TRY(cudaMemsetAsync(w.dead, 0, sizeof(int) * g.B, Bt.st));
   const int ndc = g.d / NB;
-  for (int p = 0; p < npanel; ++p) {
+  // diagonal block and panel p: their grid depends only on the longest problem
+  auto head = [&](int p, cudaStream_t st) -> int {
     const int j0 = p * NB;
-    k_chol_diag<<<g.B, 256, 0, Bt.st>>>(a, j0);
+    k_chol_diag<<<g.B, 256, 0, st>>>(a, j0);
     KVS_LAUNCH_CHECK("k_chol_diag");
     const int n2 = g.max_c - j0 - NB;
-    if (n2 <= 0) continue;
-    const int nt = (n2 + NB - 1) / NB;
-    k_chol_panel<<<dim3(nt, g.B), 256, 0, Bt.st>>>(a, j0);
-    KVS_LAUNCH_CHECK("k_chol_panel");
-    k_chol_update<<<dim3(nt * (nt + 1) / 2 + nt * ndc, g.B), 256, 0, Bt.st>>>(a, j0);
+    if (n2 > 0) {
+      k_chol_panel<<<dim3((n2 + NB - 1) / NB, g.B), 256, 0, st>>>(a, j0);
+      KVS_LAUNCH_CHECK("k_chol_panel");
+    }
+    return KVS_OK;
+  };
+  int rc = head(0, Bt.st);
+  if (rc) return rc;
+  for (int p = 0; p + 1 < npanel; ++p) {
+    const int j0 = p * NB;
+    const int nt = (g.max_c - j0 - NB + NB - 1) / NB;  // trailing block rows of the longest problem
+    k_chol_update<<<dim3(nt + ndc, g.B), 256, 0, Bt.st>>>(a, j0, 1);
     KVS_LAUNCH_CHECK("k_chol_update");
+    KVS_CUDA_TRY(cudaEventRecord(la->fork, Bt.st));
+    KVS_CUDA_TRY(cudaStreamWaitEvent(la->side, la->fork, 0));
+    if ((rc = head(p + 1, la->side))) return rc;
+    KVS_CUDA_TRY(cudaEventRecord(la->join, la->side));
+    if (nt > 1) {
+      k_chol_update<<<dim3(nt * (nt - 1) / 2 + (nt - 1) * ndc, g.B), 256, 0, Bt.st>>>(a, j0, 2);
+      KVS_LAUNCH_CHECK("k_chol_update");
+    }
+    KVS_CUDA_TRY(cudaStreamWaitEvent(Bt.st, la->join, 0));
   }
   k_chol_backward<<<dim3(ndc, g.B), 256, BWD_SMEM, Bt.st>>>(a);
   KVS_LAUNCH_CHECK("k_chol_backward");
