@@ -97,7 +97,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     mbar_init(&bars.k_full, 1);
     mbar_init(&bars.v_full, 2 * BK);
     for (int i = 0; i < NSTAGE; ++i) {
-      mbar_init(&bars.q_full[i], 1);
+      mbar_init(&bars.q_full[i], 2);  // the copies' arrival and the staged l / delta
       mbar_init(&bars.q_empty[i], 1 + BK);
     }
     for (int i = 0; i < 2; ++i) {
@@ -137,13 +137,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
           break;
         }
       }
-      for (int e = lane; e < BQ; e += 32) {
-        const int q = (t0 + i) * BQ + e;
-        const bool v = q < nq;
-        bars.lse2[st][e] = v ? a.lse[q_begin + q] * L2E : INFINITY;
-        bars.del[st][e] = (v && C::DK) ? a.delta[q_begin + q] : 0.f;
-      }
-      __syncwarp();
+      // the tile's copies first, then its l and delta (their loads overlap the copies)
       if (lane == 0) {
         issued = i + 1;
         unsigned char *base = sm + C::OFF_ST + st * C::STAGE;
@@ -156,6 +150,14 @@ __global__ void __launch_bounds__(NTHREADS, 1)
             tma_load_2d(base + 2 * C::Q_BYTES + r * BQ * 128, &mG, &bars.q_full[st], 64 * r, qrow);
         }
       }
+      for (int e = lane; e < BQ; e += 32) {
+        const int q = (t0 + i) * BQ + e;
+        const bool v = q < nq;
+        bars.lse2[st][e] = v ? a.lse[q_begin + q] * L2E : INFINITY;
+        bars.del[st][e] = (v && C::DK) ? a.delta[q_begin + q] : 0.f;
+      }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&bars.q_full[st]);
     }
     if (lane == 0 && *abort) {  // let issued copies land before shared memory is released
       mbar_wait(&bars.k_full, 0);
@@ -168,7 +170,6 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       const uint32_t id_s = idesc_bf16(BK, BQ, false, false);
       const uint32_t id_dk = idesc_bf16(BK, D, false, true);
       bool ok = mbar_wait(&bars.k_full, 0, abort);
-      if (C::DK) ok = ok && mbar_wait(&bars.v_full, 0, abort);
       fence_after_sync();
       const uint64_t kh0 = sdesc(smem_u32(sm), 16, 1024), kl0 = sdesc_add(kh0, C::K_BYTES);
       const uint32_t tv_hi = tmem + C::COL_V, tv_lo = tmem + C::COL_V + D / 2;
@@ -207,7 +208,17 @@ __global__ void __launch_bounds__(NTHREADS, 1)
           mma_bf16(tmem + sb * BQ, kh, qh, id_s, kk > 0 ? 1u : 0u);
           mma_bf16(tmem + sb * BQ, kl, qh, id_s, 1u);
           mma_bf16(tmem + sb * BQ, kh, ql, id_s, 1u);
-          if (C::DK) {
+        }
+        if (C::DK) {
+          // V reaches tensor memory through the row threads: the first score product
+          // runs while they store it
+          if (i == 0) {
+            if (!mbar_wait(&bars.v_full, 0, abort)) { ok = false; break; }
+            fence_after_sync();
+          }
+#pragma unroll
+          for (int kk = 0; kk < D / 16; ++kk) {
+            const uint32_t oq = (kk >> 2) * (BQ * 128) + (kk & 3) * 32;
             const uint64_t gd = sdesc_add(gd0, oq);
             mma_bf16_ts(tmem + C::COL_DP + sb * BQ, tv_hi + kk * 8, gd, id_s, kk > 0 ? 1u : 0u);
             mma_bf16_ts(tmem + C::COL_DP + sb * BQ, tv_lo + kk * 8, gd, id_s, 1u);
