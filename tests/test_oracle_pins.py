@@ -312,6 +312,48 @@ def test_lbfgs_failed_search_keeps_x():
     assert st.trials == 6
 
 
+def test_lbfgs_block_on_the_loss_meets_armijo_every_step():
+    """On the distillation loss itself (fixed V_c): every accepted step satisfies
+    f(x + t d) <= f(x) + c1 t g.d with the g.d of a descent direction, so f never
+    rises inside an L-BFGS block; checked against f and g recomputed from scratch."""
+    Q, Kz, Vz, Kc, _ = tiny(n_q=40, z=20, k=5, d=8, seed=21)
+    Y, lse = O.targets(Q, Kz, Vz)
+    V, _ = O.ridge_fit(Q, Kc, Y, 1e-3)
+    d = Q.shape[1]
+    fl = lambda x: O.loss_only(Q, x.reshape(-1, d), V, Y, lse)
+    fg = lambda x: O.loss_grad(Q, x.reshape(-1, d), V, Y, lse)[1].ravel()
+    f0, g0, _ = O.loss_grad(Q, Kc, V, Y, lse)
+    st = O.LBFGSState(x=Kc.ravel().copy(), f=f0, g=g0.ravel())
+    for _ in range(8):
+        x_old, f_old, g_old = st.x.copy(), st.f, st.g.copy()
+        assert O.lbfgs_step(st, fl, fg)
+        step = st.x - x_old
+        assert float(g_old @ step) < 0.0                      # a descent step
+        assert st.f <= f_old + 1e-4 * float(g_old @ step)     # Armijo with t d = step
+        assert abs(st.f - fl(st.x)) <= 1e-12 * max(1.0, abs(st.f))
+        np.testing.assert_allclose(st.g, fg(st.x), rtol=1e-10, atol=1e-14)
+
+
+def test_ridge_fit_minimises_the_penalised_objective():
+    """The fitted V_c is the minimiser of |A V - Y|^2 + lam |V|^2: random
+    perturbations of either sign raise the objective by exactly |A E|^2 + lam |E|^2
+    (a quadratic with zero gradient at the minimiser)."""
+    Q, Kz, Vz, Kc, _ = tiny(n_q=30, z=12, k=5, d=6, seed=22)
+    Y, lse = O.targets(Q, Kz, Vz)
+    lam = 0.05
+    V, _ = O.ridge_fit(Q, Kc, Y, lam)
+    A, _ = O.attention(Q, Kc)
+    obj = lambda W: float(np.sum((A @ W - Y) ** 2) + lam * np.sum(W ** 2))
+    base = obj(V)
+    r = np.random.default_rng(5)
+    for _ in range(5):
+        E = r.standard_normal(V.shape) * 1e-2
+        for sgn in (1.0, -1.0):
+            rise = obj(V + sgn * E) - base
+            expect = float(np.sum((A @ E) ** 2) + lam * np.sum(E ** 2))
+            assert abs(rise - expect) <= 1e-9 * max(1.0, base)
+
+
 def test_compress_trace_and_select_fit():
     """Loss never rises across L-BFGS blocks followed by value re-fits in this
     small case, iteration 0 is Select+Fit, and the solve beats it."""
