@@ -174,7 +174,12 @@ int kvs_loss_grad_static(const kvs_batch *batch, const float *Q, const float *Kc
 /* Closed-form values (section 2 "Value Optimization"): with A = softmax(s Q Kc^T)
  * fixed, Vc = (A^T A + lambda I)^-1 A^T Y, by Cholesky.  A problem whose Gram
  * matrix is not positive definite gets KVS_ST_NOT_PD in status[b] (OR-ed in)
- * and keeps its previous Vc. */
+ * and keeps its previous Vc.
+ * The factorisation forks part of its work onto one internal high-priority
+ * stream (created once per host thread and device) through events recorded on
+ * `stream`, and joins it back to `stream` before returning: the call stays
+ * ordered on `stream` and can be captured into a graph like any other.  This
+ * holds for every entry point that fits values (kvs_compress_batch too). */
 int kvs_fit_values(const kvs_batch *batch, const float *Q, const float *Kc, const float *Y,
                    float lambda, float *Vc, int32_t *status, void *ws, size_t ws_bytes,
                    void *stream);
