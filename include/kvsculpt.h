@@ -177,9 +177,9 @@ int kvs_loss_grad_static(const kvs_batch *batch, const float *Q, const float *Kc
  * and keeps its previous Vc.
  * The factorisation forks part of its work onto one internal high-priority
  * stream (created once per host thread and device) through events recorded on
- * `stream`, and joins it back to `stream` before returning: the call stays
- * ordered on `stream` and can be captured into a graph like any other.  This
- * holds for every entry point that fits values (kvs_compress_batch too). */
+ * `stream`, and joins it back to `stream` before returning, so the call stays
+ * ordered on `stream` (every entry point that fits values, kvs_compress_batch
+ * too, behaves this way). */
 int kvs_fit_values(const kvs_batch *batch, const float *Q, const float *Kc, const float *Y,
                    float lambda, float *Vc, int32_t *status, void *ws, size_t ws_bytes,
                    void *stream);
