@@ -18,7 +18,7 @@ __all__ = [
     "rope_inv_freq", "rope", "derope", "build_queries",
     "attention", "targets", "importance", "topk_select", "ridge_fit",
     "loss_grad", "loss_only", "two_loop_direction", "LBFGSState", "lbfgs_step",
-    "Schedule", "compress", "pilot_allocate", "adaptive_compress",
+    "Schedule", "compress", "restart_search", "pilot_allocate", "adaptive_compress",
 ]
 
 ST_OK = 0
@@ -330,6 +330,18 @@ def compress(Q, Kz, Vz, k: int, sched: Schedule, idx: Optional[np.ndarray] = Non
 # ---------------------------------------------------------------------------
 # Adaptive budget allocation (Summary 2 "Adaptive Budget Allocation"; Abstract).
 # ---------------------------------------------------------------------------
+
+
+def restart_search(Q, Kz, Vz, k: int, sched: Schedule, inits):
+    """Random-restart search over the initial keys ("KVSculpt: KV Cache Compression
+    as Distillation", summary §4 "Optimizer Efficacy": a single L-BFGS run is
+    compared with the best of 100 random restarts).  Each restart runs the whole
+    schedule of `compress` from the zone keys inits[r] (k positions) instead of
+    the top-k ones; returns the results and the index of the lowest final loss
+    (the first one on ties)."""
+    runs = [compress(Q, Kz, Vz, k, sched, idx=np.asarray(ix)) for ix in inits]
+    losses = [r["loss"] for r in runs]
+    return runs, int(np.argmin(losses))
 
 def _clamped_shares(w, lo, hi, total):
     """x_b = clip(c * w_b, lo_b, hi_b) with the scalar c >= 0 chosen so that sum x = total.

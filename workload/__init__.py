@@ -41,7 +41,7 @@ import numpy as np
 
 __all__ = [
     "Workload", "Batch", "WORKLOADS", "k_from_ratio", "generate", "make_batch",
-    "subset",
+    "subset", "restart_inits",
 ]
 
 
@@ -253,3 +253,24 @@ def subset(wl: Workload, count: int, seed: int = 0) -> list:
     rng = _stream(seed, 7 << 20)
     pick = np.sort(rng.choice(len(allids), min(count, len(allids)), replace=False))
     return [allids[i] for i in pick]
+
+
+def restart_inits(z_counts: Sequence[int], k_counts: Sequence[int], restarts: int,
+                  seed: int = 0) -> np.ndarray:
+    """Initial key subsets of a random-restart search: for restart r and problem b,
+    k_b distinct zone positions drawn uniformly without replacement from
+    [0, z_b), sorted ascending.  Returns int32 [restarts, sum k_b] (problem b's
+    entries at its c_off[b] ..).  The draw is the search's own random choice,
+    passed to both sides as an input; each (restart, problem) has its own stream."""
+    z_counts = [int(z) for z in z_counts]
+    k_counts = [int(k) for k in k_counts]
+    if len(z_counts) != len(k_counts) or any(not 1 <= k <= z for k, z in zip(k_counts, z_counts)):
+        raise ValueError("each problem needs 1 <= k_b <= z_b")
+    out = np.empty((restarts, sum(k_counts)), np.int32)
+    for r in range(restarts):
+        c = 0
+        for b, (z, k) in enumerate(zip(z_counts, k_counts)):
+            rng = _stream(seed, 9 << 20, r, b)
+            out[r, c:c + k] = np.sort(rng.choice(z, k, replace=False))
+            c += k
+    return out
