@@ -204,6 +204,19 @@ int kvs_lbfgs_step(const kvs_batch *batch, const kvs_schedule *sched, const floa
                    void *state, size_t state_bytes, int32_t *status, float *f_out,
                    void *ws, size_t ws_bytes, void *stream);
 
+/* One Adam step on Kc, the ablation of the key optimiser (section 4 "Optimizer
+ * Efficacy": Adam in place of L-BFGS leaves a much larger per-layer error).
+ * With g = dKc [sum_c, d] (e.g. from kvs_loss_grad), elementwise over all
+ * sum_c x d values of the batch:
+ *   m <- beta1 m + (1 - beta1) g,   v <- beta2 v + (1 - beta2) g^2,
+ *   Kc <- Kc - lr (m / (1 - beta1^t)) / (sqrt(v / (1 - beta2^t)) + eps).
+ * m, v: caller buffers [sum_c, d] (float32, 16-byte aligned), zero before the
+ * first step and carried between steps; t >= 1 counts the steps taken so far
+ * including this one.  Errors: KVS_EINVAL for a null or unaligned pointer,
+ * t < 1, lr <= 0, beta outside [0, 1) or eps <= 0. */
+int kvs_adam_step(const kvs_batch *batch, float *Kc, const float *dKc, float *m, float *v,
+                  int32_t t, float lr, float beta1, float beta2, float eps, void *stream);
+
 /* The whole alternating solve for a batch (Abstract; section 2): targets,
  * importance, top-k keys, ridge values (the Select+Fit state), then
  * sched->outer times { sched->steps L-BFGS steps; ridge re-fit }.

@@ -20,7 +20,7 @@ __all__ = [
     "ST_NONFINITE", "ST_NOT_PD", "ST_LS_FAIL",
     "kvs_version", "kvs_launch_count", "kvs_workspace_bytes", "kvs_lbfgs_state_bytes", "kvs_build_queries",
     "kvs_targets", "kvs_init_topk", "kvs_loss_grad", "kvs_loss_grad_static", "kvs_fit_values", "kvs_lbfgs_reset",
-    "kvs_lbfgs_step", "kvs_compress_batch", "kvs_pilot_allocate",
+    "kvs_lbfgs_step", "kvs_compress_batch", "kvs_pilot_allocate", "kvs_adam_step",
     "alloc_workspace", "alloc_state",
 ]
 
@@ -74,6 +74,7 @@ _SIGS = {
     "kvs_compress_batch": (ctypes.c_int, [_BP, _SP, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp,
                                           _vp, _vp, _sz, _vp, _sz, _vp]),
     "kvs_pilot_allocate": (ctypes.c_int, [_i32, _vp, _i64, _i32, _vp, _f32, _vp]),
+    "kvs_adam_step": (ctypes.c_int, [_BP, _vp, _vp, _vp, _vp, _i32, _f32, _f32, _f32, _f32, _vp]),
 }
 for _name, (_res, _args) in _SIGS.items():
     _fn = getattr(lib, _name)
@@ -307,6 +308,14 @@ def kvs_compress_batch(batch: KvsBatch, sched: Schedule, Q, Kz, Vz, Kc, Vc, idx,
         _ptr(Vz, torch.float32), _ptr(Kc, torch.float32), _ptr(Vc, torch.float32),
         _ptr(idx, torch.int32), _ptr(loss_trace, torch.float32), _ptr(parts, torch.float32),
         _ptr(status, torch.int32), _ptr(state), state.numel(), _ptr(ws), ws.numel(),
+        _stream(stream)))
+
+
+def kvs_adam_step(batch: KvsBatch, Kc, dKc, m, v, t: int, lr: float, beta1: float = 0.9,
+                  beta2: float = 0.999, eps: float = 1e-8, stream=None):
+    _check("kvs_adam_step", lib.kvs_adam_step(
+        batch.ref, _ptr(Kc, torch.float32), _ptr(dKc, torch.float32), _ptr(m, torch.float32),
+        _ptr(v, torch.float32), int(t), float(lr), float(beta1), float(beta2), float(eps),
         _stream(stream)))
 
 

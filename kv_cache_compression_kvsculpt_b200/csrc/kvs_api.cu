@@ -461,6 +461,21 @@ int kvs_lbfgs_step(const kvs_batch *batch, const kvs_schedule *sched, const floa
   return fold_err(Bt, w, status);
 }
 
+int kvs_adam_step(const kvs_batch *batch, float *Kc, const float *dKc, float *m, float *v,
+                  int32_t t, float lr, float beta1, float beta2, float eps, void *stream) {
+  HostGeom g;
+  int rc = geom_from_batch(batch, &g, true);
+  if (rc) return rc;
+  if (!ok_ptr(Kc) || !ok_ptr(dKc) || !ok_ptr(m) || !ok_ptr(v)) return KVS_EINVAL;
+  if (t < 1 || !(lr > 0.f) || !isfinite(lr) || !(beta1 >= 0.f && beta1 < 1.f) ||
+      !(beta2 >= 0.f && beta2 < 1.f) || !(eps > 0.f) || !isfinite(eps))
+    return KVS_EINVAL;
+  const double bc1 = 1.0 - pow((double)beta1, (double)t);
+  const double bc2 = 1.0 - pow((double)beta2, (double)t);
+  return launch_adam(Kc, dKc, m, v, g.sum_c * g.d, lr, beta1, beta2, eps, (float)bc1, (float)bc2,
+                     static_cast<cudaStream_t>(stream));
+}
+
 int kvs_compress_batch(const kvs_batch *batch, const kvs_schedule *sched, const float *Q,
                        const float *Kz, const float *Vz, float *Kc, float *Vc, int32_t *idx,
                        float *loss_trace, float *parts, int32_t *status, void *state,

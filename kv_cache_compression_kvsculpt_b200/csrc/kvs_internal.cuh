@@ -142,4 +142,9 @@ int launch_lbfgs_update(const Batch &B, const State &s, float *Kc, int32_t *stat
                         float *f_out);
 int launch_copy_f(const Batch &B, const State &s, float *dst, int64_t stride, int64_t col);
 
+// Adam ablation (kvs_adam.cu): one elementwise Adam step over n key values
+// (bc1, bc2: the bias corrections 1 - beta^t).
+int launch_adam(float *Kc, const float *dKc, float *m, float *v, int64_t n, float lr, float b1,
+                float b2, float eps, float bc1, float bc2, cudaStream_t st);
+
 }  // namespace kvs

@@ -18,7 +18,8 @@ __all__ = [
     "rope_inv_freq", "rope", "derope", "build_queries",
     "attention", "targets", "importance", "topk_select", "ridge_fit",
     "loss_grad", "loss_only", "two_loop_direction", "LBFGSState", "lbfgs_step",
-    "Schedule", "compress", "restart_search", "pilot_allocate", "adaptive_compress",
+    "Schedule", "compress", "restart_search", "adam_step", "adam_compress",
+    "pilot_allocate", "adaptive_compress",
 ]
 
 ST_OK = 0
@@ -342,6 +343,49 @@ def restart_search(Q, Kz, Vz, k: int, sched: Schedule, inits):
     runs = [compress(Q, Kz, Vz, k, sched, idx=np.asarray(ix)) for ix in inits]
     losses = [r["loss"] for r in runs]
     return runs, int(np.argmin(losses))
+
+
+def adam_step(x, g, m, v, t: int, lr: float, beta1=0.9, beta2=0.999, eps=1e-8):
+    """One Adam step (Kingma & Ba, bias-corrected moments); returns (x, m, v)."""
+    m = beta1 * m + (1.0 - beta1) * g
+    v = beta2 * v + (1.0 - beta2) * g * g
+    mh = m / (1.0 - beta1 ** t)
+    vh = v / (1.0 - beta2 ** t)
+    return x - lr * mh / (np.sqrt(vh) + eps), m, v
+
+
+def adam_compress(Q, Kz, Vz, k: int, sched: Schedule, lr: float, beta1=0.9, beta2=0.999,
+                  eps=1e-8, idx: Optional[np.ndarray] = None):
+    """The schedule of `compress` with Adam on K_c in place of L-BFGS: the
+    optimiser ablation of the page ("KVSculpt: KV Cache Compression as
+    Distillation", summary §4 "Optimizer Efficacy").  `steps` Adam steps per
+    outer iteration, one step per loss/gradient evaluation; the moments and the
+    step count persist across value re-fits (one optimiser across outers)."""
+    Q = np.asarray(Q, np.float64)
+    d = Q.shape[1]
+    Y, lse = targets(Q, Kz, Vz)
+    if idx is None:
+        idx = topk_select(importance(Q, Kz, lse), k)
+    Kc = np.asarray(Kz, np.float64)[idx].copy()
+    Vc, status = ridge_fit(Q, Kc, Y, sched.lam)
+    if Vc is None:
+        Vc = np.zeros((len(idx), d))
+    trace = [loss_only(Q, Kc, Vc, Y, lse, sched.w_out, sched.w_lse)]
+    m = np.zeros_like(Kc)
+    v = np.zeros_like(Kc)
+    t = 0
+    for _o in range(sched.outer):
+        for _s in range(sched.steps):
+            t += 1
+            _, g, _ = loss_grad(Q, Kc, Vc, Y, lse, sched.w_out, sched.w_lse)
+            Kc, m, v = adam_step(Kc, g, m, v, t, lr, beta1, beta2, eps)
+        V_new, st_fit = ridge_fit(Q, Kc, Y, sched.lam)
+        status |= st_fit
+        if V_new is not None:
+            Vc = V_new
+        trace.append(loss_only(Q, Kc, Vc, Y, lse, sched.w_out, sched.w_lse))
+    return dict(Kc=Kc, Vc=Vc, trace=np.array(trace), loss=float(trace[-1]), idx=idx,
+                status=status)
 
 def _clamped_shares(w, lo, hi, total):
     """x_b = clip(c * w_b, lo_b, hi_b) with the scalar c >= 0 chosen so that sum x = total.
