@@ -605,7 +605,8 @@ __global__ void __launch_bounds__(256) k_chol_store(CholArgs a, float *Vc) {
 // A side stream (highest priority) and two events per host thread and device: the
 // next panel's diagonal block and panel run on the side stream while the caller's
 // stream finishes the current trailing update (disjoint tiles).  Per-thread objects
-// keep concurrent callers from sharing events.
+// keep concurrent callers from sharing events; they are created on a thread's first
+// solve and kept for the life of the process (three handles per thread and device).
 struct Lookahead {
   cudaStream_t side = nullptr;
   cudaEvent_t fork = nullptr, join = nullptr;
