@@ -334,7 +334,7 @@ def run_gpu(args):
                    "parallelism": f"problem-sharded x{world}, no collective"},
         "e2e": {"value": round(e2e_value, 4), "unit": "head-problems/s",
                 "h2d_bytes_per_step": job.h2d_bytes(), "d2h_bytes_per_step": job.d2h_bytes()},
-        "loss_grad_evals_per_s": round(wl.B / (lg_ms * 1e-3), 1),
+        "loss_grad_evals_per_s": round(job.batch.B / (lg_ms * 1e-3), 1),  # per rank's batch
         "roofline": {"kernel": "kvs_loss_grad (forward + dKc backward, whole batch)",
                      "bound": args.bound, "achieved": round(lg_tflops, 3), "peak": peak,
                      "unit": "TFLOP/s", "frac": round(lg_tflops / peak, 4),
@@ -350,7 +350,7 @@ def run_gpu(args):
                     "final_loss_mean": float(np.mean(final)),
                     "status_nonzero": int((status != 0).sum())},
     }
-    if rank == 0 and not args.no_cpu_baseline:
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:  # the oracle beside one GPU only
         out["cpu_baseline"] = cpu_baseline(wl, budget_s=args.cpu_budget)
     if rank == 0:
         print(json.dumps(out), flush=True)
