@@ -71,3 +71,19 @@ def test_adam_step_argument_errors(K=None):
     unaligned = ctypes.c_void_p((1 << 20) + 4)
     assert lib.kvs_adam_step(b.ref, fake, unaligned, fake, fake, 1, 1e-2, 0.9, 0.999, 1e-8,
                              None) != 0
+
+
+def test_adam_moments_persist_across_refits():
+    """One Adam step per outer iteration: the first step moves every key
+    coordinate by exactly lr (zero moments, bias correction), while the second,
+    taken after the value re-fit with the moments carried over, does not."""
+    r = np.random.default_rng(43)
+    Q = r.standard_normal((20, 4))
+    Kz = r.standard_normal((9, 4))
+    Vz = r.standard_normal((9, 4))
+    one = O.adam_compress(Q, Kz, Vz, 3, O.Schedule(outer=1, steps=1), lr=1e-2, eps=1e-14)
+    two = O.adam_compress(Q, Kz, Vz, 3, O.Schedule(outer=2, steps=1), lr=1e-2, eps=1e-14)
+    K0 = Kz[one["idx"]]
+    np.testing.assert_allclose(np.abs(one["Kc"] - K0), 1e-2, rtol=1e-9)
+    step2 = np.abs(two["Kc"] - one["Kc"])
+    assert np.abs(step2 - 1e-2).max() > 1e-4
