@@ -277,13 +277,16 @@ class Schedule:
     persist_history: bool = True
 
 
-def compress(Q, Kz, Vz, k: int, sched: Schedule, idx: Optional[np.ndarray] = None):
+def compress(Q, Kz, Vz, k: int, sched: Schedule, idx: Optional[np.ndarray] = None,
+             record: Optional[list] = None):
     """Distil one compress zone (K_z, V_z) into k pairs for the training queries Q.
 
     targets -> importance -> top-k keys -> ridge values (Select+Fit state) ->
     [steps x L-BFGS on K_c, ridge re-fit of V_c] x outer.  Returns a dict with
     K_c, V_c, the loss trace after every fit (outer + 1 entries), the final
-    loss terms, the top-k indices and the status bits.
+    loss terms, the top-k indices and the status bits.  When `record` is a
+    list, a copy of (K_c, V_c, number of stored L-BFGS pairs) is appended to
+    it after every fit (outer + 1 entries); nothing else changes.
     """
     Q = np.asarray(Q, np.float64)
     d = Q.shape[1]
@@ -306,6 +309,8 @@ def compress(Q, Kz, Vz, k: int, sched: Schedule, idx: Optional[np.ndarray] = Non
     f, g, _ = loss_grad(Q, Kc, Vc, Y, lse, sched.w_out, sched.w_lse)
     st = LBFGSState(x=Kc.ravel().copy(), f=f, g=g.ravel())
     trace = [f]
+    if record is not None:
+        record.append((Kc.copy(), Vc.copy(), 0))
     for _o in range(sched.outer):
         for _t in range(sched.steps):
             lbfgs_step(st, fl, fg, sched.history, sched.c1, sched.backtrack, sched.max_bt)
@@ -320,6 +325,8 @@ def compress(Q, Kz, Vz, k: int, sched: Schedule, idx: Optional[np.ndarray] = Non
         f, g, _ = loss_grad(Q, Kc, Vc, Y, lse, sched.w_out, sched.w_lse)
         st.f, st.g = f, g.ravel()
         trace.append(f)
+        if record is not None:
+            record.append((Kc.copy(), Vc.copy(), len(st.hist_s)))
     f, _, info = loss_grad(Q, Kc, Vc, Y, lse, sched.w_out, sched.w_lse)
     if not math.isfinite(f):
         status |= ST_NONFINITE
