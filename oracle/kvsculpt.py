@@ -125,13 +125,17 @@ def ridge_fit(Q, Kc, Y, lam: float):
     With the attention weights A induced by the current keys fixed,
     V_c = argmin ||A V - Y||_F^2 + lam ||V||_F^2 = (A^T A + lam I)^-1 A^T Y.
     Returns (V_c, status); a Gram matrix that is not positive definite gives
-    ST_NOT_PD and V_c = None.
+    ST_NOT_PD and V_c = None, and so does one with a non-finite entry (it has
+    no Cholesky factor); a finite Gram matrix with a non-finite solution (e.g.
+    a NaN in Y) gives ST_NONFINITE and V_c = None.
     """
     A, _ = attention(Q, Kc)
     G = A.T @ A + lam * np.eye(A.shape[1])
     R = A.T @ np.asarray(Y, np.float64)
+    if not np.all(np.isfinite(G)):
+        return None, ST_NOT_PD
     try:
-        V = scipy.linalg.solve(G, R, assume_a="pos")
+        V = scipy.linalg.solve(G, R, assume_a="pos", check_finite=False)
     except np.linalg.LinAlgError:
         return None, ST_NOT_PD
     if not np.all(np.isfinite(V)):
@@ -239,6 +243,8 @@ def lbfgs_step(st: LBFGSState, fun_loss, fun_grad, history=10, c1=1e-4, backtrac
         xt = st.x + t * d
         ft = fun_loss(xt)
         st.trials += 1
+        if not math.isfinite(ft):  # rejected below (a NaN comparison is false)
+            st.status |= ST_NONFINITE
         if ft <= st.f + c1 * t * gtd:
             gt = fun_grad(xt)
             s = xt - st.x

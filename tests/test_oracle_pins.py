@@ -440,3 +440,27 @@ def test_allocation_zero_signal_absorbs_leftover():
     assert k.tolist() == [20, 10, 20]
     k = O.pilot_allocate([0.0, 4.0, 0.0], 20, 5, [30, 10, 30], 0.5)
     assert k.tolist() == [5, 10, 5]
+
+
+def test_ridge_non_finite_inputs():
+    """A NaN in Y leaves the Gram matrix finite and the solution NaN
+    (ST_NONFINITE); a NaN in Q makes the Gram matrix non-finite, which has no
+    Cholesky factor (ST_NOT_PD)."""
+    Q, _, _, Kc, Vc = tiny(n_q=9, k=3, d=4, seed=4)
+    Y = np.random.default_rng(5).standard_normal((9, 4))
+    Y[2, 1] = np.nan
+    V, st = O.ridge_fit(Q, Kc, Y, 1e-3)
+    assert V is None and st == O.ST_NONFINITE
+    Q2 = Q.copy()
+    Q2[0, 0] = np.nan
+    V, st = O.ridge_fit(Q2, Kc, np.nan_to_num(Y), 1e-3)
+    assert V is None and st == O.ST_NOT_PD
+
+
+def test_lbfgs_non_finite_trial_is_rejected_and_flagged():
+    x0 = np.array([1.0, -2.0])
+    st = O.LBFGSState(x=x0.copy(), f=2.5, g=x0.copy())
+    ok = O.lbfgs_step(st, lambda x: float("nan"), lambda x: x, max_bt=4)
+    assert not ok and st.trials == 4
+    assert st.status & O.ST_NONFINITE and st.status & O.ST_LS_FAIL
+    np.testing.assert_array_equal(st.x, x0)
