@@ -103,6 +103,18 @@ const char *kvs_version(void);
 const char *kvs_last_cuda_error(void);     /* text of the last CUDA error seen by this thread */
 uint64_t kvs_launch_count(void);           /* kernels this library has launched in this process */
 
+/* Failure detection.  Every wait inside the tensor-core kernels is bounded: a
+ * kernel whose pipeline wait spins longer than the limit stops, lets the
+ * copies and MMAs it already issued complete, and raises the call's timeout
+ * flag.  Calls with a status array report it as KVS_ST_TIMEOUT in every
+ * problem; kvs_targets, kvs_loss_grad and kvs_loss_grad_static, which have no
+ * status array, then write NaN into every element of their outputs instead.
+ * kvs_set_wait_limit sets the limit in SM clock cycles for launches issued
+ * after it, process-wide (0 restores the default, about 2 s; a CUDA graph
+ * keeps the limit it was recorded with).  It exists to test this path with a
+ * limit too short for any wait to succeed; KVS_EINVAL for cycles < 0. */
+int kvs_set_wait_limit(int64_t cycles);
+
 /* Bytes of scratch workspace needed by every call below for this batch
  * (and schedule; may be NULL when no L-BFGS call will use the workspace).
  * Returns 0 for an invalid batch. */
@@ -110,6 +122,26 @@ size_t kvs_workspace_bytes(const kvs_batch *batch, const kvs_schedule *sched);
 
 /* Bytes of persistent L-BFGS state for this batch and history length. */
 size_t kvs_lbfgs_state_bytes(const kvs_batch *batch, int32_t history);
+
+/* Where the L-BFGS state of kvs_lbfgs_step lives inside a state buffer
+ * (host only; for inspection and tests: the solver needs none of it).  All
+ * offsets are in bytes from the start of the buffer.
+ *   scalars + b * scalar_bytes: problem b's record, holding at off_f the
+ *     float loss f at x, at off_count the int32 number of stored pairs and at
+ *     off_head the int32 ring slot the next pair goes to;
+ *   x, g, dir: float [sum k_b * d] vectors (problem b at c_off[b] * d): the
+ *     accepted keys, the gradient there and the last search direction;
+ *   ring_s, ring_y: `slots` = history + 1 vectors each, ring_stride bytes
+ *     apart, holding s = x_new - x_old and y = g_new - g_old of the stored
+ *     pairs: pair p (p = 0 the newest, p < count) of a problem sits in slot
+ *     (head - 1 - p) mod slots.
+ * KVS_EINVAL for a null `out`, an invalid batch or history outside 1..15. */
+typedef struct kvs_lbfgs_layout {
+  uint64_t scalars, scalar_bytes, off_f, off_count, off_head;
+  uint64_t x, g, dir, ring_s, ring_y, ring_stride;
+  int32_t slots;
+} kvs_lbfgs_layout;
+int kvs_lbfgs_state_layout(const kvs_batch *batch, int32_t history, kvs_lbfgs_layout *out);
 
 /* Training queries (section 2 "Training Query Construction").
  * q_retain [B*g*m_q, d]: retain queries, already RoPE'd at their positions,
@@ -126,7 +158,8 @@ int kvs_build_queries(const kvs_query_spec *spec, const float *q_retain, const f
  * Y = softmax(S0) Vz.  If `importance` is non-NULL it also receives
  * importance[j] = sum_i exp(S0[i,j] - lse[i]) over the problem's z_b keys
  * (section 2 "Initialization": attention importance), rows by z_off.
- * Q [sum n_q, d], Kz/Vz [sum z, d]; Y [sum n_q, d]; lse [sum n_q]. */
+ * Q [sum n_q, d], Kz/Vz [sum z, d]; Y [sum n_q, d]; lse [sum n_q].
+ * If a kernel's bounded wait gave up, Y, lse and importance are all NaN. */
 int kvs_targets(const kvs_batch *batch, const float *Q, const float *Kz, const float *Vz,
                 float *Y, float *lse, float *importance, void *ws, size_t ws_bytes, void *stream);
 
@@ -142,7 +175,8 @@ int kvs_init_topk(const kvs_batch *batch, const float *importance, const float *
  * Function"):  A = softmax(s Q Kc^T), Yh = A Vc, lh = LSE(s Q Kc^T),
  * loss[b] = w_out/(n_q d) ||Yh - Y||_F^2 + w_lse/n_q ||lh - lse||^2, and
  * dKc = dloss/dKc [sum k_b, d].  dKc may be NULL (loss only).
- * parts (nullable) [B,2] receives the unweighted output-MSE and LSE-MSE. */
+ * parts (nullable) [B,2] receives the unweighted output-MSE and LSE-MSE.
+ * If a kernel's bounded wait gave up, loss, parts and dKc are all NaN. */
 int kvs_loss_grad(const kvs_batch *batch, const float *Q, const float *Kc, const float *Vc,
                   const float *Y, const float *lse, float w_out, float w_lse,
                   float *loss, float *parts, float *dKc, void *ws, size_t ws_bytes,
@@ -160,8 +194,10 @@ int kvs_loss_grad(const kvs_batch *batch, const float *Q, const float *Kc, const
  * - Batches whose kvs_workspace_bytes() exceeds 32 MiB return KVS_EWORKSPACE
  *   (one head-problem with d = 128, n_q = 3840 and k = 960 fits; two do not).
  * - The first call on a device looks up the array's device address with that
- *   device current (cudaGetSymbolAddress) and caches it; make that first call
- *   before any stream capture.
+ *   device current (cudaGetSymbolAddress) and caches it with the context it
+ *   belongs to; a call under another context (after cudaDeviceReset, or with
+ *   another driver context current) looks it up again.  Make the first call
+ *   in each context before any stream capture.
  * - Every call on a device shares the one array and the array keeps the last
  *   call's contents.  No part of it needs to start at zero for this call.
  *   Calls whose work overlaps on the GPU (other streams, other host threads)
@@ -174,7 +210,9 @@ int kvs_loss_grad_static(const kvs_batch *batch, const float *Q, const float *Kc
 /* Closed-form values (section 2 "Value Optimization"): with A = softmax(s Q Kc^T)
  * fixed, Vc = (A^T A + lambda I)^-1 A^T Y, by Cholesky.  A problem whose Gram
  * matrix is not positive definite gets KVS_ST_NOT_PD in status[b] (OR-ed in)
- * and keeps its previous Vc.
+ * and keeps its previous Vc; so does a problem whose solution is not finite,
+ * which gets KVS_ST_NONFINITE (a Gram matrix with a non-finite entry counts
+ * as not positive definite).
  * The factorisation forks part of its work onto one internal high-priority
  * stream (created once per host thread and device) through events recorded on
  * `stream`, and joins it back to `stream` before returning, so the call stays
@@ -197,7 +235,9 @@ int kvs_lbfgs_reset(const kvs_batch *batch, const kvs_schedule *sched, const flo
  * backtracking Armijo search (first trial 1, or min(1, 1/||g||) with empty
  * history; factor sched->backtrack; at most sched->max_bt trials), history
  * update when s^T y > 1e-10 y^T y.  Kc is updated in place; a failed search
- * leaves Kc unchanged, clears the history and sets KVS_ST_LS_FAIL.
+ * leaves Kc unchanged, clears the history and sets KVS_ST_LS_FAIL.  A loss
+ * that evaluates to inf or NaN (at a trial point, or at the point the last
+ * reset started from) sets KVS_ST_NONFINITE; such a trial is rejected.
  * f_out (nullable) [B] receives the loss after the step. */
 int kvs_lbfgs_step(const kvs_batch *batch, const kvs_schedule *sched, const float *Q,
                    const float *Y, const float *lse, const float *Vc, float *Kc,

@@ -18,7 +18,7 @@ import torch
 __all__ = [
     "KvsError", "KvsBatch", "Schedule", "QuerySpec", "LIB_PATH", "lib",
     "ST_NONFINITE", "ST_NOT_PD", "ST_LS_FAIL",
-    "kvs_version", "kvs_launch_count", "kvs_workspace_bytes", "kvs_lbfgs_state_bytes", "kvs_build_queries",
+    "kvs_version", "kvs_launch_count", "kvs_set_wait_limit", "kvs_workspace_bytes", "kvs_lbfgs_state_bytes", "kvs_lbfgs_state_layout", "kvs_build_queries",
     "kvs_targets", "kvs_init_topk", "kvs_loss_grad", "kvs_loss_grad_static", "kvs_fit_values", "kvs_lbfgs_reset",
     "kvs_lbfgs_step", "kvs_compress_batch", "kvs_pilot_allocate", "kvs_adam_step",
     "alloc_workspace", "alloc_state",
@@ -52,13 +52,21 @@ class _QSpec(ctypes.Structure):
                 ("N", _i32), ("rope_base", _f32)]
 
 
+class _Layout(ctypes.Structure):
+    _fields_ = [(n, ctypes.c_uint64) for n in ("scalars", "scalar_bytes", "off_f", "off_count",
+                                                "off_head", "x", "g", "dir", "ring_s", "ring_y",
+                                                "ring_stride")] + [("slots", _i32)]
+
+
 _BP, _SP, _QP = ctypes.POINTER(_Batch), ctypes.POINTER(_Sched), ctypes.POINTER(_QSpec)
 _SIGS = {
     "kvs_version": (ctypes.c_char_p, []),
     "kvs_last_cuda_error": (ctypes.c_char_p, []),
     "kvs_launch_count": (ctypes.c_uint64, []),
+    "kvs_set_wait_limit": (ctypes.c_int, [_i64]),
     "kvs_workspace_bytes": (_sz, [_BP, _SP]),
     "kvs_lbfgs_state_bytes": (_sz, [_BP, _i32]),
+    "kvs_lbfgs_state_layout": (ctypes.c_int, [_BP, _i32, ctypes.POINTER(_Layout)]),
     "kvs_build_queries": (ctypes.c_int, [_QP, _vp, _vp, _vp, _vp, _vp]),
     "kvs_targets": (ctypes.c_int, [_BP, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _sz, _vp]),
     "kvs_init_topk": (ctypes.c_int, [_BP, _vp, _vp, _vp, _vp, _vp]),
@@ -211,6 +219,12 @@ def kvs_launch_count() -> int:
     return int(lib.kvs_launch_count())
 
 
+def kvs_set_wait_limit(cycles: int) -> None:
+    """Bound on the tensor-core kernels' pipeline waits, in SM cycles (0: the default);
+    for tests of the timeout path."""
+    _check("kvs_set_wait_limit", lib.kvs_set_wait_limit(int(cycles)))
+
+
 def kvs_workspace_bytes(batch: KvsBatch, sched: Optional[Schedule] = None) -> int:
     s = None if sched is None else ctypes.byref(sched.struct())
     return int(lib.kvs_workspace_bytes(batch.ref, s))
@@ -218,6 +232,14 @@ def kvs_workspace_bytes(batch: KvsBatch, sched: Optional[Schedule] = None) -> in
 
 def kvs_lbfgs_state_bytes(batch: KvsBatch, history: int) -> int:
     return int(lib.kvs_lbfgs_state_bytes(batch.ref, history))
+
+
+def kvs_lbfgs_state_layout(batch: KvsBatch, history: int) -> dict:
+    """Byte offsets of the L-BFGS state fields inside a state buffer (see the header)."""
+    out = _Layout()
+    _check("kvs_lbfgs_state_layout", lib.kvs_lbfgs_state_layout(batch.ref, int(history),
+                                                                ctypes.byref(out)))
+    return {n: int(getattr(out, n)) for n, _ in _Layout._fields_}
 
 
 def alloc_workspace(batch: KvsBatch, sched: Optional[Schedule] = None, device="cuda"):

@@ -18,8 +18,14 @@ namespace kvs {
 
 static thread_local char g_err[256] = "no error";
 static std::atomic<uint64_t> g_launches{0};
+static std::atomic<long long> g_wait_limit{0};  // 0: the default limit
 
 void count_launch() { g_launches.fetch_add(1, std::memory_order_relaxed); }
+
+long long wait_limit() {
+  const long long v = g_wait_limit.load(std::memory_order_relaxed);
+  return v > 0 ? v : tc_wait_default();
+}
 
 cudaError_t set_smem_once_impl(const void *kern, int bytes) {
   static std::mutex mu;
@@ -170,6 +176,30 @@ static int fold_err(const Batch &Bt, const Work &w, int32_t *status) {
   if (!status) return KVS_OK;
   k_fold_err<<<(Bt.g.B + 127) / 128, 128, 0, Bt.st>>>(w.err, status, Bt.g.B);
   KVS_LAUNCH_CHECK("k_fold_err");
+  return KVS_OK;
+}
+
+// For the calls without a status array: when a kernel of the call gave up
+// waiting, every output element becomes NaN, so partial results cannot pass
+// for finite ones.
+struct NanOut {
+  float *p[3];
+  int64_t n[3];
+};
+
+__global__ void k_nan_if_err(const int *err, NanOut o) {
+  if (!*err) return;
+  for (int k = 0; k < 3; ++k)
+    for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < o.n[k];
+         i += (int64_t)gridDim.x * blockDim.x)
+      o.p[k][i] = __int_as_float(0x7fc00000);
+}
+
+static int nan_if_err(const Batch &Bt, const Work &w, float *p0, int64_t n0, float *p1, int64_t n1,
+                      float *p2, int64_t n2) {
+  NanOut o{{p0, p1, p2}, {p0 ? n0 : 0, p1 ? n1 : 0, p2 ? n2 : 0}};
+  k_nan_if_err<<<64, 256, 0, Bt.st>>>(w.err, o);
+  KVS_LAUNCH_CHECK("k_nan_if_err");
   return KVS_OK;
 }
 
@@ -335,6 +365,12 @@ const char *kvs_last_cuda_error(void) { return g_err; }
 
 uint64_t kvs_launch_count(void) { return g_launches.load(std::memory_order_relaxed); }
 
+int kvs_set_wait_limit(int64_t cycles) {
+  if (cycles < 0) return KVS_EINVAL;
+  g_wait_limit.store((long long)cycles, std::memory_order_relaxed);
+  return KVS_OK;
+}
+
 size_t kvs_workspace_bytes(const kvs_batch *batch, const kvs_schedule *) {
   HostGeom g;
   if (geom_from_batch(batch, &g, false)) return 0;
@@ -347,6 +383,29 @@ size_t kvs_lbfgs_state_bytes(const kvs_batch *batch, int32_t history) {
   if (history < 1 || history > 15 || geom_from_batch(batch, &g, true)) return 0;
   State s;
   return carve_state(g, history, nullptr, &s);
+}
+
+int kvs_lbfgs_state_layout(const kvs_batch *batch, int32_t history, kvs_lbfgs_layout *out) {
+  HostGeom g;
+  if (!out || history < 1 || history > 15 || geom_from_batch(batch, &g, true)) return KVS_EINVAL;
+  State s;
+  carve_state(g, history, reinterpret_cast<void *>(uintptr_t{1} << 40), &s);
+  const char *base = reinterpret_cast<const char *>(uintptr_t{1} << 40);
+  auto at = [&](const void *p) { return (uint64_t)(static_cast<const char *>(p) - base); };
+  *out = kvs_lbfgs_layout{};
+  out->scalars = at(s.sc);
+  out->scalar_bytes = sizeof(LbfgsScal);
+  out->off_f = offsetof(LbfgsScal, f);
+  out->off_count = offsetof(LbfgsScal, count);
+  out->off_head = offsetof(LbfgsScal, head);
+  out->x = at(s.x);
+  out->g = at(s.g);
+  out->dir = at(s.dir);
+  out->ring_s = at(s.ring_s);
+  out->ring_y = at(s.ring_y);
+  out->ring_stride = (uint64_t)(g.sum_c * g.d) * sizeof(float);
+  out->slots = history + 1;
+  return KVS_OK;
 }
 
 int kvs_build_queries(const kvs_query_spec *sp, const float *q_retain, const float *q_ctx,
@@ -372,7 +431,9 @@ int kvs_targets(const kvs_batch *batch, const float *Q, const float *Kz, const f
       (importance && !ok_ptr(importance)))
     return KVS_EINVAL;
   if ((rc = begin(Bt, w))) return rc;
-  return launch_targets(Bt, Q, Kz, Vz, Y, lse, importance, w);
+  if ((rc = launch_targets(Bt, Q, Kz, Vz, Y, lse, importance, w))) return rc;
+  const HostGeom &g = Bt.g;
+  return nan_if_err(Bt, w, Y, g.sum_q * g.d, lse, g.sum_q, importance, g.sum_z);
 }
 
 int kvs_init_topk(const kvs_batch *batch, const float *importance, const float *Kz,
@@ -400,9 +461,11 @@ int kvs_loss_grad(const kvs_batch *batch, const float *Q, const float *Kc, const
       (parts && !ok_ptr(parts)) || (dKc && !ok_ptr(dKc)))
     return KVS_EINVAL;
   if ((rc = begin(Bt, w))) return rc;
-  rc = launch_forward(Bt, Q, Kc, Vc, Y, lse, w_out, w_lse, loss, parts, ALL, false, w);
-  if (rc || !dKc) return rc;
-  return launch_backward(Bt, dKc, ALL, w);
+  if ((rc = launch_forward(Bt, Q, Kc, Vc, Y, lse, w_out, w_lse, loss, parts, ALL, false, w)))
+    return rc;
+  if (dKc && (rc = launch_backward(Bt, dKc, ALL, w))) return rc;
+  const HostGeom &g = Bt.g;
+  return nan_if_err(Bt, w, loss, g.B, parts, 2 * (int64_t)g.B, dKc, g.sum_c * g.d);
 }
 
 int kvs_fit_values(const kvs_batch *batch, const float *Q, const float *Kc, const float *Y,

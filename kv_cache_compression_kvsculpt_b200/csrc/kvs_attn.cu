@@ -13,6 +13,7 @@
 #include <math.h>
 
 #include <algorithm>
+#include <atomic>
 #include <mutex>
 #include <unordered_map>
 
@@ -153,13 +154,18 @@ __global__ void k_loss_reduce(const float *partials, int tiles, const int64_t *q
 
 int max_qtiles(const HostGeom &g) { return (g.max_q + 127) / 128; }
 
+// Multiprocessor count of the current device, cached per device (several host
+// threads may ask at once: relaxed atomics, the value is the same for all).
 int sm_count() {
-  static int n[64] = {0};
+  static std::atomic<int> n[64];
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 148;
-  if (!n[dev] && cudaDeviceGetAttribute(&n[dev], cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
-    n[dev] = 148;
-  return n[dev];
+  int v = n[dev].load(std::memory_order_relaxed);
+  if (v > 0) return v;
+  if (cudaDeviceGetAttribute(&v, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || v <= 0)
+    v = 148;
+  n[dev].store(v, std::memory_order_relaxed);
+  return v;
 }
 
 // Query-range splits of the key-gradient kernel: the one whose last wave of
@@ -232,6 +238,7 @@ int targets_d(const Batch &Bt, const float *Q, const float *Kz, const float *Vz,
   a.y_lo = w.yl;
   a.lse_out = lse;
   a.err = w.err;
+  a.wait = wait_limit();
   if ((rc = launch_fwd_tc<D, FWD_TARGETS>(fm, a, max_qtiles(g), g.B, Bt.st))) return rc;
   if (!imp) return KVS_OK;
   BwdMaps bm;
@@ -249,6 +256,7 @@ int targets_d(const Batch &Bt, const float *Q, const float *Kz, const float *Vz,
   ba.lse = lse;
   ba.imp = imp;
   ba.err = w.err;
+  ba.wait = wait_limit();
   ba.nsplit = 1;
   return launch_bwd_tc<D, BWD_COLSUM>(bm, ba, (g.max_z + 127) / 128, g.B, Bt.st);
 }
@@ -295,6 +303,7 @@ int forward_d(const Batch &Bt, const float *Q, const float *Kc, const float *Vc,
   a.w_out = w_out;
   a.w_lse = w_lse;
   a.err = w.err;
+  a.wait = wait_limit();
   if ((rc = launch_fwd_tc<D, FWD_LOSS>(fm, a, max_qtiles(g), g.B, Bt.st))) return rc;
   if (!reduce) return KVS_OK;
   k_loss_reduce<<<(g.B + 127) / 128, 128, 0, Bt.st>>>(w.partials, max_qtiles(g), Bt.b->q_off, D,
@@ -325,6 +334,7 @@ int backward_d(const Batch &Bt, float *dKc, Filter flt, const Work &w) {
   ba.v_lo = w.vl;
   ba.dk = dKc;
   ba.err = w.err;
+  ba.wait = wait_limit();
   ba.nsplit = 1;
   const int ktiles = (g.max_c + 127) / 128;
   const int ns = bwd_split(ktiles * g.B, (g.max_q + 63) / 64);
@@ -368,6 +378,7 @@ int fit_d(const Batch &Bt, const float *Q, const float *Kc, const float *Y, floa
   a.scale = 1.f / sqrtf((float)D);
   a.lse_out = w.lse_h;
   a.err = w.err;
+  a.wait = wait_limit();
   if ((rc = launch_fwd_tc<D, FWD_STATS>(fm, a, max_qtiles(g), g.B, Bt.st))) return rc;
   a.flt = Filter{nullptr, 0, 0};
   k_pad_offsets<<<1, 1, 0, Bt.st>>>(Bt.b->q_off, g.B, w.a_pad_off);
@@ -393,6 +404,7 @@ int fit_d(const Batch &Bt, const float *Q, const float *Kc, const float *Y, floa
   ga.ldc = g.ld_g;
   ga.diag = lam;
   ga.err = w.err;
+  ga.wait = wait_limit();
   const int tm = (g.max_c + 127) / 128;
   if ((rc = launch_gemm3_tc(gm, ga, tm, 1, g.B, Bt.st))) return rc;
   if ((rc = make_map_bf16(&gm.bh, w.yh, g.sum_q, D, 64)) ||

@@ -131,7 +131,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       const int st = i % C::NS;
       if (i >= C::NS) {
         const bool w = __all_sync(0xffffffffu,
-                                  mbar_wait(&bars.q_empty[st], ((i / C::NS) - 1) & 1, abort));
+                                  mbar_wait(&bars.q_empty[st], ((i / C::NS) - 1) & 1, abort, a.wait));
         if (!w) {
           *abort = 1;
           break;
@@ -169,13 +169,13 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     if (lane == 0) {
       const uint32_t id_s = idesc_bf16(BK, BQ, false, false);
       const uint32_t id_dk = idesc_bf16(BK, D, false, true);
-      bool ok = mbar_wait(&bars.k_full, 0, abort);
+      bool ok = mbar_wait(&bars.k_full, 0, abort, a.wait);
       fence_after_sync();
       const uint64_t kh0 = sdesc(smem_u32(sm), 16, 1024), kl0 = sdesc_add(kh0, C::K_BYTES);
       const uint32_t tv_hi = tmem + C::COL_V, tv_lo = tmem + C::COL_V + D / 2;
       auto issue_dk = [&](int i) -> bool {
         const int db = i & 1;
-        if (!mbar_wait(&bars.ds_full[db], (i >> 1) & 1, abort)) return false;
+        if (!mbar_wait(&bars.ds_full[db], (i >> 1) & 1, abort, a.wait)) return false;
         fence_after_sync();
         const uint64_t qh0 = sdesc(smem_u32(sm + C::OFF_ST + (i % C::NS) * C::STAGE), BQ * 128,
                                    1024);
@@ -194,8 +194,8 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       };
       for (int i = 0; ok && i < nqt; ++i) {
         const int st = i % C::NS, sb = i & 1;
-        if (!mbar_wait(&bars.q_full[st], (i / C::NS) & 1, abort)) { ok = false; break; }
-        if (i >= 2 && !mbar_wait(&bars.sd_free[sb], ((i >> 1) - 1) & 1, abort)) { ok = false; break; }
+        if (!mbar_wait(&bars.q_full[st], (i / C::NS) & 1, abort, a.wait)) { ok = false; break; }
+        if (i >= 2 && !mbar_wait(&bars.sd_free[sb], ((i >> 1) - 1) & 1, abort, a.wait)) { ok = false; break; }
         fence_after_sync();
         const uint64_t qh0 = sdesc(smem_u32(sm + C::OFF_ST + st * C::STAGE), 16, 1024);
         const uint64_t ql0 = sdesc_add(qh0, C::Q_BYTES), gd0 = sdesc_add(qh0, 2 * C::Q_BYTES);
@@ -213,7 +213,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
           // V reaches tensor memory through the row threads: the first score product
           // runs while they store it
           if (i == 0) {
-            if (!mbar_wait(&bars.v_full, 0, abort)) { ok = false; break; }
+            if (!mbar_wait(&bars.v_full, 0, abort, a.wait)) { ok = false; break; }
             fence_after_sync();
           }
 #pragma unroll
@@ -267,9 +267,9 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     bool ok = true;
     for (int i = wg; i < nqt; i += 2) {
       const int sb = i & 1, st = i % C::NS;
-      ok = __all_sync(0xffffffffu, mbar_wait(&bars.sd_full[sb], (i >> 1) & 1, abort));
+      ok = __all_sync(0xffffffffu, mbar_wait(&bars.sd_full[sb], (i >> 1) & 1, abort, a.wait));
       // the tile's l and delta were staged by the producer lanes: acquire them directly
-      ok = ok && __all_sync(0xffffffffu, mbar_wait(&bars.q_full[st], (i / C::NS) & 1, abort));
+      ok = ok && __all_sync(0xffffffffu, mbar_wait(&bars.q_full[st], (i / C::NS) & 1, abort, a.wait));
       if (!ok) break;
       fence_after_sync();
       float s[BQ];
@@ -314,7 +314,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     }
     if (!ok) *abort = 1;
     if (C::DK) {
-      if (!mbar_wait(&bars.done, 0, abort)) *abort = 1;
+      if (!mbar_wait(&bars.done, 0, abort, a.wait)) *abort = 1;
       fence_after_sync();
 #pragma unroll 1
       for (int c0 = wg * (D / 2); c0 < (wg + 1) * (D / 2); c0 += 32) {

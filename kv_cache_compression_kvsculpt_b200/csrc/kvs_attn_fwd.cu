@@ -159,7 +159,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       int k_issued = 0, v_issued = 0;
       auto load_k = [&](int j) -> bool {
         const int st = j % C::NSK;
-        if (j >= C::NSK && !mbar_wait(&bars.k_empty[st], ((j / C::NSK) - 1) & 1, abort))
+        if (j >= C::NSK && !mbar_wait(&bars.k_empty[st], ((j / C::NSK) - 1) & 1, abort, a.wait))
           return false;
         k_issued = j + 1;
         unsigned char *base = sm + C::OFF_K + st * 2 * C::T_BYTES;
@@ -173,7 +173,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       };
       auto load_v = [&](int j) -> bool {
         const int st = j % C::NSVI;
-        if (j >= C::NSVI && !mbar_wait(&bars.v_empty[st], ((j / C::NSVI) - 1) & 1, abort))
+        if (j >= C::NSVI && !mbar_wait(&bars.v_empty[st], ((j / C::NSVI) - 1) & 1, abort, a.wait))
           return false;
         v_issued = j + 1;
         unsigned char *base = sm + C::OFF_V + st * 2 * C::T_BYTES;
@@ -212,13 +212,13 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       const uint32_t id_s128 = idesc_bf16(BM, BN, false, false);
       const uint32_t id_s64 = idesc_bf16(BM, 64, false, false);
       const uint32_t id_pv = idesc_bf16(BM, 2 * D, false, true);  // N = [V_hi | V_lo]
-      bool ok = mbar_wait(&bars.q_full, 0, abort);
+      bool ok = mbar_wait(&bars.q_full, 0, abort, a.wait);
       fence_after_sync();
       const uint64_t qh0 = sdesc(smem_u32(sm), 16, 1024), ql0 = sdesc_add(qh0, C::T_BYTES);
       auto issue_pv = [&](int i) -> bool {
         const int pb = i & 1;
-        if (!mbar_wait(&bars.p_full[pb], (i >> 1) & 1, abort)) return false;
-        if (!mbar_wait(&bars.v_full[i % C::NSVI], (i / C::NSVI) & 1, abort)) return false;
+        if (!mbar_wait(&bars.p_full[pb], (i >> 1) & 1, abort, a.wait)) return false;
+        if (!mbar_wait(&bars.v_full[i % C::NSVI], (i / C::NSVI) & 1, abort, a.wait)) return false;
         fence_after_sync();
         // V_hi and V_lo boxes sit back to back with one stride: one N = 2d operand
         const uint64_t v0 = sdesc(smem_u32(sm + C::OFF_V + (i % C::NSVI) * 2 * C::T_BYTES),
@@ -237,8 +237,8 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       };
       for (int j = 0; ok && j < ntiles; ++j) {
         const int st = j % C::NSK, sb = j & 1;
-        if (!mbar_wait(&bars.k_full[st], (j / C::NSK) & 1, abort)) { ok = false; break; }
-        if (j >= 2 && !mbar_wait(&bars.s_free[sb], ((j >> 1) - 1) & 1, abort)) { ok = false; break; }
+        if (!mbar_wait(&bars.k_full[st], (j / C::NSK) & 1, abort, a.wait)) { ok = false; break; }
+        if (j >= 2 && !mbar_wait(&bars.s_free[sb], ((j >> 1) - 1) & 1, abort, a.wait)) { ok = false; break; }
         fence_after_sync();
         // a last tile with at most 64 keys takes the narrower product
         const uint32_t id_s = (nk - j * BN) > 64 ? id_s128 : id_s64;
@@ -277,7 +277,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     bool ok = true;
     for (int j = 0; j < ntiles; ++j) {
       const int sb = j & 1;
-      ok = ok && __all_sync(0xffffffffu, mbar_wait(&bars.s_full[sb], (j >> 1) & 1, abort));
+      ok = ok && __all_sync(0xffffffffu, mbar_wait(&bars.s_full[sb], (j >> 1) & 1, abort, a.wait));
       if (MODE == FWD_WRITE_A && !ok) break;  // no barrier below in this mode
       float s[HB];
       if (ok) {
@@ -369,7 +369,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
           // rows' rescale decisions are the same in both warpgroups; each scales
           // one output half.
           const int pj = j - 1;
-          ok = __all_sync(0xffffffffu, mbar_wait(&bars.s_free[pj & 1], (pj >> 1) & 1, abort));
+          ok = __all_sync(0xffffffffu, mbar_wait(&bars.s_free[pj & 1], (pj >> 1) & 1, abort, a.wait));
           if (ok) {  // a failed wait ends the loop at the next tile's row barrier
             fence_after_sync();
 #pragma unroll 1
@@ -395,7 +395,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       lsum = bars.ls[0][row] + bars.ls[1][row];
       const float lse = (mref + log2f(lsum)) * 0.6931471805599453f;
       if (C::PV) {
-        if (!mbar_wait(&bars.o_done, 0, abort)) *abort = 1;
+        if (!mbar_wait(&bars.o_done, 0, abort, a.wait)) *abort = 1;
         fence_after_sync();
       }
       const float inv = 1.f / lsum;

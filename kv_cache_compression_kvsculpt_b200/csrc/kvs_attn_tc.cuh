@@ -48,6 +48,7 @@ struct FwdArgs {
   int64_t ld_a;
   const int64_t *a_pad_off;    // [B+1] padded query-row offsets of the A buffer
   int *err;               // timeout flag
+  long long wait;         // cycles a pipeline wait may spin (wait_limit())
 };
 
 struct BwdMaps {
@@ -66,6 +67,7 @@ struct BwdArgs {
   float *dk;              // [sum_k, d] (DK): dL/dK, or nsplit partial sums dk_stride apart
   float *imp;             // [sum_k] (COLSUM): column sums of probabilities
   int *err;
+  long long wait;
   int nsplit;             // query tiles of a problem split over this many CTAs (COLSUM: 1)
   int64_t dk_stride;      // floats between the partial sums of two splits
 };
@@ -84,6 +86,7 @@ struct GemmArgs3 {
   float diag;                // added on the diagonal (Gram: lambda)
   int b_col_shift;           // Gram: 0 ; R: 0 (B columns start at 0)
   int *err;
+  long long wait;
 };
 
 template <int D, int MODE>

@@ -12,6 +12,11 @@ namespace kvs {
 void set_cuda_error(cudaError_t e, const char *where);
 // Counts kernel launches (kvs_launch_count); called once per launch.
 void count_launch();
+// Cycles a kernel's pipeline wait may spin before the kernel gives up
+// (kvs_set_wait_limit; about 2 s by default).
+long long wait_limit();
+// The default of wait_limit() (the tensor-core kernels' kWaitCycles).
+constexpr long long tc_wait_default() { return 4000000000LL; }
 
 #define KVS_CUDA_TRY(expr)                                     \
   do {                                                         \

@@ -122,7 +122,7 @@ __global__ void __launch_bounds__(192, 1)
       int issued = 0;
       for (int i = 0; i < nkt; ++i) {
         const int st = i % NS;
-        if (i >= NS && !mbar_wait(&bars.empty[st], ((i / NS) - 1) & 1, abort)) {
+        if (i >= NS && !mbar_wait(&bars.empty[st], ((i / NS) - 1) & 1, abort, a.wait)) {
           *abort = 1;
           break;
         }
@@ -150,7 +150,7 @@ __global__ void __launch_bounds__(192, 1)
       bool ok = true;
       for (int i = 0; i < nkt; ++i) {
         const int st = i % NS;
-        if (!mbar_wait(&bars.full[st], (i / NS) & 1, abort)) { ok = false; break; }
+        if (!mbar_wait(&bars.full[st], (i / NS) & 1, abort, a.wait)) { ok = false; break; }
         fence_after_sync();
         const uint64_t d0 = sdesc(smem_u32(sm + st * C::STAGE), TKQ * 128, 1024);
 #pragma unroll
@@ -177,7 +177,7 @@ __global__ void __launch_bounds__(192, 1)
   } else {
     const int row = tid;
     const int gi = ti * TM + row;
-    if (!mbar_wait(&bars.done, 0, abort)) *abort = 1;
+    if (!mbar_wait(&bars.done, 0, abort, a.wait)) *abort = 1;
     fence_after_sync();
     const uint32_t lane_base = (uint32_t)(warp * 32) << 16;
     float *crow = a.c + (m_begin + gi) * a.ldc;

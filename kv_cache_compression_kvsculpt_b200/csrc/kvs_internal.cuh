@@ -23,7 +23,8 @@ struct LbfgsScal {
   int phase;      // Phase
   int trials;     // trials of the current search
   int lse_stale;  // 1: the workspace l_hat is not that of the accepted keys (failed search)
-  int pad[2];
+  int nonfinite;  // 1: a loss or gradient evaluated since the last report was inf / NaN
+  int pad;
 };
 
 // Scratch buffers carved from the caller's workspace.

@@ -256,7 +256,7 @@ __global__ void __launch_bounds__(PT) k_pairs(PairArgs a) {
         count = min(count0 + 1, a.h);
       }
       s.f = s.ft;
-      if (!isfinite(s.f) && a.status) a.status[b] |= KVS_ST_NONFINITE;
+      if (!isfinite(s.f) || !isfinite(tot[4])) s.nonfinite = 1;
     } else if (phase == PH_FAIL) {
       count = 0;
       head = 0;
@@ -264,12 +264,16 @@ __global__ void __launch_bounds__(PT) k_pairs(PairArgs a) {
     }
     s.phase = PH_IDLE;
     s.lse_stale = phase == PH_FAIL;  // the last loss forward ran at a rejected trial
+    if (s.nonfinite && a.status) a.status[b] |= KVS_ST_NONFINITE;
+    s.nonfinite = 0;
     if (a.f_out) a.f_out[b] = s.f;
   } else {
     s.f = a.f[b];
     s.phase = PH_IDLE;
     s.trials = 0;
     s.lse_stale = 0;
+    // reported by the next step (the reset itself has no status array)
+    s.nonfinite = !isfinite(s.f) || !isfinite(tot[4]);
     if (a.clear) {
       count = 0;
       head = 0;
@@ -387,6 +391,7 @@ __global__ void __launch_bounds__(256) k_armijo(LbfgsScal *sc, int B, const floa
     }
     const float f = (float)(w_out * (so / ((double)nq * d)) + w_lse * (sl / (double)nq));
     s.trials += 1;
+    if (!isfinite(f)) s.nonfinite = 1;
     if (isfinite(f) && f <= s.f + c1 * s.t * s.gtd) {
       s.ft = f;
       s.phase = PH_ACCEPT;

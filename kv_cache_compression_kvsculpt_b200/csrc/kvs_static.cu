@@ -12,6 +12,8 @@
 // The array is KVS_STATIC_WS_BYTES bytes of device memory on every GPU that
 // loads the library, held until the process exits.  Batches whose workspace
 // (kvs_workspace_bytes) exceeds it are rejected with KVS_EWORKSPACE.
+#include <cuda.h>
+
 #include <mutex>
 
 #include "kvs_common.cuh"
@@ -23,12 +25,33 @@ static __device__ __align__(256) unsigned char g_static_ws[KVS_STATIC_WS_BYTES];
 
 namespace {
 
-std::mutex g_static_mu;
-void *g_static_ptr[KVS_STATIC_MAX_DEVICES];
+typedef CUresult (*CtxGetCurrentFn)(CUcontext *);
 
-// Device address of g_static_ws on the current device.  The host-side name
-// of the array is only a handle: the address must come from
-// cudaGetSymbolAddress, once per device, with that device current.
+std::mutex g_static_mu;
+struct Cached {
+  CUcontext ctx;  // the context the address belongs to
+  void *ptr;
+};
+Cached g_static[KVS_STATIC_MAX_DEVICES];
+
+CtxGetCurrentFn ctx_get_current() {
+  static CtxGetCurrentFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    cudaDriverEntryPointQueryResult q;
+    void *p = nullptr;
+    if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<CtxGetCurrentFn>(p);
+  });
+  return fn;
+}
+
+// Device address of g_static_ws in the current device's current context.  The
+// host-side name of the array is only a handle: the address must come from
+// cudaGetSymbolAddress with that device current.  It is looked up once per
+// device and again whenever the current context is not the one it was looked
+// up in (after cudaDeviceReset, or under another driver context).
 int static_workspace(void **out) {
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
@@ -37,17 +60,25 @@ int static_workspace(void **out) {
     return KVS_ECUDA;
   }
   if (dev < 0 || dev >= KVS_STATIC_MAX_DEVICES) return KVS_ENOTSUP;
+  CtxGetCurrentFn get = ctx_get_current();
+  if (!get) return KVS_ECUDA;
+  // null before the runtime's first call on this thread has made a context current
+  CUcontext ctx = nullptr;
+  if (get(&ctx) != CUDA_SUCCESS) return KVS_ECUDA;
   std::lock_guard<std::mutex> lock(g_static_mu);
-  if (!g_static_ptr[dev]) {
+  Cached &c = g_static[dev];
+  if (!c.ptr || !ctx || c.ctx != ctx) {
     void *p = nullptr;
-    e = cudaGetSymbolAddress(&p, g_static_ws);
+    e = cudaGetSymbolAddress(&p, g_static_ws);  // makes the device's context current
     if (e != cudaSuccess) {
       kvs::set_cuda_error(e, "cudaGetSymbolAddress(g_static_ws)");
       return KVS_ECUDA;
     }
-    g_static_ptr[dev] = p;
+    if (get(&ctx) != CUDA_SUCCESS || !ctx) return KVS_ECUDA;
+    c.ctx = ctx;
+    c.ptr = p;
   }
-  *out = g_static_ptr[dev];
+  *out = c.ptr;
   return KVS_OK;
 }
 

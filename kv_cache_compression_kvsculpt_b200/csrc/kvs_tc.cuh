@@ -12,13 +12,18 @@
 #include <cuda_bf16.h>
 #include <stdint.h>
 
+#include "kvs_common.cuh"
+
 namespace kvs {
 namespace tc {
 
 // Longest time any wait may spin before the kernel gives up (SM clock cycles,
 // about 2 s at 1.9 GHz).  A timed-out wait sets an error flag; the caller
-// then unwinds without touching the data it waited for.
-constexpr long long kWaitCycles = 4000000000LL;
+// then unwinds without touching the data it waited for.  The pipeline waits
+// (those that also watch the CTA's abort flag) take their limit from the
+// kernel's arguments, which default to this value; the waits of the unwinding
+// itself (copies and MMAs already issued) always use it.
+constexpr long long kWaitCycles = tc_wait_default();
 
 __device__ __forceinline__ uint32_t smem_u32(const void *p) {
   return (uint32_t)__cvta_generic_to_shared(p);
@@ -57,14 +62,15 @@ __device__ __forceinline__ bool mbar_test(uint64_t *bar, uint32_t parity) {
   return done != 0;
 }
 
-// Wait until the phase of parity `parity` completes; false after kWaitCycles
-// or as soon as *abort is set by another thread of the CTA.
+// Wait until the phase of parity `parity` completes; false after `limit`
+// cycles or as soon as *abort is set by another thread of the CTA.
 __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity,
-                                          volatile int *abort = nullptr) {
+                                          volatile int *abort = nullptr,
+                                          long long limit = kWaitCycles) {
   const long long t0 = clock64();
   while (!mbar_test(bar, parity)) {
     if (abort && *abort) return false;
-    if (clock64() - t0 > kWaitCycles) return false;
+    if (clock64() - t0 > limit) return false;
   }
   return true;
 }
@@ -293,105 +299,6 @@ __device__ __forceinline__ float ex2(float x) {
   float y;
   asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
   return y;
-}
-
-// ------------------------------------------------------------- CTA pairs
-// A cluster of two CTAs runs one tcgen05 product of M = 256 (cta_group::2): each
-// CTA holds 128 rows of A and of the accumulator, and half of B's N extent
-// (columns n < N/2 from CTA 0's operand rows 0 .., the rest from CTA 1's rows
-// 0 ..).  One thread of CTA 0 issues; commits signal both CTAs.
-
-__device__ __forceinline__ uint32_t cta_rank() {
-  uint32_t r;
-  asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
-  return r;
-}
-
-__device__ __forceinline__ void cluster_sync() {
-  asm volatile(
-      "barrier.cluster.arrive.release.aligned;\n\t"
-      "barrier.cluster.wait.acquire.aligned;" ::: "memory");
-}
-
-// shared::cluster address of the variable at `p` in CTA `rank` of the cluster
-__device__ __forceinline__ uint32_t peer_addr(const void *p, uint32_t rank) {
-  uint32_t a;
-  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(a) : "r"(smem_u32(p)), "r"(rank));
-  return a;
-}
-
-// arrive (release, cluster scope) on an mbarrier given by its shared::cluster address
-__device__ __forceinline__ void mbar_arrive_cluster(uint32_t addr) {
-  asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(addr)
-               : "memory");
-}
-
-__device__ __forceinline__ bool mbar_test_cluster(uint64_t *bar, uint32_t parity) {
-  uint32_t done;
-  asm volatile(
-      "{\n\t.reg .pred p;\n\t"
-      "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n\t"
-      "selp.u32 %0, 1, 0, p;\n\t}"
-      : "=r"(done)
-      : "r"(smem_u32(bar)), "r"(parity)
-      : "memory");
-  return done != 0;
-}
-
-// mbar_wait for barriers that the peer CTA arrives on (cluster-scope acquire)
-__device__ __forceinline__ bool mbar_wait_cluster(uint64_t *bar, uint32_t parity,
-                                                  volatile int *abort = nullptr) {
-  const long long t0 = clock64();
-  while (!mbar_test_cluster(bar, parity)) {
-    if (abort && *abort) return false;
-    if (clock64() - t0 > kWaitCycles) return false;
-  }
-  return true;
-}
-
-// Tensor memory of both CTAs of the pair; one warp of each CTA executes these.
-__device__ __forceinline__ void tmem_alloc_pair(uint32_t *slot, uint32_t ncols) {
-  asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
-                   smem_u32(slot)),
-               "r"(ncols)
-               : "memory");
-  asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;" ::: "memory");
-}
-
-__device__ __forceinline__ void tmem_dealloc_pair(uint32_t taddr, uint32_t ncols) {
-  asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols)
-               : "memory");
-}
-
-// D (+)= A[smem] * B[smem] over the pair (M = 256).
-__device__ __forceinline__ void mma_pair(uint32_t d_tmem, uint64_t a, uint64_t b, uint32_t idesc,
-                                         uint32_t accumulate) {
-  asm volatile(
-      "{\n\t.reg .pred p;\n\t"
-      "setp.ne.b32 p, %4, 0;\n\t"
-      "tcgen05.mma.cta_group::2.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
-      "l"(a), "l"(b), "r"(idesc), "r"(accumulate)
-      : "memory");
-}
-
-// D (+)= A[tmem of each CTA] * B[smem] over the pair (M = 256).
-__device__ __forceinline__ void mma_pair_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t b,
-                                            uint32_t idesc, uint32_t accumulate) {
-  asm volatile(
-      "{\n\t.reg .pred p;\n\t"
-      "setp.ne.b32 p, %4, 0;\n\t"
-      "tcgen05.mma.cta_group::2.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
-      "r"(a_tmem), "l"(b), "r"(idesc), "r"(accumulate)
-      : "memory");
-}
-
-// Arrive once on `bar` in both CTAs when the pair's MMAs issued so far have completed.
-__device__ __forceinline__ void mma_commit_pair(uint64_t *bar) {
-  asm volatile(
-      "tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64"
-      " [%0], %1;" ::"r"(smem_u32(bar)),
-      "h"((uint16_t)3)
-      : "memory");
 }
 
 // Byte offset of 16-byte chunk `chunk` of row `row` in a 128-byte-swizzled tile.

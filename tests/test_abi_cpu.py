@@ -118,3 +118,23 @@ def test_pilot_allocate_rejects_infeasible(K):
         K.kvs_pilot_allocate([1.0, 2.0], 100, 16, [40, 40])
     with pytest.raises(K.KvsError):
         K.kvs_pilot_allocate([1.0, 2.0], 10, 16, [40, 40])
+
+
+def test_lbfgs_state_layout(K):
+    b = K.KvsBatch(128, [0, 40, 70], [0, 30, 60], [0, 7, 12], device="cpu")
+    for h in (1, 3, 10, 15):
+        L = K.kvs_lbfgs_state_layout(b, h)
+        total = K.kvs_lbfgs_state_bytes(b, h)
+        n = 12 * 128 * 4  # sum k_b * d floats
+        assert L["slots"] == h + 1 and L["ring_stride"] == n
+        assert L["scalar_bytes"] >= 16 and L["scalars"] + 2 * L["scalar_bytes"] <= L["x"]
+        for f in ("off_f", "off_count", "off_head"):
+            assert 0 <= L[f] <= L["scalar_bytes"] - 4 and L[f] % 4 == 0
+        assert len({L["off_f"], L["off_count"], L["off_head"]}) == 3
+        vecs = [L["x"], L["g"], L["dir"]]
+        assert all(v % 256 == 0 for v in vecs + [L["ring_s"], L["ring_y"]])
+        assert all(b1 - a >= n for a, b1 in zip(vecs, vecs[1:]))
+        assert L["ring_s"] >= L["dir"] + n and L["ring_y"] >= L["ring_s"] + (h + 1) * n
+        assert L["ring_y"] + (h + 1) * n <= total
+    with pytest.raises(K.KvsError):
+        K.kvs_lbfgs_state_layout(b, 16)

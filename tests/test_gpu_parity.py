@@ -120,21 +120,28 @@ def test_topk_bit_exact(case):
 
 # ----------------------------------------------------------- loss and grad
 
-def grad_close(g_gpu, g_or, Q, lse):
-    """Gradient parity: cosine >= 0.999, i.e. |dg| <= 0.0447 |g|, with a floor.
+def grad_close(g_gpu, g_or, Q, lse, floor_ok=False):
+    """Gradient parity: cosine >= 0.999, i.e. |dg| <= 0.0447 |g|.
 
-    The scores carry about 16 significant bits, so the GPU's l_hat may differ
-    from the float64 one by ~2^-16 max|l| per row; through dL/dl_hat =
-    2/n_q (l_hat - l) that moves the gradient by about
+    Returns the branch that decided ("rel" or "floor") and raises on failure.
+    The floor applies only where the caller allows it (floor_ok: k = z with
+    K_c = K_z, where the true gradient vanishes) and only when the true
+    gradient is below it: the scores carry about 16 significant bits, so the
+    GPU's l_hat may differ from the float64 one by ~2^-16 max|l| per row;
+    through dL/dl_hat = 2/n_q (l_hat - l) that moves the gradient by about
     tau = s (2/n_q) 2^-16 max|l| sqrt(sum_i |q_i|^2) (root-mean-square
-    estimate).  Where the true gradient is that small (e.g. k = z with K_c = K_z)
-    the comparison is against tau instead."""
+    estimate).  There the comparison is |dg| <= tau."""
     g_gpu = np.asarray(g_gpu, np.float64)
     g_or = np.asarray(g_or, np.float64)
     n_q, d = Q.shape
     tau = (1 / np.sqrt(d)) * (2.0 / n_q) * 2.0 ** -16 * np.abs(lse).max() * np.sqrt(
         (np.asarray(Q, np.float64) ** 2).sum())
-    return np.linalg.norm(g_gpu - g_or) <= max(0.0447 * np.linalg.norm(g_or), tau)
+    err, gn = np.linalg.norm(g_gpu - g_or), np.linalg.norm(g_or)
+    if floor_ok and gn < tau / 0.0447:
+        assert err <= tau, ("floor", err, tau, gn)
+        return "floor"
+    assert err <= 0.0447 * gn, ("rel", err, gn, tau)
+    return "rel"
 
 
 def select_fit_point(c, perturb=0.0, seed=0):
@@ -181,7 +188,51 @@ def test_loss_grad(case, perturb):
         floor_out = (2.0 ** -16) ** 2 * float((tgt[b][0].astype(np.float64) ** 2).mean())
         assert abs(gp[b, 0] - info["out"]) <= 1e-3 * info["out"] + floor_out
         assert abs(gp[b, 1] - info["lse"]) <= 1e-3 * info["lse"] + floor_lse
-        assert grad_close(gd[co[b]:co[b + 1]], g, c.Qs[b], tgt[b][1]), b
+        full = int(c.k[b]) == len(c.Zk[b])  # K_c = K_z: the true gradient vanishes
+        branch = grad_close(gd[co[b]:co[b + 1]], g, c.Qs[b], tgt[b][1],
+                            floor_ok=full and perturb == 0.0)
+        assert branch == "rel" or full, b
+
+
+OPTIMISED = {
+    # name: (case, oracle schedule run before the comparison)
+    "single_d64": ("single_d64", O.Schedule(outer=20, steps=5)),
+    "small_d64": ("small_d64", O.Schedule(outer=10, steps=5)),
+    "qwen_layer": ("qwen_layer", O.Schedule(outer=6, steps=5)),
+}
+
+
+@pytest.mark.parametrize("name", sorted(OPTIMISED))
+def test_loss_grad_at_an_optimised_point(name):
+    """Loss and gradient at the point an oracle run reaches after many L-BFGS
+    steps and value fits: near an optimum the gradient is a small sum of large
+    terms, where the arithmetic's precision matters most."""
+    cname, osched = OPTIMISED[name]
+    c = cases()[cname]()
+    K = c.K
+    Kcs, Vcs, tgt = [], [], []
+    for b in range(c.bt.B):
+        r = O.compress(c.Qs[b], c.Zk[b], c.Zv[b], int(c.k[b]), osched)
+        assert r["loss"] < 0.5 * r["trace"][0]
+        Kcs.append(r["Kc"].astype(np.float32))
+        Vcs.append(r["Vc"].astype(np.float32))
+        tgt.append((r["Y"].astype(np.float32), r["lse"].astype(np.float32)))
+    B = c.bt.B
+    loss = torch.empty(B, device="cuda")
+    dK = torch.empty((c.batch.sum_c, c.wl.d), device="cuda")
+    K.kvs_loss_grad(c.batch, c.Q, dev(np.concatenate(Kcs)), dev(np.concatenate(Vcs)),
+                    dev(np.concatenate([t[0] for t in tgt])),
+                    dev(np.concatenate([t[1] for t in tgt])), 1.0, 1.0, loss, None, dK, c.ws)
+    torch.cuda.synchronize()
+    gl, gd = host(loss), host(dK)
+    co = c.batch.c_off_h
+    for b in range(B):
+        # the oracle at the same float32 point
+        f, g, _ = O.loss_grad(c.Qs[b], Kcs[b], Vcs[b], tgt[b][0], tgt[b][1])
+        assert abs(gl[b] - f) <= 1e-3 * f, (b, gl[b], f)
+        full = int(c.k[b]) == len(c.Zk[b])
+        branch = grad_close(gd[co[b]:co[b + 1]], g, c.Qs[b], tgt[b][1], floor_ok=full)
+        assert branch == "rel" or full, b
 
 
 def test_loss_only_matches_loss_grad(case):
@@ -334,7 +385,9 @@ def test_compress_small(name):
         check_topk_valid(gi, c.Qs[b], c.Zk[b], c.Zv[b], int(c.k[b]))
         assert abs(r["trace"][b, 0] - res["trace"][0]) <= 1e-3 * res["trace"][0] + 1e-7, b
         f_gpu, f_or = float(r["trace"][b, -1]), float(res["loss"])
-        assert f_gpu <= 1.05 * f_or + 1e-7, (b, f_gpu, f_or)
+        # within 5 % of the oracle's final loss on either side (plus a floor for
+        # losses near zero)
+        assert abs(f_gpu - f_or) <= 0.05 * f_or + 1e-7, (b, f_gpu, f_or, f_gpu / f_or)
         assert f_gpu <= r["trace"][b, 0]
         assert abs(r["parts"][b, 0] * 1.0 + r["parts"][b, 1] - f_gpu) <= 1e-3 * f_gpu + 1e-7
 
@@ -350,7 +403,8 @@ def test_compress_qwen_layer_head():
     res = O.compress(c.Qs[0], c.Zk[0], c.Zv[0], wl.k, O.Schedule(outer=wl.outer, steps=wl.steps))
     assert check_topk_valid(r["idx"], c.Qs[0], c.Zk[0], c.Zv[0], wl.k)
     assert abs(r["trace"][0, 0] - res["trace"][0]) <= 1e-3 * res["trace"][0]
-    assert float(r["trace"][0, -1]) <= 1.05 * res["loss"]
+    ratio = float(r["trace"][0, -1]) / res["loss"]
+    assert 0.95 <= ratio <= 1.05, ratio
 
 
 @pytest.mark.slow
@@ -380,4 +434,4 @@ def test_longctx_head_targets_fit_loss_grad():
     torch.cuda.synchronize()
     f, g, _ = O.loss_grad(c.Qs[0], Kcs[0], Vcs[0], tgt[0][0], tgt[0][1])
     assert abs(host(loss)[0] - f) <= 1e-3 * f
-    assert grad_close(host(dK), g, c.Qs[0], tgt[0][1])
+    assert grad_close(host(dK), g, c.Qs[0], tgt[0][1]) == "rel"

@@ -52,6 +52,13 @@ def test_static_matches_workspace_call_twice(name):
         dK = torch.full_like(Kc, float("nan"))
         K.kvs_loss_grad_static(c.batch, c.Q, Kc, Vc, Y, lse, 1.0, 1.0, loss, parts, dK)
         torch.cuda.synchronize()
+        if call == 1:
+            # the call itself allocates no device memory: after a first call has
+            # loaded the library's kernels, the free device memory does not move
+            free0 = torch.cuda.mem_get_info()[0]
+            K.kvs_loss_grad_static(c.batch, c.Q, Kc, Vc, Y, lse, 1.0, 1.0, loss, parts, dK)
+            torch.cuda.synchronize()
+            assert torch.cuda.mem_get_info()[0] == free0
         rl, l = host(ref_loss), host(loss)
         assert np.all(np.abs(l - rl) <= 1e-3 * np.abs(rl)), (call, l, rl)
         np.testing.assert_allclose(host(parts), host(ref_parts), rtol=1e-3, atol=1e-9)
@@ -62,11 +69,12 @@ def test_static_matches_workspace_call_twice(name):
 
 
 def test_static_rejects_batches_beyond_its_array():
+    assert torch.cuda.is_available()
     c = Case(W.WORKLOADS["qwen_layer"])  # both KV heads of one layer
     K = c.K
     assert K.kvs_workspace_bytes(c.batch) > 32 << 20
     Kc = torch.zeros((c.batch.sum_c, c.wl.d), device="cuda")
-    loss = torch.empty(1, device="cuda")
+    loss = torch.empty(c.bt.B, device="cuda")
     with pytest.raises(K.KvsError) as e:
         K.kvs_loss_grad_static(c.batch, c.Q, Kc, Kc, c.Q, c.Q[:, 0].contiguous(), 1.0, 1.0,
                                loss, None, None)
