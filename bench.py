@@ -33,7 +33,16 @@ sys.path.insert(0, ROOT)
 
 import workload as W  # noqa: E402
 
-METRIC = "head-problems compressed/sec at N=2048,r=0.5"
+METRIC = "head-problems compressed/sec at N=2048,r=0.5"  # the default workload's metric
+
+
+def metric_for(wl: W.Workload) -> str:
+    """The throughput metric of a workload, labelled with its context length and ratio."""
+    r = round(wl.k / wl.z, 2)
+    label = f"head-problems compressed/sec at N={wl.N},r={r:g}"
+    return label + (" (adaptive allocation)" if wl.adaptive else "")
+
+
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 # CUDA-core fp32 FMA peak from unit counts and clock: 148 SMs x 128 lanes x 2 flop x 1.965 GHz
 DERIVED_PEAKS = {"fp32_simt_tflops": 148 * 128 * 2 * 1.965e9 / 1e12}
@@ -317,7 +326,7 @@ def run_gpu(args):
     final = job.trace[:, -1].cpu().numpy()
     first = job.trace[:, 0].cpu().numpy()
     out = {
-        "metric": METRIC,
+        "metric": metric_for(wl),
         "value": round(value, 4),
         "unit": "head-problems/s",
         "n_gpus": world,
@@ -361,45 +370,59 @@ def run_gpu(args):
 
 # ---------------------------------------------------------------- oracle
 
-def oracle_sample(wl, budget_s, pid=(0, 0, 0)):
-    """The oracle's schedule on one problem, run until budget_s of outer
-    iterations have elapsed; returns the per-problem time extrapolated to the
-    full schedule and a description of the sample."""
-    import oracle as O
-    t0 = time.perf_counter()
-    bt = W.make_batch(wl, 0, [pid])
-    p = bt.problem(0)
-    Q = O.build_queries(p["q_retain"], p["q_ctx"], p["pos"], wl.g, wl.m_q, wl.n_syn, wl.N,
-                        wl.rope_base)
-    Y, lse = O.targets(Q, p["Kz"], p["Vz"])
-    idx = O.topk_select(O.importance(Q, p["Kz"], lse), wl.k)
-    Kc = np.asarray(p["Kz"], np.float64)[idx]
-    Vc, _ = O.ridge_fit(Q, Kc, Y, wl.lam)
-    f, g, _ = O.loss_grad(Q, Kc, Vc, Y, lse)
-    st = O.LBFGSState(x=Kc.ravel().copy(), f=f, g=g.ravel())
-    d = wl.d
-    t_setup = time.perf_counter() - t0
-    done = 0
-    t1 = time.perf_counter()
-    while done < wl.outer and (done == 0 or time.perf_counter() - t1 < budget_s):
+class OracleRun:
+    """The oracle's schedule on one problem of the workload: the set-up (query
+    build, targets, top-k, first fit) once, then outer iterations one at a time."""
+
+    def __init__(self, wl, pid=(0, 0, 0)):
+        import oracle as O
+        self.O, self.wl, self.pid = O, wl, pid
+        t0 = time.perf_counter()
+        bt = W.make_batch(wl, 0, [pid])
+        p = bt.problem(0)
+        Q = O.build_queries(p["q_retain"], p["q_ctx"], p["pos"], wl.g, wl.m_q, wl.n_syn, wl.N,
+                            wl.rope_base)
+        Y, lse = O.targets(Q, p["Kz"], p["Vz"])
+        idx = O.topk_select(O.importance(Q, p["Kz"], lse), wl.k)
+        Kc = np.asarray(p["Kz"], np.float64)[idx]
+        self.Vc, _ = O.ridge_fit(Q, Kc, Y, wl.lam)
+        f, g, _ = O.loss_grad(Q, Kc, self.Vc, Y, lse)
+        self.st = O.LBFGSState(x=Kc.ravel().copy(), f=f, g=g.ravel())
+        self.Q, self.Y, self.lse = Q, Y, lse
+        self.t_setup = time.perf_counter() - t0
+
+    def outer(self):
+        """One outer iteration (steps L-BFGS steps, value re-fit); returns its seconds."""
+        O, wl, d = self.O, self.wl, self.wl.d
+        Q, Y, lse, Vc, st = self.Q, self.Y, self.lse, self.Vc, self.st
+        t0 = time.perf_counter()
         fl = lambda x: O.loss_only(Q, x.reshape(-1, d), Vc, Y, lse)
         fg = lambda x: O.loss_grad(Q, x.reshape(-1, d), Vc, Y, lse)[1].ravel()
         for _ in range(wl.steps):
             O.lbfgs_step(st, fl, fg, wl.history)
-        Vc, _ = O.ridge_fit(Q, st.x.reshape(-1, d), Y, wl.lam)
-        f, g, _ = O.loss_grad(Q, st.x.reshape(-1, d), Vc, Y, lse)
+        self.Vc, _ = O.ridge_fit(Q, st.x.reshape(-1, d), Y, wl.lam)
+        f, g, _ = O.loss_grad(Q, st.x.reshape(-1, d), self.Vc, Y, lse)
         st.f, st.g = f, g.ravel()
-        done += 1
-    t_outer = (time.perf_counter() - t1) / done
-    total = t_setup + t_outer * wl.outer
-    sample = (f"1 problem {pid} of {wl.name}: query build, targets, top-k, first fit, then "
-              f"{done} of {wl.outer} outer iterations ({wl.steps} L-BFGS steps + re-fit each) "
-              f"timed; per-problem time extrapolated to the full schedule")
-    if wl.adaptive:
-        # the pilot repeats the setup and runs pilot_outer outer iterations at uniform k
-        total += t_setup + t_outer * wl.pilot_outer * wl.pilot_steps / wl.steps
-        sample += f", plus a {wl.pilot_outer}x{wl.pilot_steps} pilot extrapolated the same way"
-    return total, sample
+        return time.perf_counter() - t0
+
+    def per_problem(self, t_outer):
+        """Seconds per head-problem of the whole schedule from the measured set-up and
+        mean outer-iteration time (plus the pilot run of an adaptive workload)."""
+        wl = self.wl
+        total = self.t_setup + t_outer * wl.outer
+        if wl.adaptive:
+            total += self.t_setup + t_outer * wl.pilot_outer * wl.pilot_steps / wl.steps
+        return total
+
+    def describe(self, n_outer, threads):
+        wl = self.wl
+        s = (f"1 problem {self.pid} of {wl.name} on {threads} thread(s): query build, targets, "
+             f"top-k and first fit timed once, then {n_outer} of the {wl.outer} outer "
+             f"iterations ({wl.steps} L-BFGS steps + re-fit each) timed; per-problem time "
+             f"extrapolated to the full schedule")
+        if wl.adaptive:
+            s += f", plus a {wl.pilot_outer}x{wl.pilot_steps} pilot extrapolated the same way"
+        return s
 
 
 def _cores():
@@ -414,38 +437,105 @@ def _cores():
 
 
 def cpu_baseline(wl, budget_s=20.0):
-    t, sample = oracle_sample(wl, budget_s)
-    return {"value": round(1.0 / t, 6), "unit": "head-problems/s", "cores": _cores(),
-            "kind": "oracle", "sample": sample, "seconds_per_problem": round(t, 2)}
+    """The oracle as it stands on the host's cores (BLAS threads = all cores), outer
+    iterations until budget_s, and one outer iteration on a single thread."""
+    run = OracleRun(wl)
+    times = [run.outer()]
+    while len(times) < wl.outer and sum(times) < budget_s:
+        times.append(run.outer())
+    t = run.per_problem(float(np.mean(times)))
+    out = {"value": round(1.0 / t, 6), "unit": "head-problems/s", "cores": _cores(),
+           "kind": "oracle", "extrapolated": True, "sample": run.describe(len(times), _cores()),
+           "seconds_per_problem": round(t, 2)}
+    try:
+        from threadpoolctl import threadpool_limits
+        with threadpool_limits(limits=1):
+            one = OracleRun(wl)
+            t1 = one.per_problem(one.outer())
+        out["single_thread"] = {"value": round(1.0 / t1, 6), "unit": "head-problems/s",
+                                "cores": 1, "seconds_per_problem": round(t1, 1),
+                                "sample": one.describe(1, 1)}
+    except ImportError:
+        pass
+    return out
 
 
 def run_reference(args):
+    """The oracle timed on the host cores.  One step = one outer iteration of the
+    schedule on one problem (a bounded sample); the value extrapolates the measured
+    set-up and outer-iteration times to whole head-problems per second."""
     rank = int(os.environ.get("RANK", "0"))
     if rank != 0:
         return
     wl = W.WORKLOADS[args.workload]
     if args.outer is not None:
         wl = wl.with_(outer=args.outer)
-    budget = max(2.0, min(args.cpu_budget, 20.0))
-    for _ in range(args.warmup if args.warmup < 1 else 1):
-        oracle_sample(wl, 1.0)
-    times = []
-    sample = ""
-    for _ in range(args.steps):
-        t, sample = oracle_sample(wl, budget)
-        times.append(t)
-    per = float(np.mean(times))
+    run = OracleRun(wl)
+    for _ in range(args.warmup):
+        run.outer()
+    times = [run.outer() for _ in range(args.steps)]
+    per = run.per_problem(float(np.mean(times)))
     value = 1.0 / per
-    out = {"impl": "reference", "metric": METRIC, "value": round(value, 6),
+    sample = run.describe(args.steps, _cores())
+    out = {"impl": "reference", "metric": metric_for(wl), "value": round(value, 6),
            "unit": "head-problems/s", "n_gpus": int(os.environ.get("WORLD_SIZE", "1")),
-           "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(per * 1e3, 1),
+           "steps": args.steps, "warmup": args.warmup,
+           "ms_per_step": round(float(np.mean(times)) * 1e3, 1),
+           "step": "one outer iteration of one problem's schedule (value: whole problems/s, "
+                   "extrapolated)",
+           "extrapolated": True, "seconds_per_problem": round(per, 2),
            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
            "data": "synthetic (seeded generator)", "config": {"workload": describe(wl)},
            "cpu_baseline": {"value": round(value, 6), "unit": "head-problems/s",
-                            "cores": _cores(), "kind": "oracle", "sample": sample},
+                            "cores": _cores(), "kind": "oracle", "sample": sample,
+                            "extrapolated": True},
            "e2e": {"value": round(value, 6), "unit": "head-problems/s",
                    "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(out), flush=True)
+
+
+# ---------------------------------------------------------------- ranks
+
+def rank_env(base_env, world, rank, port):
+    """Environment of rank `rank` of `world` processes on this node (one GPU each)."""
+    env = dict(base_env)
+    env.update(RANK=str(rank), WORLD_SIZE=str(world), LOCAL_RANK=str(rank),
+               LOCAL_WORLD_SIZE=str(world), MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    return env
+
+
+def free_port():
+    import socket
+    with socket.socket() as sk:
+        sk.bind(("127.0.0.1", 0))
+        return sk.getsockname()[1]
+
+
+def spawn_ranks(world, argv, timeout_s=3600):
+    """Run this script as `world` processes (rank 0 prints the JSON line); returns the
+    first non-zero exit code, or 0.  A rank that fails ends the others."""
+    port = free_port()
+    procs = [subprocess.Popen([sys.executable, os.path.abspath(__file__), *argv],
+                              env=rank_env(os.environ, world, r, port))
+             for r in range(world)]
+    rc = 0
+    t_end = time.time() + timeout_s
+    while procs:
+        for p in list(procs):
+            code = p.poll()
+            if code is None:
+                continue
+            procs.remove(p)
+            if code != 0 and rc == 0:
+                rc = code
+                t_end = min(t_end, time.time() + 60)  # give the others a minute
+        if time.time() > t_end:
+            for p in procs:
+                p.kill()
+            rc = rc or 124
+            break
+        time.sleep(0.2)
+    return rc
 
 
 def main():
@@ -462,6 +552,12 @@ def main():
     ap.add_argument("--peak-key", default="bf16_tflops")
     ap.add_argument("--dtype-label", default="bf16x3-f32acc")
     args = ap.parse_args()
+    if args.gpus > 1 and "WORLD_SIZE" not in os.environ:
+        # one process per GPU, launched here (torchrun sets WORLD_SIZE itself)
+        sys.exit(spawn_ranks(args.gpus, sys.argv[1:]))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    if args.gpus != world:
+        raise SystemExit(f"--gpus {args.gpus} but WORLD_SIZE={world}")
     if args.impl == "reference":
         run_reference(args)
     else:

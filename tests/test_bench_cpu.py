@@ -26,7 +26,8 @@ def test_reference_line_contract():
     assert len(lines) == 1
     d = json.loads(lines[0])
     assert d["impl"] == "reference"
-    assert d["metric"] == bench.METRIC and d["unit"] == "head-problems/s"
+    assert d["metric"] == bench.metric_for(W.WORKLOADS["single_d64"])
+    assert d["unit"] == "head-problems/s" and d["extrapolated"] is True
     assert d["value"] > 0 and d["higher_is_better"] is True
     assert d["steps"] == 1 and d["warmup"] == 0 and d["n_gpus"] == 1
     assert d["dtype"] == "f64" and d["vs_baseline"] is None
@@ -91,3 +92,43 @@ def test_reference_arm_under_torchrun_prints_once():
     assert len(lines) == 1
     d = json.loads(lines[0])
     assert d["impl"] == "reference" and d["n_gpus"] == 2
+
+
+def test_gpus_flag_launches_the_ranks_itself():
+    # without torchrun, --gpus 2 starts two processes with their own rank environment;
+    # rank 0 alone prints the line, which reports both ranks
+    r = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--impl", "reference",
+                        "--gpus", "2", "--workload", "single_d64", "--steps", "1", "--warmup",
+                        "0"], capture_output=True, text=True, timeout=900, cwd=ROOT,
+                       env={k: v for k, v in os.environ.items() if k not in
+                            ("RANK", "WORLD_SIZE", "LOCAL_RANK")})
+    assert r.returncode == 0, r.stderr[-2000:]
+    lines = [l for l in r.stdout.splitlines() if l.startswith("{")]
+    assert len(lines) == 1
+    d = json.loads(lines[0])
+    assert d["impl"] == "reference" and d["n_gpus"] == 2
+
+
+def test_rank_env():
+    base = {"PATH": "/bin", "RANK": "7"}
+    envs = [bench.rank_env(base, 4, r, 29500) for r in range(4)]
+    assert [e["RANK"] for e in envs] == ["0", "1", "2", "3"]
+    assert [e["LOCAL_RANK"] for e in envs] == ["0", "1", "2", "3"]
+    assert all(e["WORLD_SIZE"] == "4" and e["MASTER_ADDR"] == "127.0.0.1" and
+               e["MASTER_PORT"] == "29500" and e["PATH"] == "/bin" for e in envs)
+    assert base["RANK"] == "7"  # the caller's environment is left alone
+
+
+def test_spawn_reports_a_failing_rank(tmp_path, monkeypatch):
+    script = tmp_path / "fail_rank1.py"
+    script.write_text("import os, sys\nsys.exit(3 if os.environ['RANK'] == '1' else 0)\n")
+    monkeypatch.setattr(bench, "__file__", str(script))
+    assert bench.spawn_ranks(2, [], timeout_s=120) == 3
+
+
+def test_metric_labels():
+    assert bench.metric_for(W.WORKLOADS["qwen_cache_r05"]) == bench.METRIC
+    assert bench.metric_for(W.WORKLOADS["qwen_cache_r03"]).endswith("N=2048,r=0.3")
+    assert bench.metric_for(W.WORKLOADS["qwen_cache_r07"]).endswith("N=2048,r=0.7")
+    assert bench.metric_for(W.WORKLOADS["longctx"]).endswith("N=8192,r=0.3")
+    assert "adaptive" in bench.metric_for(W.WORKLOADS["qwen_cache_adaptive"])
