@@ -284,7 +284,7 @@ class Schedule:
 
 
 def compress(Q, Kz, Vz, k: int, sched: Schedule, idx: Optional[np.ndarray] = None,
-             record: Optional[list] = None):
+             record: Optional[list] = None, evaluate=None):
     """Distil one compress zone (K_z, V_z) into k pairs for the training queries Q.
 
     targets -> importance -> top-k keys -> ridge values (Select+Fit state) ->
@@ -292,8 +292,13 @@ def compress(Q, Kz, Vz, k: int, sched: Schedule, idx: Optional[np.ndarray] = Non
     K_c, V_c, the loss trace after every fit (outer + 1 entries), the final
     loss terms, the top-k indices and the status bits.  When `record` is a
     list, a copy of (K_c, V_c, number of stored L-BFGS pairs) is appended to
-    it after every fit (outer + 1 entries); nothing else changes.
+    it after every fit (outer + 1 entries); nothing else changes.  `evaluate`
+    (a pair of functions with the signatures of loss_only and loss_grad)
+    replaces the loss and gradient evaluations that steer the schedule, e.g. by
+    perturbed ones to measure how sensitive the trajectory is; the reported
+    losses are still evaluated exactly.  Default: the plain ones.
     """
+    ev_loss, ev_grad = evaluate if evaluate is not None else (loss_only, loss_grad)
     Q = np.asarray(Q, np.float64)
     d = Q.shape[1]
     Y, lse = targets(Q, Kz, Vz)
@@ -307,14 +312,14 @@ def compress(Q, Kz, Vz, k: int, sched: Schedule, idx: Optional[np.ndarray] = Non
         Vc = np.zeros((len(idx), d))
 
     def fl(x):
-        return loss_only(Q, x.reshape(-1, d), Vc, Y, lse, sched.w_out, sched.w_lse)
+        return ev_loss(Q, x.reshape(-1, d), Vc, Y, lse, sched.w_out, sched.w_lse)
 
     def fg(x):
-        return loss_grad(Q, x.reshape(-1, d), Vc, Y, lse, sched.w_out, sched.w_lse)[1].ravel()
+        return ev_grad(Q, x.reshape(-1, d), Vc, Y, lse, sched.w_out, sched.w_lse)[1].ravel()
 
-    f, g, _ = loss_grad(Q, Kc, Vc, Y, lse, sched.w_out, sched.w_lse)
+    f, g, _ = ev_grad(Q, Kc, Vc, Y, lse, sched.w_out, sched.w_lse)
     st = LBFGSState(x=Kc.ravel().copy(), f=f, g=g.ravel())
-    trace = [f]
+    trace = [loss_only(Q, Kc, Vc, Y, lse, sched.w_out, sched.w_lse) if evaluate else f]
     if record is not None:
         record.append((Kc.copy(), Vc.copy(), 0))
     for _o in range(sched.outer):
@@ -328,9 +333,9 @@ def compress(Q, Kz, Vz, k: int, sched: Schedule, idx: Optional[np.ndarray] = Non
         if not sched.persist_history:
             st.hist_s.clear()
             st.hist_y.clear()
-        f, g, _ = loss_grad(Q, Kc, Vc, Y, lse, sched.w_out, sched.w_lse)
+        f, g, _ = ev_grad(Q, Kc, Vc, Y, lse, sched.w_out, sched.w_lse)
         st.f, st.g = f, g.ravel()
-        trace.append(f)
+        trace.append(loss_only(Q, Kc, Vc, Y, lse, sched.w_out, sched.w_lse) if evaluate else f)
         if record is not None:
             record.append((Kc.copy(), Vc.copy(), len(st.hist_s)))
     f, _, info = loss_grad(Q, Kc, Vc, Y, lse, sched.w_out, sched.w_lse)
