@@ -116,11 +116,12 @@ uint64_t kvs_launch_count(void);           /* kernels this library has launched 
 int kvs_set_wait_limit(int64_t cycles);
 
 /* Bytes of scratch workspace needed by every call below for this batch
- * (and schedule; may be NULL when no L-BFGS call will use the workspace).
- * Returns 0 for an invalid batch. */
+ * (and schedule; may be NULL when no L-BFGS call will use the workspace),
+ * kvs_compress_batch's sub-batches included.  Returns 0 for an invalid batch. */
 size_t kvs_workspace_bytes(const kvs_batch *batch, const kvs_schedule *sched);
 
-/* Bytes of persistent L-BFGS state for this batch and history length. */
+/* Bytes of persistent L-BFGS state for this batch and history length (enough
+ * for kvs_lbfgs_reset / kvs_lbfgs_step and for kvs_compress_batch). */
 size_t kvs_lbfgs_state_bytes(const kvs_batch *batch, int32_t history);
 
 /* Where the L-BFGS state of kvs_lbfgs_step lives inside a state buffer
@@ -266,7 +267,13 @@ int kvs_adam_step(const kvs_batch *batch, float *Kc, const float *dKc, float *m,
  * After its first step each L-BFGS step runs as one CUDA graph whose trial
  * loop is a conditional node; with the environment variable
  * KVS_STEP_GRAPHS=0 (read once per process) the same kernels are launched
- * one by one instead, for kernel-level profilers. */
+ * one by one instead, for kernel-level profilers.
+ * A batch of 8 or more problems is solved as two sub-batches of contiguous
+ * problems (cut where the work n_q k (d + k) splits evenly), the second on an
+ * internal stream forked from and joined back to `stream`, so that the
+ * latency-bound steps of one overlap the tensor-core work of the other; the
+ * results are those of solving each problem on its own.  `state` is then
+ * scratch laid out per sub-batch (kvs_lbfgs_state_layout does not apply). */
 int kvs_compress_batch(const kvs_batch *batch, const kvs_schedule *sched, const float *Q,
                        const float *Kz, const float *Vz, float *Kc, float *Vc, int32_t *idx,
                        float *loss_trace, float *parts, int32_t *status,

@@ -74,8 +74,11 @@ int geom_from_batch(const kvs_batch *b, HostGeom *g, bool need_c) {
   } else if (b->c_off_h) {
     if (check_offsets(b->c_off_h, b->B, &g->sum_c, &g->max_c, true)) return KVS_EINVAL;
   }
-  for (int bb = 0; bb < b->B; ++bb)
+  for (int bb = 0; bb < b->B; ++bb) {
     g->sum_qpad += align_up(b->q_off_h[bb + 1] - b->q_off_h[bb], 128);
+    g->sum_zpad += align_up(b->z_off_h[bb + 1] - b->z_off_h[bb], 128);
+    if (b->c_off_h) g->sum_cpad += align_up(b->c_off_h[bb + 1] - b->c_off_h[bb], 128);
+  }
   g->ld_a = align_up(std::max(g->max_c, 1), 128);
   g->ld_g = align_up(std::max(g->max_c, 1), 4);
   return KVS_OK;
@@ -96,22 +99,26 @@ struct Carver {
 
 size_t carve_work(const HostGeom &g, void *base, Work *w) {
   Carver c{static_cast<char *>(base)};
-  const int64_t kz = std::max(g.sum_z, g.sum_c);
-  w->qh = c.take<__nv_bfloat16>(g.sum_q * g.d);
-  w->ql = c.take<__nv_bfloat16>(g.sum_q * g.d);
+  // tensor-core operands: rows padded to 128 per problem (zero rows), so that no
+  // tile reaches into another problem's rows
+  const int64_t kz = std::max(g.sum_zpad, g.sum_cpad);
+  w->qh = c.take<__nv_bfloat16>(g.sum_qpad * g.d);
+  w->ql = c.take<__nv_bfloat16>(g.sum_qpad * g.d);
   w->kh = c.take<__nv_bfloat16>(kz * g.d);
   w->kl = c.take<__nv_bfloat16>(kz * g.d);
   w->vh = c.take<__nv_bfloat16>(kz * g.d);
   w->vl = c.take<__nv_bfloat16>(kz * g.d);
-  w->go = c.take<__nv_bfloat16>(g.sum_q * g.d);
-  w->yh = c.take<__nv_bfloat16>(g.sum_q * g.d);
-  w->yl = c.take<__nv_bfloat16>(g.sum_q * g.d);
+  w->go = c.take<__nv_bfloat16>(g.sum_qpad * g.d);
+  w->yh = c.take<__nv_bfloat16>(g.sum_qpad * g.d);
+  w->yl = c.take<__nv_bfloat16>(g.sum_qpad * g.d);
   w->ahi = c.take<__nv_bfloat16>(g.sum_qpad * g.ld_a);
   w->alo = c.take<__nv_bfloat16>(g.sum_qpad * g.ld_a);
   w->lse_h = c.take<float>(g.sum_q);
   w->delta = c.take<float>(g.sum_q);
   w->partials = c.take<float>((int64_t)g.B * ((g.max_q + 127) / 128) * 2);
   w->a_pad_off = c.take<int64_t>(g.B + 1);
+  w->z_pad = c.take<int64_t>(g.B + 1);
+  w->c_pad = c.take<int64_t>(g.B + 1);
   w->gram = c.take<float>(g.sum_c * g.ld_g);
   w->R = c.take<float>(g.sum_c * g.d);
   w->X = c.take<float>(g.sum_c * g.d);
@@ -160,10 +167,11 @@ static int prep(const kvs_batch *b, bool need_c, void *ws, size_t ws_bytes, void
   return KVS_OK;
 }
 
-// First device work of a call, after every argument check has passed.
+// First device work of a call, after every argument check has passed: clear the
+// timeout flag and lay out the padded operand rows.
 static int begin(const Batch &Bt, const Work &w) {
   KVS_CUDA_TRY(cudaMemsetAsync(w.err, 0, sizeof(int), Bt.st));
-  return KVS_OK;
+  return launch_pad_offsets(Bt, w);
 }
 
 // status[b] |= KVS_ST_TIMEOUT when a kernel of the call gave up waiting.
@@ -353,6 +361,142 @@ static int build_step_graph(const Batch &Bcaller, const kvs_schedule &sc, const 
   return KVS_OK;
 }
 
+// ------------------------------------------------------------ sub-batches
+// kvs_compress_batch runs a large batch as independent sub-batches of
+// contiguous problems, each on its own stream, so that the latency-bound parts
+// of one (the Cholesky panels, the single-CTA L-BFGS control kernels) overlap
+// the tensor-core work of the other.  Each sub-batch is a batch in its own
+// right: offsets rebased to zero (on the device, in the caller's workspace),
+// data pointers moved to its first rows, its own workspace and state carved
+// from the caller's buffers, its own step graph and internal streams.
+
+struct Partition {
+  int n = 1;
+  int cut[KVS_MAX_PARTS + 1] = {0};
+};
+
+// Two sub-batches once the batch has at least 8 problems (each half still fills
+// the GPU in the attention kernels), cut where the estimated work
+// n_q k (d + k) of the problems splits most evenly.
+static Partition partition_of(const kvs_batch *b, const HostGeom &g) {
+  Partition P;
+  P.cut[1] = g.B;
+  if (g.B < 8 || !b->c_off_h) return P;
+  std::vector<double> acc(g.B + 1, 0.0);
+  for (int i = 0; i < g.B; ++i) {
+    const double nq = (double)(b->q_off_h[i + 1] - b->q_off_h[i]);
+    const double k = (double)(b->c_off_h[i + 1] - b->c_off_h[i]);
+    acc[i + 1] = acc[i] + nq * k * (g.d + k);
+  }
+  int best = 1;
+  for (int c = 2; c < g.B; ++c)
+    if (std::fabs(acc[c] - acc[g.B] / 2) < std::fabs(acc[best] - acc[g.B] / 2)) best = c;
+  P.n = 2;
+  P.cut[1] = best;
+  P.cut[2] = g.B;
+  return P;
+}
+
+// Placeholder for device offset pointers while sizing (never dereferenced).
+static const int64_t *const kSizingOnly = reinterpret_cast<const int64_t *>(uintptr_t{256});
+
+struct Part {
+  int b0 = 0, b1 = 0;
+  std::vector<int64_t> q_h, z_h, c_h;  // rebased host offsets
+  kvs_batch kb{};
+  HostGeom g;
+  size_t ws_off = 0, st_off = 0;       // this part's pieces of the caller's buffers
+};
+
+// Host geometry of every part and where its workspace, state and rebased device
+// offsets sit; returns false for an invalid batch.  *ws_need / *st_need: bytes.
+static bool plan_parts(const kvs_batch *b, const HostGeom &g, int history, const Partition &P,
+                       Part *parts, size_t *ws_need, size_t *st_need, size_t *off_at) {
+  size_t ws = 0, st = 0;
+  for (int p = 0; p < P.n; ++p) {
+    Part &pt = parts[p];
+    pt.b0 = P.cut[p];
+    pt.b1 = P.cut[p + 1];
+    const int n = pt.b1 - pt.b0;
+    pt.q_h.resize(n + 1);
+    pt.z_h.resize(n + 1);
+    pt.c_h.resize(n + 1);
+    for (int i = 0; i <= n; ++i) {
+      pt.q_h[i] = b->q_off_h[pt.b0 + i] - b->q_off_h[pt.b0];
+      pt.z_h[i] = b->z_off_h[pt.b0 + i] - b->z_off_h[pt.b0];
+      pt.c_h[i] = b->c_off_h[pt.b0 + i] - b->c_off_h[pt.b0];
+    }
+    pt.kb = kvs_batch{n, b->d, kSizingOnly, kSizingOnly, kSizingOnly,
+                      pt.q_h.data(), pt.z_h.data(), pt.c_h.data()};
+    if (geom_from_batch(&pt.kb, &pt.g, true)) return false;
+    Work w;
+    State s;
+    pt.ws_off = ws = (size_t)align_up((int64_t)ws, 256);
+    ws += carve_work(pt.g, nullptr, &w);
+    pt.st_off = st = (size_t)align_up((int64_t)st, 256);
+    st += carve_state(pt.g, history, nullptr, &s);
+  }
+  *off_at = ws = (size_t)align_up((int64_t)ws, 256);
+  ws += sizeof(int64_t) * 3 * (size_t)(g.B + P.n);  // rebased q, z, c offsets of every part
+  *ws_need = (size_t)align_up((int64_t)ws, 256);
+  *st_need = (size_t)align_up((int64_t)st, 256);
+  return true;
+}
+
+// dst receives, part after part, the rebased offsets q, z and c of each part
+// (3 arrays of n_p + 1 entries).
+__global__ void k_rebase(const int64_t *q_off, const int64_t *z_off, const int64_t *c_off,
+                         Partition P, int64_t *dst) {
+  int64_t *o = dst;
+  for (int p = 0; p < P.n; ++p) {
+    const int b0 = P.cut[p], n = P.cut[p + 1] - b0;
+    for (int i = threadIdx.x; i <= n; i += blockDim.x) {
+      o[i] = q_off[b0 + i] - q_off[b0];
+      o[n + 1 + i] = z_off[b0 + i] - z_off[b0];
+      o[2 * (n + 1) + i] = c_off[b0 + i] - c_off[b0];
+    }
+    o += 3 * (n + 1);
+  }
+}
+
+// The stream of sub-batch `slot` >= 1 and the events that fork it from and join it
+// to the caller's stream (per host thread and device, created on first use).
+struct PartStreams {
+  cudaStream_t st[KVS_MAX_PARTS] = {nullptr};
+  cudaEvent_t fork = nullptr, join[KVS_MAX_PARTS] = {nullptr};
+};
+
+static cudaError_t part_streams(PartStreams **out) {
+  constexpr int kMaxDev = 64;
+  static thread_local PartStreams ps[kMaxDev];
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev < 0 || dev >= kMaxDev) return cudaErrorInvalidDevice;
+  PartStreams &p = ps[dev];
+  if (!p.fork) {
+    if ((e = cudaEventCreateWithFlags(&p.fork, cudaEventDisableTiming)) != cudaSuccess) return e;
+    for (int i = 1; i < KVS_MAX_PARTS; ++i)
+      if ((e = cudaStreamCreateWithFlags(&p.st[i], cudaStreamNonBlocking)) != cudaSuccess ||
+          (e = cudaEventCreateWithFlags(&p.join[i], cudaEventDisableTiming)) != cudaSuccess)
+        return e;
+  }
+  *out = &p;
+  return cudaSuccess;
+}
+
+// One sub-batch's solve: its batch view, buffers and step graph.
+struct Solve {
+  Batch Bt;
+  Work w;
+  State s;
+  const float *Q, *Kz, *Vz;
+  float *Kc, *Vc, *trace, *parts;
+  int32_t *idx, *status;
+  StepGraph sg;
+  bool have_graph = false;
+};
+
 }  // namespace kvs
 
 using namespace kvs;
@@ -375,14 +519,30 @@ size_t kvs_workspace_bytes(const kvs_batch *batch, const kvs_schedule *) {
   HostGeom g;
   if (geom_from_batch(batch, &g, false)) return 0;
   Work w;
-  return carve_work(g, nullptr, &w);
+  size_t need = carve_work(g, nullptr, &w);
+  const Partition P = partition_of(batch, g);
+  if (P.n > 1) {  // the sub-batches of kvs_compress_batch
+    Part parts[KVS_MAX_PARTS];
+    size_t ws = 0, st = 0, off = 0;
+    if (!plan_parts(batch, g, 1, P, parts, &ws, &st, &off)) return 0;
+    need = std::max(need, ws);
+  }
+  return need;
 }
 
 size_t kvs_lbfgs_state_bytes(const kvs_batch *batch, int32_t history) {
   HostGeom g;
   if (history < 1 || history > 15 || geom_from_batch(batch, &g, true)) return 0;
   State s;
-  return carve_state(g, history, nullptr, &s);
+  size_t need = carve_state(g, history, nullptr, &s);
+  const Partition P = partition_of(batch, g);
+  if (P.n > 1) {
+    Part parts[KVS_MAX_PARTS];
+    size_t ws = 0, st = 0, off = 0;
+    if (!plan_parts(batch, g, history, P, parts, &ws, &st, &off)) return 0;
+    need = std::max(need, st);
+  }
+  return need;
 }
 
 int kvs_lbfgs_state_layout(const kvs_batch *batch, int32_t history, kvs_lbfgs_layout *out) {
@@ -558,18 +718,74 @@ int kvs_compress_batch(const kvs_batch *batch, const kvs_schedule *sched, const 
     if (batch->c_off_h[b + 1] - batch->c_off_h[b] > batch->z_off_h[b + 1] - batch->z_off_h[b])
       return KVS_EINVAL;
   const kvs_schedule &sc = *sched;
-  int32_t *ix = idx ? idx : w.idx;
-  if ((rc = begin(Bt, w))) return rc;
-  KVS_CUDA_TRY(cudaMemsetAsync(status, 0, sizeof(int32_t) * Bt.g.B, Bt.st));
-  if ((rc = launch_targets(Bt, Q, Kz, Vz, w.Yt, w.lset, w.imp, w))) return rc;
-  if ((rc = launch_topk(Bt, w.imp, Kz, ix, Kc))) return rc;
-  // from here on the bf16 splits of Q and of the targets Y stay in the workspace
-  if ((rc = launch_fit(Bt, Q, Kc, w.Yt, sc.lambda, Vc, status, true, true, w))) return rc;
-  if ((rc = lbfgs_restart(Bt, sc, Q, w.Yt, w.lset, Vc, Kc, s, 1, true, w))) return rc;
   const int64_t tstride = sc.outer + 1;
-  if (loss_trace && (rc = launch_copy_f(Bt, s, loss_trace, tstride, 0))) return rc;
-  StepGraph sg;
-  bool have_graph = false;
+  const int d = Bt.g.d;
+
+  // the sub-batches: one (the whole batch, as given) or several
+  const Partition P = partition_of(batch, Bt.g);
+  Part pt[KVS_MAX_PARTS];
+  Solve sv[KVS_MAX_PARTS];
+  PartStreams *ps = nullptr;
+  if (P.n == 1) {
+    sv[0].Bt = Bt;
+    sv[0].w = w;
+    sv[0].s = s;
+  } else {
+    size_t ws_need = 0, st_need = 0, off_at = 0;
+    if (!plan_parts(batch, Bt.g, sc.history, P, pt, &ws_need, &st_need, &off_at))
+      return KVS_EINVAL;
+    if (ws_need > ws_bytes || st_need > state_bytes) return KVS_EWORKSPACE;
+    KVS_CUDA_TRY(part_streams(&ps));
+    int64_t *dev_off = reinterpret_cast<int64_t *>(static_cast<char *>(ws) + off_at);
+    k_rebase<<<1, 256, 0, Bt.st>>>(batch->q_off, batch->z_off, batch->c_off, P, dev_off);
+    KVS_LAUNCH_CHECK("k_rebase");
+    KVS_CUDA_TRY(cudaEventRecord(ps->fork, Bt.st));
+    for (int p = 0; p < P.n; ++p) {
+      const int n = pt[p].b1 - pt[p].b0;
+      pt[p].kb.q_off = dev_off;
+      pt[p].kb.z_off = dev_off + (n + 1);
+      pt[p].kb.c_off = dev_off + 2 * (n + 1);
+      dev_off += 3 * (n + 1);
+      Solve &v = sv[p];
+      v.Bt.g = pt[p].g;
+      v.Bt.b = &pt[p].kb;
+      v.Bt.slot = p;
+      v.Bt.st = p == 0 ? Bt.st : ps->st[p];
+      if (p > 0) KVS_CUDA_TRY(cudaStreamWaitEvent(v.Bt.st, ps->fork, 0));
+      carve_work(v.Bt.g, static_cast<char *>(ws) + pt[p].ws_off, &v.w);
+      carve_state(v.Bt.g, sc.history, static_cast<char *>(state) + pt[p].st_off, &v.s);
+    }
+  }
+  for (int p = 0; p < P.n; ++p) {
+    Solve &v = sv[p];
+    const int b0 = P.cut[p];
+    const int64_t q0 = batch->q_off_h[b0], z0 = batch->z_off_h[b0], c0 = batch->c_off_h[b0];
+    v.Q = Q + q0 * d;
+    v.Kz = Kz + z0 * d;
+    v.Vz = Vz + z0 * d;
+    v.Kc = Kc + c0 * d;
+    v.Vc = Vc + c0 * d;
+    v.idx = idx ? idx + c0 : v.w.idx;
+    v.status = status + b0;
+    v.trace = loss_trace ? loss_trace + b0 * tstride : nullptr;
+    v.parts = parts ? parts + 2 * b0 : nullptr;
+  }
+
+  // initial state of every sub-batch: targets, top-k keys, Select+Fit, L-BFGS reset
+  for (int p = 0; p < P.n; ++p) {
+    Solve &v = sv[p];
+    const Batch &B = v.Bt;
+    if ((rc = begin(B, v.w))) return rc;
+    KVS_CUDA_TRY(cudaMemsetAsync(v.status, 0, sizeof(int32_t) * B.g.B, B.st));
+    if ((rc = launch_targets(B, v.Q, v.Kz, v.Vz, v.w.Yt, v.w.lset, v.w.imp, v.w))) return rc;
+    if ((rc = launch_topk(B, v.w.imp, v.Kz, v.idx, v.Kc))) return rc;
+    // from here on the bf16 splits of Q and of the targets Y stay in the workspace
+    if ((rc = launch_fit(B, v.Q, v.Kc, v.w.Yt, sc.lambda, v.Vc, v.status, true, true, v.w)))
+      return rc;
+    if ((rc = lbfgs_restart(B, sc, v.Q, v.w.Yt, v.w.lset, v.Vc, v.Kc, v.s, 1, true, v.w)))
+      return rc;
+    if (v.trace && (rc = launch_copy_f(B, v.s, v.trace, tstride, 0))) return rc;
+  }
   // KVS_STEP_GRAPHS=0 launches every kernel of a step individually (the same
   // arithmetic; kernel profilers do not look inside graphs with conditional nodes)
   static const bool use_graphs = [] {
@@ -578,34 +794,49 @@ int kvs_compress_batch(const kvs_batch *batch, const kvs_schedule *sched, const 
   }();
   for (int o = 0; o < sc.outer; ++o) {
     for (int t = 0; t < sc.steps; ++t) {
-      if (use_graphs && !have_graph && o + t > 0) {
-        // every kernel has been launched once outside capture: record the step now
-        if ((rc = build_step_graph(Bt, sc, Q, w.Yt, w.lset, Vc, Kc, s, status, w, &sg))) return rc;
-        have_graph = true;
-      }
-      if (have_graph) {
-        KVS_CUDA_TRY(cudaGraphLaunch(sg.exec, Bt.st));
-        g_launches.fetch_add(sg.kernels, std::memory_order_relaxed);
-      } else if ((rc = lbfgs_one_step(Bt, sc, Q, w.Yt, w.lset, Vc, Kc, s, status, nullptr, true,
-                                      w))) {
-        return rc;
+      for (int p = 0; p < P.n; ++p) {
+        Solve &v = sv[p];
+        if (use_graphs && !v.have_graph && o + t > 0) {
+          // every kernel has been launched once outside capture: record the step now
+          if ((rc = build_step_graph(v.Bt, sc, v.Q, v.w.Yt, v.w.lset, v.Vc, v.Kc, v.s,
+                                     v.status, v.w, &v.sg)))
+            return rc;
+          v.have_graph = true;
+        }
+        if (v.have_graph) {
+          KVS_CUDA_TRY(cudaGraphLaunch(v.sg.exec, v.Bt.st));
+          g_launches.fetch_add(v.sg.kernels, std::memory_order_relaxed);
+        } else if ((rc = lbfgs_one_step(v.Bt, sc, v.Q, v.w.Yt, v.w.lset, v.Vc, v.Kc, v.s,
+                                        v.status, nullptr, true, v.w))) {
+          return rc;
+        }
       }
     }
-    // every problem's l_hat at Kc is in the workspace from its accepted trial's
-    // loss forward, except after a failed search
-    if ((rc = launch_fit(Bt, Q, Kc, w.Yt, sc.lambda, Vc, status, true, true, w,
-                         sc.steps > 0 ? stale_filter(s) : ALL)))
-      return rc;
-    if ((rc = lbfgs_restart(Bt, sc, Q, w.Yt, w.lset, Vc, Kc, s, sc.persist_history ? 0 : 1, true,
-                            w)))
-      return rc;
-    if (loss_trace && (rc = launch_copy_f(Bt, s, loss_trace, tstride, o + 1))) return rc;
+    for (int p = 0; p < P.n; ++p) {
+      Solve &v = sv[p];
+      // every problem's l_hat at Kc is in the workspace from its accepted trial's
+      // loss forward, except after a failed search
+      if ((rc = launch_fit(v.Bt, v.Q, v.Kc, v.w.Yt, sc.lambda, v.Vc, v.status, true, true, v.w,
+                           sc.steps > 0 ? stale_filter(v.s) : ALL)))
+        return rc;
+      if ((rc = lbfgs_restart(v.Bt, sc, v.Q, v.w.Yt, v.w.lset, v.Vc, v.Kc, v.s,
+                              sc.persist_history ? 0 : 1, true, v.w)))
+        return rc;
+      if (v.trace && (rc = launch_copy_f(v.Bt, v.s, v.trace, tstride, o + 1))) return rc;
+    }
   }
-  if (parts &&
-      (rc = launch_forward(Bt, Q, Kc, Vc, w.Yt, w.lset, sc.w_out, sc.w_lse, w.fbuf, parts, ALL,
-                           true, w)))
-    return rc;
-  return fold_err(Bt, w, status);
+  for (int p = 0; p < P.n; ++p) {
+    Solve &v = sv[p];
+    if (v.parts && (rc = launch_forward(v.Bt, v.Q, v.Kc, v.Vc, v.w.Yt, v.w.lset, sc.w_out,
+                                        sc.w_lse, v.w.fbuf, v.parts, ALL, true, v.w)))
+      return rc;
+    if ((rc = fold_err(v.Bt, v.w, v.status))) return rc;
+    if (p > 0) {
+      KVS_CUDA_TRY(cudaEventRecord(ps->join[p], v.Bt.st));
+      KVS_CUDA_TRY(cudaStreamWaitEvent(Bt.st, ps->join[p], 0));
+    }
+  }
+  return KVS_OK;
 }
 
 // Host-only budget allocation.  The real shares x_b(c) = clip(c w_b, k_min,

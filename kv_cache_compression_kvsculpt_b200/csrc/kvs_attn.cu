@@ -87,49 +87,57 @@ namespace {
 
 // ------------------------------------------------------ elementwise helpers
 
-// x -> (hi, lo) bf16 with hi = rn(x), lo = rn(x - hi); lo may be null (hi only).
-__global__ void k_split(const float *__restrict__ x, __nv_bfloat16 *__restrict__ hi,
-                        __nv_bfloat16 *__restrict__ lo, int64_t n4) {
+// Problem b's rows x[off[b] ..] split into (hi, lo) at rows pad[b] .. of the padded
+// operand buffers; the rows between its own count and the padded count are zero.
+__global__ void k_split_pad(const float *__restrict__ x, const int64_t *off, const int64_t *pad,
+                            int d, __nv_bfloat16 *__restrict__ hi,
+                            __nv_bfloat16 *__restrict__ lo) {
+  const int b = blockIdx.y;
+  const int64_t v4 = (off[b + 1] - off[b]) * d / 4;  // d is a multiple of 4
+  const int64_t n4 = (pad[b + 1] - pad[b]) * d / 4;
+  const float4 *src = reinterpret_cast<const float4 *>(x + off[b] * d);
+  uint2 *h = reinterpret_cast<uint2 *>(hi + pad[b] * d);
+  uint2 *l = reinterpret_cast<uint2 *>(lo + pad[b] * d);
   for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < n4;
        i += (int64_t)gridDim.x * blockDim.x) {
-    const float4 v = reinterpret_cast<const float4 *>(x)[i];
-    const float e[4] = {v.x, v.y, v.z, v.w};
-    __nv_bfloat16 h[4], l[4];
-#pragma unroll
-    for (int u = 0; u < 4; ++u) tc::split_bf16(e[u], h[u], l[u]);
-    uint2 hv, lv;
-    hv.x = (uint32_t)__bfloat16_as_ushort(h[0]) | ((uint32_t)__bfloat16_as_ushort(h[1]) << 16);
-    hv.y = (uint32_t)__bfloat16_as_ushort(h[2]) | ((uint32_t)__bfloat16_as_ushort(h[3]) << 16);
-    reinterpret_cast<uint2 *>(hi)[i] = hv;
-    if (lo) {
-      lv.x = (uint32_t)__bfloat16_as_ushort(l[0]) | ((uint32_t)__bfloat16_as_ushort(l[1]) << 16);
-      lv.y = (uint32_t)__bfloat16_as_ushort(l[2]) | ((uint32_t)__bfloat16_as_ushort(l[3]) << 16);
-      reinterpret_cast<uint2 *>(lo)[i] = lv;
-    }
+    const float4 v = i < v4 ? src[i] : make_float4(0.f, 0.f, 0.f, 0.f);
+    uint32_t h0, h1, l0, l1;
+    tc::split_pack(v.x, v.y, h0, l0);
+    tc::split_pack(v.z, v.w, h1, l1);
+    h[i] = make_uint2(h0, h1);
+    l[i] = make_uint2(l0, l1);
   }
 }
 
-int split(const float *x, __nv_bfloat16 *hi, __nv_bfloat16 *lo, int64_t n, cudaStream_t st) {
-  const int64_t n4 = n / 4;  // row length d is a multiple of 4
+// x [rows by off] -> padded (hi, lo) by pad; max_rows: the largest padded count.
+int split_pad(const float *x, const int64_t *off, const int64_t *pad, int64_t max_rows, int d,
+              __nv_bfloat16 *hi, __nv_bfloat16 *lo, int B, cudaStream_t st) {
+  const int64_t n4 = max_rows * d / 4;
   if (n4 == 0) return KVS_OK;
-  const int blocks = (int)std::min<int64_t>((n4 + 255) / 256, 148 * 16);
-  k_split<<<blocks, 256, 0, st>>>(x, hi, lo, n4);
-  KVS_LAUNCH_CHECK("k_split");
+  const int per = (int)std::max<int64_t>(1, std::min<int64_t>((n4 + 255) / 256,
+                                                              std::max(1, 4096 / B)));
+  k_split_pad<<<dim3(per, B), 256, 0, st>>>(x, off, pad, d, hi, lo);
+  KVS_LAUNCH_CHECK("k_split_pad");
   return KVS_OK;
 }
 
-// padded row offsets of the A buffer: pad[b] = sum_{b' < b} round_up(n_q_b', 128)
-__global__ void k_pad_offsets(const int64_t *q_off, int B, int64_t *pad) {
-  if (blockIdx.x == 0 && threadIdx.x == 0) {
-    int64_t s = 0;
-    pad[0] = 0;
-    for (int b = 0; b < B; ++b) {
-      const int64_t n = q_off[b + 1] - q_off[b];
-      s += (n + 127) / 128 * 128;
-      pad[b + 1] = s;
-    }
+// pad[b] = sum_{b' < b} round_up(n_b', 128) for the queries, zones and (when
+// present) pairs of the batch.
+__global__ void k_pad_offsets(const int64_t *q_off, const int64_t *z_off, const int64_t *c_off,
+                              int B, int64_t *qp, int64_t *zp, int64_t *cp) {
+  const int64_t *src[3] = {q_off, z_off, c_off};
+  int64_t *dst[3] = {qp, zp, cp};
+  const int k = threadIdx.x;
+  if (k >= 3 || !src[k]) return;
+  int64_t s = 0;
+  dst[k][0] = 0;
+  for (int b = 0; b < B; ++b) {
+    s += (src[k][b + 1] - src[k][b] + 127) / 128 * 128;
+    dst[k][b + 1] = s;
   }
 }
+
+int max_pad(int n) { return (n + 127) / 128 * 128; }
 
 // loss[b] from the per-CTA partial sums of the loss forward (fixed order).
 __global__ void k_loss_reduce(const float *partials, int tiles, const int64_t *q_off, int d,
@@ -214,21 +222,25 @@ int targets_d(const Batch &Bt, const float *Q, const float *Kz, const float *Vz,
               float *lse, float *imp, const Work &w) {
   const HostGeom &g = Bt.g;
   int rc;
-  if ((rc = split(Q, w.qh, w.ql, g.sum_q * D, Bt.st))) return rc;
-  if ((rc = split(Kz, w.kh, w.kl, g.sum_z * D, Bt.st))) return rc;
-  if ((rc = split(Vz, w.vh, w.vl, g.sum_z * D, Bt.st))) return rc;
-  FwdMaps fm;
-  if ((rc = make_map_bf16(&fm.kh, w.kh, g.sum_z, D, FWD_BN)) ||
-      (rc = make_map_bf16(&fm.kl, w.kl, g.sum_z, D, FWD_BN)) ||
-      (rc = make_map_bf16(&fm.vh, w.vh, g.sum_z, D, FWD_BN)) ||
-      (rc = make_map_bf16(&fm.vl, w.vl, g.sum_z, D, FWD_BN)))
+  const kvs_batch *bb = Bt.b;
+  if ((rc = split_pad(Q, bb->q_off, w.a_pad_off, max_pad(g.max_q), D, w.qh, w.ql, g.B, Bt.st)) ||
+      (rc = split_pad(Kz, bb->z_off, w.z_pad, max_pad(g.max_z), D, w.kh, w.kl, g.B, Bt.st)) ||
+      (rc = split_pad(Vz, bb->z_off, w.z_pad, max_pad(g.max_z), D, w.vh, w.vl, g.B, Bt.st)))
     return rc;
-  if ((rc = make_map_bf16(&fm.qh, w.qh, g.sum_q, D, FWD_BN)) ||
-      (rc = make_map_bf16(&fm.ql, w.ql, g.sum_q, D, FWD_BN)))
+  FwdMaps fm;
+  if ((rc = make_map_bf16(&fm.kh, w.kh, g.sum_zpad, D, FWD_BN)) ||
+      (rc = make_map_bf16(&fm.kl, w.kl, g.sum_zpad, D, FWD_BN)) ||
+      (rc = make_map_bf16(&fm.vh, w.vh, g.sum_zpad, D, FWD_BN)) ||
+      (rc = make_map_bf16(&fm.vl, w.vl, g.sum_zpad, D, FWD_BN)))
+    return rc;
+  if ((rc = make_map_bf16(&fm.qh, w.qh, g.sum_qpad, D, FWD_BN)) ||
+      (rc = make_map_bf16(&fm.ql, w.ql, g.sum_qpad, D, FWD_BN)))
     return rc;
   FwdArgs a{};
   a.q_off = Bt.b->q_off;
   a.k_off = Bt.b->z_off;
+  a.a_pad_off = w.a_pad_off;
+  a.k_pad = w.z_pad;
   a.q_hi = w.qh;
   a.q_lo = w.ql;
   a.flt = Filter{nullptr, 0, 0};
@@ -242,15 +254,17 @@ int targets_d(const Batch &Bt, const float *Q, const float *Kz, const float *Vz,
   if ((rc = launch_fwd_tc<D, FWD_TARGETS>(fm, a, max_qtiles(g), g.B, Bt.st))) return rc;
   if (!imp) return KVS_OK;
   BwdMaps bm;
-  if ((rc = make_map_bf16(&bm.kh, w.kh, g.sum_z, D, 128)) ||
-      (rc = make_map_bf16(&bm.kl, w.kl, g.sum_z, D, 128)) ||
-      (rc = make_map_bf16(&bm.qh, w.qh, g.sum_q, D, BWD_BQ)) ||
-      (rc = make_map_bf16(&bm.ql, w.ql, g.sum_q, D, BWD_BQ)))
+  if ((rc = make_map_bf16(&bm.kh, w.kh, g.sum_zpad, D, 128)) ||
+      (rc = make_map_bf16(&bm.kl, w.kl, g.sum_zpad, D, 128)) ||
+      (rc = make_map_bf16(&bm.qh, w.qh, g.sum_qpad, D, BWD_BQ)) ||
+      (rc = make_map_bf16(&bm.ql, w.ql, g.sum_qpad, D, BWD_BQ)))
     return rc;
   bm.g = bm.qh;
   BwdArgs ba{};
   ba.q_off = Bt.b->q_off;
   ba.k_off = Bt.b->z_off;
+  ba.q_pad = w.a_pad_off;
+  ba.k_pad = w.z_pad;
   ba.flt = Filter{nullptr, 0, 0};
   ba.scale = a.scale;
   ba.lse = lse;
@@ -264,9 +278,10 @@ int targets_d(const Batch &Bt, const float *Q, const float *Kz, const float *Vz,
 // bf16 hi/lo copies of the keys and values of the compressed pairs.
 template <int D>
 int prep_pairs(const Batch &Bt, const float *Kc, const float *Vc, const Work &w) {
-  int rc = split(Kc, w.kh, w.kl, Bt.g.sum_c * D, Bt.st);
+  const HostGeom &g = Bt.g;
+  int rc = split_pad(Kc, Bt.b->c_off, w.c_pad, max_pad(g.max_c), D, w.kh, w.kl, g.B, Bt.st);
   if (rc || !Vc) return rc;
-  return split(Vc, w.vh, w.vl, Bt.g.sum_c * D, Bt.st);
+  return split_pad(Vc, Bt.b->c_off, w.c_pad, max_pad(g.max_c), D, w.vh, w.vl, g.B, Bt.st);
 }
 
 template <int D>
@@ -275,20 +290,24 @@ int forward_d(const Batch &Bt, const float *Q, const float *Kc, const float *Vc,
               bool q_ready, bool pairs_ready, bool reduce, const Work &w) {
   const HostGeom &g = Bt.g;
   int rc;
-  if (!q_ready && (rc = split(Q, w.qh, w.ql, g.sum_q * D, Bt.st))) return rc;
+  if (!q_ready && (rc = split_pad(Q, Bt.b->q_off, w.a_pad_off, max_pad(g.max_q), D, w.qh, w.ql,
+                                  g.B, Bt.st)))
+    return rc;
   if (!pairs_ready && (rc = prep_pairs<D>(Bt, Kc, Vc, w))) return rc;
   FwdMaps fm;
-  if ((rc = make_map_bf16(&fm.kh, w.kh, g.sum_c, D, FWD_BN)) ||
-      (rc = make_map_bf16(&fm.kl, w.kl, g.sum_c, D, FWD_BN)) ||
-      (rc = make_map_bf16(&fm.vh, w.vh, g.sum_c, D, FWD_BN)) ||
-      (rc = make_map_bf16(&fm.vl, w.vl, g.sum_c, D, FWD_BN)))
+  if ((rc = make_map_bf16(&fm.kh, w.kh, g.sum_cpad, D, FWD_BN)) ||
+      (rc = make_map_bf16(&fm.kl, w.kl, g.sum_cpad, D, FWD_BN)) ||
+      (rc = make_map_bf16(&fm.vh, w.vh, g.sum_cpad, D, FWD_BN)) ||
+      (rc = make_map_bf16(&fm.vl, w.vl, g.sum_cpad, D, FWD_BN)))
     return rc;
-  if ((rc = make_map_bf16(&fm.qh, w.qh, g.sum_q, D, FWD_BN)) ||
-      (rc = make_map_bf16(&fm.ql, w.ql, g.sum_q, D, FWD_BN)))
+  if ((rc = make_map_bf16(&fm.qh, w.qh, g.sum_qpad, D, FWD_BN)) ||
+      (rc = make_map_bf16(&fm.ql, w.ql, g.sum_qpad, D, FWD_BN)))
     return rc;
   FwdArgs a{};
   a.q_off = Bt.b->q_off;
   a.k_off = Bt.b->c_off;
+  a.a_pad_off = w.a_pad_off;
+  a.k_pad = w.c_pad;
   a.q_hi = w.qh;
   a.q_lo = w.ql;
   a.flt = flt;
@@ -317,15 +336,17 @@ int backward_d(const Batch &Bt, float *dKc, Filter flt, const Work &w) {
   const HostGeom &g = Bt.g;
   int rc;
   BwdMaps bm;
-  if ((rc = make_map_bf16(&bm.kh, w.kh, g.sum_c, D, 128)) ||
-      (rc = make_map_bf16(&bm.kl, w.kl, g.sum_c, D, 128)) ||
-      (rc = make_map_bf16(&bm.qh, w.qh, g.sum_q, D, BWD_BQ)) ||
-      (rc = make_map_bf16(&bm.ql, w.ql, g.sum_q, D, BWD_BQ)) ||
-      (rc = make_map_bf16(&bm.g, w.go, g.sum_q, D, BWD_BQ)))
+  if ((rc = make_map_bf16(&bm.kh, w.kh, g.sum_cpad, D, 128)) ||
+      (rc = make_map_bf16(&bm.kl, w.kl, g.sum_cpad, D, 128)) ||
+      (rc = make_map_bf16(&bm.qh, w.qh, g.sum_qpad, D, BWD_BQ)) ||
+      (rc = make_map_bf16(&bm.ql, w.ql, g.sum_qpad, D, BWD_BQ)) ||
+      (rc = make_map_bf16(&bm.g, w.go, g.sum_qpad, D, BWD_BQ)))
     return rc;
   BwdArgs ba{};
   ba.q_off = Bt.b->q_off;
   ba.k_off = Bt.b->c_off;
+  ba.q_pad = w.a_pad_off;
+  ba.k_pad = w.c_pad;
   ba.flt = flt;
   ba.scale = 1.f / sqrtf((float)D);
   ba.lse = w.lse_h;
@@ -357,21 +378,28 @@ int fit_d(const Batch &Bt, const float *Q, const float *Kc, const float *Y, floa
           int32_t *status, bool q_ready, bool y_ready, Filter stats, const Work &w) {
   const HostGeom &g = Bt.g;
   int rc;
-  if (!q_ready && (rc = split(Q, w.qh, w.ql, g.sum_q * D, Bt.st))) return rc;
-  if (!y_ready && (rc = split(Y, w.yh, w.yl, g.sum_q * D, Bt.st))) return rc;
+  const kvs_batch *bb = Bt.b;
+  if (!q_ready && (rc = split_pad(Q, bb->q_off, w.a_pad_off, max_pad(g.max_q), D, w.qh, w.ql,
+                                  g.B, Bt.st)))
+    return rc;
+  if (!y_ready && (rc = split_pad(Y, bb->q_off, w.a_pad_off, max_pad(g.max_q), D, w.yh, w.yl,
+                                  g.B, Bt.st)))
+    return rc;
   if ((rc = prep_pairs<D>(Bt, Kc, nullptr, w))) return rc;
   FwdMaps fm;
-  if ((rc = make_map_bf16(&fm.kh, w.kh, g.sum_c, D, FWD_BN)) ||
-      (rc = make_map_bf16(&fm.kl, w.kl, g.sum_c, D, FWD_BN)))
+  if ((rc = make_map_bf16(&fm.kh, w.kh, g.sum_cpad, D, FWD_BN)) ||
+      (rc = make_map_bf16(&fm.kl, w.kl, g.sum_cpad, D, FWD_BN)))
     return rc;
-  if ((rc = make_map_bf16(&fm.qh, w.qh, g.sum_q, D, FWD_BN)) ||
-      (rc = make_map_bf16(&fm.ql, w.ql, g.sum_q, D, FWD_BN)))
+  if ((rc = make_map_bf16(&fm.qh, w.qh, g.sum_qpad, D, FWD_BN)) ||
+      (rc = make_map_bf16(&fm.ql, w.ql, g.sum_qpad, D, FWD_BN)))
     return rc;
   fm.vh = fm.kh;
   fm.vl = fm.kl;
   FwdArgs a{};
   a.q_off = Bt.b->q_off;
   a.k_off = Bt.b->c_off;
+  a.a_pad_off = w.a_pad_off;
+  a.k_pad = w.c_pad;
   a.q_hi = w.qh;
   a.q_lo = w.ql;
   a.flt = stats;  // problems whose l_hat in the workspace is not that of Kc
@@ -381,8 +409,6 @@ int fit_d(const Batch &Bt, const float *Q, const float *Kc, const float *Y, floa
   a.wait = wait_limit();
   if ((rc = launch_fwd_tc<D, FWD_STATS>(fm, a, max_qtiles(g), g.B, Bt.st))) return rc;
   a.flt = Filter{nullptr, 0, 0};
-  k_pad_offsets<<<1, 1, 0, Bt.st>>>(Bt.b->q_off, g.B, w.a_pad_off);
-  KVS_LAUNCH_CHECK("k_pad_offsets");
   a.lse_in = w.lse_h;
   a.a_hi = w.ahi;
   a.a_lo = w.alo;
@@ -407,11 +433,11 @@ int fit_d(const Batch &Bt, const float *Q, const float *Kc, const float *Y, floa
   ga.wait = wait_limit();
   const int tm = (g.max_c + 127) / 128;
   if ((rc = launch_gemm3_tc(gm, ga, tm, 1, g.B, Bt.st))) return rc;
-  if ((rc = make_map_bf16(&gm.bh, w.yh, g.sum_q, D, 64)) ||
-      (rc = make_map_bf16(&gm.bl, w.yl, g.sum_q, D, 64)))
+  if ((rc = make_map_bf16(&gm.bh, w.yh, g.sum_qpad, D, 64)) ||
+      (rc = make_map_bf16(&gm.bl, w.yl, g.sum_qpad, D, 64)))
     return rc;
   ga.n_fixed = D;
-  ga.b_row_off = Bt.b->q_off;
+  ga.b_row_off = w.a_pad_off;  // Y at the padded query rows: zero rows past each problem
   ga.c = w.R;
   ga.ldc = D;
   ga.diag = 0.f;
@@ -420,6 +446,13 @@ int fit_d(const Batch &Bt, const float *Q, const float *Kc, const float *Y, floa
 }
 
 }  // namespace
+
+int launch_pad_offsets(const Batch &Bt, const Work &w) {
+  k_pad_offsets<<<1, 32, 0, Bt.st>>>(Bt.b->q_off, Bt.b->z_off, Bt.b->c_off, Bt.g.B, w.a_pad_off,
+                                      w.z_pad, w.c_pad);
+  KVS_LAUNCH_CHECK("k_pad_offsets");
+  return KVS_OK;
+}
 
 int launch_targets(const Batch &Bt, const float *Q, const float *Kz, const float *Vz, float *Y,
                    float *lse, float *imp, const Work &w) {

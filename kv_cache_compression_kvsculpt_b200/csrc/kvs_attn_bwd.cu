@@ -119,7 +119,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
   if (warp == 8) {
     // ------------------------------------------------------------ producer
     if (lane == 0) {
-      const int krow = (int)(k_begin + k0);
+      const int krow = (int)(a.k_pad[b] + k0);
       mbar_arrive_expect_tx(&bars.k_full, 2 * C::K_BYTES);
       for (int r = 0; r < C::KD; ++r) {
         tma_load_2d(sm + r * BK * 128, &mKh, &bars.k_full, 64 * r, krow);
@@ -141,7 +141,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       if (lane == 0) {
         issued = i + 1;
         unsigned char *base = sm + C::OFF_ST + st * C::STAGE;
-        const int qrow = (int)(q_begin + (t0 + i) * BQ);
+        const int qrow = (int)(a.q_pad[b] + (t0 + i) * BQ);
         mbar_arrive_expect_tx(&bars.q_full[st], C::STAGE);
         for (int r = 0; r < C::KD; ++r) {
           tma_load_2d(base + r * BQ * 128, &mQh, &bars.q_full[st], 64 * r, qrow);
@@ -243,8 +243,8 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     if (C::DK) {
       // this warpgroup's half of the value row (hi, lo) into tensor memory: the A
       // operand of dP^T = V Go^T
-      const uint4 *vh = reinterpret_cast<const uint4 *>(a.v_hi + (k_begin + kr) * D);
-      const uint4 *vl = reinterpret_cast<const uint4 *>(a.v_lo + (k_begin + kr) * D);
+      const uint4 *vh = reinterpret_cast<const uint4 *>(a.v_hi + (a.k_pad[b] + kr) * D);
+      const uint4 *vl = reinterpret_cast<const uint4 *>(a.v_lo + (a.k_pad[b] + kr) * D);
 #pragma unroll 1
       for (int c0 = wg * 32; c0 < D / 2; c0 += 64) {
         uint32_t wh[32], wl[32];

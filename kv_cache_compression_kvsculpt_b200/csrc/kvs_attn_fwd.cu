@@ -149,8 +149,8 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     // ------------------------------------------------------------ TMA producer
     if (lane == 0) {
       tma_prefetch_map(&mKh);
-      // the CTA's query tile, hi and lo
-      const int qrow = (int)(q_begin + q0);
+      // the CTA's query tile, hi and lo (padded rows: zeros past the problem)
+      const int qrow = (int)(a.a_pad_off[b] + q0);
       mbar_arrive_expect_tx(&bars.q_full, 2 * C::T_BYTES);
       for (int r = 0; r < C::KD; ++r) {
         tma_load_2d(sm + r * BM * 128, &mQh, &bars.q_full, 64 * r, qrow);
@@ -163,7 +163,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
           return false;
         k_issued = j + 1;
         unsigned char *base = sm + C::OFF_K + st * 2 * C::T_BYTES;
-        const int krow = (int)(k_begin + j * BN);
+        const int krow = (int)(a.k_pad[b] + j * BN);
         mbar_arrive_expect_tx(&bars.k_full[st], 2 * C::T_BYTES);
         for (int r = 0; r < C::KD; ++r) {
           tma_load_2d(base + r * BN * 128, &mKh, &bars.k_full[st], 64 * r, krow);
@@ -177,7 +177,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
           return false;
         v_issued = j + 1;
         unsigned char *base = sm + C::OFF_V + st * 2 * C::T_BYTES;
-        const int krow = (int)(k_begin + j * BN);
+        const int krow = (int)(a.k_pad[b] + j * BN);
         mbar_arrive_expect_tx(&bars.v_full[st], 2 * C::T_BYTES);
         for (int r = 0; r < C::KD; ++r) {
           tma_load_2d(base + r * BN * 128, &mVh, &bars.v_full[st], 64 * r, krow);
@@ -402,6 +402,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       const float c_out = 2.f * a.w_out / ((float)nq * (float)D);
       const float c_lse = 2.f * a.w_lse / (float)nq;
       const int64_t grow = q_begin + q;
+      const int64_t prow = a.a_pad_off[b] + q;  // row of the padded bf16 buffers
       float se = 0.f, ls = 0.f, gy = 0.f;
       if (C::PV) {
         // this warpgroup's half of the row's output columns
@@ -410,7 +411,22 @@ __global__ void __launch_bounds__(NTHREADS, 1)
           float o[32], ob[32];
           tmem_ld32(tmem + lane_base + C::COL_O + c0, o);
           tmem_ld32(tmem + lane_base + C::COL_O + D + c0, ob);
-          if (!valid) continue;
+          if (!valid) {
+            // rows past the problem: zero padding of the bf16 operand buffers (this
+            // CTA's tile ends within the problem's padded rows)
+            const uint4 z4 = make_uint4(0u, 0u, 0u, 0u);
+            if (MODE == FWD_TARGETS) {
+#pragma unroll
+              for (int ch = 0; ch < 4; ++ch) {
+                reinterpret_cast<uint4 *>(a.y_hi + prow * D + c0)[ch] = z4;
+                reinterpret_cast<uint4 *>(a.y_lo + prow * D + c0)[ch] = z4;
+              }
+            } else {
+#pragma unroll
+              for (int ch = 0; ch < 4; ++ch) reinterpret_cast<uint4 *>(a.go + prow * D + c0)[ch] = z4;
+            }
+            continue;
+          }
 #pragma unroll
           for (int e = 0; e < 32; ++e) o[e] = (o[e] + ob[e]) * inv;  // O = O_a + O_b
           if (MODE == FWD_TARGETS) {
@@ -418,8 +434,8 @@ __global__ void __launch_bounds__(NTHREADS, 1)
 #pragma unroll
             for (int e = 0; e < 8; ++e)
               y4[e] = make_float4(o[4 * e], o[4 * e + 1], o[4 * e + 2], o[4 * e + 3]);
-            uint4 *yh = reinterpret_cast<uint4 *>(a.y_hi + grow * D + c0);
-            uint4 *yl = reinterpret_cast<uint4 *>(a.y_lo + grow * D + c0);
+            uint4 *yh = reinterpret_cast<uint4 *>(a.y_hi + prow * D + c0);
+            uint4 *yl = reinterpret_cast<uint4 *>(a.y_lo + prow * D + c0);
 #pragma unroll
             for (int ch = 0; ch < 4; ++ch) {
               uint32_t h[4], l[4];
@@ -440,7 +456,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
               ev[4 * e + 2] = o[4 * e + 2] - v.z;
               ev[4 * e + 3] = o[4 * e + 3] - v.w;
             }
-            uint4 *g4 = reinterpret_cast<uint4 *>(a.go + grow * D + c0);
+            uint4 *g4 = reinterpret_cast<uint4 *>(a.go + prow * D + c0);
 #pragma unroll
             for (int ch = 0; ch < 4; ++ch) {
               uint32_t h[4];

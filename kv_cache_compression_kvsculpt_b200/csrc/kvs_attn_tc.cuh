@@ -46,7 +46,8 @@ struct FwdArgs {
   // WRITE_A
   __nv_bfloat16 *a_hi, *a_lo;  // [sum padded q, ld_a]
   int64_t ld_a;
-  const int64_t *a_pad_off;    // [B+1] padded query-row offsets of the A buffer
+  const int64_t *a_pad_off;    // [B+1] padded query rows of q_hi/lo, go, y_hi/lo and the A buffer
+  const int64_t *k_pad;        // [B+1] padded key / value rows of the bf16 key and value maps
   int *err;               // timeout flag
   long long wait;         // cycles a pipeline wait may spin (wait_limit())
 };
@@ -63,7 +64,8 @@ struct BwdArgs {
   float scale;
   const float *lse;       // [sum_q] row lse used to form the probabilities
   const float *delta;     // [sum_q] (DK)
-  const __nv_bfloat16 *v_hi, *v_lo;  // [sum_k, d] value split (DK; loaded into tensor memory)
+  const __nv_bfloat16 *v_hi, *v_lo;  // [padded k, d] value split (DK; loaded into tensor memory)
+  const int64_t *q_pad, *k_pad;      // [B+1] padded rows of the query / Go and key / value maps
   float *dk;              // [sum_k, d] (DK): dL/dK, or nsplit partial sums dk_stride apart
   float *imp;             // [sum_k] (COLSUM): column sums of probabilities
   int *err;

@@ -75,6 +75,8 @@ struct HostGeom {
   int64_t sum_q = 0, sum_z = 0, sum_c = 0;
   int max_q = 0, max_z = 0, max_c = 0;
   int64_t sum_qpad = 0;  // sum over problems of n_q rounded up to 128
+  int64_t sum_zpad = 0;  // ... of z rounded up to 128
+  int64_t sum_cpad = 0;  // ... of k rounded up to 128
   int64_t ld_a = 0;      // columns of the attention-weight buffer (max_c rounded up to 128)
   int64_t ld_g = 0;      // columns of the Gram / factor buffer (max_c rounded up to 4)
 };

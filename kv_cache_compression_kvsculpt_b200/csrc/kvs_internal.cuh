@@ -7,6 +7,9 @@
 
 namespace kvs {
 
+// Most sub-batches a solve runs concurrently (kvs_compress_batch).
+constexpr int KVS_MAX_PARTS = 4;
+
 // L-BFGS line-search phase of a problem.
 enum Phase : int { PH_IDLE = 0, PH_SEARCH = 1, PH_ACCEPT = 2, PH_FAIL = 3 };
 
@@ -28,17 +31,21 @@ struct LbfgsScal {
 };
 
 // Scratch buffers carved from the caller's workspace.
+// The bf16 operand copies hold each problem's rows at padded offsets (rows
+// rounded up to 128 per problem) with zero rows in the padding.
 struct Work {
-  __nv_bfloat16 *qh, *ql;    // [sum_q, d]             training queries, hi/lo
-  __nv_bfloat16 *kh, *kl;    // [max(sum_z, sum_c), d] keys, hi/lo
-  __nv_bfloat16 *vh, *vl;    // [max(sum_z, sum_c), d] values, hi (and lo for targets)
-  __nv_bfloat16 *go;         // [sum_q, d]             dloss/dY_hat
-  __nv_bfloat16 *yh, *yl;    // [sum_q, d]             targets Y, hi/lo
+  __nv_bfloat16 *qh, *ql;    // [sum_qpad, d]          training queries, hi/lo
+  __nv_bfloat16 *kh, *kl;    // [max(zpad, cpad), d]   keys, hi/lo
+  __nv_bfloat16 *vh, *vl;    // [max(zpad, cpad), d]   values, hi/lo
+  __nv_bfloat16 *go;         // [sum_qpad, d]          dloss/dY_hat
+  __nv_bfloat16 *yh, *yl;    // [sum_qpad, d]          targets Y, hi/lo
   __nv_bfloat16 *ahi, *alo;  // [sum_qpad, ld_a]       attention weights for the ridge fit
   float *lse_h;              // [sum_q]                row lse of the compressed keys
   float *delta;              // [sum_q]
   float *partials;           // [B, max q tiles, 2]    per-CTA loss sums
-  int64_t *a_pad_off;        // [B+1]                  padded row offsets of ahi/alo
+  int64_t *a_pad_off;        // [B+1]                  padded query-row offsets (qh, ql, go,
+                             //                        yh, yl, ahi, alo): n_q rounded up to 128
+  int64_t *z_pad, *c_pad;    // [B+1] each             padded zone / pair rows of kh .. vl
   float *gram;               // [sum_c, ld_g]          A^T A + lam I, then its Cholesky factor
   float *R;                  // [sum_c, d]             A^T Y, then the forward-solved rows
   float *X;                  // [sum_c, d]             solution of the ridge system
@@ -97,9 +104,13 @@ struct Batch {
   HostGeom g;
   const kvs_batch *b;
   cudaStream_t st;
+  int slot = 0;  // sub-batch index of a partitioned solve (its own internal streams)
 };
 
 // ---- attention contractions (kvs_attn.cu) ----
+// Padded row offsets of the batch's queries, zones and (if any) pairs into the
+// workspace (w.a_pad_off, w.z_pad, w.c_pad).
+int launch_pad_offsets(const Batch &B, const Work &w);
 // targets: Y, lse and (optionally) importance; leaves the Q split in w.qh/ql
 // and the Y split in w.yh/yl.
 int launch_targets(const Batch &B, const float *Q, const float *Kz, const float *Vz, float *Y,
@@ -133,7 +144,8 @@ int launch_chol_solve(const Batch &B, float *Vc, int32_t *status, const Work &w)
 int launch_lbfgs_reset(const Batch &B, const State &s, const float *Kc, const float *f,
                        const float *g, int clear);
 int launch_lbfgs_direction(const Batch &B, const State &s, const kvs_schedule &sc);
-// Kc = x + t d for searching problems, with its bf16 hi/lo split into w.kh/w.kl.
+// Kc = x + t d for searching problems, with its bf16 hi/lo split into w.kh/w.kl
+// (at the padded pair rows).
 int launch_lbfgs_trial(const Batch &B, const State &s, float *Kc, const Work &w);
 // Armijo test on the trial loss summed from the forward's per-CTA partials;
 // with `cond`, also sets that graph condition to "a problem is still searching".

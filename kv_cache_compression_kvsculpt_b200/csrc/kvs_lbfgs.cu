@@ -351,10 +351,11 @@ __global__ void __launch_bounds__(PT) k_direction(LbfgsScal *sc, const DirCoef *
 __global__ void k_trial(const LbfgsScal *sc, const float *__restrict__ x,
                         const float *__restrict__ dir, float *__restrict__ Kc,
                         __nv_bfloat16 *__restrict__ kh, __nv_bfloat16 *__restrict__ kl,
-                        const int64_t *c_off, int d) {
+                        const int64_t *c_off, const int64_t *c_pad, int d) {
   const int b = blockIdx.y;
   if (sc[b].phase != PH_SEARCH) return;
   const int64_t o = seg0(c_off, b, d), n = c_off[b + 1] * (int64_t)d - o;
+  const int64_t op = c_pad[b] * (int64_t)d;  // the split at the padded pair rows
   const float t = sc[b].t;
   for (int64_t i = 2 * (blockIdx.x * (int64_t)blockDim.x + threadIdx.x); i < n;
        i += 2 * (int64_t)gridDim.x * blockDim.x) {
@@ -364,8 +365,8 @@ __global__ void k_trial(const LbfgsScal *sc, const float *__restrict__ x,
     *reinterpret_cast<float2 *>(Kc + o + i) = make_float2(k0, k1);
     const __nv_bfloat162 h = __floats2bfloat162_rn(k0, k1);
     const float2 hf = __bfloat1622float2(h);
-    *reinterpret_cast<__nv_bfloat162 *>(kh + o + i) = h;
-    *reinterpret_cast<__nv_bfloat162 *>(kl + o + i) = __floats2bfloat162_rn(k0 - hf.x, k1 - hf.y);
+    *reinterpret_cast<__nv_bfloat162 *>(kh + op + i) = h;
+    *reinterpret_cast<__nv_bfloat162 *>(kl + op + i) = __floats2bfloat162_rn(k0 - hf.x, k1 - hf.y);
   }
 }
 
@@ -457,7 +458,7 @@ int launch_lbfgs_trial(const Batch &Bt, const State &s, float *Kc, const Work &w
   const int64_t n = (int64_t)Bt.g.max_c * Bt.g.d / 2;
   const int blocks = (int)std::min<int64_t>((n + 255) / 256, 64);
   k_trial<<<dim3(blocks, Bt.g.B), 256, 0, Bt.st>>>(s.sc, s.x, s.dir, Kc, w.kh, w.kl,
-                                                   Bt.b->c_off, Bt.g.d);
+                                                   Bt.b->c_off, w.c_pad, Bt.g.d);
   KVS_LAUNCH_CHECK("k_trial");
   return KVS_OK;
 }

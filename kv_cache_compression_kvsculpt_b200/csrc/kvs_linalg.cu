@@ -602,24 +602,26 @@ __global__ void __launch_bounds__(256) k_chol_store(CholArgs a, float *Vc) {
 
 }  // namespace
 
-// A side stream (highest priority) and two events per host thread and device: the
-// next panel's diagonal block and panel run on the side stream while the caller's
-// stream finishes the current trailing update (disjoint tiles).  Per-thread objects
-// keep concurrent callers from sharing events; they are created on a thread's first
-// solve and kept for the life of the process (three handles per thread and device).
+// A side stream (highest priority) and two events per host thread, device and
+// sub-batch slot: the next panel's diagonal block and panel run on the side stream
+// while the caller's stream finishes the current trailing update (disjoint tiles).
+// Per-thread objects keep concurrent callers from sharing events, and per-slot ones
+// the concurrent sub-batches of one solve; they are created on first use and kept
+// for the life of the process (three handles per thread, device and slot).
 struct Lookahead {
   cudaStream_t side = nullptr;
   cudaEvent_t fork = nullptr, join = nullptr;
 };
 
-static cudaError_t lookahead(Lookahead **out) {
+static cudaError_t lookahead(int slot, Lookahead **out) {
   constexpr int kMaxDev = 64;
-  static thread_local Lookahead la[kMaxDev];
+  static thread_local Lookahead la[kMaxDev][KVS_MAX_PARTS];
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
-  if (dev < 0 || dev >= kMaxDev) return cudaErrorInvalidDevice;
-  Lookahead &l = la[dev];
+  if (dev < 0 || dev >= kMaxDev || slot < 0 || slot >= KVS_MAX_PARTS)
+    return cudaErrorInvalidDevice;
+  Lookahead &l = la[dev][slot];
   if (!l.side) {
     // the highest priority: the next panel's few CTAs take SMs as soon as update
     // CTAs retire instead of queueing behind all of them
@@ -640,7 +642,7 @@ int launch_chol_solve(const Batch &Bt, float *Vc, int32_t *status, const Work &w
   CholArgs a{w.gram, w.R, w.X, w.chol_t, npanel, w.dead, status, Bt.b->c_off, g.ld_g, g.d};
   KVS_CUDA_TRY(set_smem_once(k_chol_backward, BWD_SMEM));
   Lookahead *la = nullptr;
-  KVS_CUDA_TRY(lookahead(&la));
+  KVS_CUDA_TRY(lookahead(Bt.slot, &la));
   KVS_CUDA_TRY(cudaMemsetAsync(w.dead, 0, sizeof(int) * g.B, Bt.st));
   const int ndc = g.d / NB;
   // diagonal block and panel p: their grid depends only on the longest problem

@@ -21,7 +21,13 @@ Inputs are the training queries built by the oracle and rounded to float32
 workload's float32 zone keys and values.  Checksums of those inputs are stored
 so that a test can tell when the generator has changed.
 
-Run:  python tests/golden/make_fullsize.py   (about 15 minutes on 8 cores)
+Each solve is also repeated with loss and gradient evaluations perturbed at the
+relative precision of the library's arithmetic (oracle.perturb, two seeds):
+the final losses of those runs ("band") show how far a run of that precision
+can legitimately end from the exact one on this (non-convex, fixed-length)
+trajectory.  The adaptive case's band is taken at the oracle's allocation.
+
+Run:  python tests/golden/make_fullsize.py   (about 45 minutes on 8 cores)
 """
 from __future__ import annotations
 
@@ -37,6 +43,9 @@ sys.path.insert(0, ROOT)
 
 import oracle as O  # noqa: E402
 import workload as W  # noqa: E402
+from oracle.perturb import GPU_LEVELS, noisy_evaluations  # noqa: E402
+
+BAND_SEEDS = 2
 
 OUT = os.path.join(os.path.dirname(os.path.abspath(__file__)), "fullsize_oracle.json")
 
@@ -76,6 +85,12 @@ def result_record(r):
             "status": int(r["status"]), "trials": int(r["trials"])}
 
 
+def band(Q, Kz, Vz, k, sched):
+    """Final losses of the schedule with perturbed evaluations (oracle.perturb)."""
+    return [float(O.compress(Q, Kz, Vz, k, sched, evaluate=noisy_evaluations(*GPU_LEVELS, s))
+                  ["loss"]) for s in range(BAND_SEEDS)]
+
+
 def uniform_case(name, ids):
     wl = W.WORKLOADS[name]
     t0 = time.time()
@@ -83,6 +98,7 @@ def uniform_case(name, ids):
     for (Q, Kz, Vz), pid in zip(float32_inputs(wl, ids), ids):
         r = O.compress(Q, Kz, Vz, wl.k, schedule(wl))
         rec = result_record(r)
+        rec["band"] = band(Q, Kz, Vz, wl.k, schedule(wl))
         rec.update(id=list(pid), k=wl.k, checksum_Q=checksum(Q), checksum_Kz=checksum(Kz),
                    checksum_Vz=checksum(Vz))
         probs.append(rec)
@@ -100,6 +116,7 @@ def adaptive_case(ids):
     probs = []
     for b, (pid, (Q, Kz, Vz)) in enumerate(zip(ids, inp)):
         rec = result_record(res["results"][b])
+        rec["band"] = band(Q, Kz, Vz, int(res["k"][b]), schedule(wl))
         rec.update(id=list(pid), k=int(res["k"][b]), pilot_mse=float(res["pilot_mse"][b]),
                    checksum_Q=checksum(Q), checksum_Kz=checksum(Kz), checksum_Vz=checksum(Vz))
         probs.append(rec)
@@ -108,7 +125,8 @@ def adaptive_case(ids):
 
 
 def main():
-    out = {"generator": "tests/golden/make_fullsize.py (oracle/ only)", "seed": 0, "cases": {}}
+    out = {"generator": "tests/golden/make_fullsize.py (oracle/ only)", "seed": 0,
+           "band_levels": list(GPU_LEVELS), "cases": {}}
     for name in ("qwen_cache_r03", "qwen_cache_r05", "qwen_cache_r07"):
         out["cases"][name] = uniform_case(name, CACHE_IDS)
     out["cases"]["qwen_cache_adaptive"] = adaptive_case(ADAPTIVE_IDS)

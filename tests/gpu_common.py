@@ -71,3 +71,38 @@ class Case:
 
     def targets_oracle(self, b):
         return O.targets(self.Qs[b], self.Zk[b], self.Zv[b])
+
+
+# Final-loss parity of the whole (non-convex, fixed-length) schedule.  The
+# oracle's run is repeated with its loss and gradient evaluations perturbed at
+# the relative precision of the library's arithmetic (oracle.perturb); the
+# final losses of those runs and of the exact run span a band that arithmetic
+# of that precision can legitimately reach.  The GPU's final loss must lie
+# within 5 % of that band.  A trajectory whose band spans more than a factor
+# 1.25 is ill-conditioned (a tiny change of the arithmetic sends it elsewhere):
+# there the result is only required to improve on Select+Fit.
+ILL_CONDITIONED = 0.25
+
+
+def final_loss_bar(f_or, band, bar=0.05):
+    """(low, high, spread) of the accepted final losses."""
+    vals = [float(f_or)] + [float(v) for v in band]
+    lo, hi = min(vals), max(vals)
+    return lo * (1 - bar), hi * (1 + bar), hi / lo - 1.0
+
+
+def oracle_band(Q, Kz, Vz, k, sched, seeds=3):
+    """Final losses of the oracle's schedule with perturbed evaluations."""
+    from oracle.perturb import GPU_LEVELS, noisy_evaluations
+    return [float(O.compress(Q, Kz, Vz, k, sched, evaluate=noisy_evaluations(*GPU_LEVELS, s))
+                  ["loss"]) for s in range(seeds)]
+
+
+def check_final_loss(f_gpu, f_sf, f_or, band, what=""):
+    """Assert the parity bar above; returns 'ok' or 'ill-conditioned'."""
+    lo, hi, spread = final_loss_bar(f_or, band)
+    if spread > ILL_CONDITIONED:
+        assert f_gpu < f_sf, (what, f_gpu, f_sf)
+        return "ill-conditioned"
+    assert lo - 1e-7 <= f_gpu <= hi + 1e-7, (what, f_gpu, f_or, band, f_gpu / f_or)
+    return "ok"
