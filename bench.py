@@ -160,11 +160,13 @@ def group_size(group):
 class Job:
     """Device buffers of one rank's batch and the calls of one step."""
 
-    def __init__(self, wl, seqs, dev, group=None):
+    def __init__(self, wl, seqs, dev, group=None, problems=None):
         import torch
         import kv_cache_compression_kvsculpt_b200 as K
         self.K, self.torch, self.wl, self.group = K, torch, wl, group
         ids = [(s, l, h) for s in seqs for l in range(wl.n_layers) for h in range(wl.n_kv_heads)]
+        if problems:
+            ids = ids[:problems]  # a reduced batch (kernel profiling)
         self.bt = W.make_batch(wl, 0, ids)
         B = self.bt.B
         self.host = {
@@ -282,6 +284,47 @@ def loss_grad_roofline(job, peaks, reps=20):
     return ms, flops, achieved
 
 
+def run_loss_grad_only(args, job, wl, rank, world, dist):
+    """The dominant evaluation alone: kvs_loss_grad over the batch at its Select+Fit
+    point (one solve with no outer iterations first), `--steps` timed calls after
+    `--warmup` untimed ones.  A kernel-level measurement, not the bench step."""
+    torch, K = job.torch, job.K
+    job.sched.outer = 0
+    job.step()
+    B = job.batch.B
+    Y = torch.empty_like(job.Q)
+    lse = torch.empty(job.batch.sum_q, device=job.Q.device)
+    K.kvs_targets(job.batch, job.Q, job.dev["Kz"], job.dev["Vz"], Y, lse, None, job.ws)
+    loss = torch.empty(B, device=job.Q.device)
+    dK = torch.empty_like(job.Kc)
+
+    def ev():
+        K.kvs_loss_grad(job.batch, job.Q, job.Kc, job.Vc, Y, lse, 1.0, 1.0, loss, None, dK, job.ws)
+
+    for _ in range(args.warmup):
+        ev()
+    ms = time_region(torch, ev, args.steps, dist) / args.steps
+    # each call on its own, with the finiteness of its results (a kernel whose
+    # bounded wait gave up returns NaN)
+    per, bad = [], 0
+    for _ in range(args.steps):
+        per.append(time_region(torch, ev, 1, dist))
+        bad += int(not (torch.isfinite(loss).all() and torch.isfinite(dK).all()))
+    flops = 8.0 * wl.n_q * wl.k * wl.d * B
+    peaks, peak_src = load_peaks()
+    peak = peaks.get(args.peak_key, FALLBACK_PEAKS.get(args.peak_key))
+    if rank == 0:
+        print(json.dumps({"metric": "kvs_loss_grad ms per call (whole batch)", "value": round(ms, 4),
+                          "unit": "ms", "problems": B, "workload": wl.name,
+                          "achieved_tflops": round(flops / (ms * 1e-3) / 1e12, 2),
+                          "frac": round(flops / (ms * 1e-3) / 1e12 / peak, 4),
+                          "per_call_ms": {"min": round(min(per), 4), "median":
+                                          round(statistics.median(per), 4),
+                                          "max": round(max(per), 4)},
+                          "calls_with_nan": bad,
+                          "peak_source": f"{peak_src} {args.peak_key}"}), flush=True)
+
+
 def run_gpu(args):
     import torch
     import kv_cache_compression_kvsculpt_b200 as K
@@ -300,7 +343,10 @@ def run_gpu(args):
     if args.outer is not None:
         wl = wl.with_(outer=args.outer)
     seqs, scaling = rank_sequences(wl, rank, world)
-    job = Job(wl, seqs, dev="cuda", group=dist.group.WORLD if dist else None)
+    job = Job(wl, seqs, dev="cuda", group=dist.group.WORLD if dist else None,
+              problems=args.problems)
+    if args.loss_grad_only:
+        return run_loss_grad_only(args, job, wl, rank, world, dist)
     for _ in range(args.warmup):
         job.step()
     torch.cuda.synchronize()
@@ -547,6 +593,10 @@ def main():
     ap.add_argument("--workload", default="qwen_cache_r05", choices=sorted(W.WORKLOADS))
     ap.add_argument("--outer", type=int, default=None, help="override the outer iterations")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--problems", type=int, default=None,
+                    help="only the first N problems of the workload (kernel profiling)")
+    ap.add_argument("--loss-grad-only", action="store_true",
+                    help="time kvs_loss_grad alone (kernel measurement, not the bench step)")
     ap.add_argument("--cpu-budget", type=float, default=20.0)
     ap.add_argument("--bound", default="tensor")
     ap.add_argument("--peak-key", default="bf16_tflops")

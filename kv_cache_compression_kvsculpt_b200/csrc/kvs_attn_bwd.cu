@@ -8,20 +8,27 @@
 //
 // One CTA owns 128 keys of one problem and streams its training queries in
 // tiles of 64.  Per tile, with A = exp(S - l_row):
-//   S^T  = K Q^T                    K_hi Q_hi + K_lo Q_hi + K_hi Q_lo  (K in smem)
-//   DK:     dP^T = V Go^T           V_hi Go + V_lo Go  (V in TMEM, Go bf16; delta was
-//                                   formed from the same rounded Go)
-//           dS = A (dP - delta_row) written as bf16 hi/lo over the S buffer in TMEM
-//           dK += dS Q              dS_hi Q_hi + dS_hi Q_lo + dS_lo Q_hi
+//   S^T  = K Q^T      K_hi [Q_hi | Q_lo] (one N = 128 product into two column
+//                     halves) + K_lo Q_hi (into the first half); S = sum of the
+//                     halves, i.e. K_hi Q_hi + K_hi Q_lo + K_lo Q_hi  (K in smem)
+//   DK:  dP^T = V Go^T  V_hi Go + V_lo Go  (V in TMEM, Go bf16; delta was formed
+//                       from the same rounded Go)
+//        dS = A (dP - delta_row), written as bf16 hi/lo over the tile's dP buffer
+//        dK += dS Q     dS_hi Q_hi + dS_hi Q_lo + dS_lo Q_hi  (Q as the N-major operand)
 //   COLSUM: importance += sum over the tile's queries of A
 // Near an optimum the key gradient is a small sum of large terms, so every
-// product keeps about 16 significant bits.
-// Tensor memory (512 columns): S buffers at 0 and 64, dP at 128 and 192,
-// dK at 256, V hi at 384, V lo at 384 + D/2.
-// Two row warpgroups take alternate query tiles (each owns one of the two S /
-// dP buffers).  Warp roles: warps 0-7 one thread per key row (warp w <-> TMEM
-// lanes 32 (w % 4) ..), warp 8 TMA producer (also stages l and delta of the
-// tile), warp 9 MMA issuer.
+// product keeps about 16 significant bits.  Each tcgen05.mma instruction costs
+// about the same for any N up to 128, so the score product takes Q_hi and Q_lo
+// side by side: two instructions per 16-deep step instead of three.
+// Tensor memory (512 columns, DK): one S buffer (two 64-column halves) at 0,
+// dP / dS buffers at 128 and 192 (one per tile parity), dK at 256, V hi at 384,
+// V lo at 384 + D/2.  COLSUM: two S buffers at 0 and 128.
+// DK issue order: S(i), dP(i), dK(i-1): the next tile's scores run while the
+// row threads form dS of the last tile, and dP(i + 2) reuses the buffer of dS(i)
+// once dK(i) has drained it, behind S(i + 2) in the tensor pipe.
+// Two row warpgroups take alternate query tiles.  Warp roles: warps 0-7 one
+// thread per key row (warp w <-> TMEM lanes 32 (w % 4) ..), warp 8 TMA
+// producer (also stages l and delta of the tile), warp 9 MMA issuer.
 #include <math.h>
 
 #include "kvs_attn_tc.cuh"
@@ -43,13 +50,17 @@ struct Bwd {
   static constexpr bool DK = (MODE == BWD_DK);
   static constexpr int NS = NSTAGE;
   static constexpr int K_BYTES = BK * D * 2;   // one copy of the key tile
-  static constexpr int Q_BYTES = BQ * D * 2;   // one copy of a query tile
-  static constexpr int STAGE = (DK ? 3 : 2) * Q_BYTES;  // Q hi, Q lo (, Go)
+  static constexpr int QB = BQ * 128;          // one 64-column box of a query tile
+  static constexpr int Q_BYTES = KD * QB;      // one copy of a query tile
+  // stage: per 64-column box r, Q_hi then Q_lo (the score product reads them as one
+  // N = 2 BQ operand); then the Go boxes
+  static constexpr int STAGE = (DK ? 3 : 2) * Q_BYTES;
+  static constexpr int OFF_GO = 2 * Q_BYTES;
   static constexpr int OFF_ST = 2 * K_BYTES;
   static constexpr int BYTES = OFF_ST + NS * STAGE;
   static constexpr int SMEM = BYTES + 1024;
-  static constexpr uint32_t TMEM_COLS = DK ? 512 : 128;
-  static constexpr uint32_t COL_DP = 128;
+  static constexpr uint32_t TMEM_COLS = DK ? 512 : 256;
+  static constexpr uint32_t COL_DP = 128;      // DK: dP / dS buffers, 64 columns each
   static constexpr uint32_t COL_DK = 256;
   static constexpr uint32_t COL_V = 384;
 };
@@ -57,8 +68,9 @@ struct Bwd {
 struct BwdBars {
   uint64_t k_full, v_full;
   uint64_t q_full[NSTAGE], q_empty[NSTAGE];
-  uint64_t sd_full[2], sd_free[2];
-  uint64_t ds_full[2];
+  uint64_t s_full[2];               // S of tile i done: [i & 1]
+  uint64_t s_free[2];               // S read by the rows: DK [0] (one buffer), COLSUM [i & 1]
+  uint64_t dp_full[2], ds_full[2], dk_done[2];  // DK, per tile parity
   uint64_t done;
   uint32_t tmem;
   int abort;
@@ -101,9 +113,11 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       mbar_init(&bars.q_empty[i], 1 + BK);
     }
     for (int i = 0; i < 2; ++i) {
-      mbar_init(&bars.sd_full[i], 1);
-      mbar_init(&bars.sd_free[i], C::DK ? 1 : BK);
+      mbar_init(&bars.s_full[i], 1);
+      mbar_init(&bars.s_free[i], BK);
+      mbar_init(&bars.dp_full[i], 1);
       mbar_init(&bars.ds_full[i], BK);
+      mbar_init(&bars.dk_done[i], 1);
     }
     mbar_init(&bars.done, 1);
     bars.abort = 0;
@@ -144,10 +158,10 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         const int qrow = (int)(a.q_pad[b] + (t0 + i) * BQ);
         mbar_arrive_expect_tx(&bars.q_full[st], C::STAGE);
         for (int r = 0; r < C::KD; ++r) {
-          tma_load_2d(base + r * BQ * 128, &mQh, &bars.q_full[st], 64 * r, qrow);
-          tma_load_2d(base + C::Q_BYTES + r * BQ * 128, &mQl, &bars.q_full[st], 64 * r, qrow);
+          tma_load_2d(base + 2 * r * C::QB, &mQh, &bars.q_full[st], 64 * r, qrow);
+          tma_load_2d(base + (2 * r + 1) * C::QB, &mQl, &bars.q_full[st], 64 * r, qrow);
           if (C::DK)
-            tma_load_2d(base + 2 * C::Q_BYTES + r * BQ * 128, &mG, &bars.q_full[st], 64 * r, qrow);
+            tma_load_2d(base + C::OFF_GO + r * C::QB, &mG, &bars.q_full[st], 64 * r, qrow);
         }
       }
       for (int e = lane; e < BQ; e += 32) {
@@ -167,66 +181,88 @@ __global__ void __launch_bounds__(NTHREADS, 1)
   } else if (warp == 9) {
     // ------------------------------------------------------------- MMA issuer
     if (lane == 0) {
-      const uint32_t id_s = idesc_bf16(BK, BQ, false, false);
+      const uint32_t id_s2 = idesc_bf16(BK, 2 * BQ, false, false);  // K_hi [Q_hi | Q_lo]
+      const uint32_t id_s1 = idesc_bf16(BK, BQ, false, false);      // K_lo Q_hi, V Go
       const uint32_t id_dk = idesc_bf16(BK, D, false, true);
       bool ok = mbar_wait(&bars.k_full, 0, abort, a.wait);
       fence_after_sync();
       const uint64_t kh0 = sdesc(smem_u32(sm), 16, 1024), kl0 = sdesc_add(kh0, C::K_BYTES);
       const uint32_t tv_hi = tmem + C::COL_V, tv_lo = tmem + C::COL_V + D / 2;
+      // S^T of tile i into the S buffer at column col
+      auto issue_s = [&](int i, uint32_t col) {
+        const uint32_t base = smem_u32(sm + C::OFF_ST + (i % C::NS) * C::STAGE);
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const int r = kk >> 2;
+          const uint32_t in = (kk & 3) * 32;
+          const uint64_t kh = sdesc_add(kh0, r * (BK * 128) + in), kl = sdesc_add(kl0, r * (BK * 128) + in);
+          const uint64_t qcat = sdesc(base + 2 * r * C::QB + in, 16, 1024);  // Q_hi box r, Q_lo box r
+          mma_bf16(tmem + col, kh, qcat, id_s2, kk > 0 ? 1u : 0u);
+          mma_bf16(tmem + col, kl, qcat, id_s1, 1u);  // first N = BQ rows: Q_hi
+        }
+      };
+      // dP^T of tile i into dP buffer i & 1
+      auto issue_dp = [&](int i) {
+        const uint32_t base = smem_u32(sm + C::OFF_ST + (i % C::NS) * C::STAGE + C::OFF_GO);
+        const uint32_t col = C::COL_DP + (i & 1) * BQ;
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint64_t gd = sdesc(base + (kk >> 2) * C::QB + (kk & 3) * 32, 16, 1024);
+          mma_bf16_ts(tmem + col, tv_hi + kk * 8, gd, id_s1, kk > 0 ? 1u : 0u);
+          mma_bf16_ts(tmem + col, tv_lo + kk * 8, gd, id_s1, 1u);
+        }
+      };
+      // dK += dS(i) Q(i): dS hi / lo over dP buffer i & 1, Q as the N-major operand
+      // (64-wide d blocks of Q_hi 2 QB apart, Q_lo one box further)
       auto issue_dk = [&](int i) -> bool {
         const int db = i & 1;
         if (!mbar_wait(&bars.ds_full[db], (i >> 1) & 1, abort, a.wait)) return false;
         fence_after_sync();
-        const uint64_t qh0 = sdesc(smem_u32(sm + C::OFF_ST + (i % C::NS) * C::STAGE), BQ * 128,
-                                   1024);
-        const uint64_t ql0 = sdesc_add(qh0, C::Q_BYTES);
-        const uint32_t tds = tmem + db * BQ;  // dS hi at +0, lo at +32 columns
+        const uint32_t base = smem_u32(sm + C::OFF_ST + (i % C::NS) * C::STAGE);
+        const uint64_t qh0 = sdesc(base, 2 * C::QB, 1024), ql0 = sdesc(base + C::QB, 2 * C::QB, 1024);
+        const uint32_t tds = tmem + C::COL_DP + db * BQ;  // dS hi at +0, lo at +BQ/2 columns
 #pragma unroll
         for (int kk = 0; kk < BQ / 16; ++kk) {
           const uint64_t qh = sdesc_add(qh0, kk * 2048), ql = sdesc_add(ql0, kk * 2048);
           mma_bf16_ts(tmem + C::COL_DK, tds + kk * 8, qh, id_dk, (i > 0 || kk > 0) ? 1u : 0u);
           mma_bf16_ts(tmem + C::COL_DK, tds + kk * 8, ql, id_dk, 1u);
-          mma_bf16_ts(tmem + C::COL_DK, tds + 32 + kk * 8, qh, id_dk, 1u);
+          mma_bf16_ts(tmem + C::COL_DK, tds + BQ / 2 + kk * 8, qh, id_dk, 1u);
         }
         mma_commit(&bars.q_empty[i % C::NS]);
-        mma_commit(&bars.sd_free[db]);
+        mma_commit(&bars.dk_done[db]);
         return true;
       };
       for (int i = 0; ok && i < nqt; ++i) {
-        const int st = i % C::NS, sb = i & 1;
+        const int st = i % C::NS;
         if (!mbar_wait(&bars.q_full[st], (i / C::NS) & 1, abort, a.wait)) { ok = false; break; }
-        if (i >= 2 && !mbar_wait(&bars.sd_free[sb], ((i >> 1) - 1) & 1, abort, a.wait)) { ok = false; break; }
-        fence_after_sync();
-        const uint64_t qh0 = sdesc(smem_u32(sm + C::OFF_ST + st * C::STAGE), 16, 1024);
-        const uint64_t ql0 = sdesc_add(qh0, C::Q_BYTES), gd0 = sdesc_add(qh0, 2 * C::Q_BYTES);
-#pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk) {
-          const uint32_t ok_ = (kk >> 2) * (BK * 128) + (kk & 3) * 32;
-          const uint32_t oq = (kk >> 2) * (BQ * 128) + (kk & 3) * 32;
-          const uint64_t kh = sdesc_add(kh0, ok_), kl = sdesc_add(kl0, ok_);
-          const uint64_t qh = sdesc_add(qh0, oq), ql = sdesc_add(ql0, oq);
-          mma_bf16(tmem + sb * BQ, kh, qh, id_s, kk > 0 ? 1u : 0u);
-          mma_bf16(tmem + sb * BQ, kl, qh, id_s, 1u);
-          mma_bf16(tmem + sb * BQ, kh, ql, id_s, 1u);
-        }
         if (C::DK) {
-          // V reaches tensor memory through the row threads: the first score product
-          // runs while they store it
-          if (i == 0) {
-            if (!mbar_wait(&bars.v_full, 0, abort, a.wait)) { ok = false; break; }
-            fence_after_sync();
+          // one S buffer: the rows of tile i - 1 have read it
+          if (i >= 1 && !mbar_wait(&bars.s_free[0], (i - 1) & 1, abort, a.wait)) { ok = false; break; }
+          fence_after_sync();
+          issue_s(i, 0);
+          mma_commit(&bars.s_full[i & 1]);  // per tile parity: each warpgroup waits its own
+          // V reaches tensor memory through the row threads (the first S runs meanwhile);
+          // dP buffer i & 1 held dS(i - 2) until dK(i - 2) drained it
+          if (i == 0 && !mbar_wait(&bars.v_full, 0, abort, a.wait)) { ok = false; break; }
+          if (i >= 2 && !mbar_wait(&bars.dk_done[i & 1], ((i >> 1) - 1) & 1, abort, a.wait)) {
+            ok = false;
+            break;
           }
-#pragma unroll
-          for (int kk = 0; kk < D / 16; ++kk) {
-            const uint32_t oq = (kk >> 2) * (BQ * 128) + (kk & 3) * 32;
-            const uint64_t gd = sdesc_add(gd0, oq);
-            mma_bf16_ts(tmem + C::COL_DP + sb * BQ, tv_hi + kk * 8, gd, id_s, kk > 0 ? 1u : 0u);
-            mma_bf16_ts(tmem + C::COL_DP + sb * BQ, tv_lo + kk * 8, gd, id_s, 1u);
+          fence_after_sync();
+          issue_dp(i);
+          mma_commit(&bars.dp_full[i & 1]);
+          if (i >= 1 && !issue_dk(i - 1)) { ok = false; break; }
+        } else {
+          const int sb = i & 1;
+          if (i >= 2 && !mbar_wait(&bars.s_free[sb], ((i >> 1) - 1) & 1, abort, a.wait)) {
+            ok = false;
+            break;
           }
+          fence_after_sync();
+          issue_s(i, sb * 128);
+          mma_commit(&bars.s_full[sb]);
+          mma_commit(&bars.q_empty[st]);
         }
-        mma_commit(&bars.sd_full[sb]);
-        if (!C::DK) mma_commit(&bars.q_empty[st]);
-        if (C::DK && i >= 1 && !issue_dk(i - 1)) { ok = false; break; }
       }
       if (ok && C::DK && nqt > 0) ok = issue_dk(nqt - 1);
       mma_commit(&bars.done);
@@ -267,17 +303,24 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     bool ok = true;
     for (int i = wg; i < nqt; i += 2) {
       const int sb = i & 1, st = i % C::NS;
-      ok = __all_sync(0xffffffffu, mbar_wait(&bars.sd_full[sb], (i >> 1) & 1, abort, a.wait));
+      // S of tile i is signalled on s_full[i & 1] (phase i / 2) in both modes
+      ok = __all_sync(0xffffffffu, mbar_wait(&bars.s_full[sb], (i >> 1) & 1, abort, a.wait));
       // the tile's l and delta were staged by the producer lanes: acquire them directly
       ok = ok && __all_sync(0xffffffffu, mbar_wait(&bars.q_full[st], (i / C::NS) & 1, abort, a.wait));
       if (!ok) break;
       fence_after_sync();
       float s[BQ];
+      {
+        float t[BQ];  // the two halves of the score product
+        const uint32_t col = C::DK ? 0u : (uint32_t)sb * 128u;
+        tmem_ld64x2(tmem + lane_base + col, s, tmem + lane_base + col + BQ, t);
+#pragma unroll
+        for (int c = 0; c < BQ; ++c) s[c] += t[c];
+      }
+      fence_before_sync();
+      mbar_arrive(&bars.s_free[C::DK ? 0 : sb]);
+      const float4 *l4 = reinterpret_cast<const float4 *>(bars.lse2[st]);
       if (!C::DK) {
-        tmem_ld64(tmem + lane_base + sb * BQ, s);
-        fence_before_sync();
-        mbar_arrive(&bars.sd_free[sb]);
-        const float4 *l4 = reinterpret_cast<const float4 *>(bars.lse2[st]);
 #pragma unroll
         for (int c4 = 0; c4 < BQ / 4; ++c4) {  // l = +inf past the problem
           const float4 l = l4[c4];
@@ -285,15 +328,19 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                  ex2(fmaf(s[4 * c4 + 2], sl2, -l.z)) + ex2(fmaf(s[4 * c4 + 3], sl2, -l.w));
         }
       } else {
+        ok = __all_sync(0xffffffffu, mbar_wait(&bars.dp_full[sb], (i >> 1) & 1, abort, a.wait));
+        if (!ok) break;
+        fence_after_sync();
+        const uint32_t tdp = tmem + lane_base + C::COL_DP + sb * BQ;
         float dp[BQ];
-        tmem_ld64x2(tmem + lane_base + sb * BQ, s, tmem + lane_base + C::COL_DP + sb * BQ, dp);
-        uint32_t hh[32], ll[32];
-        const float4 *l4 = reinterpret_cast<const float4 *>(bars.lse2[st]);
+        tmem_ld64(tdp, dp);
+        uint32_t hh[BQ / 2], ll[BQ / 2];
         const float4 *d4 = reinterpret_cast<const float4 *>(bars.del[st]);
 #pragma unroll
         for (int c4 = 0; c4 < BQ / 4; ++c4) {
-          // queries past the problem have l = +inf (p = 0) and delta = 0; rows of keys
-          // past it only feed their own dK rows, which are not stored
+          // queries past the problem have l = +inf (p = 0), delta = 0 and zero Q and
+          // Go rows; rows of keys past it only feed their own dK rows, which are not
+          // stored
           const float4 l = l4[c4], dl = d4[c4];
           const int c = 4 * c4;
           const float v0 = ex2(fmaf(s[c], sl2, -l.x)) * (dp[c] - dl.x);
@@ -303,9 +350,9 @@ __global__ void __launch_bounds__(NTHREADS, 1)
           split_pack(v0, v1, hh[2 * c4], ll[2 * c4]);
           split_pack(v2, v3, hh[2 * c4 + 1], ll[2 * c4 + 1]);
         }
-        // dS (hi, lo) over the S buffer: the A operand of dK += dS Q
-        tmem_st32u(tmem + lane_base + sb * BQ, hh);
-        tmem_st32u(tmem + lane_base + sb * BQ + 32, ll);
+        // dS (hi, lo) over this tile's dP buffer: the A operand of dK += dS Q
+        tmem_st32u(tdp, hh);
+        tmem_st32u(tdp + BQ / 2, ll);
         tmem_wait_st();
         fence_before_sync();
         mbar_arrive(&bars.ds_full[sb]);
