@@ -242,7 +242,7 @@ static int lbfgs_restart(const Batch &Bt, const kvs_schedule &sc, const float *Q
   int rc = launch_forward(Bt, Q, Kc, Vc, Y, lse, sc.w_out, sc.w_lse, w.fbuf, nullptr, ALL, q_ready,
                           w);
   if (rc) return rc;
-  rc = launch_backward(Bt, s.gn, ALL, w);
+  rc = launch_backward(Bt, Vc, sc.w_out, s.gn, ALL, w);
   if (rc) return rc;
   return launch_lbfgs_reset(Bt, s, Kc, w.fbuf, s.gn, clear);
 }
@@ -267,9 +267,9 @@ static int step_trial(const Batch &Bt, const kvs_schedule &sc, const float *Q, c
   return launch_lbfgs_armijo(Bt, s, sc, w, cond);
 }
 
-static int step_tail(const Batch &Bt, float *Kc, const State &s, int32_t *status, float *f_out,
-                     const Work &w) {
-  int rc = launch_backward(Bt, s.gn, phase_filter(s, PH_ACCEPT), w);
+static int step_tail(const Batch &Bt, const kvs_schedule &sc, const float *Vc, float *Kc,
+                     const State &s, int32_t *status, float *f_out, const Work &w) {
+  int rc = launch_backward(Bt, Vc, sc.w_out, s.gn, phase_filter(s, PH_ACCEPT), w);
   if (rc) return rc;
   return launch_lbfgs_update(Bt, s, Kc, status, f_out);
 }
@@ -282,7 +282,7 @@ static int lbfgs_one_step(const Batch &Bt, const kvs_schedule &sc, const float *
   if (rc) return rc;
   for (int t = 0; t < sc.max_bt; ++t)  // problems that have left the search skip each trial
     if ((rc = step_trial(Bt, sc, Q, Y, lse, Vc, Kc, s, q_ready || t > 0, w, nullptr))) return rc;
-  return step_tail(Bt, Kc, s, status, f_out, w);
+  return step_tail(Bt, sc, Vc, Kc, s, status, f_out, w);
 }
 
 // One L-BFGS step as a CUDA graph whose trial loop is a conditional WHILE node:
@@ -344,7 +344,7 @@ static int build_step_graph(const Batch &Bcaller, const kvs_schedule &sc, const 
       if (e2 != cudaSuccess) e = e2;
     }
   }
-  if (!rc && e == cudaSuccess) rc = step_tail(Bt, Kc, s, status, nullptr, w);
+  if (!rc && e == cudaSuccess) rc = step_tail(Bt, sc, Vc, Kc, s, status, nullptr, w);
   cudaGraph_t graph = nullptr;
   const cudaError_t e3 = cudaStreamEndCapture(Bt.st, &graph);
   sg->graph = graph;
@@ -623,7 +623,7 @@ int kvs_loss_grad(const kvs_batch *batch, const float *Q, const float *Kc, const
   if ((rc = begin(Bt, w))) return rc;
   if ((rc = launch_forward(Bt, Q, Kc, Vc, Y, lse, w_out, w_lse, loss, parts, ALL, false, w)))
     return rc;
-  if (dKc && (rc = launch_backward(Bt, dKc, ALL, w))) return rc;
+  if (dKc && (rc = launch_backward(Bt, Vc, w_out, dKc, ALL, w))) return rc;
   const HostGeom &g = Bt.g;
   return nan_if_err(Bt, w, loss, g.B, parts, 2 * (int64_t)g.B, dKc, g.sum_c * g.d);
 }

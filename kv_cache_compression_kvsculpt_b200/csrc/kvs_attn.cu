@@ -332,7 +332,8 @@ int forward_d(const Batch &Bt, const float *Q, const float *Kc, const float *Vc,
 }
 
 template <int D>
-int backward_d(const Batch &Bt, float *dKc, Filter flt, const Work &w) {
+int backward_d(const Batch &Bt, const float *Vc, float w_out, float *dKc, Filter flt,
+               const Work &w) {
   const HostGeom &g = Bt.g;
   int rc;
   BwdMaps bm;
@@ -351,8 +352,8 @@ int backward_d(const Batch &Bt, float *dKc, Filter flt, const Work &w) {
   ba.scale = 1.f / sqrtf((float)D);
   ba.lse = w.lse_h;
   ba.delta = w.delta;
-  ba.v_hi = w.vh;
-  ba.v_lo = w.vl;
+  ba.v32 = Vc;
+  ba.w_out = w_out;
   ba.dk = dKc;
   ba.err = w.err;
   ba.wait = wait_limit();
@@ -474,8 +475,10 @@ int launch_split_pairs(const Batch &Bt, const float *Kc, const float *Vc, const 
   return Bt.g.d == 64 ? prep_pairs<64>(Bt, Kc, Vc, w) : prep_pairs<128>(Bt, Kc, Vc, w);
 }
 
-int launch_backward(const Batch &Bt, float *dKc, Filter flt, const Work &w) {
-  return Bt.g.d == 64 ? backward_d<64>(Bt, dKc, flt, w) : backward_d<128>(Bt, dKc, flt, w);
+int launch_backward(const Batch &Bt, const float *Vc, float w_out, float *dKc, Filter flt,
+                    const Work &w) {
+  return Bt.g.d == 64 ? backward_d<64>(Bt, Vc, w_out, dKc, flt, w)
+                      : backward_d<128>(Bt, Vc, w_out, dKc, flt, w);
 }
 
 int launch_fit(const Batch &Bt, const float *Q, const float *Kc, const float *Y, float lam,

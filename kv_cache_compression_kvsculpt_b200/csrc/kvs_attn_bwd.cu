@@ -11,8 +11,9 @@
 //   S^T  = K Q^T      K_hi [Q_hi | Q_lo] (one N = 128 product into two column
 //                     halves) + K_lo Q_hi (into the first half); S = sum of the
 //                     halves, i.e. K_hi Q_hi + K_hi Q_lo + K_lo Q_hi  (K in smem)
-//   DK:  dP^T = V Go^T  V_hi Go + V_lo Go  (V in TMEM, Go bf16; delta was formed
-//                       from the same rounded Go)
+//   DK:  dP^T = V Go^T  V_hi Go + V_lo Go  (fp16: V split by the row threads into
+//                       TMEM, Go written by the loss forward, scaled into fp16's
+//                       range; delta was formed from the same rounded Go)
 //        dS = A (dP - delta_row), written as bf16 hi/lo over the tile's dP buffer
 //        dK += dS Q     dS_hi Q_hi + dS_hi Q_lo + dS_lo Q_hi  (Q as the N-major operand)
 //   COLSUM: importance += sum over the tile's queries of A
@@ -182,7 +183,8 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     // ------------------------------------------------------------- MMA issuer
     if (lane == 0) {
       const uint32_t id_s2 = idesc_bf16(BK, 2 * BQ, false, false);  // K_hi [Q_hi | Q_lo]
-      const uint32_t id_s1 = idesc_bf16(BK, BQ, false, false);      // K_lo Q_hi, V Go
+      const uint32_t id_s1 = idesc_bf16(BK, BQ, false, false);      // K_lo Q_hi
+      const uint32_t id_dp = idesc_f16(BK, BQ, false, false);       // V Go (fp16)
       const uint32_t id_dk = idesc_bf16(BK, D, false, true);
       bool ok = mbar_wait(&bars.k_full, 0, abort, a.wait);
       fence_after_sync();
@@ -208,8 +210,8 @@ __global__ void __launch_bounds__(NTHREADS, 1)
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
           const uint64_t gd = sdesc(base + (kk >> 2) * C::QB + (kk & 3) * 32, 16, 1024);
-          mma_bf16_ts(tmem + col, tv_hi + kk * 8, gd, id_s1, kk > 0 ? 1u : 0u);
-          mma_bf16_ts(tmem + col, tv_lo + kk * 8, gd, id_s1, 1u);
+          mma_bf16_ts(tmem + col, tv_hi + kk * 8, gd, id_dp, kk > 0 ? 1u : 0u);
+          mma_bf16_ts(tmem + col, tv_lo + kk * 8, gd, id_dp, 1u);
         }
       };
       // dK += dS(i) Q(i): dS hi / lo over dP buffer i & 1, Q as the N-major operand
@@ -277,19 +279,17 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     const bool kvalid = kr < nk;
     const uint32_t lane_base = (uint32_t)((warp & 3) * 32) << 16;
     if (C::DK) {
-      // this warpgroup's half of the value row (hi, lo) into tensor memory: the A
-      // operand of dP^T = V Go^T
-      const uint4 *vh = reinterpret_cast<const uint4 *>(a.v_hi + (a.k_pad[b] + kr) * D);
-      const uint4 *vl = reinterpret_cast<const uint4 *>(a.v_lo + (a.k_pad[b] + kr) * D);
+      // this warpgroup's half of the value row, split into fp16 hi / lo, into tensor
+      // memory: the A operand of dP^T = V Go^T (rows past the problem are zero)
+      const float4 *v4 = reinterpret_cast<const float4 *>(a.v32 + (k_begin + kr) * D);
 #pragma unroll 1
-      for (int c0 = wg * 32; c0 < D / 2; c0 += 64) {
+      for (int c0 = wg * 32; c0 < D / 2; c0 += 64) {  // packed columns c0 .. c0 + 31
         uint32_t wh[32], wl[32];
 #pragma unroll
-        for (int e = 0; e < 8; ++e) {
-          const uint4 h = kvalid ? vh[c0 / 4 + e] : make_uint4(0, 0, 0, 0);
-          const uint4 l = kvalid ? vl[c0 / 4 + e] : make_uint4(0, 0, 0, 0);
-          wh[4 * e] = h.x; wh[4 * e + 1] = h.y; wh[4 * e + 2] = h.z; wh[4 * e + 3] = h.w;
-          wl[4 * e] = l.x; wl[4 * e + 1] = l.y; wl[4 * e + 2] = l.z; wl[4 * e + 3] = l.w;
+        for (int e = 0; e < 16; ++e) {
+          const float4 v = kvalid ? v4[c0 / 2 + e] : make_float4(0.f, 0.f, 0.f, 0.f);
+          split_pack_f16(v.x, v.y, wh[2 * e], wl[2 * e]);
+          split_pack_f16(v.z, v.w, wh[2 * e + 1], wl[2 * e + 1]);
         }
         tmem_st32u(tmem + lane_base + C::COL_V + c0, wh);
         tmem_st32u(tmem + lane_base + C::COL_V + D / 2 + c0, wl);
@@ -363,6 +363,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     if (C::DK) {
       if (!mbar_wait(&bars.done, 0, abort, a.wait)) *abort = 1;
       fence_after_sync();
+      const float dks = a.scale / go_scale(nq, D, a.w_out);  // score scale, Go's scale undone
 #pragma unroll 1
       for (int c0 = wg * (D / 2); c0 < (wg + 1) * (D / 2); c0 += 32) {
         float o[32];
@@ -376,8 +377,8 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                                                    (k_begin + kr) * D + c0);
 #pragma unroll
           for (int e = 0; e < 8; ++e)
-            dst[e] = make_float4(o[4 * e] * a.scale, o[4 * e + 1] * a.scale,
-                                 o[4 * e + 2] * a.scale, o[4 * e + 3] * a.scale);
+            dst[e] = make_float4(o[4 * e] * dks, o[4 * e + 1] * dks, o[4 * e + 2] * dks,
+                                 o[4 * e + 3] * dks);
         }
       }
     } else {

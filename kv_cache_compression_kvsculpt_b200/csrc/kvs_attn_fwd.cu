@@ -18,8 +18,9 @@
 // while P V of the previous tile runs, the value tile while S of the next runs.
 // Tensor memory (512 columns): S/P buffers at 0 and 128, O_a | O_b at 256.
 // Modes:
-//   LOSS     keys K_c, values V_c: writes l_hat, Go = dL/dY_hat (bf16),
-//            delta = Go . Y_hat - dL/dl_hat (with the rounded Go), loss partials
+//   LOSS     keys K_c, values V_c: writes l_hat, Go = dL/dY_hat (fp16, scaled by
+//            go_scale), delta = Go . Y_hat - dL/dl_hat (same scale, with the
+//            rounded Go), loss partials
 //   TARGETS  keys K_z, values V_z: writes Y (fp32 and bf16 hi/lo) and l
 //   STATS    row log-sum-exp only
 //   WRITE_A  given l_hat: writes A = exp(S - l_hat) as bf16 hi/lo
@@ -399,8 +400,9 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         fence_after_sync();
       }
       const float inv = 1.f / lsum;
-      const float c_out = 2.f * a.w_out / ((float)nq * (float)D);
-      const float c_lse = 2.f * a.w_lse / (float)nq;
+      const float sig = go_scale(nq, D, a.w_out);
+      const float c_out = 2.f * a.w_out / ((float)nq * (float)D) * sig;  // scaled
+      const float c_lse = 2.f * a.w_lse / (float)nq * sig;
       const int64_t grow = q_begin + q;
       const int64_t prow = a.a_pad_off[b] + q;  // row of the padded bf16 buffers
       float se = 0.f, ls = 0.f, gy = 0.f;
@@ -463,11 +465,11 @@ __global__ void __launch_bounds__(NTHREADS, 1)
 #pragma unroll
               for (int e = 0; e < 4; ++e) {
                 const int i0 = ch * 8 + 2 * e;
-                // delta uses the bf16-rounded Go that the backward's dP product sees,
+                // delta uses the fp16-rounded Go that the backward's dP product sees,
                 // so the rounding of Go cancels exactly in dP - delta.
-                h[e] = pack_bf16(c_out * ev[i0], c_out * ev[i0 + 1]);
-                const float g0 = __uint_as_float(h[e] << 16);
-                const float g1 = __uint_as_float(h[e] & 0xffff0000u);
+                h[e] = pack_f16(c_out * ev[i0], c_out * ev[i0 + 1]);
+                const float2 gg = unpack_f16(h[e]);
+                const float g0 = gg.x, g1 = gg.y;
                 se = fmaf(ev[i0], ev[i0], se);
                 se = fmaf(ev[i0 + 1], ev[i0 + 1], se);
                 gy = fmaf(g0, o[i0], gy);

@@ -19,6 +19,16 @@ constexpr int FWD_BN = 128;
 // and Go maps).
 constexpr int BWD_BQ = 64;
 
+// dL/dY_hat = c (Y_hat - Y), c = 2 w_out / (n_q d), is carried as fp16 scaled by
+// sigma = 2^-round(log2 c) (so that it sits in fp16's normal range; 1 when c = 0):
+// the loss forward writes Go = fp16(sigma c (Y_hat - Y)) and delta in the same
+// scale, the key gradient divides dK by sigma.  Powers of two keep the scaling
+// exact.
+__device__ __forceinline__ float go_scale(int nq, int d, float w_out) {
+  const float c = 2.f * w_out / ((float)nq * (float)d);
+  return c > 0.f ? exp2f(-rintf(log2f(c))) : 1.f;
+}
+
 // Tensor maps of the bf16 operands (2-D, [rows, d], box 64 columns x FWD_BN rows).
 struct FwdMaps {
   CUtensorMap kh, kl, vh, vl;
@@ -35,8 +45,8 @@ struct FwdArgs {
   const float *y_in;      // [sum_q, d] targets
   const float *lse_in;    // [sum_q] target lse (LOSS) or given row lse (WRITE_A)
   float *lse_out;         // [sum_q] row lse of these keys
-  __nv_bfloat16 *go;      // [sum_q, d] dL/dY_hat, bf16
-  float *delta;           // [sum_q]
+  __nv_bfloat16 *go;      // [padded q, d] dL/dY_hat, fp16 bits scaled by go_scale
+  float *delta;           // [sum_q] Go . Y_hat - dL/dl_hat, in the scale of Go
   float *partials;        // [B, tiles_per_problem, 2]
   int tiles_per_problem;
   float w_out, w_lse;     // loss weights (means over n_q d and n_q)
@@ -64,7 +74,8 @@ struct BwdArgs {
   float scale;
   const float *lse;       // [sum_q] row lse used to form the probabilities
   const float *delta;     // [sum_q] (DK)
-  const __nv_bfloat16 *v_hi, *v_lo;  // [padded k, d] value split (DK; loaded into tensor memory)
+  const float *v32;       // [sum_k, d] values (DK; split into fp16 hi/lo in tensor memory)
+  float w_out;            // output-term weight (DK: the scale of Go, go_scale)
   const int64_t *q_pad, *k_pad;      // [B+1] padded rows of the query / Go and key / value maps
   float *dk;              // [sum_k, d] (DK): dL/dK, or nsplit partial sums dk_stride apart
   float *imp;             // [sum_k] (COLSUM): column sums of probabilities

@@ -117,7 +117,7 @@ int launch_targets(const Batch &B, const float *Q, const float *Kz, const float 
                    float *lse, float *imp, const Work &w);
 // Loss forward over the compressed pairs for the problems selected by `flt`:
 // writes loss[b] (and parts[2b..2b+1] if non-null) and leaves lse_h, go and
-// delta (plus the bf16 copies of Kc, Vc) for launch_backward.  q_ready: the
+// delta (plus the bf16 copies of Kc) for launch_backward.  q_ready: the
 // Q split in w.qh/ql is current.
 int launch_forward(const Batch &B, const float *Q, const float *Kc, const float *Vc,
                    const float *Y, const float *lse, float w_out, float w_lse, float *loss,
@@ -125,8 +125,10 @@ int launch_forward(const Batch &B, const float *Q, const float *Kc, const float 
                    bool pairs_ready = false, bool reduce = true);
 // bf16 hi/lo copies of the compressed pairs (keys; values unless Vc is null).
 int launch_split_pairs(const Batch &B, const float *Kc, const float *Vc, const Work &w);
-// dKc from the state left by launch_forward for the same problems.
-int launch_backward(const Batch &B, float *dKc, Filter flt, const Work &w);
+// dKc from the state left by launch_forward for the same problems (with the same
+// values Vc and output weight w_out).
+int launch_backward(const Batch &B, const float *Vc, float w_out, float *dKc, Filter flt,
+                    const Work &w);
 // Ridge fit: Vc = (A^T A + lam I)^-1 A^T Y (y_ready: the Y split is current).  The
 // row log-sum-exp of Kc is recomputed for the problems `stats` selects; the others
 // take the one the last loss forward left in the workspace.

@@ -10,6 +10,7 @@
 
 #include <cuda.h>
 #include <cuda_bf16.h>
+#include <cuda_fp16.h>
 #include <stdint.h>
 
 #include "kvs_common.cuh"
@@ -62,11 +63,28 @@ __device__ __forceinline__ bool mbar_test(uint64_t *bar, uint32_t parity) {
   return done != 0;
 }
 
+// Non-blocking test of the same phase.
+__device__ __forceinline__ bool mbar_test_now(uint64_t *bar, uint32_t parity) {
+  uint32_t done;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(done)
+      : "r"(smem_u32(bar)), "r"(parity)
+      : "memory");
+  return done != 0;
+}
+
 // Wait until the phase of parity `parity` completes; false after `limit`
-// cycles or as soon as *abort is set by another thread of the CTA.
+// cycles or as soon as *abort is set by another thread of the CTA.  A phase
+// that has already completed is seen by one non-blocking test, without
+// starting the clock: the MMA-issuing thread checks mostly such phases, and
+// the tensor pipe idles while it waits.
 __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity,
                                           volatile int *abort = nullptr,
                                           long long limit = kWaitCycles) {
+  if (mbar_test_now(bar, parity)) return true;
   const long long t0 = clock64();
   while (!mbar_test(bar, parity)) {
     if (abort && *abort) return false;
@@ -220,6 +238,12 @@ __host__ __device__ constexpr uint32_t idesc_bf16(int M, int N, bool a_mn, bool 
          ((uint32_t)(N >> 3) << 17) | ((uint32_t)(M >> 4) << 24);
 }
 
+// Instruction descriptor: f16 x f16 -> f32 (A and B types 0), dense, shape M x N.
+__host__ __device__ constexpr uint32_t idesc_f16(int M, int N, bool a_mn, bool b_mn) {
+  return (1u << 4) | ((uint32_t)a_mn << 15) | ((uint32_t)b_mn << 16) | ((uint32_t)(N >> 3) << 17) |
+         ((uint32_t)(M >> 4) << 24);
+}
+
 // D[tmem] (+)= A[smem] * B[smem]; one thread issues.
 __device__ __forceinline__ void mma_bf16(uint32_t d_tmem, uint64_t a, uint64_t b, uint32_t idesc,
                                          uint32_t accumulate) {
@@ -291,6 +315,21 @@ __device__ __forceinline__ void split_pack(float a, float b, uint32_t &hi, uint3
   const __nv_bfloat162 l = __floats2bfloat162_rn(a - ha, b - hb);
   hi = hw;
   lo = *reinterpret_cast<const uint32_t *>(&l);
+}
+
+// fp16 pair packing (round to nearest even), a in the low half, and its values.
+__device__ __forceinline__ uint32_t pack_f16(float a, float b) {
+  __half2 h = __floats2half2_rn(a, b);
+  return *reinterpret_cast<uint32_t *>(&h);
+}
+__device__ __forceinline__ float2 unpack_f16(uint32_t w) {
+  return __half22float2(*reinterpret_cast<const __half2 *>(&w));
+}
+// fp16 hi and lo words of the pair (a, b): hi = rn(x), lo = rn(x - hi).
+__device__ __forceinline__ void split_pack_f16(float a, float b, uint32_t &hi, uint32_t &lo) {
+  hi = pack_f16(a, b);
+  const float2 h = unpack_f16(hi);
+  lo = pack_f16(a - h.x, b - h.y);
 }
 
 // 2^x on the special-function unit; subnormal results flush to zero (softmax

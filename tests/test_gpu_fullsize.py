@@ -81,7 +81,8 @@ def test_full_schedule_matches_oracle(name):
                          [round(x / p["loss"], 4) for x in p["band"]]))
         check_topk_valid(r["idx"][co[b]:co[b + 1]], c.Qs[b], c.Zk[b], c.Zv[b], int(c.k[b]))
     print(f"{name}: (problem, verdict, GPU / oracle, band / oracle) = {verdicts}")
-    assert sum(v == "ok" for _, v, _, _ in verdicts) >= 2, "most problems must be comparable"
+    assert sum(v == "ok" for _, v, _, _ in verdicts) >= (2 * len(verdicts) + 2) // 3, \
+        "most problems must be comparable"
 
 
 def test_adaptive_matches_oracle():

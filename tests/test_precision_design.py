@@ -109,3 +109,36 @@ def test_split_gram_and_fp32_cholesky_meet_the_value_bar(point):
     rel = lambda V: float(np.linalg.norm(V - Vo) / np.linalg.norm(Vo))
     assert rel(fit_emulated(mm_split, Q, Kc, Y)) <= 1e-4   # bar 1e-3
     assert rel(fit_emulated(mm_single, Q, Kc, Y)) > 1e-3
+
+
+def f16(x):
+    return np.asarray(x, np.float32).astype(np.float16).astype(np.float64)
+
+
+def grad_with_go(Q, Kc, Vc, Y, lse, rnd):
+    """Exact gradient except that dL/dY_hat is rounded by rnd before both the
+    value product and delta (as in the key-gradient kernel)."""
+    n_q, d = Q.shape
+    A, l = O.attention(Q, Kc)
+    Yh = A @ Vc
+    G = rnd(2.0 / (n_q * d) * (Yh - Y))
+    delta = (G * Yh).sum(1) - 2.0 / n_q * (l - lse)
+    return ((A * (G @ Vc.T - delta[:, None])).T @ Q) / np.sqrt(d)
+
+
+def test_go_in_scaled_fp16_beats_bf16(point):
+    """Go = dL/dY_hat is the one operand that enters its product without a lo
+    part.  In bf16 (8-bit mantissa) its rounding moves the gradient near an
+    optimum by a few 1e-4, enough to steer some full-length solves several
+    percent away from the float64 one; fp16 (11 bits) after scaling by a power
+    of two into fp16's normal range moves it about eight times less, at the
+    same MMA cost."""
+    Q, Kc, Vc, Y, lse = point
+    n_q, d = Q.shape
+    _, g0, _ = O.loss_grad(Q, Kc, Vc, Y, lse)
+    sig = 2.0 ** -np.rint(np.log2(2.0 / (n_q * d)))
+    err = lambda g: float(np.linalg.norm(g - g0) / np.linalg.norm(g0))
+    e_bf = err(grad_with_go(Q, Kc, Vc, Y, lse, bf16))
+    e_f16 = err(grad_with_go(Q, Kc, Vc, Y, lse, lambda G: f16(G * sig) / sig))
+    assert e_f16 <= e_bf / 4, (e_f16, e_bf)
+    assert e_f16 < 1e-4
