@@ -265,13 +265,15 @@ def loss_grad_roofline(job, peaks, reps=20):
     """Time kvs_loss_grad (the dominant evaluation) over the batch at the solved point."""
     torch, K, wl = job.torch, job.K, job.wl
     B = job.batch.B
+    # the solve's workspace when it is large enough for the batch's (possibly
+    # allocated) k, else one of that size
+    ws = (job.ws if K.kvs_workspace_bytes(job.batch) <= job.ws.numel()
+          else K.alloc_workspace(job.batch))
     Y = torch.empty_like(job.Q)
     lse = torch.empty(job.batch.sum_q, device=job.Q.device)
-    K.kvs_targets(job.batch, job.Q, job.dev["Kz"], job.dev["Vz"], Y, lse, None,
-                  K.alloc_workspace(job.batch))
+    K.kvs_targets(job.batch, job.Q, job.dev["Kz"], job.dev["Vz"], Y, lse, None, ws)
     loss = torch.empty(B, device=job.Q.device)
     dK = torch.empty_like(job.Kc)
-    ws = K.alloc_workspace(job.batch)  # sized for the batch's (possibly allocated) k
 
     def ev():
         K.kvs_loss_grad(job.batch, job.Q, job.Kc, job.Vc, Y, lse, 1.0, 1.0, loss, None, dK, ws)
