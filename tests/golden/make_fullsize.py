@@ -22,12 +22,16 @@ workload's float32 zone keys and values.  Checksums of those inputs are stored
 so that a test can tell when the generator has changed.
 
 Each solve is also repeated with loss and gradient evaluations perturbed at the
-relative precision of the library's arithmetic (oracle.perturb, two seeds):
-the final losses of those runs ("band") show how far a run of that precision
-can legitimately end from the exact one on this (non-convex, fixed-length)
-trajectory.  The adaptive case's band is taken at the oracle's allocation.
+relative precision of the library's arithmetic (oracle.perturb, two seeds), and
+once with the library's own rounding emulated in float64 (oracle.perturb
+emulated_evaluations): the final losses of those runs ("band", "emulated")
+show how far a run of that precision can legitimately end from the exact one
+on this (non-convex, fixed-length) trajectory.  The adaptive case's runs are
+taken at the oracle's allocation.
 
-Run:  python tests/golden/make_fullsize.py   (about 45 minutes on 8 cores)
+Run:  python tests/golden/make_fullsize.py   (about 2 hours on 8 cores)
+      python tests/golden/make_fullsize.py --add-emulated   (only the emulated
+      runs, added to an existing file)
 """
 from __future__ import annotations
 
@@ -43,7 +47,7 @@ sys.path.insert(0, ROOT)
 
 import oracle as O  # noqa: E402
 import workload as W  # noqa: E402
-from oracle.perturb import GPU_LEVELS, noisy_evaluations  # noqa: E402
+from oracle.perturb import GPU_LEVELS, emulated_evaluations, noisy_evaluations  # noqa: E402
 
 BAND_SEEDS = 2
 
@@ -91,6 +95,11 @@ def band(Q, Kz, Vz, k, sched):
                   ["loss"]) for s in range(BAND_SEEDS)]
 
 
+def emulated(Q, Kz, Vz, k, sched):
+    """Final loss of the schedule with the library's rounding emulated."""
+    return float(O.compress(Q, Kz, Vz, k, sched, evaluate=emulated_evaluations())["loss"])
+
+
 def uniform_case(name, ids):
     wl = W.WORKLOADS[name]
     t0 = time.time()
@@ -99,6 +108,7 @@ def uniform_case(name, ids):
         r = O.compress(Q, Kz, Vz, wl.k, schedule(wl))
         rec = result_record(r)
         rec["band"] = band(Q, Kz, Vz, wl.k, schedule(wl))
+        rec["emulated"] = emulated(Q, Kz, Vz, wl.k, schedule(wl))
         rec.update(id=list(pid), k=wl.k, checksum_Q=checksum(Q), checksum_Kz=checksum(Kz),
                    checksum_Vz=checksum(Vz))
         probs.append(rec)
@@ -117,6 +127,7 @@ def adaptive_case(ids):
     for b, (pid, (Q, Kz, Vz)) in enumerate(zip(ids, inp)):
         rec = result_record(res["results"][b])
         rec["band"] = band(Q, Kz, Vz, int(res["k"][b]), schedule(wl))
+        rec["emulated"] = emulated(Q, Kz, Vz, int(res["k"][b]), schedule(wl))
         rec.update(id=list(pid), k=int(res["k"][b]), pilot_mse=float(res["pilot_mse"][b]),
                    checksum_Q=checksum(Q), checksum_Kz=checksum(Kz), checksum_Vz=checksum(Vz))
         probs.append(rec)
@@ -124,7 +135,27 @@ def adaptive_case(ids):
     return {"workload": wl.name, "total": int(total), "problems": probs}
 
 
+def add_emulated():
+    """Add the emulated-rounding run to every problem of an existing file."""
+    with open(OUT) as fh:
+        out = json.load(fh)
+    for name, case in out["cases"].items():
+        wl = W.WORKLOADS[name]
+        ids = [tuple(p["id"]) for p in case["problems"]]
+        for (Q, Kz, Vz), p in zip(float32_inputs(wl, ids), case["problems"]):
+            if "emulated" in p:
+                continue
+            t0 = time.time()
+            p["emulated"] = emulated(Q, Kz, Vz, int(p["k"]), schedule(wl))
+            print(f"{name} {p['id']}: emulated {p['emulated'] / p['loss']:.4f}x "
+                  f"({time.time() - t0:.0f} s)", flush=True)
+            with open(OUT, "w") as fh:
+                json.dump(out, fh, indent=1)
+
+
 def main():
+    if "--add-emulated" in sys.argv:
+        return add_emulated()
     out = {"generator": "tests/golden/make_fullsize.py (oracle/ only)", "seed": 0,
            "band_levels": list(GPU_LEVELS), "cases": {}}
     for name in ("qwen_cache_r03", "qwen_cache_r05", "qwen_cache_r07"):

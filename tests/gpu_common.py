@@ -98,9 +98,18 @@ def oracle_band(Q, Kz, Vz, k, sched, seeds=3):
                   ["loss"]) for s in range(seeds)]
 
 
-def check_final_loss(f_gpu, f_sf, f_or, band, what=""):
-    """Assert the parity bar above; returns 'ok' or 'ill-conditioned'."""
+def check_final_loss(f_gpu, f_sf, f_or, band, what="", emulated=None):
+    """Assert the parity bar above; returns 'ok', 'ok (emulated)' or 'ill-conditioned'.
+    `emulated`: the final loss of the oracle's run with the library's own rounding
+    emulated (oracle.perturb.emulated_evaluations), a member of the band when
+    given; 'ok (emulated)' says the result needed it."""
     lo, hi, spread = final_loss_bar(f_or, band)
+    if emulated is not None and not (lo - 1e-7 <= f_gpu <= hi + 1e-7):
+        lo2, hi2, spread2 = final_loss_bar(f_or, list(band) + [emulated])
+        if spread2 <= ILL_CONDITIONED:
+            assert lo2 - 1e-7 <= f_gpu <= hi2 + 1e-7, (what, f_gpu, f_or, band, emulated,
+                                                       f_gpu / f_or)
+            return "ok (emulated)"
     if spread > ILL_CONDITIONED:
         assert f_gpu < f_sf, (what, f_gpu, f_sf)
         return "ill-conditioned"

@@ -76,12 +76,12 @@ def test_full_schedule_matches_oracle(name):
         sf_gpu, sf_or = float(r["trace"][b, 0]), p["trace"][0]
         assert abs(sf_gpu - sf_or) <= 1e-3 * sf_or, (p["id"], sf_gpu, sf_or)
         f_gpu = float(r["trace"][b, -1])
-        v = check_final_loss(f_gpu, sf_gpu, p["loss"], p["band"], p["id"])
+        v = check_final_loss(f_gpu, sf_gpu, p["loss"], p["band"], p["id"], p.get("emulated"))
         verdicts.append((p["id"], v, round(f_gpu / p["loss"], 4),
                          [round(x / p["loss"], 4) for x in p["band"]]))
         check_topk_valid(r["idx"][co[b]:co[b + 1]], c.Qs[b], c.Zk[b], c.Zv[b], int(c.k[b]))
     print(f"{name}: (problem, verdict, GPU / oracle, band / oracle) = {verdicts}")
-    assert sum(v == "ok" for _, v, _, _ in verdicts) >= (2 * len(verdicts) + 2) // 3, \
+    assert sum(v.startswith("ok") for _, v, _, _ in verdicts) >= (2 * len(verdicts) + 2) // 3, \
         "most problems must be comparable"
 
 
@@ -121,7 +121,7 @@ def test_adaptive_matches_oracle():
         sf_gpu = float(r["trace"][b, 0])
         assert abs(sf_gpu - p["trace"][0]) <= 1e-3 * p["trace"][0], (p["id"], sf_gpu)
         f_gpu = float(r["trace"][b, -1])
-        v = check_final_loss(f_gpu, sf_gpu, p["loss"], p["band"], p["id"])
+        v = check_final_loss(f_gpu, sf_gpu, p["loss"], p["band"], p["id"], p.get("emulated"))
         verdicts.append((p["id"], int(p["k"]), v, round(f_gpu / p["loss"], 4)))
     print(f"{name}: GPU k = {k.tolist()}, oracle k = {k_or.tolist()}; "
           f"(problem, k, verdict, GPU / oracle) = {verdicts}")

@@ -142,3 +142,17 @@ def test_go_in_scaled_fp16_beats_bf16(point):
     e_f16 = err(grad_with_go(Q, Kc, Vc, Y, lse, lambda G: f16(G * sig) / sig))
     assert e_f16 <= e_bf / 4, (e_f16, e_bf)
     assert e_f16 < 1e-4
+
+
+def test_emulated_evaluations_model_the_library_rounding(point):
+    """oracle.perturb.emulated_evaluations (used to bound the final-loss parity
+    bar) rounds like the library: close to the exact loss and gradient at the
+    16-bit level, and not identical to them."""
+    from oracle.perturb import emulated_evaluations
+    Q, Kc, Vc, Y, lse = point
+    f0, g0, _ = O.loss_grad(Q, Kc, Vc, Y, lse)
+    fo, fg = emulated_evaluations()
+    f1, g1, _ = fg(Q, Kc, Vc, Y, lse)
+    assert abs(f1 - f0) <= 1e-5 * f0 and f1 != f0
+    assert _cos(g1, g0) >= 0.99999 and not np.array_equal(g1, g0)
+    assert fo(Q, Kc, Vc, Y, lse) == f1
