@@ -268,11 +268,12 @@ int kvs_adam_step(const kvs_batch *batch, float *Kc, const float *dKc, float *m,
  * loop is a conditional node; with the environment variable
  * KVS_STEP_GRAPHS=0 (read once per process) the same kernels are launched
  * one by one instead, for kernel-level profilers.
- * A batch of 8 or more problems is solved as two sub-batches of contiguous
- * problems (cut where the work n_q k (d + k) splits evenly), the second on an
- * internal stream forked from and joined back to `stream`, so that the
- * latency-bound steps of one overlap the tensor-core work of the other; the
- * results are those of solving each problem on its own.  `state` is then
+ * A batch of 8 or more problems is solved as sub-batches of contiguous
+ * problems (two from 8 problems, four from 16; cut where the work
+ * n_q k (d + k) splits evenly), all but the first on internal streams forked
+ * from and joined back to `stream`, so that the latency-bound steps of one
+ * overlap the tensor-core work of the others; the results are those of solving
+ * each problem on its own.  `state` is then
  * scratch laid out per sub-batch (kvs_lbfgs_state_layout does not apply). */
 int kvs_compress_batch(const kvs_batch *batch, const kvs_schedule *sched, const float *Q,
                        const float *Kz, const float *Vz, float *Kc, float *Vc, int32_t *idx,

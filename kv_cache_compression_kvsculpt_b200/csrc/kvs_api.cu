@@ -375,25 +375,31 @@ struct Partition {
   int cut[KVS_MAX_PARTS + 1] = {0};
 };
 
-// Two sub-batches once the batch has at least 8 problems (each half still fills
-// the GPU in the attention kernels), cut where the estimated work
-// n_q k (d + k) of the problems splits most evenly.
+// Sub-batches: four once the batch has at least 16 problems, two from 8 (each
+// part still fills the GPU in the attention kernels), cut where the estimated
+// work n_q k (d + k) of the problems reaches 1/n, 2/n, .. of the total.
 static Partition partition_of(const kvs_batch *b, const HostGeom &g) {
   Partition P;
   P.cut[1] = g.B;
   if (g.B < 8 || !b->c_off_h) return P;
+  const int n = g.B >= 16 ? 4 : 2;
+  static_assert(KVS_MAX_PARTS >= 4, "parts");
   std::vector<double> acc(g.B + 1, 0.0);
   for (int i = 0; i < g.B; ++i) {
     const double nq = (double)(b->q_off_h[i + 1] - b->q_off_h[i]);
     const double k = (double)(b->c_off_h[i + 1] - b->c_off_h[i]);
     acc[i + 1] = acc[i] + nq * k * (g.d + k);
   }
-  int best = 1;
-  for (int c = 2; c < g.B; ++c)
-    if (std::fabs(acc[c] - acc[g.B] / 2) < std::fabs(acc[best] - acc[g.B] / 2)) best = c;
-  P.n = 2;
-  P.cut[1] = best;
-  P.cut[2] = g.B;
+  P.n = n;
+  for (int p = 1; p < n; ++p) {
+    // the cut nearest to the target that leaves at least one problem per part
+    const double target = acc[g.B] * p / n;
+    int best = P.cut[p - 1] + 1;
+    for (int c = best; c <= g.B - (n - p); ++c)
+      if (std::fabs(acc[c] - target) < std::fabs(acc[best] - target)) best = c;
+    P.cut[p] = best;
+  }
+  P.cut[n] = g.B;
   return P;
 }
 

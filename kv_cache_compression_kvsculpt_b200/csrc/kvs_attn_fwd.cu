@@ -9,11 +9,11 @@
 // bits through a bf16 hi/lo split, with fp32 accumulation in tensor memory:
 //   S = Q K^T     Q_hi K_hi + Q_hi K_lo + Q_lo K_hi   (Q and K in smem; N = 128)
 //   online softmax, one thread per query row, lazy rescaling of O
-//   O += P V      P_hi [V_hi | V_lo] + P_lo [V_hi | V_lo]  (P in TMEM over S; N = 2d)
-// Each tcgen05.mma instruction costs about the same for any N up to 256, so
-// the key tile is 128 wide and the value product takes V_hi and V_lo side by
-// side: two instructions per 16 keys instead of three, into two output halves
-// O_a = P V_hi, O_b = P V_lo (plus the negligible P_lo V_lo) summed at the end.
+//   O += P V      P_hi [V_hi | V_lo] (N = 2d) + P_lo V_hi (N = d)  (P in TMEM over S)
+// An instruction of N = 128 costs half as much as one of N = 256, so the value
+// product takes V_hi and V_lo side by side for P_hi: two instructions per 16
+// keys instead of three, into two output halves O_a = P_hi V_hi + P_lo V_hi and
+// O_b = P_hi V_lo, summed at the end.
 // Keys and values have separate shared-memory rings: the next key tile loads
 // while P V of the previous tile runs, the value tile while S of the next runs.
 // Tensor memory (512 columns): S/P buffers at 0 and 128, O_a | O_b at 256.
@@ -213,6 +213,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       const uint32_t id_s128 = idesc_bf16(BM, BN, false, false);
       const uint32_t id_s64 = idesc_bf16(BM, 64, false, false);
       const uint32_t id_pv = idesc_bf16(BM, 2 * D, false, true);  // N = [V_hi | V_lo]
+      const uint32_t id_pvh = idesc_bf16(BM, D, false, true);     // N = V_hi
       bool ok = mbar_wait(&bars.q_full, 0, abort, a.wait);
       fence_after_sync();
       const uint64_t qh0 = sdesc(smem_u32(sm), 16, 1024), ql0 = sdesc_add(qh0, C::T_BYTES);
@@ -229,8 +230,9 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         const int nks = (kv + 15) / 16;      // key steps that hold valid keys
         for (int kk = 0; kk < nks; ++kk) {
           const uint64_t v = sdesc_add(v0, kk * 2048);
+          // P_hi [V_hi | V_lo] into both halves, P_lo V_hi into the first
           mma_bf16_ts(tmem + C::COL_O, tp + kk * 8, v, id_pv, (i > 0 || kk > 0) ? 1u : 0u);
-          mma_bf16_ts(tmem + C::COL_O, tp + BN / 2 + kk * 8, v, id_pv, 1u);
+          mma_bf16_ts(tmem + C::COL_O, tp + BN / 2 + kk * 8, v, id_pvh, 1u);
         }
         mma_commit(&bars.v_empty[i % C::NSVI]);
         mma_commit(&bars.s_free[pb]);

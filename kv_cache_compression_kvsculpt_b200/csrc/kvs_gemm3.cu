@@ -31,7 +31,8 @@ struct G3 {
   static constexpr int NS = TN > 128 ? 2 : 3;
   static constexpr int SMEM = NS * STAGE + 1024;
   // tiles up to 128 wide take B_hi and B_lo side by side as one operand of N = 2 TN
-  // (two instructions per 16-row step instead of three), into two summed halves
+  // for A_hi, and B_hi alone (N = TN) for A_lo: two instructions per 16-row step
+  // instead of three, into two summed halves
   static constexpr bool CAT = TN <= 128;
   static constexpr int MMA_N = CAT ? 2 * TN : TN;
   static constexpr uint32_t TMEM_COLS = MMA_N < 32 ? 32 : MMA_N;
@@ -147,6 +148,7 @@ __global__ void __launch_bounds__(192, 1)
   } else if (warp == 5) {
     if (lane == 0) {
       const uint32_t id = idesc_bf16(TM, C::MMA_N, true, true);
+      const uint32_t id_h = idesc_bf16(TM, TN, true, true);  // CAT: B_hi alone
       bool ok = true;
       for (int i = 0; i < nkt; ++i) {
         const int st = i % NS;
@@ -159,9 +161,9 @@ __global__ void __launch_bounds__(192, 1)
           const uint64_t al = sdesc_add(ah, A_BYTES);
           const uint64_t bh = sdesc_add(ah, 2 * A_BYTES);
           const uint64_t bl = sdesc_add(ah, 2 * A_BYTES + C::B_BYTES);
-          if (C::CAT) {  // A_hi [B_hi | B_lo] + A_lo [B_hi | B_lo]
+          if (C::CAT) {  // A_hi [B_hi | B_lo] into both halves + A_lo B_hi into the first
             mma_bf16(tmem, ah, bh, id, (i > 0 || kk > 0) ? 1u : 0u);
-            mma_bf16(tmem, al, bh, id, 1u);
+            mma_bf16(tmem, al, bh, id_h, 1u);
           } else {
             mma_bf16(tmem, ah, bh, id, (i > 0 || kk > 0) ? 1u : 0u);
             mma_bf16(tmem, ah, bl, id, 1u);

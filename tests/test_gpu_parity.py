@@ -27,6 +27,10 @@ SMALL64 = W.Workload("small_d64", 1, 2, 2, d=64, N=200, m=40, g=3, n_syn=30, k=5
 SPLIT10 = W.Workload("split10", 1, 5, 2, d=128, N=260, m=36, g=2, n_syn=50, k=60,
                      layer_scale=True, outer=3, steps=4)
 SPLIT10_K = [60, 17, 224, 1, 90, 33, 128, 60, 200, 5]
+# sixteen problems: four concurrent sub-batches
+SPLIT16 = W.Workload("split16", 1, 8, 2, d=64, N=200, m=40, g=2, n_syn=40, k=40,
+                     layer_scale=True, outer=3, steps=4)
+SPLIT16_K = [40, 3, 160, 71, 12, 40, 99, 150, 8, 40, 64, 1, 130, 27, 45, 160]
 
 
 @pytest.fixture(scope="module", autouse=True)
@@ -45,6 +49,7 @@ def cases():
         # problem's query tiles over several CTAs and some splits of the short one are empty
         "uneven": lambda: Case(W.WORKLOADS["qwen_layer"], k=[960, 200], n_q=[3840, 100]),
         "split10": lambda: Case(SPLIT10, k=SPLIT10_K),
+        "split16": lambda: Case(SPLIT16, k=SPLIT16_K),
     }
 
 
@@ -375,7 +380,7 @@ def check_topk_valid(gidx, Qb, Zk, Zv, k, tol=1e-4):
     return np.array_equal(gidx, O.topk_select(imp, k))
 
 
-@pytest.mark.parametrize("name", ["single_d64", "ragged", "small_d64", "split10"])
+@pytest.mark.parametrize("name", ["single_d64", "ragged", "small_d64", "split10", "split16"])
 def test_compress_small(name):
     c = cases()[name]()
     wl = c.wl
