@@ -64,13 +64,16 @@ struct Fwd {
   static constexpr int SMEM = BYTES + 1024;
   static constexpr uint32_t TMEM_COLS = 512;
   static constexpr uint32_t COL_O = 2 * BN;     // O_a at +0, O_b at +D
+  // the single key / value stages are freed by the commits that signal S and P V
+  static_assert(!PV || (NSK == 1 && NSVI == 1), "stage release through s_full / s_free");
+  static_assert(!WA || NSK == 1, "stage release through s_full");
 };
 static_assert(BM == BN, "the Q tile shares the key tile's layout");
 
 struct FwdBars {
   uint64_t q_full;
   uint64_t k_full[3], k_empty[3];
-  uint64_t v_full[1], v_empty[1];
+  uint64_t v_full[1];
   uint64_t s_full[2], s_free[2];
   uint64_t p_full[2];
   uint64_t o_done;
@@ -126,10 +129,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       mbar_init(&bars.k_full[i], 1);
       mbar_init(&bars.k_empty[i], 1);
     }
-    for (int i = 0; i < C::NSV; ++i) {
-      mbar_init(&bars.v_full[i], 1);
-      mbar_init(&bars.v_empty[i], 1);
-    }
+    for (int i = 0; i < C::NSV; ++i) mbar_init(&bars.v_full[i], 1);
     for (int i = 0; i < 2; ++i) {
       mbar_init(&bars.s_full[i], 1);
       mbar_init(&bars.s_free[i], C::PV ? 1 : 2 * BM);
@@ -160,8 +160,14 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       int k_issued = 0, v_issued = 0;
       auto load_k = [&](int j) -> bool {
         const int st = j % C::NSK;
-        if (j >= C::NSK && !mbar_wait(&bars.k_empty[st], ((j / C::NSK) - 1) & 1, abort, a.wait))
-          return false;
+        if (j >= C::NSK) {
+          // one stage: free once S(j - 1) has completed, which its commit on s_full
+          // signals (a separate commit per tile would cost the tensor pipe a slot)
+          const bool w = C::NSK == 1
+                             ? mbar_wait(&bars.s_full[(j - 1) & 1], ((j - 1) >> 1) & 1, abort, a.wait)
+                             : mbar_wait(&bars.k_empty[st], ((j / C::NSK) - 1) & 1, abort, a.wait);
+          if (!w) return false;
+        }
         k_issued = j + 1;
         unsigned char *base = sm + C::OFF_K + st * 2 * C::T_BYTES;
         const int krow = (int)(a.k_pad[b] + j * BN);
@@ -174,7 +180,8 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       };
       auto load_v = [&](int j) -> bool {
         const int st = j % C::NSVI;
-        if (j >= C::NSVI && !mbar_wait(&bars.v_empty[st], ((j / C::NSVI) - 1) & 1, abort, a.wait))
+        // one stage: free once P V of tile j - 1 has completed (its commit on s_free)
+        if (j >= 1 && !mbar_wait(&bars.s_free[(j - 1) & 1], ((j - 1) >> 1) & 1, abort, a.wait))
           return false;
         v_issued = j + 1;
         unsigned char *base = sm + C::OFF_V + st * 2 * C::T_BYTES;
@@ -234,8 +241,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
           mma_bf16_ts(tmem + C::COL_O, tp + kk * 8, v, id_pv, (i > 0 || kk > 0) ? 1u : 0u);
           mma_bf16_ts(tmem + C::COL_O, tp + BN / 2 + kk * 8, v, id_pvh, 1u);
         }
-        mma_commit(&bars.v_empty[i % C::NSVI]);
-        mma_commit(&bars.s_free[pb]);
+        mma_commit(&bars.s_free[pb]);  // also frees the value stage
         return true;
       };
       for (int j = 0; ok && j < ntiles; ++j) {
@@ -257,7 +263,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
           mma_bf16(tmem + sb * BN, ql, kh, id_s, 1u);
         }
         mma_commit(&bars.s_full[sb]);
-        mma_commit(&bars.k_empty[st]);
+        if (C::NSK > 1) mma_commit(&bars.k_empty[st]);  // one stage: freed through s_full
         if (C::PV && j >= 1 && !issue_pv(j - 1)) { ok = false; break; }
       }
       if (ok && C::PV && ntiles > 0) ok = issue_pv(ntiles - 1);
