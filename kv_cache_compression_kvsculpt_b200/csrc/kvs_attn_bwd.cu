@@ -71,7 +71,8 @@ struct BwdBars {
   uint64_t q_full[NSTAGE], q_empty[NSTAGE];
   uint64_t s_full[2];               // S of tile i done: [i & 1]
   uint64_t s_free[2];               // S read by the rows: DK [0] (one buffer), COLSUM [i & 1]
-  uint64_t dp_full[2], ds_full[2], dk_done[2];  // DK, per tile parity
+  uint64_t dp_full[2], ds_full[2];  // DK, per tile parity
+  uint64_t dk_done[NSTAGE];         // DK: dK of tile i done, [i % NSTAGE]; frees the stage
   uint64_t done;
   uint32_t tmem;
   int abort;
@@ -111,14 +112,14 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     mbar_init(&bars.v_full, 2 * BK);
     for (int i = 0; i < NSTAGE; ++i) {
       mbar_init(&bars.q_full[i], 2);  // the copies' arrival and the staged l / delta
-      mbar_init(&bars.q_empty[i], 1 + BK);
+      mbar_init(&bars.q_empty[i], BK);  // COLSUM: the rows are done with the stage
+      mbar_init(&bars.dk_done[i], 1);
     }
     for (int i = 0; i < 2; ++i) {
       mbar_init(&bars.s_full[i], 1);
       mbar_init(&bars.s_free[i], BK);
       mbar_init(&bars.dp_full[i], 1);
       mbar_init(&bars.ds_full[i], BK);
-      mbar_init(&bars.dk_done[i], 1);
     }
     mbar_init(&bars.done, 1);
     bars.abort = 0;
@@ -145,8 +146,11 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     for (int i = 0; i < nqt; ++i) {
       const int st = i % C::NS;
       if (i >= C::NS) {
-        const bool w = __all_sync(0xffffffffu,
-                                  mbar_wait(&bars.q_empty[st], ((i / C::NS) - 1) & 1, abort, a.wait));
+        // DK: the last product that reads the stage is dK of tile i - NS, which starts
+        // after the rows are done with its l and delta; COLSUM: only S reads it, and
+        // the rows arrive after S has completed
+        uint64_t *fr = C::DK ? &bars.dk_done[st] : &bars.q_empty[st];
+        const bool w = __all_sync(0xffffffffu, mbar_wait(fr, ((i / C::NS) - 1) & 1, abort, a.wait));
         if (!w) {
           *abort = 1;
           break;
@@ -230,8 +234,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
           mma_bf16_ts(tmem + C::COL_DK, tds + kk * 8, ql, id_dk, 1u);
           mma_bf16_ts(tmem + C::COL_DK, tds + BQ / 2 + kk * 8, qh, id_dk, 1u);
         }
-        mma_commit(&bars.q_empty[i % C::NS]);
-        mma_commit(&bars.dk_done[db]);
+        mma_commit(&bars.dk_done[i % C::NS]);  // frees dP buffer i & 1 and stage i % NS
         return true;
       };
       for (int i = 0; ok && i < nqt; ++i) {
@@ -246,7 +249,8 @@ __global__ void __launch_bounds__(NTHREADS, 1)
           // V reaches tensor memory through the row threads (the first S runs meanwhile);
           // dP buffer i & 1 held dS(i - 2) until dK(i - 2) drained it
           if (i == 0 && !mbar_wait(&bars.v_full, 0, abort, a.wait)) { ok = false; break; }
-          if (i >= 2 && !mbar_wait(&bars.dk_done[i & 1], ((i >> 1) - 1) & 1, abort, a.wait)) {
+          if (i >= 2 && !mbar_wait(&bars.dk_done[(i - 2) % C::NS], ((i - 2) / C::NS) & 1, abort,
+                                   a.wait)) {
             ok = false;
             break;
           }
@@ -263,7 +267,6 @@ __global__ void __launch_bounds__(NTHREADS, 1)
           fence_after_sync();
           issue_s(i, sb * 128);
           mma_commit(&bars.s_full[sb]);
-          mma_commit(&bars.q_empty[st]);
         }
       }
       if (ok && C::DK && nqt > 0) ok = issue_dk(nqt - 1);
@@ -357,7 +360,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         fence_before_sync();
         mbar_arrive(&bars.ds_full[sb]);
       }
-      mbar_arrive(&bars.q_empty[st]);
+      if (!C::DK) mbar_arrive(&bars.q_empty[st]);
     }
     if (!ok) *abort = 1;
     if (C::DK) {
