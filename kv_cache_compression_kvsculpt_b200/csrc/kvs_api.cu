@@ -45,6 +45,10 @@ void set_cuda_error(cudaError_t e, const char *where) {
   snprintf(g_err, sizeof g_err, "%s: %s (%s)", where, cudaGetErrorName(e), cudaGetErrorString(e));
 }
 
+void set_driver_error(int code, const char *where) {
+  snprintf(g_err, sizeof g_err, "%s: CUresult %d", where, code);
+}
+
 static bool aligned(const void *p, size_t a) { return ((uintptr_t)p % a) == 0; }
 
 static int check_offsets(const int64_t *off, int B, int64_t *sum, int *mx, bool allow_empty) {
@@ -122,8 +126,10 @@ size_t carve_work(const HostGeom &g, void *base, Work *w) {
   w->gram = c.take<float>(g.sum_c * g.ld_g);
   w->R = c.take<float>(g.sum_c * g.d);
   w->X = c.take<float>(g.sum_c * g.d);
-  w->dkp = c.take<float>(4 * g.sum_c * g.d);
+  w->dkp = c.take<float>(4 * g.sum_c * g.d);  // 4 d >= 2 x 2 x 64 floats per row (d >= 64)
+  w->chol_p = w->dkp;
   w->chol_t = c.take<float>((int64_t)g.B * ((g.max_c + 63) / 64) * 64 * 64);
+  w->chol_y = c.take<float>(4 * (int64_t)g.B * g.d * 64);
   w->dead = c.take<int>(g.B);
   w->fbuf = c.take<float>(g.B);
   w->Yt = c.take<float>(g.sum_q * g.d);

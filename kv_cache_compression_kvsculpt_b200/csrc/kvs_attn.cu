@@ -13,6 +13,7 @@
 #include <math.h>
 
 #include <algorithm>
+#include <cstdio>
 #include <atomic>
 #include <mutex>
 #include <unordered_map>
@@ -41,24 +42,28 @@ namespace {
 struct MapKey {
   const void *base;
   uint64_t rows, cols;
-  uint32_t box;
+  uint32_t box_rows, box_cols, elem;
   bool operator==(const MapKey &o) const {
-    return base == o.base && rows == o.rows && cols == o.cols && box == o.box;
+    return base == o.base && rows == o.rows && cols == o.cols && box_rows == o.box_rows &&
+           box_cols == o.box_cols && elem == o.elem;
   }
 };
 struct MapKeyHash {
   size_t operator()(const MapKey &k) const {
     return std::hash<const void *>()(k.base) ^ (k.rows * 0x9E3779B97F4A7C15ull) ^
-           (k.cols << 20) ^ ((uint64_t)k.box << 40);
+           (k.cols << 20) ^ ((uint64_t)k.box_rows << 40) ^ ((uint64_t)k.box_cols << 52) ^
+           ((uint64_t)k.elem << 60);
   }
 };
 std::mutex g_map_mu;
 std::unordered_map<MapKey, CUtensorMap, MapKeyHash> g_maps;  // encoded descriptors, reused
-}  // namespace
 
-int make_map_bf16(CUtensorMap *m, const void *base, uint64_t rows, uint64_t cols,
-                  uint32_t box_rows) {
-  const MapKey key{base, rows, cols, box_rows};
+// 2-D map over a row-major [rows, cols] array of `elem`-byte elements, box
+// [box_rows, box_cols] with 128 bytes per box row (128-byte swizzle).
+int make_map_2d(CUtensorMap *m, CUtensorMapDataType type, uint32_t elem, const void *base,
+                uint64_t rows, uint64_t cols, uint32_t box_rows) {
+  const uint32_t box_cols = 128 / elem;
+  const MapKey key{base, rows, cols, box_rows, box_cols, elem};
   {
     std::lock_guard<std::mutex> lock(g_map_mu);
     auto it = g_maps.find(key);
@@ -68,19 +73,39 @@ int make_map_bf16(CUtensorMap *m, const void *base, uint64_t rows, uint64_t cols
     }
   }
   auto fn = encode_fn();
-  if (!fn) return KVS_ECUDA;
+  if (!fn) {
+    set_driver_error(-1, "cuTensorMapEncodeTiled entry point");
+    return KVS_ECUDA;
+  }
   cuuint64_t dims[2] = {(cuuint64_t)cols, (cuuint64_t)(rows > 0 ? rows : 1)};
-  cuuint64_t strides[1] = {(cuuint64_t)cols * 2};
-  cuuint32_t box[2] = {64, box_rows};
+  cuuint64_t strides[1] = {(cuuint64_t)cols * elem};
+  cuuint32_t box[2] = {box_cols, box_rows};
   cuuint32_t es[2] = {1, 1};
-  CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(base), dims, strides,
-                  box, es, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+  CUresult r = fn(m, type, 2, const_cast<void *>(base), dims, strides, box, es,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-  if (r != CUDA_SUCCESS) return KVS_ECUDA;
+  if (r != CUDA_SUCCESS) {
+    char where[160];
+    snprintf(where, sizeof where, "cuTensorMapEncodeTiled (%llu x %llu, elem %u, box %u x %u, base %p)",
+             (unsigned long long)rows, (unsigned long long)cols, elem, box_rows, box_cols, base);
+    set_driver_error((int)r, where);
+    return KVS_ECUDA;
+  }
   std::lock_guard<std::mutex> lock(g_map_mu);
   if (g_maps.size() > 4096) g_maps.clear();
   g_maps.emplace(key, *m);
   return KVS_OK;
+}
+}  // namespace
+
+int make_map_bf16(CUtensorMap *m, const void *base, uint64_t rows, uint64_t cols,
+                  uint32_t box_rows) {
+  return make_map_2d(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, base, rows, cols, box_rows);
+}
+
+int make_map_f32(CUtensorMap *m, const void *base, uint64_t rows, uint64_t cols,
+                 uint32_t box_rows) {
+  return make_map_2d(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, base, rows, cols, box_rows);
 }
 
 namespace {

@@ -109,9 +109,43 @@ int launch_bwd_tc(const BwdMaps &m, const BwdArgs &a, int max_tiles, int B, cuda
 int launch_gemm3_tc(const GemmMaps &m, const GemmArgs3 &a, int tiles_m, int gram, int B,
                     cudaStream_t st);
 
+// Trailing update of the blocked ridge Cholesky (64-column panels) on tensor
+// cores.  The panel's factor columns L (rows below the diagonal block) and the
+// forward-solved rows y of the diagonal block are held as tf32 hi / lo pairs,
+// written by the panel and diagonal-block kernels:
+//   P: [2 parities][hi, lo][sum_c][64]     P[par][h][c_off[b] + i][t] = L[i][j0 + t]
+//   Y: [2 parities][hi, lo][B * d][64]     Y[par][h][b d + c][t] = y[j0 + t][c]
+// with par = (j0 / 64) % 2, so that the next panel can be written while the
+// current update still reads its own.
+struct CholTcMaps {
+  CUtensorMap p;  // fp32, box 32 columns x 128 rows
+  CUtensorMap y;  // fp32, box 32 columns x d rows
+};
+
+struct CholTcArgs {
+  float *G;              // [sum_c, ld] Gram matrix / factor (lower triangle)
+  float *R;              // [sum_c, d] right-hand sides
+  const int64_t *c_off;  // [B+1]
+  const int *dead;       // [B] problems whose factorisation stopped
+  int64_t ld;            // multiple of 4
+  int64_t sum_c;
+  int B, d;
+  int *err;
+  long long wait;
+};
+
+// The trailing lower triangle and right-hand-side rows from j0 + 128 (the next
+// panel's column block takes its update in the diagonal-block and panel kernels).
+// max_c: the longest problem (grid size).
+int launch_chol_update_tc(const CholTcMaps &m, const CholTcArgs &a, int j0, int max_c,
+                          cudaStream_t st);
+
 // Host: a 2-D bf16 tensor map over [rows, cols] (row-major) with a
 // [box_rows, 64]-element box and 128-byte swizzle.
 int make_map_bf16(CUtensorMap *m, const void *base, uint64_t rows, uint64_t cols,
                   uint32_t box_rows);
+// The same for fp32 elements ([box_rows, 32]-element box).
+int make_map_f32(CUtensorMap *m, const void *base, uint64_t rows, uint64_t cols,
+                 uint32_t box_rows);
 
 }  // namespace kvs

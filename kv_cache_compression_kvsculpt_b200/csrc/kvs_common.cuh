@@ -10,6 +10,8 @@ namespace kvs {
 
 // Per-thread text of the last CUDA error (kvs_last_cuda_error).
 void set_cuda_error(cudaError_t e, const char *where);
+// The same for a driver-API failure (CUresult code).
+void set_driver_error(int code, const char *where);
 // Counts kernel launches (kvs_launch_count); called once per launch.
 void count_launch();
 // Cycles a kernel's pipeline wait may spin before the kernel gives up

@@ -34,31 +34,35 @@ struct LbfgsScal {
 // The bf16 operand copies hold each problem's rows at padded offsets (rows
 // rounded up to 128 per problem) with zero rows in the padding.
 struct Work {
-  __nv_bfloat16 *qh, *ql;    // [sum_qpad, d]          training queries, hi/lo
-  __nv_bfloat16 *kh, *kl;    // [max(zpad, cpad), d]   keys, hi/lo
-  __nv_bfloat16 *vh, *vl;    // [max(zpad, cpad), d]   values, hi/lo
-  __nv_bfloat16 *go;         // [sum_qpad, d]          dloss/dY_hat
-  __nv_bfloat16 *yh, *yl;    // [sum_qpad, d]          targets Y, hi/lo
-  __nv_bfloat16 *ahi, *alo;  // [sum_qpad, ld_a]       attention weights for the ridge fit
-  float *lse_h;              // [sum_q]                row lse of the compressed keys
-  float *delta;              // [sum_q]
-  float *partials;           // [B, max q tiles, 2]    per-CTA loss sums
-  int64_t *a_pad_off;        // [B+1]                  padded query-row offsets (qh, ql, go,
-                             //                        yh, yl, ahi, alo): n_q rounded up to 128
-  int64_t *z_pad, *c_pad;    // [B+1] each             padded zone / pair rows of kh .. vl
-  float *gram;               // [sum_c, ld_g]          A^T A + lam I, then its Cholesky factor
-  float *R;                  // [sum_c, d]             A^T Y, then the forward-solved rows
-  float *X;                  // [sum_c, d]             solution of the ridge system
-  float *dkp;                // [4, sum_c, d]          key-gradient partial sums of query splits
-  float *chol_t;             // [B, panels, 64, 64]    transposed inverses of the diagonal blocks
-  int *dead;                 // [B]                    factorisation failed
-  float *fbuf;               // [B]                    loss scratch
-  float *Yt;                 // [sum_q, d]             targets (kvs_compress_batch)
-  float *lset;               // [sum_q]                target log-sum-exp (kvs_compress_batch)
-  float *imp;                // [sum_z]                importance (kvs_compress_batch)
-  int32_t *idx;              // [sum_c]                top-k positions (kvs_compress_batch)
-  int *err;                  // [1]                    set when a kernel wait timed out
-  size_t bytes;
+  __nv_bfloat16 *qh = nullptr, *ql = nullptr;    // [sum_qpad, d]        training queries, hi/lo
+  __nv_bfloat16 *kh = nullptr, *kl = nullptr;    // [max(zpad, cpad), d] keys, hi/lo
+  __nv_bfloat16 *vh = nullptr, *vl = nullptr;    // [max(zpad, cpad), d] values, hi/lo
+  __nv_bfloat16 *go = nullptr;                   // [sum_qpad, d]        dloss/dY_hat
+  __nv_bfloat16 *yh = nullptr, *yl = nullptr;    // [sum_qpad, d]        targets Y, hi/lo
+  __nv_bfloat16 *ahi = nullptr, *alo = nullptr;  // [sum_qpad, ld_a]     attention weights for the ridge fit
+  float *lse_h = nullptr;          // [sum_q]              row lse of the compressed keys
+  float *delta = nullptr;          // [sum_q]
+  float *partials = nullptr;       // [B, max q tiles, 2]  per-CTA loss sums
+  int64_t *a_pad_off = nullptr;    // [B+1]                padded query-row offsets (qh, ql, go,
+                                   //                      yh, yl, ahi, alo): n_q rounded up to 128
+  int64_t *z_pad = nullptr, *c_pad = nullptr;  // [B+1] each  padded zone / pair rows of kh .. vl
+  float *gram = nullptr;           // [sum_c, ld_g]        A^T A + lam I, then its Cholesky factor
+  float *R = nullptr;              // [sum_c, d]           A^T Y, then the forward-solved rows
+  float *X = nullptr;              // [sum_c, d]           solution of the ridge system
+  float *dkp = nullptr;            // [4, sum_c, d]        key-gradient partial sums of query splits
+  float *chol_t = nullptr;         // [B, panels, 64, 64]  transposed inverses of the diagonal blocks
+  float *chol_p = nullptr;         // [2, 2, sum_c, 64]    tf32 hi / lo of a panel's factor rows;
+                                   //                      shares dkp's memory (the fit and the key
+                                   //                      gradient never run at once on one workspace)
+  float *chol_y = nullptr;         // [2, 2, B d, 64]      tf32 hi / lo of the forward-solved rows
+  int *dead = nullptr;             // [B]                  factorisation failed
+  float *fbuf = nullptr;           // [B]                  loss scratch
+  float *Yt = nullptr;             // [sum_q, d]           targets (kvs_compress_batch)
+  float *lset = nullptr;           // [sum_q]              target log-sum-exp (kvs_compress_batch)
+  float *imp = nullptr;            // [sum_z]              importance (kvs_compress_batch)
+  int32_t *idx = nullptr;          // [sum_c]              top-k positions (kvs_compress_batch)
+  int *err = nullptr;              // [1]                  set when a kernel wait timed out
+  size_t bytes = 0;
 };
 
 // Persistent L-BFGS state carved from the caller's state buffer.

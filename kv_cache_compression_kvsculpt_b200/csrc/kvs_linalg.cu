@@ -6,17 +6,23 @@
 // Right-looking blocked algorithm over panels of NB = 64 columns, float32,
 // every problem of the batch advancing together so that all SMs share the work:
 //   per panel j:
-//     diag    factor the diagonal block G_jj = L_jj L_jj^T in shared memory,
+//     diag    apply panel j-1's update to the diagonal block and its
+//             right-hand-side rows, factor G_jj = L_jj L_jj^T in shared memory,
 //             keep T_j = L_jj^-1 and forward-solve its rows y_j = T_j r_j
-//     panel   L_ij = G_ij T_j^T for the rows below
-//     update  G_ik -= L_ij L_kj^T on the trailing lower triangle and
-//             r_i -= L_ij y_j on the right-hand sides
+//     panel   apply panel j-1's update to the column below, L_ij = G_ij T_j^T
+//     update  G_ik -= L_ij L_kj^T on the trailing lower triangle from column
+//             block j+2 on and r_i -= L_ij y_j on those right-hand-side rows,
+//             on tensor cores (kvs_chol_tc.cu) from tf32 hi / lo splits of L_ij
+//             and y_j that the panel and diagonal-block kernels write beside
+//             their results
 //   then one kernel sweeps the panels from the last one: x_j = T_j^T y_j,
 //   y_i -= L_ji^T x_j.
-// Look-ahead: the update is split into the next panel's column and the rest, and
-// the next diagonal block and panel are computed on a second stream while the
-// rest of the update runs.
-// Every 64 x 64 x 64 product runs from shared memory with both operands stored
+// Look-ahead: diag and panel run on a second stream, and the update of panel j
+// on the caller's stream beside diag and panel of j+1, which need only the
+// update of panel j-1 (the splits alternate between two buffers by panel parity,
+// so the next panel never overwrites the operands of the running update).
+// The 64 x 64 x 64 products of the diagonal block, the panel and the backward
+// sweep run from shared memory with both operands stored
 // contraction-index-major (S[t][row]): each thread owns a 4 x 4 output block
 // and forms a rank-1 update from two 128-bit loads per t.  The diagonal block
 // is factored 16 columns at a time: one warp factors and inverts the 16 x 16
@@ -29,7 +35,7 @@
 // steps are skipped.
 #include <math.h>
 
-#include "kvs_internal.cuh"
+#include "kvs_attn_tc.cuh"
 
 namespace kvs {
 namespace {
@@ -44,6 +50,10 @@ struct CholArgs {
   float *R;              // [sum_c, d] right-hand sides -> forward-solved rows
   float *X;              // [sum_c, d] solution
   float *Tt;             // [B, npanel, NB, NB] transposes of the diagonal-block inverses
+  float *P;              // [2, 2, sum_c, NB] tf32 hi / lo of the panel's factor rows
+  float *Y;              // [2, 2, B d, NB] tf32 hi / lo of the forward-solved rows, transposed
+  int64_t sum_c;
+  int B;
   int npanel;
   int *dead;             // [B] DEAD_* bits
   int32_t *status;
@@ -54,6 +64,13 @@ struct CholArgs {
 
 __device__ __forceinline__ int kdim(const CholArgs &a, int b) {
   return (int)(a.c_off[b + 1] - a.c_off[b]);
+}
+
+// x = hi + lo with hi = x rounded toward zero to tf32 (low 13 mantissa bits
+// cleared); lo is exact in fp32.
+__device__ __forceinline__ void split_tf32(float x, float &hi, float &lo) {
+  hi = __uint_as_float(__float_as_uint(x) & 0xffffe000u);
+  lo = x - hi;
 }
 
 __device__ __forceinline__ float4 ld4(const float *p) { return *reinterpret_cast<const float4 *>(p); }
@@ -183,18 +200,58 @@ __device__ __forceinline__ bool factor16(float (*L)[SP], float (*Ts)[SP], int c0
 // transposed) and forward-solve the block's rows of the right-hand sides, y_j = T_j r_j.
 // Rows past jb (the last panel of a problem whose k is not a multiple of 64) are
 // factored as identity rows, so T_j is the identity there.
+// The previous panel's update of this block and of its right-hand-side rows
+// (G_jj -= L_j,j-1 L_j,j-1^T, r_j -= L_j,j-1 y_j-1) is applied here first, in
+// fp32; the trailing update leaves those to this kernel, so that it is not on
+// the path from one panel to the next.
+constexpr int DIAG_SMEM = 3 * NB * SP * 4;
+
 __global__ void __launch_bounds__(256) k_chol_diag(CholArgs a, int j0) {
   const int b = blockIdx.x;
   const int k = kdim(a, b);
   if (j0 >= k || a.dead[b]) return;
   const int jb = min(NB, k - j0);
-  __shared__ __align__(16) float L[NB][SP];   // the block; then T_j^T
-  __shared__ __align__(16) float Ts[NB][SP];  // T_j; then right-hand-side tiles
+  extern __shared__ __align__(16) float dsm[];
+  float (*L)[SP] = reinterpret_cast<float (*)[SP]>(dsm);             // the block; then T_j^T
+  float (*Ts)[SP] = reinterpret_cast<float (*)[SP]>(dsm + NB * SP);  // T_j; then rhs tiles
+  float (*Xs)[SP] = reinterpret_cast<float (*)[SP]>(dsm + 2 * NB * SP);
   __shared__ int bad;
-  float *G = a.G + (a.c_off[b] + j0) * a.ld + j0;
+  const int64_t row0 = a.c_off[b];
+  float *G = a.G + (row0 + j0) * a.ld + j0;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int tx = tid & 15, ty = tid >> 4;
   if (tid == 0) bad = 0;
   load_d(L, G, a.ld, 0, jb, 0, jb);
+  if (j0 > 0) {
+    // Xs[t][r] = L_j,j-1[r][t]: the previous panel's factor rows of this block
+    load_t(Xs, a.G + row0 * a.ld, a.ld, j0, k, j0 - NB, j0);
+    __syncthreads();
+    float acc[4][4];
+    zero_acc(acc);
+    mmk(Xs, Xs, acc, tx, ty);
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+#pragma unroll
+      for (int j = 0; j < 4; ++j) L[4 * ty + i][4 * tx + j] -= acc[i][j];
+    // r_j -= L_j,j-1 y_j-1, 64 right-hand-side columns at a time
+    float *R = a.R + row0 * a.d;
+    for (int c0 = 0; c0 < a.d; c0 += NB) {
+      load_d(Ts, R, a.d, j0 - NB, j0, c0, a.d);  // Ts[t][c] = y_j-1[t][c0 + c]
+      __syncthreads();
+      zero_acc(acc);
+      mmk(Xs, Ts, acc, tx, ty);
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const int r = j0 + 4 * ty + i;
+        if (r < k) {
+          float *p = R + (int64_t)r * a.d + c0 + 4 * tx;
+          const float4 v = ld4(p);
+          st4(p, make_float4(v.x - acc[i][0], v.y - acc[i][1], v.z - acc[i][2], v.w - acc[i][3]));
+        }
+      }
+      __syncthreads();
+    }
+  }
   for (int e = tid; e < NB * SP; e += blockDim.x) (&Ts[0][0])[e] = 0.f;
   __syncthreads();
 #pragma unroll 1
@@ -355,8 +412,7 @@ __global__ void __launch_bounds__(256) k_chol_diag(CholArgs a, int j0) {
   }
   __syncthreads();
   // y_j = T_j r_j, 64 right-hand-side columns at a time (the tile reuses Ts)
-  const int tx = tid & 15, ty = tid >> 4;
-  float *R = a.R + (a.c_off[b] + j0) * a.d;
+  float *R = a.R + (row0 + j0) * a.d;
   for (int c0 = 0; c0 < a.d; c0 += NB) {
     load_d(Ts, R, a.d, 0, jb, c0, a.d);
     __syncthreads();
@@ -369,11 +425,26 @@ __global__ void __launch_bounds__(256) k_chol_diag(CholArgs a, int j0) {
       if (r < jb)
         st4(R + (int64_t)r * a.d + c0 + 4 * tx, make_float4(acc[i][0], acc[i][1], acc[i][2], acc[i][3]));
     }
+    // the trailing update's B operand: Y[par][h][b d + c][t] = split of y[t][c]
+    const int par = (j0 / NB) & 1;
+    float *Yh = a.Y + ((int64_t)(par * 2) * a.B * a.d + (int64_t)b * a.d) * NB;
+    float *Yl = Yh + (int64_t)a.B * a.d * NB;
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      float h[4], l[4];
+#pragma unroll
+      for (int i = 0; i < 4; ++i) split_tf32(acc[i][j], h[i], l[i]);
+      const int64_t o = (int64_t)(c0 + 4 * tx + j) * NB + 4 * ty;
+      st4(Yh + o, make_float4(h[0], h[1], h[2], h[3]));
+      st4(Yl + o, make_float4(l[0], l[1], l[2], l[3]));
+    }
     __syncthreads();
   }
 }
 
 // L_ij = G_ij T_j^T for 64 rows of the panel below the diagonal block.
+// The previous panel's update of these rows of the column block,
+// G_ij -= L_i,j-1 L_j,j-1^T, is applied here first (fp32), as in the diagonal block.
 __global__ void __launch_bounds__(256) k_chol_panel(CholArgs a, int j0) {
   const int b = blockIdx.y;
   const int k = kdim(a, b);
@@ -383,118 +454,44 @@ __global__ void __launch_bounds__(256) k_chol_panel(CholArgs a, int j0) {
   __shared__ __align__(16) float As[NB][SP];  // As[t][r] = G[i0 + r][j0 + t]
   __shared__ __align__(16) float Bs[NB][SP];  // Bs[t][c] = T[c][t]
   const int tid = threadIdx.x;
+  const int tx = tid & 15, ty = tid >> 4;
   const int64_t row0 = a.c_off[b];
+  float acc[4][4];
+  if (j0 > 0) {
+    // acc[r][t] = sum_u L[i0 + r][j0 - 64 + u] L[j0 + t][j0 - 64 + u]
+    load_t(As, a.G + row0 * a.ld, a.ld, i0, k, j0 - NB, j0);
+    load_t(Bs, a.G + row0 * a.ld, a.ld, j0, k, j0 - NB, j0);
+    __syncthreads();
+    zero_acc(acc);
+    mmk(As, Bs, acc, tx, ty);
+    __syncthreads();
+  }
   load_t(As, a.G + row0 * a.ld, a.ld, i0, k, j0, j0 + NB);
   load_d(Bs, a.Tt + ((int64_t)b * a.npanel + j0 / NB) * NB * NB, NB, 0, NB, 0, NB);
   __syncthreads();
-  const int tx = tid & 15, ty = tid >> 4;
-  float acc[4][4];
+  if (j0 > 0) {
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+#pragma unroll
+      for (int j = 0; j < 4; ++j) As[4 * tx + j][4 * ty + i] -= acc[i][j];
+    __syncthreads();
+  }
   zero_acc(acc);
   mmk(As, Bs, acc, tx, ty);
+  const int par = (j0 / NB) & 1;
+  float *Ph = a.P + ((int64_t)(par * 2) * a.sum_c + row0) * NB;
+  float *Pl = Ph + a.sum_c * NB;
 #pragma unroll
   for (int i = 0; i < 4; ++i) {
     const int r = i0 + 4 * ty + i;
-    if (r < k)
+    if (r < k) {
       st4(a.G + (row0 + r) * a.ld + j0 + 4 * tx,
           make_float4(acc[i][0], acc[i][1], acc[i][2], acc[i][3]));
-  }
-}
-
-// Trailing update: tiles (ti >= tj) of G_ik -= L_i L_k^T, and tiles of
-// r_i -= L_i y_j (columns of R in chunks of 64), 64 x 64 outputs per CTA.  The
-// diagonal tiles are written whole: their upper triangle is scratch.  The tiles
-// come in two parts so that the next panel can start early:
-//   part 1: the next panel's column (ti = 0 .. nt-1, tj = 0), then the right-hand
-//           sides of the next diagonal block (ti = 0)
-//   part 2: the other lower-triangle tiles (1 <= tj <= ti), then the other
-//           right-hand-side rows (ti >= 1)
-__global__ void __launch_bounds__(256) k_chol_update(CholArgs a, int j0, int part) {
-  const int b = blockIdx.y;
-  const int k = kdim(a, b);
-  if (j0 >= k || a.dead[b]) return;
-  const int jb = min(NB, k - j0);
-  const int s0 = j0 + jb;
-  const int n2 = k - s0;
-  if (n2 <= 0) return;
-  const int nt = (n2 + NB - 1) / NB;
-  const int ndc = a.d / NB;
-  int t = blockIdx.x;
-  bool rhs = false;
-  int ti, tj;
-  if (part == 1) {
-    if (t >= nt + ndc) return;
-    if (t < nt) {
-      ti = t;
-      tj = 0;
-    } else {
-      rhs = true;
-      ti = 0;
-      tj = t - nt;
-    }
-  } else {
-    const int ntri1 = nt * (nt - 1) / 2;  // the triangle 1 <= tj <= ti < nt
-    if (t < ntri1) {
-      int r = (int)((sqrtf(8.f * t + 1.f) - 1.f) * 0.5f);
-      while (r * (r + 1) / 2 > t) --r;
-      while ((r + 1) * (r + 2) / 2 <= t) ++r;
-      ti = r + 1;
-      tj = t - r * (r + 1) / 2 + 1;
-    } else {
-      t -= ntri1;
-      if (t >= (nt - 1) * ndc) return;
-      rhs = true;
-      ti = 1 + t / ndc;
-      tj = t % ndc;
-    }
-  }
-  __shared__ __align__(16) float As[NB][SP];  // As[t][r] = L[ri + r][j0 + t]
-  __shared__ __align__(16) float Bs[NB][SP];  // Bs[t][c] = L[rk + c][j0 + t], or y[j0 + t][c]
-  const int tid = threadIdx.x;
-  const int tx = tid & 15, ty = tid >> 4;
-  const int64_t row0 = a.c_off[b];
-  const int ri = s0 + ti * NB;
-  float *out;
-  int64_t ldo;
-  int cmax;
-  if (!rhs) {
-    out = a.G + row0 * a.ld + s0 + tj * NB + 4 * tx;
-    ldo = a.ld;
-    cmax = k - (s0 + tj * NB + 4 * tx);  // valid columns from this thread's first
-  } else {
-    out = a.R + row0 * a.d + tj * NB + 4 * tx;
-    ldo = a.d;
-    cmax = 4;
-  }
-  // the outputs' current values first: their loads overlap the tile loads
-  float4 cur[4];
+      float h[4], l[4];
 #pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    const int r = ri + 4 * ty + i;
-    cur[i] = make_float4(0.f, 0.f, 0.f, 0.f);
-    if (r < k && cmax > 0) cur[i] = ld4m(out, ldo, r, 0, cmax);
-  }
-  load_t(As, a.G + row0 * a.ld, a.ld, ri, k, j0, j0 + jb);
-  if (!rhs)
-    load_t(Bs, a.G + row0 * a.ld, a.ld, s0 + tj * NB, k, j0, j0 + jb);
-  else
-    load_d(Bs, a.R + row0 * a.d, a.d, j0, j0 + jb, tj * NB, a.d);
-  __syncthreads();
-  float acc[4][4];
-  zero_acc(acc);
-  mmk(As, Bs, acc, tx, ty);
-#pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    const int r = ri + 4 * ty + i;
-    if (r >= k || cmax <= 0) continue;
-    const float4 v = make_float4(cur[i].x - acc[i][0], cur[i].y - acc[i][1],
-                                 cur[i].z - acc[i][2], cur[i].w - acc[i][3]);
-    float *p = out + (int64_t)r * ldo;
-    if (cmax >= 4) {
-      st4(p, v);
-    } else {
-      p[0] = v.x;
-      if (cmax > 1) p[1] = v.y;
-      if (cmax > 2) p[2] = v.z;
+      for (int j = 0; j < 4; ++j) split_tf32(acc[i][j], h[j], l[j]);
+      st4(Ph + (int64_t)r * NB + 4 * tx, make_float4(h[0], h[1], h[2], h[3]));
+      st4(Pl + (int64_t)r * NB + 4 * tx, make_float4(l[0], l[1], l[2], l[3]));
     }
   }
 }
@@ -611,6 +608,7 @@ __global__ void __launch_bounds__(256) k_chol_store(CholArgs a, float *Vc) {
 struct Lookahead {
   cudaStream_t side = nullptr;
   cudaEvent_t fork = nullptr, join = nullptr;
+  cudaEvent_t updated[2] = {nullptr, nullptr};  // trailing update of panel p done, [p % 2]
 };
 
 static cudaError_t lookahead(int slot, Lookahead **out) {
@@ -629,7 +627,9 @@ static cudaError_t lookahead(int slot, Lookahead **out) {
     if ((e = cudaDeviceGetStreamPriorityRange(&least, &greatest)) != cudaSuccess ||
         (e = cudaStreamCreateWithPriority(&l.side, cudaStreamNonBlocking, greatest)) != cudaSuccess ||
         (e = cudaEventCreateWithFlags(&l.fork, cudaEventDisableTiming)) != cudaSuccess ||
-        (e = cudaEventCreateWithFlags(&l.join, cudaEventDisableTiming)) != cudaSuccess)
+        (e = cudaEventCreateWithFlags(&l.join, cudaEventDisableTiming)) != cudaSuccess ||
+        (e = cudaEventCreateWithFlags(&l.updated[0], cudaEventDisableTiming)) != cudaSuccess ||
+        (e = cudaEventCreateWithFlags(&l.updated[1], cudaEventDisableTiming)) != cudaSuccess)
       return e;
   }
   *out = &l;
@@ -638,41 +638,44 @@ static cudaError_t lookahead(int slot, Lookahead **out) {
 
 int launch_chol_solve(const Batch &Bt, float *Vc, int32_t *status, const Work &w) {
   const HostGeom &g = Bt.g;
+  if (!w.gram || !w.R || !w.X || !w.chol_t || !w.chol_p || !w.chol_y || !w.dead) return KVS_EINVAL;
   const int npanel = (g.max_c + NB - 1) / NB;
-  CholArgs a{w.gram, w.R, w.X, w.chol_t, npanel, w.dead, status, Bt.b->c_off, g.ld_g, g.d};
+  CholArgs a{w.gram, w.R, w.X, w.chol_t, w.chol_p, w.chol_y, g.sum_c, g.B, npanel,
+             w.dead, status, Bt.b->c_off, g.ld_g, g.d};
+  CholTcArgs ta{w.gram, w.R, Bt.b->c_off, w.dead, g.ld_g, g.sum_c, g.B, g.d, w.err, wait_limit()};
+  CholTcMaps tm;
+  int rc;
+  if ((rc = make_map_f32(&tm.p, w.chol_p, 4 * (uint64_t)g.sum_c, NB, 128)) ||
+      (rc = make_map_f32(&tm.y, w.chol_y, 4 * (uint64_t)g.B * g.d, NB, (uint32_t)g.d)))
+    return rc;
   KVS_CUDA_TRY(set_smem_once(k_chol_backward, BWD_SMEM));
+  KVS_CUDA_TRY(set_smem_once(k_chol_diag, DIAG_SMEM));
   Lookahead *la = nullptr;
   KVS_CUDA_TRY(lookahead(Bt.slot, &la));
   KVS_CUDA_TRY(cudaMemsetAsync(w.dead, 0, sizeof(int) * g.B, Bt.st));
   const int ndc = g.d / NB;
-  // diagonal block and panel p: their grid depends only on the longest problem
-  auto head = [&](int p, cudaStream_t st) -> int {
+  // Panel p on the side stream: its diagonal block (with the update by panel p - 1),
+  // then its column below (likewise).  The trailing update of panel p runs on the
+  // caller's stream beside panel p + 1, which waits only for the update of panel
+  // p - 1 (it covers column blocks from p + 2 on).
+  KVS_CUDA_TRY(cudaEventRecord(la->fork, Bt.st));
+  KVS_CUDA_TRY(cudaStreamWaitEvent(la->side, la->fork, 0));
+  for (int p = 0; p < npanel; ++p) {
     const int j0 = p * NB;
-    k_chol_diag<<<g.B, 256, 0, st>>>(a, j0);
+    if (p >= 2) KVS_CUDA_TRY(cudaStreamWaitEvent(la->side, la->updated[p & 1], 0));
+    k_chol_diag<<<g.B, 256, DIAG_SMEM, la->side>>>(a, j0);
     KVS_LAUNCH_CHECK("k_chol_diag");
     const int n2 = g.max_c - j0 - NB;
     if (n2 > 0) {
-      k_chol_panel<<<dim3((n2 + NB - 1) / NB, g.B), 256, 0, st>>>(a, j0);
+      k_chol_panel<<<dim3((n2 + NB - 1) / NB, g.B), 256, 0, la->side>>>(a, j0);
       KVS_LAUNCH_CHECK("k_chol_panel");
     }
-    return KVS_OK;
-  };
-  int rc = head(0, Bt.st);
-  if (rc) return rc;
-  for (int p = 0; p + 1 < npanel; ++p) {
-    const int j0 = p * NB;
-    const int nt = (g.max_c - j0 - NB + NB - 1) / NB;  // trailing block rows of the longest problem
-    k_chol_update<<<dim3(nt + ndc, g.B), 256, 0, Bt.st>>>(a, j0, 1);
-    KVS_LAUNCH_CHECK("k_chol_update");
-    KVS_CUDA_TRY(cudaEventRecord(la->fork, Bt.st));
-    KVS_CUDA_TRY(cudaStreamWaitEvent(la->side, la->fork, 0));
-    if ((rc = head(p + 1, la->side))) return rc;
     KVS_CUDA_TRY(cudaEventRecord(la->join, la->side));
-    if (nt > 1) {
-      k_chol_update<<<dim3(nt * (nt - 1) / 2 + (nt - 1) * ndc, g.B), 256, 0, Bt.st>>>(a, j0, 2);
-      KVS_LAUNCH_CHECK("k_chol_update");
-    }
     KVS_CUDA_TRY(cudaStreamWaitEvent(Bt.st, la->join, 0));
+    if (p + 1 < npanel) {
+      if ((rc = launch_chol_update_tc(tm, ta, j0, g.max_c, Bt.st))) return rc;
+      KVS_CUDA_TRY(cudaEventRecord(la->updated[p & 1], Bt.st));
+    }
   }
   k_chol_backward<<<dim3(ndc, g.B), 256, BWD_SMEM, Bt.st>>>(a);
   KVS_LAUNCH_CHECK("k_chol_backward");
