@@ -326,7 +326,8 @@ int forward_d(const Batch &Bt, const float *Q, const float *Kc, const float *Vc,
       (rc = make_map_bf16(&fm.vl, w.vl, g.sum_cpad, D, FWD_BN)))
     return rc;
   if ((rc = make_map_bf16(&fm.qh, w.qh, g.sum_qpad, D, FWD_BN)) ||
-      (rc = make_map_bf16(&fm.ql, w.ql, g.sum_qpad, D, FWD_BN)))
+      (rc = make_map_bf16(&fm.ql, w.ql, g.sum_qpad, D, FWD_BN)) ||
+      (rc = make_map_f32(&fm.y, Y, g.sum_q, D, FWD_BN)))
     return rc;
   FwdArgs a{};
   a.q_off = Bt.b->q_off;

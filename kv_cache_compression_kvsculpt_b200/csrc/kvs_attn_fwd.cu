@@ -67,6 +67,8 @@ struct Fwd {
   // the single key / value stages are freed by the commits that signal S and P V
   static_assert(!PV || (NSK == 1 && NSVI == 1), "stage release through s_full / s_free");
   static_assert(!WA || NSK == 1, "stage release through s_full");
+  // LOSS: the fp32 target tile (BM x D) takes the key stage after the last S
+  static_assert(MODE != FWD_LOSS || NSK * 2 * T_BYTES >= BM * D * 4, "target tile");
 };
 static_assert(BM == BN, "the Q tile shares the key tile's layout");
 
@@ -77,6 +79,7 @@ struct FwdBars {
   uint64_t s_full[2], s_free[2];
   uint64_t p_full[2];
   uint64_t o_done;
+  uint64_t y_full;       // LOSS: the CTA's target rows landed in the key stage
   uint32_t tmem;
   int abort;
   float red[8];
@@ -107,7 +110,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     k_attn_fwd(const __grid_constant__ CUtensorMap mKh, const __grid_constant__ CUtensorMap mKl,
                const __grid_constant__ CUtensorMap mVh, const __grid_constant__ CUtensorMap mVl,
                const __grid_constant__ CUtensorMap mQh, const __grid_constant__ CUtensorMap mQl,
-               FwdArgs a) {
+               const __grid_constant__ CUtensorMap mY, FwdArgs a) {
   using C = Fwd<D, MODE>;
   extern __shared__ unsigned char smraw[];
   unsigned char *sm = (unsigned char *)(((uintptr_t)smraw + 1023) & ~(uintptr_t)1023);
@@ -136,6 +139,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       mbar_init(&bars.p_full[i], 2 * BM);
     }
     mbar_init(&bars.o_done, 1);
+    mbar_init(&bars.y_full, 1);
     bars.abort = 0;
     fence_barrier_init();
   }
@@ -193,7 +197,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         }
         return true;
       };
-      bool ok = true;
+      bool ok = true, y_issued = false;
       if (C::PV) {
         // key tile j+1 goes ahead of value tile j: S of the next tile never waits
         // behind the value ring
@@ -201,6 +205,20 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         for (int j = 0; ok && j < ntiles; ++j) {
           if (j + 1 < ntiles) ok = load_k(j + 1);
           ok = ok && load_v(j);
+        }
+        if (MODE == FWD_LOSS && ok) {
+          // the CTA's target rows (fp32) into the key stage once the last S is done:
+          // the epilogue reads them from shared memory instead of waiting on global
+          // loads after the last P V
+          if (ntiles > 0)
+            ok = mbar_wait(&bars.s_full[(ntiles - 1) & 1], ((ntiles - 1) >> 1) & 1, abort, a.wait);
+          if (ok) {
+            y_issued = true;
+            mbar_arrive_expect_tx(&bars.y_full, BM * D * 4);
+            for (int r = 0; r < D / 32; ++r)
+              tma_load_2d(sm + C::OFF_K + r * BM * 128, &mY, &bars.y_full, 32 * r,
+                          (int)(q_begin + q0));
+          }
         }
       } else {
         for (int j = 0; ok && j < ntiles; ++j) ok = load_k(j);
@@ -212,6 +230,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
           mbar_wait(&bars.k_full[j % C::NSK], (j / C::NSK) & 1);
         for (int j = (v_issued > C::NSVI ? v_issued - C::NSVI : 0); j < v_issued; ++j)
           mbar_wait(&bars.v_full[j % C::NSVI], (j / C::NSVI) & 1);
+        if (y_issued) mbar_wait(&bars.y_full, 0);
       }
     }
   } else if (warp == 9) {
@@ -405,6 +424,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       const float lse = (mref + log2f(lsum)) * 0.6931471805599453f;
       if (C::PV) {
         if (!mbar_wait(&bars.o_done, 0, abort, a.wait)) *abort = 1;
+        if (MODE == FWD_LOSS && !mbar_wait(&bars.y_full, 0, abort, a.wait)) *abort = 1;
         fence_after_sync();
       }
       const float inv = 1.f / lsum;
@@ -456,11 +476,12 @@ __global__ void __launch_bounds__(NTHREADS, 1)
               yl[ch] = make_uint4(l[0], l[1], l[2], l[3]);
             }
           } else {
-            const float4 *y4 = reinterpret_cast<const float4 *>(a.y_in + grow * D + c0);
+            // Y[row][c0 .. c0 + 31]: one 128-byte swizzled row of box c0 / 32
+            const unsigned char *yrow = sm + C::OFF_K + (c0 >> 5) * (BM * 128) + row * 128;
             float ev[32];
 #pragma unroll
             for (int e = 0; e < 8; ++e) {
-              const float4 v = y4[e];
+              const float4 v = *reinterpret_cast<const float4 *>(yrow + ((e ^ (row & 7)) << 4));
               ev[4 * e] = o[4 * e] - v.x;
               ev[4 * e + 1] = o[4 * e + 1] - v.y;
               ev[4 * e + 2] = o[4 * e + 2] - v.z;
@@ -539,7 +560,8 @@ int launch_fwd_tc(const FwdMaps &m, const FwdArgs &a, int max_tiles, int B, cuda
   static_assert(C::SMEM + sizeof(FwdBars) <= 232448, "shared memory");
   auto kern = k_attn_fwd<D, MODE>;
   KVS_CUDA_TRY(set_smem_once(kern, C::SMEM));
-  kern<<<dim3(max_tiles, B), NTHREADS, C::SMEM, st>>>(m.kh, m.kl, m.vh, m.vl, m.qh, m.ql, a);
+  kern<<<dim3(max_tiles, B), NTHREADS, C::SMEM, st>>>(m.kh, m.kl, m.vh, m.vl, m.qh, m.ql,
+                                                      MODE == FWD_LOSS ? m.y : m.kh, a);
   KVS_LAUNCH_CHECK("k_attn_fwd");
   return KVS_OK;
 }

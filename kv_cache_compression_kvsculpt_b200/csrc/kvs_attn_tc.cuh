@@ -33,6 +33,7 @@ __device__ __forceinline__ float go_scale(int nq, int d, float w_out) {
 struct FwdMaps {
   CUtensorMap kh, kl, vh, vl;
   CUtensorMap qh, ql;     // query tiles (box 64 columns x FWD_BN rows)
+  CUtensorMap y;          // LOSS: targets, fp32 [sum_q, d], box 32 columns x FWD_BN rows
 };
 
 struct FwdArgs {
