@@ -204,7 +204,29 @@ __device__ __forceinline__ bool factor16(float (*L)[SP], float (*Ts)[SP], int c0
 // (G_jj -= L_j,j-1 L_j,j-1^T, r_j -= L_j,j-1 y_j-1) is applied here first, in
 // fp32; the trailing update leaves those to this kernel, so that it is not on
 // the path from one panel to the next.
-constexpr int DIAG_SMEM = 3 * NB * SP * 4;
+// Every input tile is requested at entry (asynchronous copies for the row-major
+// ones), and the block's right-hand-side rows stay in shared memory from the
+// update through the forward solve.
+constexpr int DIAG_SMEM = 7 * NB * SP * 4;
+
+// 16-byte asynchronous copy global -> shared; bytes past src_bytes are zero.
+__device__ __forceinline__ void cp16(void *dst, const void *src, int src_bytes) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(
+                   (uint32_t)__cvta_generic_to_shared(dst)),
+               "l"(src), "r"(src_bytes)
+               : "memory");
+}
+
+// S[r][c] = M[r0 + r][c0 + c] by asynchronous copies, zero for r0 + r >= rmax or
+// c0 + c >= cmax (M row-major, ld and c0 multiples of 4).
+__device__ __forceinline__ void cp_tile(float (*S)[SP], const float *M, int64_t ld, int r0,
+                                        int rmax, int c0, int cmax) {
+  for (int e = threadIdx.x; e < NB * NB / 4; e += blockDim.x) {
+    const int r = e >> 4, c = (e & 15) * 4;
+    const int n = (r0 + r < rmax) ? max(0, min(4, cmax - (c0 + c))) : 0;
+    cp16(&S[r][c], M + (int64_t)(n > 0 ? r0 + r : 0) * ld + (n > 0 ? c0 + c : 0), 4 * n);
+  }
+}
 
 __global__ void __launch_bounds__(256) k_chol_diag(CholArgs a, int j0) {
   const int b = blockIdx.x;
@@ -213,19 +235,34 @@ __global__ void __launch_bounds__(256) k_chol_diag(CholArgs a, int j0) {
   const int jb = min(NB, k - j0);
   extern __shared__ __align__(16) float dsm[];
   float (*L)[SP] = reinterpret_cast<float (*)[SP]>(dsm);             // the block; then T_j^T
-  float (*Ts)[SP] = reinterpret_cast<float (*)[SP]>(dsm + NB * SP);  // T_j; then rhs tiles
+  float (*Ts)[SP] = reinterpret_cast<float (*)[SP]>(dsm + NB * SP);  // T_j
   float (*Xs)[SP] = reinterpret_cast<float (*)[SP]>(dsm + 2 * NB * SP);
+  // right-hand-side rows of this block (r_j, then y_j) and of the previous one
+  // (y_j-1), 64 columns per tile
+  float (*Rb[2])[SP] = {reinterpret_cast<float (*)[SP]>(dsm + 3 * NB * SP),
+                        reinterpret_cast<float (*)[SP]>(dsm + 4 * NB * SP)};
+  float (*Yp[2])[SP] = {reinterpret_cast<float (*)[SP]>(dsm + 5 * NB * SP),
+                        reinterpret_cast<float (*)[SP]>(dsm + 6 * NB * SP)};
   __shared__ int bad;
   const int64_t row0 = a.c_off[b];
   float *G = a.G + (row0 + j0) * a.ld + j0;
+  const float *R = a.R + row0 * a.d;
+  const int ndc = a.d / NB;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int tx = tid & 15, ty = tid >> 4;
   if (tid == 0) bad = 0;
-  load_d(L, G, a.ld, 0, jb, 0, jb);
+  cp_tile(L, G, a.ld, 0, jb, 0, jb);
+  for (int ch = 0; ch < ndc; ++ch) {
+    cp_tile(Rb[ch], R, a.d, j0, k, ch * NB, a.d);
+    if (j0 > 0) cp_tile(Yp[ch], R, a.d, j0 - NB, j0, ch * NB, a.d);
+  }
+  asm volatile("cp.async.commit_group;" ::: "memory");
+  // Xs[t][r] = L_j,j-1[r][t]: the previous panel's factor rows of this block
+  if (j0 > 0) load_t(Xs, a.G + row0 * a.ld, a.ld, j0, k, j0 - NB, j0);
+  asm volatile("cp.async.wait_group 0;" ::: "memory");
+  __syncthreads();
   if (j0 > 0) {
-    // Xs[t][r] = L_j,j-1[r][t]: the previous panel's factor rows of this block
-    load_t(Xs, a.G + row0 * a.ld, a.ld, j0, k, j0 - NB, j0);
-    __syncthreads();
+    // the previous panel's update: G_jj -= L_j,j-1 L_j,j-1^T, r_j -= L_j,j-1 y_j-1
     float acc[4][4];
     zero_acc(acc);
     mmk(Xs, Xs, acc, tx, ty);
@@ -233,23 +270,13 @@ __global__ void __launch_bounds__(256) k_chol_diag(CholArgs a, int j0) {
     for (int i = 0; i < 4; ++i)
 #pragma unroll
       for (int j = 0; j < 4; ++j) L[4 * ty + i][4 * tx + j] -= acc[i][j];
-    // r_j -= L_j,j-1 y_j-1, 64 right-hand-side columns at a time
-    float *R = a.R + row0 * a.d;
-    for (int c0 = 0; c0 < a.d; c0 += NB) {
-      load_d(Ts, R, a.d, j0 - NB, j0, c0, a.d);  // Ts[t][c] = y_j-1[t][c0 + c]
-      __syncthreads();
+    for (int ch = 0; ch < ndc; ++ch) {
       zero_acc(acc);
-      mmk(Xs, Ts, acc, tx, ty);
+      mmk(Xs, Yp[ch], acc, tx, ty);
 #pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        const int r = j0 + 4 * ty + i;
-        if (r < k) {
-          float *p = R + (int64_t)r * a.d + c0 + 4 * tx;
-          const float4 v = ld4(p);
-          st4(p, make_float4(v.x - acc[i][0], v.y - acc[i][1], v.z - acc[i][2], v.w - acc[i][3]));
-        }
-      }
-      __syncthreads();
+      for (int i = 0; i < 4; ++i)
+#pragma unroll
+        for (int j = 0; j < 4; ++j) Rb[ch][4 * ty + i][4 * tx + j] -= acc[i][j];
     }
   }
   for (int e = tid; e < NB * SP; e += blockDim.x) (&Ts[0][0])[e] = 0.f;
@@ -411,24 +438,23 @@ __global__ void __launch_bounds__(256) k_chol_diag(CholArgs a, int j0) {
     L[c][r] = v;
   }
   __syncthreads();
-  // y_j = T_j r_j, 64 right-hand-side columns at a time (the tile reuses Ts)
-  float *R = a.R + (row0 + j0) * a.d;
-  for (int c0 = 0; c0 < a.d; c0 += NB) {
-    load_d(Ts, R, a.d, 0, jb, c0, a.d);
-    __syncthreads();
+  // y_j = T_j r_j, 64 right-hand-side columns at a time
+  float *Rj = a.R + (row0 + j0) * a.d;
+  const int par = (j0 / NB) & 1;
+  float *Yh = a.Y + ((int64_t)(par * 2) * a.B * a.d + (int64_t)b * a.d) * NB;
+  float *Yl = Yh + (int64_t)a.B * a.d * NB;
+  for (int ch = 0; ch < ndc; ++ch) {
+    const int c0 = ch * NB;
     float acc[4][4];
     zero_acc(acc);
-    mmk(L, Ts, acc, tx, ty);
+    mmk(L, Rb[ch], acc, tx, ty);
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
       const int r = 4 * ty + i;
       if (r < jb)
-        st4(R + (int64_t)r * a.d + c0 + 4 * tx, make_float4(acc[i][0], acc[i][1], acc[i][2], acc[i][3]));
+        st4(Rj + (int64_t)r * a.d + c0 + 4 * tx, make_float4(acc[i][0], acc[i][1], acc[i][2], acc[i][3]));
     }
     // the trailing update's B operand: Y[par][h][b d + c][t] = split of y[t][c]
-    const int par = (j0 / NB) & 1;
-    float *Yh = a.Y + ((int64_t)(par * 2) * a.B * a.d + (int64_t)b * a.d) * NB;
-    float *Yl = Yh + (int64_t)a.B * a.d * NB;
 #pragma unroll
     for (int j = 0; j < 4; ++j) {
       float h[4], l[4];
@@ -438,7 +464,6 @@ __global__ void __launch_bounds__(256) k_chol_diag(CholArgs a, int j0) {
       st4(Yh + o, make_float4(h[0], h[1], h[2], h[3]));
       st4(Yl + o, make_float4(l[0], l[1], l[2], l[3]));
     }
-    __syncthreads();
   }
 }
 
