@@ -327,6 +327,32 @@ def run_loss_grad_only(args, job, wl, rank, world, dist):
                           "peak_source": f"{peak_src} {args.peak_key}"}), flush=True)
 
 
+def run_fit_only(args, job, wl, rank, world, dist):
+    """The ridge fit alone: kvs_fit_values over the batch at its Select+Fit point
+    (one solve with no outer iterations first), `--steps` timed calls after
+    `--warmup` untimed ones.  A kernel-level measurement, not the bench step."""
+    torch, K = job.torch, job.K
+    job.sched.outer = 0
+    job.step()
+    B = job.batch.B
+    Y = torch.empty_like(job.Q)
+    lse = torch.empty(job.batch.sum_q, device=job.Q.device)
+    K.kvs_targets(job.batch, job.Q, job.dev["Kz"], job.dev["Vz"], Y, lse, None, job.ws)
+    Vc = torch.empty_like(job.Vc)
+    status = torch.zeros(B, dtype=torch.int32, device=job.Q.device)
+
+    def fit():
+        K.kvs_fit_values(job.batch, job.Q, job.Kc, Y, wl.lam, Vc, status, job.ws)
+
+    for _ in range(args.warmup):
+        fit()
+    ms = time_region(torch, fit, args.steps, dist) / args.steps
+    if rank == 0:
+        print(json.dumps({"metric": "kvs_fit_values ms per call (whole batch)", "value": round(ms, 4),
+                          "unit": "ms", "problems": B, "workload": wl.name,
+                          "status_nonzero": int((status != 0).sum())}), flush=True)
+
+
 def run_gpu(args):
     import torch
     import kv_cache_compression_kvsculpt_b200 as K
@@ -349,6 +375,8 @@ def run_gpu(args):
               problems=args.problems)
     if args.loss_grad_only:
         return run_loss_grad_only(args, job, wl, rank, world, dist)
+    if args.fit_only:
+        return run_fit_only(args, job, wl, rank, world, dist)
     for _ in range(args.warmup):
         job.step()
     torch.cuda.synchronize()
@@ -597,6 +625,8 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--problems", type=int, default=None,
                     help="only the first N problems of the workload (kernel profiling)")
+    ap.add_argument("--fit-only", action="store_true",
+                    help="time kvs_fit_values alone over the batch (kernel-level)")
     ap.add_argument("--loss-grad-only", action="store_true",
                     help="time kvs_loss_grad alone (kernel measurement, not the bench step)")
     ap.add_argument("--cpu-budget", type=float, default=20.0)
