@@ -153,9 +153,39 @@ def add_emulated():
                 json.dump(out, fh, indent=1)
 
 
+def add_pilot_bands():
+    """Add, for every adaptive problem, the pilot MSE of the pilot schedule run with
+    perturbed evaluations (the same levels and seeds as the final-loss bands) and
+    with the library's rounding emulated: the pilot is as trajectory-sensitive as
+    the full solve, so its MSE is compared with a band too."""
+    with open(OUT) as fh:
+        out = json.load(fh)
+    case = out["cases"]["qwen_cache_adaptive"]
+    wl = W.WORKLOADS["qwen_cache_adaptive"]
+    ids = [tuple(p["id"]) for p in case["problems"]]
+    k_uni = case["total"] // len(ids)
+    pilot = schedule(wl, pilot=True)
+    for (Q, Kz, Vz), p in zip(float32_inputs(wl, ids), case["problems"]):
+        if "pilot_band" in p:
+            continue
+        t0 = time.time()
+        p["pilot_band"] = [float(O.compress(Q, Kz, Vz, k_uni, pilot,
+                                            evaluate=noisy_evaluations(*GPU_LEVELS, s))["mse_out"])
+                           for s in range(BAND_SEEDS)]
+        p["pilot_emulated"] = float(O.compress(Q, Kz, Vz, k_uni, pilot,
+                                               evaluate=emulated_evaluations())["mse_out"])
+        print(f"adaptive {p['id']}: pilot band {[round(x / p['pilot_mse'], 4) for x in p['pilot_band']]}"
+              f" emulated {p['pilot_emulated'] / p['pilot_mse']:.4f} ({time.time() - t0:.0f} s)",
+              flush=True)
+        with open(OUT, "w") as fh:
+            json.dump(out, fh, indent=1)
+
+
 def main():
     if "--add-emulated" in sys.argv:
         return add_emulated()
+    if "--add-pilot-bands" in sys.argv:
+        return add_pilot_bands()
     out = {"generator": "tests/golden/make_fullsize.py (oracle/ only)", "seed": 0,
            "band_levels": list(GPU_LEVELS), "cases": {}}
     for name in ("qwen_cache_r03", "qwen_cache_r05", "qwen_cache_r07"):

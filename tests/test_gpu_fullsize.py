@@ -12,6 +12,9 @@ oracle needs minutes per problem at these sizes, so its results are stored in
 tests/golden/fullsize_oracle.json, written by tests/golden/make_fullsize.py
 from oracle/ alone; checksums of the inputs guard against a changed generator.
 
+The adaptive case's pilot MSEs are compared the same way, with the band of
+the pilot schedule's oracle runs.
+
 The problems include the layers with the largest (3.97) and the smallest
 (0.54) per-layer key scale: the largest makes attention sharpest, where
 precision and conditioning are hardest.  Bars: the Select+Fit loss within rel
@@ -105,10 +108,16 @@ def test_adaptive_matches_oracle():
     k = np.asarray(res["k"])
     mse_or = np.array([p["pilot_mse"] for p in g["problems"]])
     k_or = np.array([p["k"] for p in g["problems"]])
-    # pilot signal within 5 %; the allocation is exactly the oracle's allocation of
-    # the GPU's pilot MSEs (an integer result decided from the same floats), and
-    # within 1 % of the budget of the oracle's own allocation
-    np.testing.assert_allclose(res["pilot_mse"], mse_or, rtol=0.05)
+    # pilot signal within 5 % of the band its oracle runs span (exact, perturbed at the
+    # library's precision, rounding emulated: the 12 x 5 pilot is as trajectory-sensitive
+    # as the full solve); the allocation is exactly the oracle's allocation of the GPU's
+    # pilot MSEs (an integer result decided from the same floats), and within 1 % of the
+    # budget of the oracle's own allocation
+    for b, p in enumerate(g["problems"]):
+        ref = [p["pilot_mse"]] + p.get("pilot_band", []) + (
+            [p["pilot_emulated"]] if "pilot_emulated" in p else [])
+        assert 0.95 * min(ref) <= res["pilot_mse"][b] <= 1.05 * max(ref), \
+            (p["id"], float(res["pilot_mse"][b]), ref)
     want = O.pilot_allocate(np.asarray(res["pilot_mse"], np.float64), total, wl.k_min, z, wl.alpha)
     np.testing.assert_array_equal(k, want)
     assert np.abs(k - k_or).sum() <= 0.01 * total, (k.tolist(), k_or.tolist())
