@@ -281,6 +281,35 @@ def test_fit_values(case):
         assert rel(gv[co[b]:co[b + 1]], Vo) < 1e-3, b
 
 
+# several problems of large, ragged k in one batch: the tensor-core trailing update
+# of the Cholesky runs many 128 x 128 tiles per panel with partial row and column
+# tiles, and problems leave the panel loop at different panels
+BIGK = W.Workload("bigk", 1, 3, 2, d=128, N=1300, m=100, g=2, n_syn=500, k=64,
+                  layer_scale=True, outer=3, steps=4)
+BIGK_K = [700, 513, 129, 1000, 64, 385]
+
+
+@pytest.mark.parametrize("d", [128, 64])
+def test_fit_values_large_ragged_k(d):
+    c = Case(BIGK.with_(d=d), k=BIGK_K)
+    K = c.K
+    Kcs, _, tgt = select_fit_point(c, 0.2)
+    Y = dev(np.concatenate([t[0] for t in tgt]))
+    Vc = torch.zeros((c.batch.sum_c, c.wl.d), device="cuda")
+    status = torch.zeros(c.bt.B, dtype=torch.int32, device="cuda")
+    K.kvs_fit_values(c.batch, c.Q, dev(np.concatenate(Kcs)), Y, 1e-3, Vc, status, c.ws)
+    torch.cuda.synchronize()
+    gv = host(Vc)
+    assert not host(status).any()
+    co = c.batch.c_off_h
+    errs = []
+    for b in range(c.bt.B):
+        Vo, st = O.ridge_fit(c.Qs[b], Kcs[b], tgt[b][0], 1e-3)
+        assert st == O.ST_OK
+        errs.append(rel(gv[co[b]:co[b + 1]], Vo))
+    assert max(errs) < 1e-3, errs
+
+
 def test_fit_not_pd_keeps_values():
     c = Case(W.WORKLOADS["single_d64"], k=2)
     K = c.K
