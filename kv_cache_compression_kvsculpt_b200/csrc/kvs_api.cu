@@ -762,6 +762,7 @@ int kvs_compress_batch(const kvs_batch *batch, const kvs_schedule *sched, const 
       v.Bt.g = pt[p].g;
       v.Bt.b = &pt[p].kb;
       v.Bt.slot = p;
+      v.Bt.share = P.n;
       v.Bt.st = p == 0 ? Bt.st : ps->st[p];
       if (p > 0) KVS_CUDA_TRY(cudaStreamWaitEvent(v.Bt.st, ps->fork, 0));
       carve_work(v.Bt.g, static_cast<char *>(ws) + pt[p].ws_off, &v.w);

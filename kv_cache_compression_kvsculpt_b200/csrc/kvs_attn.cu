@@ -201,16 +201,31 @@ int sm_count() {
   return v;
 }
 
-// Query-range splits of the key-gradient kernel: the one whose last wave of
-// CTAs wastes least, with a small charge per split for the extra prologue,
-// epilogue and partial-sum traffic, and at least 8 query tiles per split.
-int bwd_split(int ctas, int nqt_max) {
+// Work items per CTA of the attention kernels.  A whole batch takes several
+// query (key) tiles per CTA, so that each CTA's setup and epilogue overlap its next
+// tile; the sub-batches of a partitioned solve, which run beside one another on
+// the same SMs, take one tile per CTA (shorter CTAs interleave better: measured
+// on the 56-problem cache, 360 against 363-372 ms per solve step).
+int fwd_items(const Batch &Bt) { return Bt.share > 1 ? FWD_ITEMS_SHARED : FWD_ITEMS; }
+int bwd_items(const Batch &Bt) { return Bt.share > 1 ? 1 : BWD_ITEMS; }
+
+// Query splits of the key gradient: the largest key-tile CTA of the batch runs
+// `items` key tiles over ceil(nqt / sp) query tiles each.  The split count
+// minimises an estimate of the kernel's time: whole waves of CTAs times the
+// CTA's time (2.3 us per query tile, 7.5 us of setup, copies and epilogue per
+// CTA, 3 us more per further key tile), plus the reduction of sp partial sums
+// (bytes_per_sum each, read and summed at 6 TB/s), with at least 8 query tiles
+// per split.
+int bwd_split(int ctas, int nqt_max, double bytes_per_sum, int items) {
   const int nsm = sm_count();
   int best = 1;
   double bc = 1e30;
-  for (int sp = 1; sp <= 4; ++sp) {
+  for (int sp = 1; sp <= 4; ++sp) {  // the workspace holds four partial sums
     if (sp > 1 && nqt_max / sp < 8) break;
-    const double cost = std::ceil((double)ctas * sp / nsm) / sp + 0.05 * sp;
+    const int per = (nqt_max + sp - 1) / sp;
+    const double waves = std::ceil((double)ctas * sp / nsm);
+    double cost = waves * (2.3 * items * per + 7.5 + 3.0 * (items - 1));
+    if (sp > 1) cost += (sp + 1) * bytes_per_sum / 6e6;  // us
     if (cost < bc - 1e-9) {
       bc = cost;
       best = sp;
@@ -276,7 +291,7 @@ int targets_d(const Batch &Bt, const float *Q, const float *Kz, const float *Vz,
   a.lse_out = lse;
   a.err = w.err;
   a.wait = wait_limit();
-  if ((rc = launch_fwd_tc<D, FWD_TARGETS>(fm, a, max_qtiles(g), g.B, Bt.st))) return rc;
+  if ((rc = launch_fwd_tc<D, FWD_TARGETS>(fm, a, max_qtiles(g), fwd_items(Bt), g.B, Bt.st))) return rc;
   if (!imp) return KVS_OK;
   BwdMaps bm;
   if ((rc = make_map_bf16(&bm.kh, w.kh, g.sum_zpad, D, 128)) ||
@@ -297,7 +312,7 @@ int targets_d(const Batch &Bt, const float *Q, const float *Kz, const float *Vz,
   ba.err = w.err;
   ba.wait = wait_limit();
   ba.nsplit = 1;
-  return launch_bwd_tc<D, BWD_COLSUM>(bm, ba, (g.max_z + 127) / 128, g.B, Bt.st);
+  return launch_bwd_tc<D, BWD_COLSUM>(bm, ba, (g.max_z + 127) / 128, bwd_items(Bt), g.B, Bt.st);
 }
 
 // bf16 hi/lo copies of the keys and values of the compressed pairs.
@@ -349,7 +364,7 @@ int forward_d(const Batch &Bt, const float *Q, const float *Kc, const float *Vc,
   a.w_lse = w_lse;
   a.err = w.err;
   a.wait = wait_limit();
-  if ((rc = launch_fwd_tc<D, FWD_LOSS>(fm, a, max_qtiles(g), g.B, Bt.st))) return rc;
+  if ((rc = launch_fwd_tc<D, FWD_LOSS>(fm, a, max_qtiles(g), fwd_items(Bt), g.B, Bt.st))) return rc;
   if (!reduce) return KVS_OK;
   k_loss_reduce<<<(g.B + 127) / 128, 128, 0, Bt.st>>>(w.partials, max_qtiles(g), Bt.b->q_off, D,
                                                       w_out, w_lse, loss, parts, flt, g.B);
@@ -385,14 +400,16 @@ int backward_d(const Batch &Bt, const float *Vc, float w_out, float *dKc, Filter
   ba.wait = wait_limit();
   ba.nsplit = 1;
   const int ktiles = (g.max_c + 127) / 128;
-  const int ns = bwd_split(ktiles * g.B, (g.max_q + 63) / 64);
+  const int items = bwd_items(Bt);
+  const int ns = bwd_split((ktiles + items - 1) / items * g.B, (g.max_q + 63) / 64,
+                           (double)g.sum_c * D * 4, items);
   if (ns > 1) {
     // partial sums of ns query ranges, then their fixed-order sum
     ba.nsplit = ns;
     ba.dk = w.dkp;
     ba.dk_stride = g.sum_c * D;
   }
-  if ((rc = launch_bwd_tc<D, BWD_DK>(bm, ba, ktiles, g.B, Bt.st))) return rc;
+  if ((rc = launch_bwd_tc<D, BWD_DK>(bm, ba, ktiles, items, g.B, Bt.st))) return rc;
   if (ns == 1) return KVS_OK;
   k_dk_reduce<<<dim3(std::min<int64_t>(((int64_t)g.max_c * D / 4 + 255) / 256, 32), g.B), 256, 0,
                 Bt.st>>>(w.dkp, ns, g.sum_c * D, Bt.b->c_off, D, flt, dKc);
@@ -434,14 +451,14 @@ int fit_d(const Batch &Bt, const float *Q, const float *Kc, const float *Y, floa
   a.lse_out = w.lse_h;
   a.err = w.err;
   a.wait = wait_limit();
-  if ((rc = launch_fwd_tc<D, FWD_STATS>(fm, a, max_qtiles(g), g.B, Bt.st))) return rc;
+  if ((rc = launch_fwd_tc<D, FWD_STATS>(fm, a, max_qtiles(g), fwd_items(Bt), g.B, Bt.st))) return rc;
   a.flt = Filter{nullptr, 0, 0};
   a.lse_in = w.lse_h;
   a.a_hi = w.ahi;
   a.a_lo = w.alo;
   a.ld_a = g.ld_a;
   a.a_pad_off = w.a_pad_off;
-  if ((rc = launch_fwd_tc<D, FWD_WRITE_A>(fm, a, max_qtiles(g), g.B, Bt.st))) return rc;
+  if ((rc = launch_fwd_tc<D, FWD_WRITE_A>(fm, a, max_qtiles(g), fwd_items(Bt), g.B, Bt.st))) return rc;
   GemmMaps gm;
   if ((rc = make_map_bf16(&gm.ah, w.ahi, g.sum_qpad, g.ld_a, 64)) ||
       (rc = make_map_bf16(&gm.al, w.alo, g.sum_qpad, g.ld_a, 64)))

@@ -73,7 +73,9 @@ struct BwdBars {
   uint64_t s_free[2];               // S read by the rows: DK [0] (one buffer), COLSUM [i & 1]
   uint64_t dp_full[2], ds_full[2];  // DK, per tile parity
   uint64_t dk_done[NSTAGE];         // DK: dK of tile i done, [i % NSTAGE]; frees the stage
-  uint64_t done;
+  uint64_t done;                    // the work item's products are done (once per item)
+  uint64_t dk_free;                 // DK: the rows have read the item's dK (once per item)
+  uint64_t all_done;                // every MMA of the CTA has completed
   uint32_t tmem;
   int abort;
   __align__(16) float lse2[NSTAGE][BQ];  // row lse in log2 units (+inf past the problem)
@@ -96,8 +98,12 @@ __global__ void __launch_bounds__(NTHREADS, 1)
   if (a.flt.skip(b)) return;
   const int64_t k_begin = a.k_off[b];
   const int nk = (int)(a.k_off[b + 1] - k_begin);
-  const int k0 = blockIdx.x * BK;
-  if (k0 >= nk) return;
+  // work items: key tiles blockIdx.x, blockIdx.x + gridDim.x, ... of problem b, one
+  // after another (each over the same query range); the next item's key tile loads
+  // while the current item's last products and epilogue run
+  const int nkt = (nk + BK - 1) / BK;
+  const int n_items = (int)blockIdx.x < nkt ? (nkt - 1 - (int)blockIdx.x) / (int)gridDim.x + 1 : 0;
+  if (n_items == 0) return;
   const int64_t q_begin = a.q_off[b];
   const int nq = (int)(a.q_off[b + 1] - q_begin);
   // split z of the problem's query tiles: tiles t0 .. t0 + nqt - 1 (DK partial sums)
@@ -122,6 +128,8 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       mbar_init(&bars.ds_full[i], BK);
     }
     mbar_init(&bars.done, 1);
+    mbar_init(&bars.dk_free, 2 * BK);
+    mbar_init(&bars.all_done, 1);
     bars.abort = 0;
     fence_barrier_init();
   }
@@ -134,54 +142,71 @@ __global__ void __launch_bounds__(NTHREADS, 1)
 
   if (warp == 8) {
     // ------------------------------------------------------------ producer
-    if (lane == 0) {
-      const int krow = (int)(a.k_pad[b] + k0);
-      mbar_arrive_expect_tx(&bars.k_full, 2 * C::K_BYTES);
-      for (int r = 0; r < C::KD; ++r) {
-        tma_load_2d(sm + r * BK * 128, &mKh, &bars.k_full, 64 * r, krow);
-        tma_load_2d(sm + C::K_BYTES + r * BK * 128, &mKl, &bars.k_full, 64 * r, krow);
-      }
-    }
-    int issued = 0;
-    for (int i = 0; i < nqt; ++i) {
-      const int st = i % C::NS;
-      if (i >= C::NS) {
-        // DK: the last product that reads the stage is dK of tile i - NS, which starts
-        // after the rows are done with its l and delta; COLSUM: only S reads it, and
-        // the rows arrive after S has completed
-        uint64_t *fr = C::DK ? &bars.dk_done[st] : &bars.q_empty[st];
-        const bool w = __all_sync(0xffffffffu, mbar_wait(fr, ((i / C::NS) - 1) & 1, abort, a.wait));
-        if (!w) {
-          *abort = 1;
-          break;
-        }
-      }
-      // the tile's copies first, then its l and delta (their loads overlap the copies)
+    int issued = 0, k_issued = 0;
+    bool pok = true;
+    for (int m = 0; pok && m < n_items; ++m) {
+      const int k0 = ((int)blockIdx.x + m * (int)gridDim.x) * BK, I0 = m * nqt;
+      // the item's key tile, once the previous item's last score product has read
+      // the buffer
       if (lane == 0) {
-        issued = i + 1;
-        unsigned char *base = sm + C::OFF_ST + st * C::STAGE;
-        const int qrow = (int)(a.q_pad[b] + (t0 + i) * BQ);
-        mbar_arrive_expect_tx(&bars.q_full[st], C::STAGE);
-        for (int r = 0; r < C::KD; ++r) {
-          tma_load_2d(base + 2 * r * C::QB, &mQh, &bars.q_full[st], 64 * r, qrow);
-          tma_load_2d(base + (2 * r + 1) * C::QB, &mQl, &bars.q_full[st], 64 * r, qrow);
-          if (C::DK)
-            tma_load_2d(base + C::OFF_GO + r * C::QB, &mG, &bars.q_full[st], 64 * r, qrow);
+        if (m > 0 && nqt > 0 &&
+            !mbar_wait(&bars.s_full[(I0 - 1) & 1], ((I0 - 1) >> 1) & 1, abort, a.wait))
+          *abort = 1;
+        if (!*abort) {
+          k_issued = m + 1;
+          const int krow = (int)(a.k_pad[b] + k0);
+          mbar_arrive_expect_tx(&bars.k_full, 2 * C::K_BYTES);
+          for (int r = 0; r < C::KD; ++r) {
+            tma_load_2d(sm + r * BK * 128, &mKh, &bars.k_full, 64 * r, krow);
+            tma_load_2d(sm + C::K_BYTES + r * BK * 128, &mKl, &bars.k_full, 64 * r, krow);
+          }
         }
       }
-      for (int e = lane; e < BQ; e += 32) {
-        const int q = (t0 + i) * BQ + e;
-        const bool v = q < nq;
-        bars.lse2[st][e] = v ? a.lse[q_begin + q] * L2E : INFINITY;
-        bars.del[st][e] = (v && C::DK) ? a.delta[q_begin + q] : 0.f;
+      if (__any_sync(0xffffffffu, *abort)) {
+        pok = false;
+        break;
       }
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&bars.q_full[st]);
+      for (int i = 0; i < nqt; ++i) {
+        const int I = I0 + i, st = I % C::NS;  // I counts query tiles over the CTA's items
+        if (I >= C::NS) {
+          // DK: the last product that reads the stage is dK of tile I - NS, which starts
+          // after the rows are done with its l and delta; COLSUM: only S reads it, and
+          // the rows arrive after S has completed
+          uint64_t *fr = C::DK ? &bars.dk_done[st] : &bars.q_empty[st];
+          const bool w = __all_sync(0xffffffffu, mbar_wait(fr, ((I / C::NS) - 1) & 1, abort, a.wait));
+          if (!w) {
+            *abort = 1;
+            pok = false;
+            break;
+          }
+        }
+        // the tile's copies first, then its l and delta (their loads overlap the copies)
+        if (lane == 0) {
+          issued = I + 1;
+          unsigned char *base = sm + C::OFF_ST + st * C::STAGE;
+          const int qrow = (int)(a.q_pad[b] + (t0 + i) * BQ);
+          mbar_arrive_expect_tx(&bars.q_full[st], C::STAGE);
+          for (int r = 0; r < C::KD; ++r) {
+            tma_load_2d(base + 2 * r * C::QB, &mQh, &bars.q_full[st], 64 * r, qrow);
+            tma_load_2d(base + (2 * r + 1) * C::QB, &mQl, &bars.q_full[st], 64 * r, qrow);
+            if (C::DK)
+              tma_load_2d(base + C::OFF_GO + r * C::QB, &mG, &bars.q_full[st], 64 * r, qrow);
+          }
+        }
+        for (int e = lane; e < BQ; e += 32) {
+          const int q = (t0 + i) * BQ + e;
+          const bool v = q < nq;
+          bars.lse2[st][e] = v ? a.lse[q_begin + q] * L2E : INFINITY;
+          bars.del[st][e] = (v && C::DK) ? a.delta[q_begin + q] : 0.f;
+        }
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&bars.q_full[st]);
+      }
     }
     if (lane == 0 && *abort) {  // let issued copies land before shared memory is released
-      mbar_wait(&bars.k_full, 0);
-      for (int i = (issued > C::NS ? issued - C::NS : 0); i < issued; ++i)
-        mbar_wait(&bars.q_full[i % C::NS], (i / C::NS) & 1);
+      if (k_issued) mbar_wait(&bars.k_full, (k_issued - 1) & 1);
+      for (int I = (issued > C::NS ? issued - C::NS : 0); I < issued; ++I)
+        mbar_wait(&bars.q_full[I % C::NS], (I / C::NS) & 1);
     }
   } else if (warp == 9) {
     // ------------------------------------------------------------- MMA issuer
@@ -190,13 +215,11 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       const uint32_t id_s1 = idesc_bf16(BK, BQ, false, false);      // K_lo Q_hi
       const uint32_t id_dp = idesc_f16(BK, BQ, false, false);       // V Go (fp16)
       const uint32_t id_dk = idesc_bf16(BK, D, false, true);
-      bool ok = mbar_wait(&bars.k_full, 0, abort, a.wait);
-      fence_after_sync();
       const uint64_t kh0 = sdesc(smem_u32(sm), 16, 1024), kl0 = sdesc_add(kh0, C::K_BYTES);
       const uint32_t tv_hi = tmem + C::COL_V, tv_lo = tmem + C::COL_V + D / 2;
-      // S^T of tile i into the S buffer at column col
-      auto issue_s = [&](int i, uint32_t col) {
-        const uint32_t base = smem_u32(sm + C::OFF_ST + (i % C::NS) * C::STAGE);
+      // S^T of tile I into the S buffer at column col
+      auto issue_s = [&](int I, uint32_t col) {
+        const uint32_t base = smem_u32(sm + C::OFF_ST + (I % C::NS) * C::STAGE);
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
           const int r = kk >> 2;
@@ -207,10 +230,10 @@ __global__ void __launch_bounds__(NTHREADS, 1)
           mma_bf16(tmem + col, kl, qcat, id_s1, 1u);  // first N = BQ rows: Q_hi
         }
       };
-      // dP^T of tile i into dP buffer i & 1
-      auto issue_dp = [&](int i) {
-        const uint32_t base = smem_u32(sm + C::OFF_ST + (i % C::NS) * C::STAGE + C::OFF_GO);
-        const uint32_t col = C::COL_DP + (i & 1) * BQ;
+      // dP^T of tile I into dP buffer I & 1
+      auto issue_dp = [&](int I) {
+        const uint32_t base = smem_u32(sm + C::OFF_ST + (I % C::NS) * C::STAGE + C::OFF_GO);
+        const uint32_t col = C::COL_DP + (I & 1) * BQ;
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
           const uint64_t gd = sdesc(base + (kk >> 2) * C::QB + (kk & 3) * 32, 16, 1024);
@@ -218,176 +241,199 @@ __global__ void __launch_bounds__(NTHREADS, 1)
           mma_bf16_ts(tmem + col, tv_lo + kk * 8, gd, id_dp, 1u);
         }
       };
-      // dK += dS(i) Q(i): dS hi / lo over dP buffer i & 1, Q as the N-major operand
-      // (64-wide d blocks of Q_hi 2 QB apart, Q_lo one box further)
-      auto issue_dk = [&](int i) -> bool {
-        const int db = i & 1;
-        if (!mbar_wait(&bars.ds_full[db], (i >> 1) & 1, abort, a.wait)) return false;
+      // dK += dS(I) Q(I): dS hi / lo over dP buffer I & 1, Q as the N-major operand
+      // (64-wide d blocks of Q_hi 2 QB apart, Q_lo one box further); `first`: the
+      // item's first tile, whose product overwrites dK once the rows have read the
+      // previous item's dK
+      auto issue_dk = [&](int I, bool first, int m) -> bool {
+        const int db = I & 1;
+        if (!mbar_wait(&bars.ds_full[db], (I >> 1) & 1, abort, a.wait)) return false;
+        if (first && m > 0 && !mbar_wait(&bars.dk_free, (m - 1) & 1, abort, a.wait)) return false;
         fence_after_sync();
-        const uint32_t base = smem_u32(sm + C::OFF_ST + (i % C::NS) * C::STAGE);
+        const uint32_t base = smem_u32(sm + C::OFF_ST + (I % C::NS) * C::STAGE);
         const uint64_t qh0 = sdesc(base, 2 * C::QB, 1024), ql0 = sdesc(base + C::QB, 2 * C::QB, 1024);
         const uint32_t tds = tmem + C::COL_DP + db * BQ;  // dS hi at +0, lo at +BQ/2 columns
 #pragma unroll
         for (int kk = 0; kk < BQ / 16; ++kk) {
           const uint64_t qh = sdesc_add(qh0, kk * 2048), ql = sdesc_add(ql0, kk * 2048);
-          mma_bf16_ts(tmem + C::COL_DK, tds + kk * 8, qh, id_dk, (i > 0 || kk > 0) ? 1u : 0u);
+          mma_bf16_ts(tmem + C::COL_DK, tds + kk * 8, qh, id_dk, (!first || kk > 0) ? 1u : 0u);
           mma_bf16_ts(tmem + C::COL_DK, tds + kk * 8, ql, id_dk, 1u);
           mma_bf16_ts(tmem + C::COL_DK, tds + BQ / 2 + kk * 8, qh, id_dk, 1u);
         }
-        mma_commit(&bars.dk_done[i % C::NS]);  // frees dP buffer i & 1 and stage i % NS
+        mma_commit(&bars.dk_done[I % C::NS]);  // frees dP buffer I & 1 and stage I % NS
         return true;
       };
-      for (int i = 0; ok && i < nqt; ++i) {
-        const int st = i % C::NS;
-        if (!mbar_wait(&bars.q_full[st], (i / C::NS) & 1, abort, a.wait)) { ok = false; break; }
-        if (C::DK) {
-          // one S buffer: the rows of tile i - 1 have read it
-          if (i >= 1 && !mbar_wait(&bars.s_free[0], (i - 1) & 1, abort, a.wait)) { ok = false; break; }
-          fence_after_sync();
-          issue_s(i, 0);
-          mma_commit(&bars.s_full[i & 1]);  // per tile parity: each warpgroup waits its own
-          // V reaches tensor memory through the row threads (the first S runs meanwhile);
-          // dP buffer i & 1 held dS(i - 2) until dK(i - 2) drained it
-          if (i == 0 && !mbar_wait(&bars.v_full, 0, abort, a.wait)) { ok = false; break; }
-          if (i >= 2 && !mbar_wait(&bars.dk_done[(i - 2) % C::NS], ((i - 2) / C::NS) & 1, abort,
-                                   a.wait)) {
-            ok = false;
-            break;
+      bool ok = true;
+      for (int m = 0; ok && m < n_items; ++m) {
+        const int I0 = m * nqt;
+        if (!mbar_wait(&bars.k_full, m & 1, abort, a.wait)) { ok = false; break; }
+        for (int i = 0; ok && i < nqt; ++i) {
+          const int I = I0 + i, st = I % C::NS;
+          if (!mbar_wait(&bars.q_full[st], (I / C::NS) & 1, abort, a.wait)) { ok = false; break; }
+          if (C::DK) {
+            // one S buffer: the rows of tile I - 1 have read it
+            if (I >= 1 && !mbar_wait(&bars.s_free[0], (I - 1) & 1, abort, a.wait)) { ok = false; break; }
+            fence_after_sync();
+            issue_s(I, 0);
+            mma_commit(&bars.s_full[I & 1]);  // per tile parity: each warpgroup waits its own
+            // V reaches tensor memory through the row threads (the item's first S runs
+            // meanwhile); dP buffer I & 1 held dS(I - 2) until dK(I - 2) drained it
+            if (i == 0 && !mbar_wait(&bars.v_full, m & 1, abort, a.wait)) { ok = false; break; }
+            if (I >= 2 && !mbar_wait(&bars.dk_done[(I - 2) % C::NS], ((I - 2) / C::NS) & 1, abort,
+                                     a.wait)) {
+              ok = false;
+              break;
+            }
+            fence_after_sync();
+            issue_dp(I);
+            mma_commit(&bars.dp_full[I & 1]);
+            if (i >= 1 && !issue_dk(I - 1, i == 1, m)) { ok = false; break; }
+          } else {
+            const int sb = I & 1;
+            if (I >= 2 && !mbar_wait(&bars.s_free[sb], ((I >> 1) - 1) & 1, abort, a.wait)) {
+              ok = false;
+              break;
+            }
+            fence_after_sync();
+            issue_s(I, sb * 128);
+            mma_commit(&bars.s_full[sb]);
           }
-          fence_after_sync();
-          issue_dp(i);
-          mma_commit(&bars.dp_full[i & 1]);
-          if (i >= 1 && !issue_dk(i - 1)) { ok = false; break; }
-        } else {
-          const int sb = i & 1;
-          if (i >= 2 && !mbar_wait(&bars.s_free[sb], ((i >> 1) - 1) & 1, abort, a.wait)) {
-            ok = false;
-            break;
-          }
-          fence_after_sync();
-          issue_s(i, sb * 128);
-          mma_commit(&bars.s_full[sb]);
         }
+        if (ok && C::DK && nqt > 0) ok = issue_dk(I0 + nqt - 1, nqt == 1, m);
+        mma_commit(&bars.done);  // this item's products (also when the loop stopped early)
       }
-      if (ok && C::DK && nqt > 0) ok = issue_dk(nqt - 1);
-      mma_commit(&bars.done);
+      mma_commit(&bars.all_done);
       if (!ok) *abort = 1;
-      mbar_wait(&bars.done, 0);  // every MMA of this CTA has completed
+      mbar_wait(&bars.all_done, 0);  // every MMA of this CTA has completed
     }
   } else {
     // --------------------------------------------------------- key rows
-    const int wg = warp >> 2;  // warpgroup: query tiles i with i % 2 == wg
+    const int wg = warp >> 2;  // warpgroup: query tiles I with I % 2 == wg
     const int row = tid & (BK - 1);
-    const int kr = k0 + row;
-    const bool kvalid = kr < nk;
     const uint32_t lane_base = (uint32_t)((warp & 3) * 32) << 16;
-    if (C::DK) {
-      // this warpgroup's half of the value row, split into fp16 hi / lo, into tensor
-      // memory: the A operand of dP^T = V Go^T (rows past the problem are zero)
-      const float4 *v4 = reinterpret_cast<const float4 *>(a.v32 + (k_begin + kr) * D);
-#pragma unroll 1
-      for (int c0 = wg * 32; c0 < D / 2; c0 += 64) {  // packed columns c0 .. c0 + 31
-        uint32_t wh[32], wl[32];
-#pragma unroll
-        for (int e = 0; e < 16; ++e) {
-          const float4 v = kvalid ? v4[c0 / 2 + e] : make_float4(0.f, 0.f, 0.f, 0.f);
-          split_pack_f16(v.x, v.y, wh[2 * e], wl[2 * e]);
-          split_pack_f16(v.z, v.w, wh[2 * e + 1], wl[2 * e + 1]);
-        }
-        tmem_st32u(tmem + lane_base + C::COL_V + c0, wh);
-        tmem_st32u(tmem + lane_base + C::COL_V + D / 2 + c0, wl);
-      }
-      tmem_wait_st();
-      fence_before_sync();
-      mbar_arrive(&bars.v_full);
-    }
     const float sl2 = a.scale * L2E;
-    float imp = 0.f;
     bool ok = true;
-    for (int i = wg; i < nqt; i += 2) {
-      const int sb = i & 1, st = i % C::NS;
-      // S of tile i is signalled on s_full[i & 1] (phase i / 2) in both modes
-      ok = __all_sync(0xffffffffu, mbar_wait(&bars.s_full[sb], (i >> 1) & 1, abort, a.wait));
-      // the tile's l and delta were staged by the producer lanes: acquire them directly
-      ok = ok && __all_sync(0xffffffffu, mbar_wait(&bars.q_full[st], (i / C::NS) & 1, abort, a.wait));
-      if (!ok) break;
-      fence_after_sync();
-      float s[BQ];
-      {
-        float t[BQ];  // the two halves of the score product
-        const uint32_t col = C::DK ? 0u : (uint32_t)sb * 128u;
-        tmem_ld64x2(tmem + lane_base + col, s, tmem + lane_base + col + BQ, t);
-#pragma unroll
-        for (int c = 0; c < BQ; ++c) s[c] += t[c];
-      }
-      fence_before_sync();
-      mbar_arrive(&bars.s_free[C::DK ? 0 : sb]);
-      const float4 *l4 = reinterpret_cast<const float4 *>(bars.lse2[st]);
-      if (!C::DK) {
-#pragma unroll
-        for (int c4 = 0; c4 < BQ / 4; ++c4) {  // l = +inf past the problem
-          const float4 l = l4[c4];
-          imp += ex2(fmaf(s[4 * c4], sl2, -l.x)) + ex2(fmaf(s[4 * c4 + 1], sl2, -l.y)) +
-                 ex2(fmaf(s[4 * c4 + 2], sl2, -l.z)) + ex2(fmaf(s[4 * c4 + 3], sl2, -l.w));
-        }
-      } else {
-        ok = __all_sync(0xffffffffu, mbar_wait(&bars.dp_full[sb], (i >> 1) & 1, abort, a.wait));
+    for (int m = 0; ok && m < n_items; ++m) {
+      const int k0 = ((int)blockIdx.x + m * (int)gridDim.x) * BK, I0 = m * nqt;
+      const int kr = k0 + row;
+      const bool kvalid = kr < nk;
+      if (C::DK) {
+        // the previous item's last dP product has read V from tensor memory
+        if (m > 0 && nqt > 0)
+          ok = __all_sync(0xffffffffu, mbar_wait(&bars.dp_full[(I0 - 1) & 1], ((I0 - 1) >> 1) & 1,
+                                                 abort, a.wait));
         if (!ok) break;
         fence_after_sync();
-        const uint32_t tdp = tmem + lane_base + C::COL_DP + sb * BQ;
-        float dp[BQ];
-        tmem_ld64(tdp, dp);
-        uint32_t hh[BQ / 2], ll[BQ / 2];
-        const float4 *d4 = reinterpret_cast<const float4 *>(bars.del[st]);
+        // this warpgroup's half of the value row, split into fp16 hi / lo, into tensor
+        // memory: the A operand of dP^T = V Go^T (rows past the problem are zero)
+        const float4 *v4 = reinterpret_cast<const float4 *>(a.v32 + (k_begin + kr) * D);
+#pragma unroll 1
+        for (int c0 = wg * 32; c0 < D / 2; c0 += 64) {  // packed columns c0 .. c0 + 31
+          uint32_t wh[32], wl[32];
 #pragma unroll
-        for (int c4 = 0; c4 < BQ / 4; ++c4) {
-          // queries past the problem have l = +inf (p = 0), delta = 0 and zero Q and
-          // Go rows; rows of keys past it only feed their own dK rows, which are not
-          // stored
-          const float4 l = l4[c4], dl = d4[c4];
-          const int c = 4 * c4;
-          const float v0 = ex2(fmaf(s[c], sl2, -l.x)) * (dp[c] - dl.x);
-          const float v1 = ex2(fmaf(s[c + 1], sl2, -l.y)) * (dp[c + 1] - dl.y);
-          const float v2 = ex2(fmaf(s[c + 2], sl2, -l.z)) * (dp[c + 2] - dl.z);
-          const float v3 = ex2(fmaf(s[c + 3], sl2, -l.w)) * (dp[c + 3] - dl.w);
-          split_pack(v0, v1, hh[2 * c4], ll[2 * c4]);
-          split_pack(v2, v3, hh[2 * c4 + 1], ll[2 * c4 + 1]);
+          for (int e = 0; e < 16; ++e) {
+            const float4 v = kvalid ? v4[c0 / 2 + e] : make_float4(0.f, 0.f, 0.f, 0.f);
+            split_pack_f16(v.x, v.y, wh[2 * e], wl[2 * e]);
+            split_pack_f16(v.z, v.w, wh[2 * e + 1], wl[2 * e + 1]);
+          }
+          tmem_st32u(tmem + lane_base + C::COL_V + c0, wh);
+          tmem_st32u(tmem + lane_base + C::COL_V + D / 2 + c0, wl);
         }
-        // dS (hi, lo) over this tile's dP buffer: the A operand of dK += dS Q
-        tmem_st32u(tdp, hh);
-        tmem_st32u(tdp + BQ / 2, ll);
         tmem_wait_st();
         fence_before_sync();
-        mbar_arrive(&bars.ds_full[sb]);
+        mbar_arrive(&bars.v_full);
       }
-      if (!C::DK) mbar_arrive(&bars.q_empty[st]);
-    }
-    if (!ok) *abort = 1;
-    if (C::DK) {
-      if (!mbar_wait(&bars.done, 0, abort, a.wait)) *abort = 1;
-      fence_after_sync();
-      const float dks = a.scale / go_scale(nq, D, a.w_out);  // score scale, Go's scale undone
+      float imp = 0.f;
+      // this warpgroup's tiles: I % 2 == wg (I counts query tiles over the CTA's items)
+      for (int I = I0 + ((I0 ^ wg) & 1); I < I0 + nqt; I += 2) {
+        const int sb = I & 1, st = I % C::NS;
+        // S of tile I is signalled on s_full[I & 1] (phase I / 2) in both modes
+        ok = __all_sync(0xffffffffu, mbar_wait(&bars.s_full[sb], (I >> 1) & 1, abort, a.wait));
+        // the tile's l and delta were staged by the producer lanes: acquire them directly
+        ok = ok && __all_sync(0xffffffffu, mbar_wait(&bars.q_full[st], (I / C::NS) & 1, abort, a.wait));
+        if (!ok) break;
+        fence_after_sync();
+        float s[BQ];
+        {
+          float t[BQ];  // the two halves of the score product
+          const uint32_t col = C::DK ? 0u : (uint32_t)sb * 128u;
+          tmem_ld64x2(tmem + lane_base + col, s, tmem + lane_base + col + BQ, t);
+#pragma unroll
+          for (int c = 0; c < BQ; ++c) s[c] += t[c];
+        }
+        fence_before_sync();
+        mbar_arrive(&bars.s_free[C::DK ? 0 : sb]);
+        const float4 *l4 = reinterpret_cast<const float4 *>(bars.lse2[st]);
+        if (!C::DK) {
+#pragma unroll
+          for (int c4 = 0; c4 < BQ / 4; ++c4) {  // l = +inf past the problem
+            const float4 l = l4[c4];
+            imp += ex2(fmaf(s[4 * c4], sl2, -l.x)) + ex2(fmaf(s[4 * c4 + 1], sl2, -l.y)) +
+                   ex2(fmaf(s[4 * c4 + 2], sl2, -l.z)) + ex2(fmaf(s[4 * c4 + 3], sl2, -l.w));
+          }
+        } else {
+          ok = __all_sync(0xffffffffu, mbar_wait(&bars.dp_full[sb], (I >> 1) & 1, abort, a.wait));
+          if (!ok) break;
+          fence_after_sync();
+          const uint32_t tdp = tmem + lane_base + C::COL_DP + sb * BQ;
+          float dp[BQ];
+          tmem_ld64(tdp, dp);
+          uint32_t hh[BQ / 2], ll[BQ / 2];
+          const float4 *d4 = reinterpret_cast<const float4 *>(bars.del[st]);
+#pragma unroll
+          for (int c4 = 0; c4 < BQ / 4; ++c4) {
+            // queries past the problem have l = +inf (p = 0), delta = 0 and zero Q and
+            // Go rows; rows of keys past it only feed their own dK rows, which are not
+            // stored
+            const float4 l = l4[c4], dl = d4[c4];
+            const int c = 4 * c4;
+            const float v0 = ex2(fmaf(s[c], sl2, -l.x)) * (dp[c] - dl.x);
+            const float v1 = ex2(fmaf(s[c + 1], sl2, -l.y)) * (dp[c + 1] - dl.y);
+            const float v2 = ex2(fmaf(s[c + 2], sl2, -l.z)) * (dp[c + 2] - dl.z);
+            const float v3 = ex2(fmaf(s[c + 3], sl2, -l.w)) * (dp[c + 3] - dl.w);
+            split_pack(v0, v1, hh[2 * c4], ll[2 * c4]);
+            split_pack(v2, v3, hh[2 * c4 + 1], ll[2 * c4 + 1]);
+          }
+          // dS (hi, lo) over this tile's dP buffer: the A operand of dK += dS Q
+          tmem_st32u(tdp, hh);
+          tmem_st32u(tdp + BQ / 2, ll);
+          tmem_wait_st();
+          fence_before_sync();
+          mbar_arrive(&bars.ds_full[sb]);
+        }
+        if (!C::DK) mbar_arrive(&bars.q_empty[st]);
+      }
+      if (!ok) *abort = 1;
+      if (C::DK) {
+        if (!mbar_wait(&bars.done, m & 1, abort, a.wait)) *abort = 1;
+        fence_after_sync();
+        const float dks = a.scale / go_scale(nq, D, a.w_out);  // score scale, Go's scale undone
 #pragma unroll 1
-      for (int c0 = wg * (D / 2); c0 < (wg + 1) * (D / 2); c0 += 32) {
-        float o[32];
-        tmem_ld32(tmem + lane_base + C::COL_DK + c0, o);
-        if (nqt == 0) {  // a split without query tiles contributes zero
+        for (int c0 = wg * (D / 2); c0 < (wg + 1) * (D / 2); c0 += 32) {
+          float o[32];
+          tmem_ld32(tmem + lane_base + C::COL_DK + c0, o);
+          if (nqt == 0) {  // a split without query tiles contributes zero
 #pragma unroll
-          for (int e = 0; e < 32; ++e) o[e] = 0.f;
-        }
-        if (kvalid) {
-          float4 *dst = reinterpret_cast<float4 *>(a.dk + blockIdx.z * a.dk_stride +
-                                                   (k_begin + kr) * D + c0);
+            for (int e = 0; e < 32; ++e) o[e] = 0.f;
+          }
+          if (kvalid) {
+            float4 *dst = reinterpret_cast<float4 *>(a.dk + blockIdx.z * a.dk_stride +
+                                                     (k_begin + kr) * D + c0);
 #pragma unroll
-          for (int e = 0; e < 8; ++e)
-            dst[e] = make_float4(o[4 * e] * dks, o[4 * e + 1] * dks, o[4 * e + 2] * dks,
-                                 o[4 * e + 3] * dks);
+            for (int e = 0; e < 8; ++e)
+              dst[e] = make_float4(o[4 * e] * dks, o[4 * e + 1] * dks, o[4 * e + 2] * dks,
+                                   o[4 * e + 3] * dks);
+          }
         }
+        // dK is read: the next item's first dK product may overwrite it
+        fence_before_sync();
+        mbar_arrive(&bars.dk_free);
+      } else {
+        if (wg == 1) bars.imp[row] = imp;
+        rows_sync();
+        if (wg == 0 && kvalid) a.imp[k_begin + kr] = imp + bars.imp[row];
+        rows_sync();  // the next item writes bars.imp again
       }
-    } else {
-      if (wg == 1) bars.imp[row] = imp;
-      rows_sync();
-      if (wg == 0 && kvalid) a.imp[k_begin + kr] = imp + bars.imp[row];
     }
   }
   fence_before_sync();
@@ -402,19 +448,22 @@ __global__ void __launch_bounds__(NTHREADS, 1)
 }  // namespace
 
 template <int D, int MODE>
-int launch_bwd_tc(const BwdMaps &m, const BwdArgs &a, int max_tiles, int B, cudaStream_t st) {
+int launch_bwd_tc(const BwdMaps &m, const BwdArgs &a, int max_tiles, int items, int B,
+                  cudaStream_t st) {
   using C = Bwd<D, MODE>;
   static_assert(C::SMEM + sizeof(BwdBars) <= 232448, "shared memory");
   auto kern = k_attn_bwd<D, MODE>;
   KVS_CUDA_TRY(set_smem_once(kern, C::SMEM));
-  kern<<<dim3(max_tiles, B, a.nsplit), NTHREADS, C::SMEM, st>>>(m.kh, m.kl, m.qh, m.ql, m.g, a);
+  // each CTA takes up to `items` key tiles of its problem, one after another
+  const int gx = (max_tiles + items - 1) / items;
+  kern<<<dim3(gx, B, a.nsplit), NTHREADS, C::SMEM, st>>>(m.kh, m.kl, m.qh, m.ql, m.g, a);
   KVS_LAUNCH_CHECK("k_attn_bwd");
   return KVS_OK;
 }
 
-template int launch_bwd_tc<64, BWD_DK>(const BwdMaps &, const BwdArgs &, int, int, cudaStream_t);
-template int launch_bwd_tc<128, BWD_DK>(const BwdMaps &, const BwdArgs &, int, int, cudaStream_t);
-template int launch_bwd_tc<64, BWD_COLSUM>(const BwdMaps &, const BwdArgs &, int, int, cudaStream_t);
-template int launch_bwd_tc<128, BWD_COLSUM>(const BwdMaps &, const BwdArgs &, int, int, cudaStream_t);
+template int launch_bwd_tc<64, BWD_DK>(const BwdMaps &, const BwdArgs &, int, int, int, cudaStream_t);
+template int launch_bwd_tc<128, BWD_DK>(const BwdMaps &, const BwdArgs &, int, int, int, cudaStream_t);
+template int launch_bwd_tc<64, BWD_COLSUM>(const BwdMaps &, const BwdArgs &, int, int, int, cudaStream_t);
+template int launch_bwd_tc<128, BWD_COLSUM>(const BwdMaps &, const BwdArgs &, int, int, int, cudaStream_t);
 
 }  // namespace kvs

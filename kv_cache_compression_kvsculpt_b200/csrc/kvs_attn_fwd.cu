@@ -44,7 +44,6 @@ constexpr int BN = FWD_BN;       // keys per tile
 constexpr int HB = BN / 2;       // keys of a tile per row warpgroup
 constexpr int NTHREADS = 320;
 constexpr float kRescale = 8.f;  // lazy rescale threshold (log2 units)
-constexpr int FWD_ITEMS = 3;     // query tiles per CTA
 constexpr float L2E = 1.4426950408889634f;
 static_assert(BN == 128, "tensor-memory layout assumes 128-key tiles");
 
@@ -600,26 +599,27 @@ __global__ void __launch_bounds__(NTHREADS, 1)
 }  // namespace
 
 template <int D, int MODE>
-int launch_fwd_tc(const FwdMaps &m, const FwdArgs &a, int max_tiles, int B, cudaStream_t st) {
+int launch_fwd_tc(const FwdMaps &m, const FwdArgs &a, int max_tiles, int items, int B,
+                  cudaStream_t st) {
   using C = Fwd<D, MODE>;
   static_assert(C::SMEM + sizeof(FwdBars) <= 232448, "shared memory");
   auto kern = k_attn_fwd<D, MODE>;
   KVS_CUDA_TRY(set_smem_once(kern, C::SMEM));
-  // each CTA takes up to FWD_ITEMS query tiles of its problem, one after another
-  const int gx = (max_tiles + FWD_ITEMS - 1) / FWD_ITEMS;
+  // each CTA takes up to `items` query tiles of its problem, one after another
+  const int gx = (max_tiles + items - 1) / items;
   kern<<<dim3(gx, B), NTHREADS, C::SMEM, st>>>(m.kh, m.kl, m.vh, m.vl, m.qh, m.ql,
                                                MODE == FWD_LOSS ? m.y : m.kh, a);
   KVS_LAUNCH_CHECK("k_attn_fwd");
   return KVS_OK;
 }
 
-template int launch_fwd_tc<64, FWD_LOSS>(const FwdMaps &, const FwdArgs &, int, int, cudaStream_t);
-template int launch_fwd_tc<128, FWD_LOSS>(const FwdMaps &, const FwdArgs &, int, int, cudaStream_t);
-template int launch_fwd_tc<64, FWD_TARGETS>(const FwdMaps &, const FwdArgs &, int, int, cudaStream_t);
-template int launch_fwd_tc<128, FWD_TARGETS>(const FwdMaps &, const FwdArgs &, int, int, cudaStream_t);
-template int launch_fwd_tc<64, FWD_STATS>(const FwdMaps &, const FwdArgs &, int, int, cudaStream_t);
-template int launch_fwd_tc<128, FWD_STATS>(const FwdMaps &, const FwdArgs &, int, int, cudaStream_t);
-template int launch_fwd_tc<64, FWD_WRITE_A>(const FwdMaps &, const FwdArgs &, int, int, cudaStream_t);
-template int launch_fwd_tc<128, FWD_WRITE_A>(const FwdMaps &, const FwdArgs &, int, int, cudaStream_t);
+template int launch_fwd_tc<64, FWD_LOSS>(const FwdMaps &, const FwdArgs &, int, int, int, cudaStream_t);
+template int launch_fwd_tc<128, FWD_LOSS>(const FwdMaps &, const FwdArgs &, int, int, int, cudaStream_t);
+template int launch_fwd_tc<64, FWD_TARGETS>(const FwdMaps &, const FwdArgs &, int, int, int, cudaStream_t);
+template int launch_fwd_tc<128, FWD_TARGETS>(const FwdMaps &, const FwdArgs &, int, int, int, cudaStream_t);
+template int launch_fwd_tc<64, FWD_STATS>(const FwdMaps &, const FwdArgs &, int, int, int, cudaStream_t);
+template int launch_fwd_tc<128, FWD_STATS>(const FwdMaps &, const FwdArgs &, int, int, int, cudaStream_t);
+template int launch_fwd_tc<64, FWD_WRITE_A>(const FwdMaps &, const FwdArgs &, int, int, int, cudaStream_t);
+template int launch_fwd_tc<128, FWD_WRITE_A>(const FwdMaps &, const FwdArgs &, int, int, int, cudaStream_t);
 
 }  // namespace kvs

@@ -18,6 +18,12 @@ constexpr int FWD_BN = 128;
 // Queries of one tile of the key-tile kernel (the TMA box height of its query
 // and Go maps).
 constexpr int BWD_BQ = 64;
+// Tiles one CTA takes in turn (its grid is ceil(tiles / items)): key tiles of the
+// key-tile kernel and query tiles of the query-tile kernel, for a whole batch and
+// for a sub-batch that shares the GPU with others.
+constexpr int BWD_ITEMS = 2;
+constexpr int FWD_ITEMS = 3;
+constexpr int FWD_ITEMS_SHARED = 3;
 
 // dL/dY_hat = c (Y_hat - Y), c = 2 w_out / (n_q d), is carried as fp16 scaled by
 // sigma = 2^-round(log2 c) (so that it sits in fp16's normal range; 1 when c = 0):
@@ -104,9 +110,11 @@ struct GemmArgs3 {
 };
 
 template <int D, int MODE>
-int launch_fwd_tc(const FwdMaps &m, const FwdArgs &a, int max_tiles, int B, cudaStream_t st);
+int launch_fwd_tc(const FwdMaps &m, const FwdArgs &a, int max_tiles, int items, int B,
+                  cudaStream_t st);
 template <int D, int MODE>
-int launch_bwd_tc(const BwdMaps &m, const BwdArgs &a, int max_tiles, int B, cudaStream_t st);
+int launch_bwd_tc(const BwdMaps &m, const BwdArgs &a, int max_tiles, int items, int B,
+                  cudaStream_t st);
 int launch_gemm3_tc(const GemmMaps &m, const GemmArgs3 &a, int tiles_m, int gram, int B,
                     cudaStream_t st);
 

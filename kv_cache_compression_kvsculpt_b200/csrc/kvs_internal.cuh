@@ -108,7 +108,8 @@ struct Batch {
   HostGeom g;
   const kvs_batch *b;
   cudaStream_t st;
-  int slot = 0;  // sub-batch index of a partitioned solve (its own internal streams)
+  int slot = 0;   // sub-batch index of a partitioned solve (its own internal streams)
+  int share = 1;  // sub-batches that run at the same time (each sizes its grids for 1/share of the SMs)
 };
 
 // ---- attention contractions (kvs_attn.cu) ----
