@@ -255,11 +255,15 @@ static int lbfgs_restart(const Batch &Bt, const kvs_schedule &sc, const float *Q
 
 // One L-BFGS step in three parts: direction (and the bf16 split of the pairs),
 // the Armijo trial loop, then dK_c at the accepted points and the history update.
+// K_c is split again every step (a failed search leaves its last rejected trial's
+// split in the workspace); V_c, fixed during a step, only when the caller has not
+// kept its split resident (inside kvs_compress_batch the L-BFGS reset after each
+// value fit split it).
 static int step_head(const Batch &Bt, const kvs_schedule &sc, const float *Kc, const float *Vc,
-                     const State &s, const Work &w) {
+                     const State &s, const Work &w, bool v_ready) {
   int rc = launch_lbfgs_direction(Bt, s, sc);
   if (rc) return rc;
-  return launch_split_pairs(Bt, Kc, Vc, w);  // V_c is fixed during the step
+  return launch_split_pairs(Bt, Kc, v_ready ? nullptr : Vc, w);
 }
 
 static int step_trial(const Batch &Bt, const kvs_schedule &sc, const float *Q, const float *Y,
@@ -284,7 +288,7 @@ static int lbfgs_one_step(const Batch &Bt, const kvs_schedule &sc, const float *
                           const float *Y, const float *lse, const float *Vc, float *Kc,
                           const State &s, int32_t *status, float *f_out, bool q_ready,
                           const Work &w) {
-  int rc = step_head(Bt, sc, Kc, Vc, s, w);
+  int rc = step_head(Bt, sc, Kc, Vc, s, w, q_ready);
   if (rc) return rc;
   for (int t = 0; t < sc.max_bt; ++t)  // problems that have left the search skip each trial
     if ((rc = step_trial(Bt, sc, Q, Y, lse, Vc, Kc, s, q_ready || t > 0, w, nullptr))) return rc;
@@ -318,7 +322,7 @@ static int build_step_graph(const Batch &Bcaller, const kvs_schedule &sc, const 
   Bt.st = sg->cap;
   const uint64_t n0 = g_launches.load(std::memory_order_relaxed);
   KVS_CUDA_TRY(cudaStreamBeginCapture(Bt.st, cudaStreamCaptureModeThreadLocal));
-  int rc = step_head(Bt, sc, Kc, Vc, s, w);
+  int rc = step_head(Bt, sc, Kc, Vc, s, w, true);
   cudaStreamCaptureStatus cst;
   cudaGraph_t g = nullptr;
   const cudaGraphNode_t *deps = nullptr;
