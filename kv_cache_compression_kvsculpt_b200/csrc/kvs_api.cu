@@ -255,15 +255,16 @@ static int lbfgs_restart(const Batch &Bt, const kvs_schedule &sc, const float *Q
 
 // One L-BFGS step in three parts: direction (and the bf16 split of the pairs),
 // the Armijo trial loop, then dK_c at the accepted points and the history update.
-// K_c is split again every step (a failed search leaves its last rejected trial's
-// split in the workspace); V_c, fixed during a step, only when the caller has not
-// kept its split resident (inside kvs_compress_batch the L-BFGS reset after each
-// value fit split it).
+// When the caller keeps the splits resident (inside kvs_compress_batch: the reset
+// after each value fit split K_c and V_c, and every accepted trial leaves its own
+// split), only the problems whose last search failed, and so left a rejected
+// trial's split in the workspace, split K_c again; otherwise K_c and V_c are split.
 static int step_head(const Batch &Bt, const kvs_schedule &sc, const float *Kc, const float *Vc,
-                     const State &s, const Work &w, bool v_ready) {
+                     const State &s, const Work &w, bool resident) {
   int rc = launch_lbfgs_direction(Bt, s, sc);
   if (rc) return rc;
-  return launch_split_pairs(Bt, Kc, v_ready ? nullptr : Vc, w);
+  if (resident) return launch_split_pairs(Bt, Kc, nullptr, w, stale_filter(s));
+  return launch_split_pairs(Bt, Kc, Vc, w);
 }
 
 static int step_trial(const Batch &Bt, const kvs_schedule &sc, const float *Q, const float *Y,

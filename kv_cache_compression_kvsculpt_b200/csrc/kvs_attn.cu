@@ -114,10 +114,12 @@ namespace {
 
 // Problem b's rows x[off[b] ..] split into (hi, lo) at rows pad[b] .. of the padded
 // operand buffers; the rows between its own count and the padded count are zero.
+// Problems the filter leaves out keep their split.
 __global__ void k_split_pad(const float *__restrict__ x, const int64_t *off, const int64_t *pad,
                             int d, __nv_bfloat16 *__restrict__ hi,
-                            __nv_bfloat16 *__restrict__ lo) {
+                            __nv_bfloat16 *__restrict__ lo, Filter flt) {
   const int b = blockIdx.y;
+  if (flt.skip(b)) return;
   const int64_t v4 = (off[b + 1] - off[b]) * d / 4;  // d is a multiple of 4
   const int64_t n4 = (pad[b + 1] - pad[b]) * d / 4;
   const float4 *src = reinterpret_cast<const float4 *>(x + off[b] * d);
@@ -136,12 +138,13 @@ __global__ void k_split_pad(const float *__restrict__ x, const int64_t *off, con
 
 // x [rows by off] -> padded (hi, lo) by pad; max_rows: the largest padded count.
 int split_pad(const float *x, const int64_t *off, const int64_t *pad, int64_t max_rows, int d,
-              __nv_bfloat16 *hi, __nv_bfloat16 *lo, int B, cudaStream_t st) {
+              __nv_bfloat16 *hi, __nv_bfloat16 *lo, int B, cudaStream_t st,
+              Filter flt = Filter{nullptr, 0, 0}) {
   const int64_t n4 = max_rows * d / 4;
   if (n4 == 0) return KVS_OK;
   const int per = (int)std::max<int64_t>(1, std::min<int64_t>((n4 + 255) / 256,
                                                               std::max(1, 4096 / B)));
-  k_split_pad<<<dim3(per, B), 256, 0, st>>>(x, off, pad, d, hi, lo);
+  k_split_pad<<<dim3(per, B), 256, 0, st>>>(x, off, pad, d, hi, lo, flt);
   KVS_LAUNCH_CHECK("k_split_pad");
   return KVS_OK;
 }
@@ -317,9 +320,10 @@ int targets_d(const Batch &Bt, const float *Q, const float *Kz, const float *Vz,
 
 // bf16 hi/lo copies of the keys and values of the compressed pairs.
 template <int D>
-int prep_pairs(const Batch &Bt, const float *Kc, const float *Vc, const Work &w) {
+int prep_pairs(const Batch &Bt, const float *Kc, const float *Vc, const Work &w,
+               Filter kflt = Filter{nullptr, 0, 0}) {
   const HostGeom &g = Bt.g;
-  int rc = split_pad(Kc, Bt.b->c_off, w.c_pad, max_pad(g.max_c), D, w.kh, w.kl, g.B, Bt.st);
+  int rc = split_pad(Kc, Bt.b->c_off, w.c_pad, max_pad(g.max_c), D, w.kh, w.kl, g.B, Bt.st, kflt);
   if (rc || !Vc) return rc;
   return split_pad(Vc, Bt.b->c_off, w.c_pad, max_pad(g.max_c), D, w.vh, w.vl, g.B, Bt.st);
 }
@@ -514,8 +518,9 @@ int launch_forward(const Batch &Bt, const float *Q, const float *Kc, const float
                                        q_ready, pairs_ready, reduce, w);
 }
 
-int launch_split_pairs(const Batch &Bt, const float *Kc, const float *Vc, const Work &w) {
-  return Bt.g.d == 64 ? prep_pairs<64>(Bt, Kc, Vc, w) : prep_pairs<128>(Bt, Kc, Vc, w);
+int launch_split_pairs(const Batch &Bt, const float *Kc, const float *Vc, const Work &w,
+                       Filter kflt) {
+  return Bt.g.d == 64 ? prep_pairs<64>(Bt, Kc, Vc, w, kflt) : prep_pairs<128>(Bt, Kc, Vc, w, kflt);
 }
 
 int launch_backward(const Batch &Bt, const float *Vc, float w_out, float *dKc, Filter flt,

@@ -129,7 +129,9 @@ int launch_forward(const Batch &B, const float *Q, const float *Kc, const float 
                    float *parts, Filter flt, bool q_ready, const Work &w,
                    bool pairs_ready = false, bool reduce = true);
 // bf16 hi/lo copies of the compressed pairs (keys; values unless Vc is null).
-int launch_split_pairs(const Batch &B, const float *Kc, const float *Vc, const Work &w);
+// kflt: the problems whose K_c split is redone (all by default).
+int launch_split_pairs(const Batch &B, const float *Kc, const float *Vc, const Work &w,
+                       Filter kflt = Filter{nullptr, 0, 0});
 // dKc from the state left by launch_forward for the same problems (with the same
 // values Vc and output weight w_out).
 int launch_backward(const Batch &B, const float *Vc, float w_out, float *dKc, Filter flt,
