@@ -108,6 +108,20 @@ int make_map_f32(CUtensorMap *m, const void *base, uint64_t rows, uint64_t cols,
   return make_map_2d(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, base, rows, cols, box_rows);
 }
 
+// Multiprocessor count of the current device, cached per device (several host
+// threads may ask at once: relaxed atomics, the value is the same for all).
+int sm_count() {
+  static std::atomic<int> n[64];
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 148;
+  int v = n[dev].load(std::memory_order_relaxed);
+  if (v > 0) return v;
+  if (cudaDeviceGetAttribute(&v, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || v <= 0)
+    v = 148;
+  n[dev].store(v, std::memory_order_relaxed);
+  return v;
+}
+
 namespace {
 
 // ------------------------------------------------------ elementwise helpers
@@ -189,20 +203,6 @@ __global__ void k_loss_reduce(const float *partials, int tiles, const int64_t *q
 }
 
 int max_qtiles(const HostGeom &g) { return (g.max_q + 127) / 128; }
-
-// Multiprocessor count of the current device, cached per device (several host
-// threads may ask at once: relaxed atomics, the value is the same for all).
-int sm_count() {
-  static std::atomic<int> n[64];
-  int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 148;
-  int v = n[dev].load(std::memory_order_relaxed);
-  if (v > 0) return v;
-  if (cudaDeviceGetAttribute(&v, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || v <= 0)
-    v = 148;
-  n[dev].store(v, std::memory_order_relaxed);
-  return v;
-}
 
 // Work items per CTA of the attention kernels.  A whole batch takes several
 // query (key) tiles per CTA, so that each CTA's setup and epilogue overlap its next
