@@ -149,9 +149,6 @@ struct CholTcArgs {
 int launch_chol_update_tc(const CholTcMaps &m, const CholTcArgs &a, int j0, int max_c,
                           cudaStream_t st);
 
-// Multiprocessor count of the current device (cached).
-int sm_count();
-
 // Host: a 2-D bf16 tensor map over [rows, cols] (row-major) with a
 // [box_rows, 64]-element box and 128-byte swizzle.
 int make_map_bf16(CUtensorMap *m, const void *base, uint64_t rows, uint64_t cols,

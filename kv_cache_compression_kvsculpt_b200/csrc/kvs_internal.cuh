@@ -143,6 +143,9 @@ int launch_fit(const Batch &B, const float *Q, const float *Kc, const float *Y, 
                float *Vc, int32_t *status, bool q_ready, bool y_ready, const Work &w,
                Filter stats = Filter{nullptr, 0, 0});
 
+// Multiprocessor count of the current device (cached).
+int sm_count();
+
 // ---- other kernels ----
 int launch_build_queries(const kvs_query_spec *sp, const float *q_retain, const float *q_ctx,
                          const int32_t *pos, float *Q, cudaStream_t st);
