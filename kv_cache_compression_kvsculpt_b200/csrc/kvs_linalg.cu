@@ -523,54 +523,62 @@ __global__ void __launch_bounds__(256) k_chol_panel(CholArgs a, int j0) {
 
 // The whole backward sweep for 64 right-hand-side columns of one problem, from
 // the last panel to the first: x_j = T_j^T y_j (stored, checked finite), then
-// y_i -= L_ji^T x_j for every i < j.  The next L_ji tile is fetched into
-// registers while the current one is multiplied (two shared tiles in turn).
-constexpr int BWD_SMEM = 3 * NB * SP * 4;
+// y_i -= L_ji^T x_j for every i < j.  Two groups of 256 threads take the
+// independent products of a step in turn (group g the rows i = g (mod 2)), so
+// that sixteen warps hide the shared-memory latency of the 64 x 64 x 64
+// products; each group fetches its next L_ji tile into registers while it
+// multiplies the current one (two shared tiles per group in turn).
+constexpr int BWD_SMEM = 5 * NB * SP * 4;
 
-__global__ void __launch_bounds__(256) k_chol_backward(CholArgs a) {
+__global__ void __launch_bounds__(512, 1) k_chol_backward(CholArgs a) {
   extern __shared__ __align__(16) float bsm[];
+  const int tid = threadIdx.x, grp = tid >> 8, tl = tid & 255;
   float (*Xs)[SP] = reinterpret_cast<float (*)[SP]>(bsm);
-  float (*At[2])[SP] = {reinterpret_cast<float (*)[SP]>(bsm + NB * SP),
-                        reinterpret_cast<float (*)[SP]>(bsm + 2 * NB * SP)};
+  float (*At[2])[SP] = {reinterpret_cast<float (*)[SP]>(bsm + (1 + 2 * grp) * NB * SP),
+                        reinterpret_cast<float (*)[SP]>(bsm + (2 + 2 * grp) * NB * SP)};
+  float (*Ts)[SP] = reinterpret_cast<float (*)[SP]>(bsm + NB * SP);  // group 0's first tile
   const int b = blockIdx.y;
   const int k = kdim(a, b);
   if (a.dead[b]) return;
   const int c0 = blockIdx.x * NB;
   const int np = (k + NB - 1) / NB;
-  const int tid = threadIdx.x;
-  const int tx = tid & 15, ty = tid >> 4;
+  const int tx = tl & 15, ty = tl >> 4;
   const int64_t row0 = a.c_off[b];
   const float *G = a.G + row0 * a.ld;
   float *R = a.R + row0 * a.d;
   for (int p = np - 1; p >= 0; --p) {
     const int j0 = p * NB, jb = min(NB, k - j0);
     const float *Tg = a.Tt + ((int64_t)b * a.npanel + p) * NB * NB;
-    load_t(At[0], Tg, NB, 0, NB, 0, NB);          // At[t][r] = T[t][r]
+    load_t(Ts, Tg, NB, 0, NB, 0, NB);             // Ts[t][r] = T[t][r]
     load_d(Xs, R, a.d, j0, j0 + jb, c0, a.d);     // Xs[t][col] = y[j0 + t][c0 + col]
     __syncthreads();
     float acc[4][4];
-    zero_acc(acc);
-    mmk(At[0], Xs, acc, tx, ty);                  // x[r][col]
-    __syncthreads();
-    bool fin = true;
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      const int r = 4 * ty + i;
-      const float4 v = make_float4(acc[i][0], acc[i][1], acc[i][2], acc[i][3]);
-      st4(&Xs[r][4 * tx], v);  // as the B operand of the updates
-      if (r < jb) {
-        st4(a.X + (row0 + j0 + r) * a.d + c0 + 4 * tx, v);
-        fin &= isfinite(v.x) && isfinite(v.y) && isfinite(v.z) && isfinite(v.w);
-      }
+    if (grp == 0) {
+      zero_acc(acc);
+      mmk(Ts, Xs, acc, tx, ty);                   // x[r][col]
     }
-    if (!fin) atomicOr(&a.dead[b], DEAD_NONFINITE);
+    __syncthreads();
+    if (grp == 0) {
+      bool fin = true;
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const int r = 4 * ty + i;
+        const float4 v = make_float4(acc[i][0], acc[i][1], acc[i][2], acc[i][3]);
+        st4(&Xs[r][4 * tx], v);  // as the B operand of the updates
+        if (r < jb) {
+          st4(a.X + (row0 + j0 + r) * a.d + c0 + 4 * tx, v);
+          fin &= isfinite(v.x) && isfinite(v.y) && isfinite(v.z) && isfinite(v.w);
+        }
+      }
+      if (!fin) atomicOr(&a.dead[b], DEAD_NONFINITE);
+    }
     if (p == 0) break;
     // y_i -= L_ji^T x_j, with At[t][r] = L[j0 + t][64 i + r]
     float4 pf[4];
     auto fetch = [&](int i) {
 #pragma unroll
       for (int u = 0; u < 4; ++u) {
-        const int e = tid + 256 * u, r = e >> 4, c = (e & 15) * 4;
+        const int e = tl + 256 * u, r = e >> 4, c = (e & 15) * 4;
         pf[u] = r < jb ? ld4(G + (int64_t)(j0 + r) * a.ld + NB * i + c)
                        : make_float4(0.f, 0.f, 0.f, 0.f);
       }
@@ -578,27 +586,37 @@ __global__ void __launch_bounds__(256) k_chol_backward(CholArgs a) {
     auto place = [&](float (*S)[SP]) {
 #pragma unroll
       for (int u = 0; u < 4; ++u) {
-        const int e = tid + 256 * u, r = e >> 4, c = (e & 15) * 4;
+        const int e = tl + 256 * u, r = e >> 4, c = (e & 15) * 4;
         st4(&S[r][c], pf[u]);
       }
     };
-    fetch(0);
-    place(At[0]);
+    // both groups take the same number of rounds (and barriers); group 1 has no
+    // product in the last round when p is odd
+    const int rounds = (p + 1) / 2;
+    if (grp < p) {
+      fetch(grp);
+      place(At[0]);
+    }
     __syncthreads();
-    for (int i = 0; i < p; ++i) {
+    for (int q = 0; q < rounds; ++q) {
+      const int i = 2 * q + grp;
+      const bool act = i < p, more = i + 2 < p;
       float4 cur[4];
+      if (act)
 #pragma unroll
-      for (int ii = 0; ii < 4; ++ii)
-        cur[ii] = ld4(R + (int64_t)(NB * i + 4 * ty + ii) * a.d + c0 + 4 * tx);
-      if (i + 1 < p) fetch(i + 1);
-      zero_acc(acc);
-      mmk(At[i & 1], Xs, acc, tx, ty);
+        for (int ii = 0; ii < 4; ++ii)
+          cur[ii] = ld4(R + (int64_t)(NB * i + 4 * ty + ii) * a.d + c0 + 4 * tx);
+      if (more) fetch(i + 2);
+      if (act) {
+        zero_acc(acc);
+        mmk(At[q & 1], Xs, acc, tx, ty);
 #pragma unroll
-      for (int ii = 0; ii < 4; ++ii)
-        st4(R + (int64_t)(NB * i + 4 * ty + ii) * a.d + c0 + 4 * tx,
-            make_float4(cur[ii].x - acc[ii][0], cur[ii].y - acc[ii][1], cur[ii].z - acc[ii][2],
-                        cur[ii].w - acc[ii][3]));
-      if (i + 1 < p) place(At[(i + 1) & 1]);
+        for (int ii = 0; ii < 4; ++ii)
+          st4(R + (int64_t)(NB * i + 4 * ty + ii) * a.d + c0 + 4 * tx,
+              make_float4(cur[ii].x - acc[ii][0], cur[ii].y - acc[ii][1], cur[ii].z - acc[ii][2],
+                          cur[ii].w - acc[ii][3]));
+      }
+      if (more) place(At[(q + 1) & 1]);
       __syncthreads();
     }
   }
@@ -702,7 +720,7 @@ int launch_chol_solve(const Batch &Bt, float *Vc, int32_t *status, const Work &w
       KVS_CUDA_TRY(cudaEventRecord(la->updated[p & 1], Bt.st));
     }
   }
-  k_chol_backward<<<dim3(ndc, g.B), 256, BWD_SMEM, Bt.st>>>(a);
+  k_chol_backward<<<dim3(ndc, g.B), 512, BWD_SMEM, Bt.st>>>(a);
   KVS_LAUNCH_CHECK("k_chol_backward");
   const int64_t n4 = (int64_t)g.max_c * g.d / 4;
   const int blocks = (int)std::min<int64_t>((n4 + 255) / 256, 64);
