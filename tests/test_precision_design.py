@@ -111,6 +111,37 @@ def test_split_gram_and_fp32_cholesky_meet_the_value_bar(point):
     assert rel(fit_emulated(mm_single, Q, Kc, Y)) > 1e-3
 
 
+def tf32(x, nearest=True):
+    """float32 values kept to tf32's 10 mantissa bits: rounded to nearest (ties to
+    even), or truncated, which is what the tensor cores do with the low bits of
+    an fp32 operand they are handed as tf32."""
+    x = np.ascontiguousarray(np.asarray(x, np.float32))
+    v = x.view(np.uint32).copy()
+    if nearest:
+        v = v + np.uint32(0xFFF) + ((v >> np.uint32(13)) & np.uint32(1))
+    v &= np.uint32(0xFFFFE000)
+    return v.view(np.float32).astype(np.float64)
+
+
+def test_single_pass_tf32_leaves_no_margin(point):
+    """tf32 operands (the other input type the tensor cores take at fp32
+    accumulation) in one pass: rounded to nearest they land just inside the
+    gradient and value bars at the optimised point, with no margin for a full
+    solve's steps to stay near the float64 trajectory; as the hardware truncates
+    raw fp32 operands they miss the gradient bar."""
+    Q, Kc, Vc, Y, lse = point
+    f0, g0, _ = O.loss_grad(Q, Kc, Vc, Y, lse)
+    Vo, _ = O.ridge_fit(Q, Kc, Y, 1e-3)
+    rel = lambda V: float(np.linalg.norm(V - Vo) / np.linalg.norm(Vo))
+    mm_rn = lambda a, b: tf32(a) @ tf32(b)
+    mm_tr = lambda a, b: tf32(a, False) @ tf32(b, False)
+    f, g = loss_grad_emulated(mm_rn, Q, Kc, Vc, Y, lse)
+    assert abs(f - f0) <= 1e-3 * f0 and 0.999 <= _cos(g, g0) < 0.9995
+    assert 5e-4 < rel(fit_emulated(mm_rn, Q, Kc, Y)) <= 1e-3
+    _, g1 = loss_grad_emulated(mm_tr, Q, Kc, Vc, Y, lse)
+    assert _cos(g1, g0) < 0.999
+
+
 def f16(x):
     return np.asarray(x, np.float32).astype(np.float16).astype(np.float64)
 
