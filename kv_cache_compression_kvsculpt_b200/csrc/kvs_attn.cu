@@ -464,8 +464,8 @@ int fit_d(const Batch &Bt, const float *Q, const float *Kc, const float *Y, floa
   a.a_pad_off = w.a_pad_off;
   if ((rc = launch_fwd_tc<D, FWD_WRITE_A>(fm, a, max_qtiles(g), fwd_items(Bt), g.B, Bt.st))) return rc;
   GemmMaps gm;
-  if ((rc = make_map_bf16(&gm.ah, w.ahi, g.sum_qpad, g.ld_a, 64)) ||
-      (rc = make_map_bf16(&gm.al, w.alo, g.sum_qpad, g.ld_a, 64)))
+  if ((rc = make_map_bf16(&gm.ah, w.ahi, g.sum_qpad, g.ld_a, 32)) ||
+      (rc = make_map_bf16(&gm.al, w.alo, g.sum_qpad, g.ld_a, 32)))
     return rc;
   gm.bh = gm.ah;
   gm.bl = gm.al;
@@ -480,8 +480,10 @@ int fit_d(const Batch &Bt, const float *Q, const float *Kc, const float *Y, floa
   ga.err = w.err;
   ga.wait = wait_limit();
   const int tm = (g.max_c + 127) / 128;
-  if ((rc = launch_gemm3_tc(gm, ga, tm, 1, g.B, Bt.st))) return rc;
-  if ((rc = make_map_bf16(&gm.bh, w.yh, g.sum_qpad, D, 64)) ||
+  if ((rc = launch_gram2_tc(gm, ga, tm, g.B, Bt.st))) return rc;
+  if ((rc = make_map_bf16(&gm.ah, w.ahi, g.sum_qpad, g.ld_a, 64)) ||
+      (rc = make_map_bf16(&gm.al, w.alo, g.sum_qpad, g.ld_a, 64)) ||
+      (rc = make_map_bf16(&gm.bh, w.yh, g.sum_qpad, D, 64)) ||
       (rc = make_map_bf16(&gm.bl, w.yl, g.sum_qpad, D, 64)))
     return rc;
   ga.n_fixed = D;
@@ -489,7 +491,7 @@ int fit_d(const Batch &Bt, const float *Q, const float *Kc, const float *Y, floa
   ga.c = w.R;
   ga.ldc = D;
   ga.diag = 0.f;
-  if ((rc = launch_gemm3_tc(gm, ga, tm, 0, g.B, Bt.st))) return rc;
+  if ((rc = launch_gemm3_tc(gm, ga, tm, g.B, Bt.st))) return rc;
   return launch_chol_solve(Bt, Vc, status, w);
 }
 

@@ -99,7 +99,7 @@ struct GemmMaps {
 struct GemmArgs3 {
   const int64_t *a_pad_off;  // [B+1] padded K (query) row offsets of both operands' buffers
   const int64_t *m_off;      // [B+1] M extents (keys)
-  int n_fixed;               // N extent when > 0 (e.g. d), else N = M extent (Gram)
+  int n_fixed;               // N extent of A^T Y (d); unused by the Gram
   const int64_t *b_row_off;  // [B+1] K-row offsets of the B operand (Gram: = a_pad_off)
   float *c;                  // output rows at m_off[b], ld = ldc
   int64_t ldc;
@@ -115,8 +115,10 @@ int launch_fwd_tc(const FwdMaps &m, const FwdArgs &a, int max_tiles, int items, 
 template <int D, int MODE>
 int launch_bwd_tc(const BwdMaps &m, const BwdArgs &a, int max_tiles, int items, int B,
                   cudaStream_t st);
-int launch_gemm3_tc(const GemmMaps &m, const GemmArgs3 &a, int tiles_m, int gram, int B,
-                    cudaStream_t st);
+// R = A^T Y (N = a.n_fixed = d) in 128 x d tiles (maps with 64-row boxes).
+int launch_gemm3_tc(const GemmMaps &m, const GemmArgs3 &a, int tiles_m, int B, cudaStream_t st);
+// The Gram matrix A^T A + diag I in 256 x 256 tiles (maps with 32-row boxes).
+int launch_gram2_tc(const GemmMaps &m, const GemmArgs3 &a, int tiles_m, int B, cudaStream_t st);
 
 // Trailing update of the blocked ridge Cholesky (64-column panels) on tensor
 // cores.  The panel's factor columns L (rows below the diagonal block) and the
